@@ -1,0 +1,312 @@
+"""Oracle arithmetic for the hybrid CSA/HCA attention layer (float64 NumPy).
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py`` for who may use it).
+
+Everything here is the plain definition, computed one entry / one query at a
+time, with no blocking, fusion or reordering beyond what the definition
+states.  Sources, by page title and section:
+
+  [Tricks]  "DeepSeek V4 Architecture Tricks" (pinktalk.online), sections
+            "CSA: Compressed Sparse Attention", "HCA: Heavily Compressed
+            Attention", "压缩 KV 的具体 trick", "Sliding Window Branch".
+  [QbitAI]  QbitAI write-up of the V4 report (admirer.cn), section
+            "混合注意力機制" (steps one to three of CSA, HCA, the sliding
+            window branch and its strict-causality remark).
+  [Report]  "[DeepSeek-5] DeepSeek-V4 Technical Report: Hybrid Attention and
+            Post-Training for Million-Token Contexts" (xutianle.me),
+            section 3 (CSA), section 4 (HCA), section 5 (heterogeneous cache).
+  [Jiedu]   "DeepSeek-V4技术报告解读" (yetianai.com), section
+            "核心创新一：混合注意力机制（CSA+HCA）".
+
+Readings taken where the pages are silent (each is also listed in the design
+notes):
+  * Overlapped CSA compression: entry i pools the 2m tokens
+    [(i-1)m, (i+1)m); positional-bias rows 0..m-1 go with the previous block,
+    rows m..2m-1 with the current block; the same candidate and logit tensors
+    serve both halves.  Entry 0 has no previous block: the missing slots are
+    left out of the softmax (not zero-padded).
+  * A trailing incomplete block produces no entry: N = floor(T / m).
+  * Causality: a query at 0-based position t sees compressed entry s iff the
+    last token of the entry's block, (s+1)*rate - 1, is <= t.
+  * Sliding window: raw tokens [max(0, t-n_win+1), t] (t itself included),
+    attended in the same softmax as the compressed entries, even where they
+    cover the same tokens.
+  * Lightning-indexer score: I(t,s) = sum_j w[t,j] * ReLU(q[t,j,:] . K[s,:]),
+    no scale; the pages only say the indexer is the lightweight one inherited
+    from DeepSeek-V3.2 ([QbitAI], CSA step two) with 64 heads of dim 128
+    ([Tricks], CSA section).
+  * Top-k order: score descending, ties by entry index ascending; all visible
+    entries when fewer than k are visible.
+  * Compressed entries are stored as bf16 (the cache format); the oracle
+    rounds its float64 compressor output to bf16 (round-to-nearest-even, via
+    float32) before it is attended or indexed.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "round_bf16", "softmax", "csa_compress", "hca_compress",
+    "compress_weights_csa", "compress_weights_hca", "n_visible",
+    "indexer_scores", "topk_select", "window_rows", "mqa_attend",
+    "mqa_partial", "combine_partials", "csa_layer_prefill",
+    "hca_layer_prefill", "csa_layer_decode", "hca_layer_decode",
+]
+
+
+# ----------------------------------------------------------------------------
+# storage format
+# ----------------------------------------------------------------------------
+def round_bf16(x) -> np.ndarray:
+    """Round to the nearest bf16 value (ties to even), returned as float64.
+
+    bf16 keeps the top 16 bits of an IEEE float32.  The value is first
+    rounded to float32 (NumPy's cast, nearest-even), then the low 16 bits
+    are rounded away with ties to even.  Finite inputs only.
+    """
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    u = (u + np.uint64(0x7FFF) + lsb) & np.uint64(0xFFFF0000)
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def softmax(z: np.ndarray, axis: int) -> np.ndarray:
+    """Max-subtracted softmax in float64."""
+    z = np.asarray(z, dtype=np.float64)
+    e = np.exp(z - np.max(z, axis=axis, keepdims=True))
+    return e / np.sum(e, axis=axis, keepdims=True)
+
+
+# ----------------------------------------------------------------------------
+# (1) KV compressor  ([Tricks] "压缩 KV 的具体 trick"; [QbitAI] CSA step one,
+#     HCA paragraph; [Report] sections 3 and 4)
+# ----------------------------------------------------------------------------
+def _csa_window(i: int, m: int, T: int):
+    """Token range pooled by CSA entry i, and the bias row of its first token."""
+    lo = max(0, (i - 1) * m)
+    hi = min(T, (i + 1) * m)
+    bias_row0 = lo - (i - 1) * m  # m for entry 0 (no previous block), else 0
+    return lo, hi, bias_row0
+
+
+def compress_weights_csa(logits: np.ndarray, pos_bias: np.ndarray, m: int, i: int) -> np.ndarray:
+    """Softmax weights [tokens, channels] that CSA entry i puts on its tokens.
+
+    Per channel j: softmax over the tokens r of the window of
+    (logit Z[r, j] + positional bias B[r - (i-1)m, j]).
+    """
+    T = logits.shape[0]
+    lo, hi, b0 = _csa_window(i, m, T)
+    z = logits[lo:hi] + pos_bias[b0:b0 + (hi - lo)]
+    return softmax(z, axis=0)
+
+
+def csa_compress(cand: np.ndarray, logits: np.ndarray, pos_bias: np.ndarray, m: int) -> np.ndarray:
+    """Overlapped CSA compression: [T, c] -> [floor(T/m), c] (float64, unrounded).
+
+    E[i, j] = sum_{r in W(i)} softmax_r(Z[r, j] + B[r - (i-1)m, j]) * C[r, j],
+    W(i) = [(i-1)m, (i+1)m) intersected with [0, T).  Each token therefore
+    contributes to its own block's entry and to the next one (the overlap
+    with the previous adjacent block that [Tricks] describes).
+    """
+    cand = np.asarray(cand, dtype=np.float64)
+    logits = np.asarray(logits, dtype=np.float64)
+    pos_bias = np.asarray(pos_bias, dtype=np.float64)
+    T, c = cand.shape
+    assert logits.shape == (T, c) and pos_bias.shape == (2 * m, c)
+    n = T // m
+    out = np.zeros((n, c), dtype=np.float64)
+    for i in range(n):
+        lo, hi, _ = _csa_window(i, m, T)
+        w = compress_weights_csa(logits, pos_bias, m, i)
+        out[i] = np.sum(w * cand[lo:hi], axis=0)
+    return out
+
+
+def compress_weights_hca(logits: np.ndarray, pos_bias: np.ndarray, m_hca: int, i: int) -> np.ndarray:
+    """Softmax weights [m', channels] of HCA entry i (block [i m', (i+1) m'))."""
+    lo = i * m_hca
+    return softmax(logits[lo:lo + m_hca] + pos_bias, axis=0)
+
+
+def hca_compress(cand: np.ndarray, logits: np.ndarray, pos_bias: np.ndarray, m_hca: int) -> np.ndarray:
+    """HCA compression, no overlap: [T, c] -> [floor(T/m'), c] (float64, unrounded).
+
+    E_h[i, j] = sum_{r in [i m', (i+1) m')} softmax_r(Z[r, j] + B[r - i m', j]) * C[r, j].
+    """
+    cand = np.asarray(cand, dtype=np.float64)
+    logits = np.asarray(logits, dtype=np.float64)
+    pos_bias = np.asarray(pos_bias, dtype=np.float64)
+    T, c = cand.shape
+    assert logits.shape == (T, c) and pos_bias.shape == (m_hca, c)
+    n = T // m_hca
+    out = np.zeros((n, c), dtype=np.float64)
+    for i in range(n):
+        w = compress_weights_hca(logits, pos_bias, m_hca, i)
+        out[i] = np.sum(w * cand[i * m_hca:(i + 1) * m_hca], axis=0)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# (4) causal visibility  ([QbitAI] sliding-window paragraph: compressed
+#     attention is strictly causal, a query cannot see its own incomplete block)
+# ----------------------------------------------------------------------------
+def n_visible(t: int, rate: int, n_entries: int) -> int:
+    """Number of compressed entries visible to a query at position t.
+
+    Entry s is visible iff (s+1)*rate - 1 <= t, i.e. s < floor((t+1)/rate);
+    the entries visible are therefore always the prefix [0, n_visible).
+    """
+    return int(min(n_entries, (t + 1) // rate))
+
+
+def window_rows(t: int, n_win: int) -> np.ndarray:
+    """Raw-token positions of the sliding window of a query at t ([Tricks]
+    "Sliding Window Branch": the most recent n_win = 128 uncompressed tokens)."""
+    return np.arange(max(0, t - n_win + 1), t + 1)
+
+
+# ----------------------------------------------------------------------------
+# (2) lightning indexer and top-k  ([QbitAI] CSA step two; [Tricks] CSA section)
+# ----------------------------------------------------------------------------
+def indexer_scores(q_idx: np.ndarray, w_idx: np.ndarray, k_idx: np.ndarray) -> np.ndarray:
+    """Scores of one query against entries: I(s) = sum_j w[j] * ReLU(q[j,:] . K[s,:]).
+
+    q_idx [H_I, d_I], w_idx [H_I], k_idx [N, d_I] -> [N] float64.
+    """
+    q = np.asarray(q_idx, dtype=np.float64)
+    w = np.asarray(w_idx, dtype=np.float64)
+    k = np.asarray(k_idx, dtype=np.float64)
+    dots = k @ q.T                      # [N, H_I]: q_j . K_s
+    return np.maximum(dots, 0.0) @ w    # sum_j w_j ReLU(.)
+
+
+def topk_select(scores: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the min(k, N) largest scores, ordered by (score desc, index asc)."""
+    scores = np.asarray(scores, dtype=np.float64)
+    n = scores.shape[0]
+    order = np.lexsort((np.arange(n), -scores))
+    return order[:min(k, n)].astype(np.int64)
+
+
+# ----------------------------------------------------------------------------
+# (3) core multi-query attention with shared K = V  ([QbitAI] CSA step three
+#     and the remark that KV entries serve as both key and value; c = 512)
+# ----------------------------------------------------------------------------
+def mqa_partial(q: np.ndarray, rows: np.ndarray, scale: float):
+    """Unnormalised softmax state of MQA over a row set.
+
+    q [H, c], rows [U, c] (each row is key and value) ->
+    (m [H], l [H], o [H, c]) with m_h = max_u s_hu, l_h = sum_u exp(s_hu - m_h),
+    o_h = sum_u exp(s_hu - m_h) rows_u, s_hu = scale * q_h . rows_u.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    rows = np.asarray(rows, dtype=np.float64)
+    s = scale * (q @ rows.T)                       # [H, U]
+    mx = np.max(s, axis=1)
+    e = np.exp(s - mx[:, None])
+    return mx, np.sum(e, axis=1), e @ rows
+
+
+def mqa_attend(q: np.ndarray, rows: np.ndarray, scale: float) -> np.ndarray:
+    """o_h = sum_u softmax_u(scale * q_h . rows_u) rows_u; q [H, c], rows [U, c]."""
+    mx, l, o = mqa_partial(q, rows, scale)
+    return o / l[:, None]
+
+
+def combine_partials(parts) -> np.ndarray:
+    """Merge softmax states of disjoint row subsets:
+    o = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i, M = max_i m_i."""
+    ms = np.stack([p[0] for p in parts])          # [P, H]
+    M = np.max(ms, axis=0)
+    num = sum(np.exp(p[0] - M)[:, None] * p[2] for p in parts)
+    den = sum(np.exp(p[0] - M) * p[1] for p in parts)
+    return num / den[:, None]
+
+
+# ----------------------------------------------------------------------------
+# whole layers
+# ----------------------------------------------------------------------------
+def csa_layer_prefill(cand, logits, kidx_cand, pos_bias, q_idx, w_idx, q, *,
+                      m, topk, d_idx, n_win, scale, queries=None):
+    """CSA layer over one sequence of T raw tokens, for the given query positions.
+
+    cand/logits [T, c]; kidx_cand [T, d_I] (per-token indexer-key candidates,
+    compressed with the same compressor using logits[:, :d_I] and
+    pos_bias[:, :d_I]); q_idx [T, H_I, d_I]; w_idx [T, H_I]; q [T, H, c].
+    Returns dict with E [N, c] and K_I [N, d_I] (bf16-valued float64), and per
+    query: the selected indices (ordered), their scores, the visible count and
+    the output o [H, c].
+    """
+    T = cand.shape[0]
+    E = round_bf16(csa_compress(cand, logits, pos_bias, m))
+    K_I = round_bf16(csa_compress(kidx_cand, np.asarray(logits)[:, :d_idx],
+                                  np.asarray(pos_bias)[:, :d_idx], m))
+    N = E.shape[0]
+    qs = range(T) if queries is None else queries
+    res = {"E": E, "K_I": K_I, "idx": {}, "scores": {}, "n_vis": {}, "O": {}}
+    cand64 = np.asarray(cand, dtype=np.float64)
+    for t in qs:
+        nv = n_visible(t, m, N)
+        sc = indexer_scores(q_idx[t], w_idx[t], K_I[:nv])
+        sel = topk_select(sc, topk)
+        rows = np.concatenate([E[sel], cand64[window_rows(t, n_win)]], axis=0)
+        res["idx"][t] = sel
+        res["scores"][t] = sc
+        res["n_vis"][t] = nv
+        res["O"][t] = mqa_attend(q[t], rows, scale)
+    return res
+
+
+def hca_layer_prefill(cand, logits, pos_bias, q, *, m_hca, n_win, scale, queries=None):
+    """HCA layer over one sequence: dense attention over every visible HCA
+    entry plus the sliding window ([Tricks] HCA section: no top-k selector)."""
+    T = cand.shape[0]
+    E = round_bf16(hca_compress(cand, logits, pos_bias, m_hca))
+    N = E.shape[0]
+    qs = range(T) if queries is None else queries
+    cand64 = np.asarray(cand, dtype=np.float64)
+    res = {"E": E, "n_vis": {}, "O": {}}
+    for t in qs:
+        nv = n_visible(t, m_hca, N)
+        rows = np.concatenate([E[:nv], cand64[window_rows(t, n_win)]], axis=0)
+        res["n_vis"][t] = nv
+        res["O"][t] = mqa_attend(q[t], rows, scale)
+    return res
+
+
+def csa_layer_decode(E, K_I, win, q, q_idx, w_idx, t, *, m, topk, n_win, scale):
+    """One decode query of one request against its CSA cache.
+
+    E [N, c] compressed entries, K_I [N, d_I] indexer keys, win [n_win, c]
+    the raw rows of the last min(n_win, t+1) tokens (first rows valid, any
+    order), q [H, c], q_idx [H_I, d_I], w_idx [H_I].
+    """
+    nv = n_visible(t, m, E.shape[0])
+    sc = indexer_scores(q_idx, w_idx, K_I[:nv])
+    sel = topk_select(sc, topk)
+    nw = min(n_win, t + 1)
+    rows = np.concatenate([np.asarray(E, dtype=np.float64)[sel],
+                           np.asarray(win, dtype=np.float64)[:nw]], axis=0)
+    return {"idx": sel, "scores": sc, "n_vis": nv, "O": mqa_attend(q, rows, scale)}
+
+
+def hca_layer_decode(E_h, block_cand, block_logits, pos_bias, win, q, t, *, m_hca, n_win, scale):
+    """One decode query of one request against its HCA cache, including the
+    compression of the newest complete block ([Report] section 5 and [Jiedu]
+    cache layout: the tail block is kept raw until it completes).
+
+    E_h [N_h, c] holds entries 0..n-2 where n = floor((t+1)/m') is the number
+    of complete blocks; block_cand/block_logits [m', c] are the raw rows of the
+    newest complete block (tokens [(n-1) m', n m')), whose entry n-1 is
+    computed here.  Returns the new entry and o [H, c].
+    """
+    n = (t + 1) // m_hca
+    assert (t + 1) % m_hca == 0, "the newest block completes at t"
+    new = round_bf16(hca_compress(block_cand, block_logits, pos_bias, m_hca))  # [1, c]
+    Eh = np.concatenate([np.asarray(E_h, dtype=np.float64)[:n - 1], new], axis=0)
+    nw = min(n_win, t + 1)
+    rows = np.concatenate([Eh, np.asarray(win, dtype=np.float64)[:nw]], axis=0)
+    return {"new_entry": new[0], "O": mqa_attend(q, rows, scale)}
