@@ -1,0 +1,550 @@
+#!/usr/bin/env python3
+"""Benchmark of the hybrid CSA/HCA attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: hybrid_decode_b8_1m -- a CSA layer and an HCA layer decoded
+back to back for 8 requests at 1,048,576 tokens of context (CSA: 262,144
+compressed entries x 512 + indexer keys x 128, 64 indexer heads, top-1024;
+HCA: 8,192 entries; 128-row windows; 64 query heads x 512).  Metric: decode
+queries per second (one query = one request's step through both layers).
+Other workloads: csa_prefill_64k (tokens/s), csa_decode_b32_128k and
+hca_decode_b16_1m (queries/s).
+
+One process per GPU; under torchrun every rank runs the same per-GPU
+workload on its own requests (weak scaling, no collective on the data path),
+timing is the max over ranks.  Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_attention_compress_b200 import workloads as wl  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+MIB = 1 << 20
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, local, ws
+
+
+def init_dist(backend):
+    import datetime
+    import torch.distributed as dist
+    rank, local, ws = dist_env()
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, local, ws
+
+
+def reduce_max(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def shard_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own requests: disjoint seeds, same distribution."""
+    return seed + 1_000_000 * rank
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.proc is None:
+            return False
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+        return False
+
+    def summary(self):
+        if not getattr(self, "rows", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ----------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def traffic_table():
+    """ncu DRAM bytes per launch, keyed by kernel, valid only for the source hash it was taken on."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return {}
+    try:
+        return json.load(open(p))
+    except ValueError:
+        return {}
+
+
+def source_hash(files):
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "long_context_attention_compress_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+class DecodeBench:
+    """Hybrid / CSA / HCA decode.  Per step: one hybrid_attn_decode call."""
+
+    def __init__(self, name, spec, seed, device):
+        import long_context_attention_compress_b200 as hca
+        self.hca = hca
+        self.name = name
+        self.spec = spec
+        s = self.shape = spec["shape"]
+        B, ctx = spec["B"], spec["ctx"]
+        self.B, self.ctx = B, ctx
+        kind = spec["kind"]
+        std = spec["cache_std"]
+        self.csa = self.hcad = None
+        if kind == "hybrid_decode":
+            d = wl.hybrid_decode_inputs(s, B, ctx, seed=seed, cache_std=std, device=device)
+            self.csa, self.hcad = d["csa"], d["hca"]
+        elif kind == "csa_decode":
+            self.csa = wl.csa_decode_inputs(s, B, ctx, seed=seed, cache_std=std, device=device)
+        else:
+            self.hcad = wl.hca_decode_inputs(s, B, ctx, seed=seed, cache_std=std, device=device)
+        self.cfg = hca.make_cfg(s)
+        dev = device
+        self.q_pos = (self.csa or self.hcad)["q_pos"]
+        self.idx = torch.empty((B, s.topk), dtype=torch.int32, device=dev) if self.csa else None
+        self.csa_out = torch.empty((B, s.n_heads, s.c), dtype=torch.bfloat16, device=dev) if self.csa else None
+        self.hca_out = torch.empty((B, s.n_heads, s.c), dtype=torch.bfloat16, device=dev) if self.hcad else None
+        self.phases = []
+        if self.hcad is not None and "block_cand" in self.hcad:
+            self.phases.append("hca_compress")
+        if self.csa is not None:
+            self.phases += ["indexer_scores", "topk_select", "csa_attention"]
+        if self.hcad is not None:
+            self.phases.append("hca_attention")
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
+        self.args, self._keep = hca.make_decode_args(B, self.q_pos, csa=self.csa, hca=self.hcad,
+                                                     csa_topk_idx=self.idx, csa_out=self.csa_out,
+                                                     hca_out=self.hca_out, events=self.events)
+        self.ws = torch.empty(max(1, hca.hybrid_attn_decode_workspace(self.cfg, self.args)), dtype=torch.uint8,
+                              device=dev)
+        self.units = B
+        self.metric = "hybrid CSA+HCA decode queries/s at 1M ctx"
+        self.unit = "queries/s"
+
+    def step(self, record=True):
+        self.args.n_events = len(self.events) if record else 0
+        self.hca.hybrid_attn_decode(self.cfg, self.args, ws=self.ws)
+
+    def launches_per_step(self):
+        return int(self.hca.lib.hca_last_launch_count())
+
+    # algorithmic HBM bytes per phase (what the method must move)
+    def phase_bytes(self):
+        s, B = self.shape, self.B
+        out = {}
+        if "hca_compress" in self.phases:
+            out["hca_compress"] = B * (2 * s.m_hca * s.c * 2 + s.c * 2)
+        if self.csa is not None:
+            N = self.csa["E"].shape[1]
+            out["indexer_scores"] = B * (N * s.d_idx * 2 + s.n_idx_heads * (s.d_idx * 2 + 4))
+            out["topk_select"] = B * s.topk * 4
+            out["csa_attention"] = B * ((min(s.topk, N) + s.n_win) * s.c * 2 + 2 * s.n_heads * s.c * 2 + s.topk * 4)
+        if self.hcad is not None:
+            Nh = self.hcad["E_h"].shape[1]
+            out["hca_attention"] = B * ((Nh + s.n_win) * s.c * 2 + 2 * s.n_heads * s.c * 2)
+        return out
+
+    def config(self):
+        s = self.shape
+        c = {"workload": self.name, "batch": self.B, "context": self.ctx, "c": s.c, "heads": s.n_heads,
+             "topk": s.topk, "indexer": f"{s.n_idx_heads}x{s.d_idx}", "n_win": s.n_win}
+        if self.csa is not None:
+            c["csa_entries"] = int(self.csa["E"].shape[1])
+        if self.hcad is not None:
+            c["hca_entries"] = int(self.hcad["E_h"].shape[1])
+        return c
+
+    # --- end to end: per-step inputs from pinned host memory, outputs back ---
+    def e2e_setup(self):
+        self.h_in, self.d_in, self.h_out, self.d_out = [], [], [], []
+        for d in (self.csa, self.hcad):
+            if d is None:
+                continue
+            for k in ("q", "q_idx", "w_idx", "win", "block_cand", "block_logits"):
+                if k in d:
+                    self.d_in.append(d[k])
+                    self.h_in.append(torch.empty(d[k].shape, dtype=d[k].dtype, pin_memory=True).copy_(d[k].cpu()))
+        for t in (self.idx, self.csa_out, self.hca_out):
+            if t is not None:
+                self.d_out.append(t)
+                self.h_out.append(torch.empty(t.shape, dtype=t.dtype, pin_memory=True))
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+
+    def e2e_step(self):
+        for h, d in zip(self.h_in, self.d_in):
+            d.copy_(h, non_blocking=True)
+        self.step(record=False)
+        for h, d in zip(self.h_out, self.d_out):
+            h.copy_(d, non_blocking=True)
+
+    # --- CPU oracle on a bounded sample of requests ---
+    def oracle_sample(self, n_req):
+        import oracle
+        s = self.shape
+        t = self.ctx - 1
+        spec = self.spec
+        t0 = time.perf_counter()
+        for b in range(n_req):
+            if self.csa is not None:
+                d = wl.csa_decode_inputs(s, 1, self.ctx, seed=900 + b, cache_std=spec["cache_std"])
+                f = lambda x: x[0].float().numpy().astype(np.float64)  # noqa: E731
+                oracle.csa_layer_decode(f(d["E"]), f(d["K_I"]), f(d["win"]), f(d["q"]), f(d["q_idx"]),
+                                        d["w_idx"][0].double().numpy(), t, m=s.m, topk=s.topk, n_win=s.n_win,
+                                        scale=s.scale)
+            if self.hcad is not None:
+                wb = "block_cand" in self.hcad
+                d = wl.hca_decode_inputs(s, 1, self.ctx, seed=900 + b, cache_std=spec["cache_std"], with_block=wb)
+                f = lambda x: x[0].float().numpy().astype(np.float64)  # noqa: E731
+                if wb:
+                    oracle.hca_layer_decode(f(d["E_h"]), f(d["block_cand"]), f(d["block_logits"]),
+                                            d["bias_hca"].double().numpy(), f(d["win"]), f(d["q"]), t,
+                                            m_hca=s.m_hca, n_win=s.n_win, scale=s.scale)
+                else:
+                    oracle.mqa_attend(f(d["q"]), np.concatenate([f(d["E_h"]), f(d["win"])]), s.scale)
+        return time.perf_counter() - t0
+
+
+class PrefillBench:
+    """CSA prefill of one 65,536-token sequence (compress, indexer + top-k, sparse MQA)."""
+
+    def __init__(self, name, spec, seed, device):
+        import long_context_attention_compress_b200 as hca
+        self.hca = hca
+        self.name = name
+        s = self.shape = spec["shape"]
+        T = self.T = spec["T"]
+        self.inp = wl.prefill_inputs(s, T, seed=seed, device=device, with_hca=False)
+        dev = device
+        Nc = T // s.m
+        self.csa_kv = torch.empty((Nc, s.c), dtype=torch.bfloat16, device=dev)
+        self.csa_k = torch.empty((Nc, s.d_idx), dtype=torch.bfloat16, device=dev)
+        self.topk = torch.empty((T, s.topk), dtype=torch.int32, device=dev)
+        self.out = torch.empty((T, s.n_heads, s.c), dtype=torch.bfloat16, device=dev)
+        self.cfg = hca.make_cfg(s)
+        self.phases = ["compress", "indexer_scores", "topk_select", "csa_attention"]
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
+        self.args, self._keep = hca.make_prefill_args(self.inp, self.csa_kv, self.csa_k, self.topk, self.out,
+                                                      events=self.events)
+        self.ws = torch.empty(max(1, hca.hybrid_attn_prefill_workspace(self.cfg, self.args)), dtype=torch.uint8,
+                              device=dev)
+        self.units = T
+        self.metric = "CSA prefill tokens/s at 64K"
+        self.unit = "tokens/s"
+
+    def step(self, record=True):
+        self.args.n_events = len(self.events) if record else 0
+        self.hca.hybrid_attn_prefill(self.cfg, self.args, ws=self.ws)
+
+    def launches_per_step(self):
+        return int(self.hca.lib.hca_last_launch_count())
+
+    def flops(self):
+        s, T = self.shape, self.T
+        pairs = sum(min(s.topk, (t + 1) // s.m) + min(s.n_win, t + 1) for t in range(T))
+        vis = sum((t + 1) // s.m for t in range(T))
+        return {"indexer_scores": 2.0 * vis * s.n_idx_heads * s.d_idx,
+                "csa_attention": 4.0 * pairs * s.n_heads * s.c}
+
+    def phase_bytes(self):
+        s, T = self.shape, self.T
+        return {"compress": T * (2 * s.c + s.d_idx) * 2 + (T // s.m) * (s.c + s.d_idx) * 2}
+
+    def config(self):
+        s = self.shape
+        return {"workload": self.name, "tokens": self.T, "c": s.c, "heads": s.n_heads, "topk": s.topk,
+                "indexer": f"{s.n_idx_heads}x{s.d_idx}", "n_win": s.n_win}
+
+    def e2e_setup(self):
+        keys = ("cand", "logits", "kidx_cand", "q_idx", "w_idx", "q")
+        self.d_in = [self.inp[k] for k in keys]
+        self.h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu()) for t in self.d_in]
+        self.d_out = [self.topk, self.out]
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in self.d_out]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+
+    def e2e_step(self):
+        for h, d in zip(self.h_in, self.d_in):
+            d.copy_(h, non_blocking=True)
+        self.step(record=False)
+        for h, d in zip(self.h_out, self.d_out):
+            h.copy_(d, non_blocking=True)
+
+    def oracle_sample(self, n_q):
+        import oracle
+        s = self.shape
+        T = self.T
+        d = wl.prefill_inputs(s, T, seed=0, with_hca=False)
+        f = lambda x: x.float().numpy().astype(np.float64)  # noqa: E731
+        qs = np.linspace(T // 2, T - 1, n_q).astype(int).tolist()
+        t0 = time.perf_counter()
+        oracle.csa_layer_prefill(f(d["cand"]), f(d["logits"]), f(d["kidx_cand"]), f(d["bias_csa"]),
+                                 d["q_idx"], d["w_idx"].double().numpy(), d["q"], m=s.m, topk=s.topk,
+                                 d_idx=s.d_idx, n_win=s.n_win, scale=s.scale, queries=qs)
+        return time.perf_counter() - t0
+
+
+def make_bench(name, seed, device):
+    spec = wl.WORKLOADS[name]
+    if spec["kind"] == "prefill":
+        return PrefillBench(name, spec, seed, device)
+    return DecodeBench(name, spec, seed, device)
+
+
+# ----------------------------------------------------------------------------
+# timing
+# ----------------------------------------------------------------------------
+def timed_steps(bench, K, flush, rank, ws, device, record=True):
+    """Run K steps, each preceded by an L2 flush outside its events.
+    Returns (total device ms, per-phase mean ms)."""
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    phase_ms = {p: 0.0 for p in bench.phases} if record else {}
+    barrier(ws)
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        starts[i].record()
+        bench.step(record=record)
+        ends[i].record()
+        if record:
+            torch.cuda.synchronize()
+            for j, p in enumerate(bench.phases):
+                phase_ms[p] += bench.events[j].elapsed_time(bench.events[j + 1])
+    torch.cuda.synchronize()
+    barrier(ws)
+    total = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    return total, {p: v / K for p, v in phase_ms.items()}
+
+
+def run_ours(a):
+    rank, local, ws = init_dist("nccl")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    bench = make_bench(a.workload, shard_seed(a.seed, rank), device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    for _ in range(a.warmup):
+        bench.step()
+    torch.cuda.synchronize()
+    launches = bench.launches_per_step()
+    # phase breakdown pass (events between kernels, one sync per step)
+    _, phase_ms = timed_steps(bench, a.steps, flush, rank, ws, device, record=True)
+    # headline: K steps without intermediate host syncs
+    with ClockSampler(local) as clk:
+        total_ms, _ = timed_steps(bench, a.steps, flush, rank, ws, device, record=False)
+    total_ms = reduce_max(total_ms, ws, device)
+    ms = total_ms / a.steps
+    value = bench.units * ws / (ms / 1e3)
+
+    # end to end through the C ABI with host buffers
+    bench.e2e_setup()
+    for _ in range(2):
+        bench.e2e_step()
+    torch.cuda.synchronize()
+    s_ev = [torch.cuda.Event(enable_timing=True) for _ in range(a.steps)]
+    e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(a.steps)]
+    barrier(ws)
+    for i in range(a.steps):
+        flush.zero_()
+        s_ev[i].record()
+        bench.e2e_step()
+        e_ev[i].record()
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(sum(x.elapsed_time(y) for x, y in zip(s_ev, e_ev)), ws, device) / a.steps
+    e2e_value = bench.units * ws / (e2e_ms / 1e3)
+
+    # roofline of the dominant kernel
+    pk = peaks()
+    dom = max(phase_ms, key=phase_ms.get) if phase_ms else None
+    roof = None
+    if dom is not None:
+        flops = bench.flops() if hasattr(bench, "flops") else {}
+        bytes_ = bench.phase_bytes()
+        dur_s = phase_ms[dom] / 1e3
+        tt = traffic_table().get(dom)
+        traffic = None
+        if tt and tt.get("source_hash") == source_hash(tt.get("files", [])) and tt.get("workload") == bench.name:
+            traffic = tt["dram_bytes_per_launch"]
+        if dom in flops:
+            ach = flops[dom] / dur_s / 1e12
+            peak = pk["bf16_tflops_sustained"] if a.workload.endswith("prefill_64k") else pk["bf16_tflops"]
+            roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": pk["source"]}
+        elif dom in bytes_:
+            ach = bytes_[dom] / dur_s / 1e9
+            roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(ach / pk["hbm_gbs"], 4), "traffic": traffic, "peak_source": pk["source"]}
+        else:
+            roof = {"bound": "alu", "kernel": dom, "achieved": None, "peak": None, "unit": None, "frac": None,
+                    "traffic": traffic, "note": "selection kernel; no algorithmic HBM bytes"}
+
+    out = {"metric": bench.metric, "value": round(value, 2), "unit": bench.unit, "n_gpus": ws, "steps": a.steps,
+           "warmup": a.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)/U(0,1) tensors of the workload's "
+           "shapes; caches drawn on the device)",
+           "config": dict(bench.config(), parallelism=f"replicas x{ws} (requests sharded, no collective)",
+                          l2="flushed before every timed step (256 MiB write, outside the step's events)"),
+           "e2e": {"value": round(e2e_value, 2), "unit": bench.unit, "h2d_bytes_per_step": bench.h2d,
+                   "d2h_bytes_per_step": bench.d2h, "ms_per_step": round(e2e_ms, 4),
+                   "note": "per-step inputs (queries, windows, new block) from pinned host memory and outputs back; "
+                           "KV caches resident on the device"},
+           "gpu_launches": launches * a.steps,
+           "phase_ms": {k: round(v, 4) for k, v in phase_ms.items()},
+           "roofline": roof,
+           "clocks": clk.summary()}
+    if rank == 0 and ws == 1 and not a.no_cpu_baseline:
+        import oracle  # noqa: F401  (timed baseline only)
+        cores = len(os.sched_getaffinity(0))
+        n = a.cpu_sample
+        secs = bench.oracle_sample(n)
+        out["cpu_baseline"] = {"value": round(n / secs, 4), "unit": bench.unit, "cores": cores, "kind": "oracle",
+                               "sample": f"{n} {'queries' if bench.unit == 'tokens/s' else 'requests'} of the same "
+                                         f"workload recipe through the float64 NumPy oracle ({secs:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(a):
+    """Reference arm: the CPU oracle as it stands, on rank 0, bounded samples per step."""
+    rank, local, ws = dist_env()
+    if rank != 0:
+        return
+    os.environ.setdefault("OMP_NUM_THREADS", str(len(os.sched_getaffinity(0))))
+    spec = wl.WORKLOADS[a.workload]
+    cores = len(os.sched_getaffinity(0))
+
+    class _Stub:
+        pass
+    if spec["kind"] == "prefill":
+        b = PrefillBench.__new__(PrefillBench)
+        b.shape, b.T, b.name = spec["shape"], spec["T"], a.workload
+        unit, metric, per = "tokens/s", "CSA prefill tokens/s at 64K", 16
+        conf = {"workload": a.workload, "tokens": b.T}
+    else:
+        b = DecodeBench.__new__(DecodeBench)
+        b.shape, b.B, b.ctx, b.spec, b.name = spec["shape"], spec["B"], spec["ctx"], spec, a.workload
+        b.csa = {} if spec["kind"] in ("hybrid_decode", "csa_decode") else None
+        b.hcad = ({"block_cand": 1} if spec["kind"] == "hca_decode" else {}) if spec["kind"] in (
+            "hybrid_decode", "hca_decode") else None
+        unit, metric, per = "queries/s", "hybrid CSA+HCA decode queries/s at 1M ctx", 1
+        conf = {"workload": a.workload, "batch": b.B, "context": b.ctx}
+    for _ in range(a.warmup):
+        b.oracle_sample(per)
+    tot = 0.0
+    for _ in range(a.steps):
+        tot += b.oracle_sample(per)
+    v = per * a.steps / tot
+    out = {"impl": "reference", "metric": metric, "value": round(v, 4), "unit": unit, "n_gpus": ws, "steps": a.steps,
+           "warmup": a.warmup, "ms_per_step": round(1e3 * tot / a.steps, 2), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": conf,
+           "cpu_baseline": {"value": round(v, 4), "unit": unit, "cores": cores, "kind": "oracle",
+                            "sample": f"{per} {'queries' if unit == 'tokens/s' else 'requests'} per step"},
+           "e2e": {"value": round(v, 4), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="hybrid_decode_b8_1m", choices=[k for k in wl.WORKLOADS
+                                                                          if k != "tiny_prefill_1k"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-sample", type=int, default=4, help="requests (decode) / queries (prefill) for the oracle")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        print("warning: fewer than 3 warm-up steps; the number is not a valid measurement", file=sys.stderr)
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

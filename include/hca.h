@@ -1,0 +1,263 @@
+/*
+ * hca.h -- C ABI of libhca.so, the hybrid CSA / HCA attention layer on B200.
+ *
+ * What the layer computes (DeepSeek-V4 write-ups; sections named per call):
+ *   "DeepSeek V4 Architecture Tricks" (pinktalk.online)        -> [Tricks]
+ *   QbitAI write-up of the V4 report (admirer.cn), "混合注意力機制" -> [QbitAI]
+ *   "DeepSeek-V4 Technical Report: Hybrid Attention and Post-Training
+ *    for Million-Token Contexts" (xutianle.me), sections 3-5   -> [Report]
+ *
+ * Conventions for every entry point
+ *   - Tensor pointers are DEVICE pointers, owned by the caller; the library
+ *     never frees or retains them.  Struct and config pointers (cfg, args)
+ *     are HOST pointers, read during the call only.
+ *   - Layouts are row-major with the strides stated; all strides are in
+ *     elements.  bf16 tensors are passed as raw 16-bit patterns (hca_bf16).
+ *     Every bf16/f32 row must start on a 16-byte boundary (base pointers
+ *     16-byte aligned, row strides multiples of 8 bf16 / 4 f32 elements).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*,
+ *     NULL = legacy default stream) and never synchronise the host.
+ *   - The library does not allocate device memory.  Scratch space comes from
+ *     the caller's `ws` (device pointer, 256-byte aligned) of at least
+ *     hca_workspace_size(...) bytes; ws may be NULL when that size is 0.
+ *   - Return value: HCA_OK, or a negative hca_status.  Arguments are checked
+ *     on the host before anything is launched; on error nothing is launched
+ *     and hca_last_error() describes the problem.  A failed launch returns
+ *     HCA_ERR_CUDA.  Device-side errors of an earlier call may surface as
+ *     HCA_ERR_CUDA from a later one (standard CUDA semantics).
+ *   - Fault injection for tests: if the environment variable
+ *     HCA_INJECT_FAULT names an entry point (or is "all"), that entry point
+ *     returns HCA_ERR_INJECTED after argument checking, launching nothing.
+ *   - Supported shapes: c in {64, 512}, d_idx in {32, 128}; n_heads,
+ *     n_idx_heads <= 64; topk <= 2048; n_win <= 256.  Other shapes return
+ *     HCA_ERR_UNSUPPORTED.
+ */
+#ifndef HCA_H_
+#define HCA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t hca_bf16; /* raw bfloat16 bit pattern */
+
+typedef enum {
+  HCA_OK = 0,
+  HCA_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, bad size, bad stride */
+  HCA_ERR_UNSUPPORTED = -2,  /* valid but not a specialised shape */
+  HCA_ERR_WORKSPACE = -3,    /* ws smaller than hca_workspace_size() */
+  HCA_ERR_CUDA = -4,         /* a CUDA call or launch failed */
+  HCA_ERR_DEVICE_CHECK = -5, /* a kernel's own bounds/wait check tripped */
+  HCA_ERR_INJECTED = -6      /* HCA_INJECT_FAULT asked for a failure */
+} hca_status;
+
+/* Hyper-parameters of one layer.
+ *   c            KV entry width = attention head dim (512 in V4-Pro, [QbitAI] CSA step four)
+ *   m            CSA compression rate (4, [Tricks] CSA section)
+ *   m_hca        HCA compression rate m' (128, [Tricks] HCA section)
+ *   topk         CSA entries selected per query (1024, [Tricks] CSA section)
+ *   n_idx_heads  lightning-indexer heads H_I (64), d_idx their dim (128)
+ *   n_heads      query heads sharing the single KV head (MQA)
+ *   n_win        sliding-window length (128, [Tricks] Sliding Window Branch)
+ *   scale        attention logit scale (1/sqrt(c)) */
+typedef struct {
+  int c, m, m_hca, topk, n_idx_heads, d_idx, n_heads, n_win;
+  float scale;
+} hca_layer_cfg;
+
+/* Query modes of the indexer and attention calls. */
+enum {
+  HCA_MODE_PREFILL = 0, /* Tq queries of ONE sequence; window rows are that
+                           sequence's raw token rows [T, c] (row r = token r) */
+  HCA_MODE_DECODE = 1   /* query i belongs to request i; each request has its
+                           own caches and its own window block [n_win, c] */
+};
+
+/* Operations, for hca_workspace_size().  The layer calls size their
+ * workspace with hybrid_attn_decode_workspace / hybrid_attn_prefill_workspace. */
+enum {
+  HCA_OP_INDEXER_TOPK = 1,
+  HCA_OP_SPARSE_MQA = 2
+};
+
+/* ---------------------------------------------------------------------------
+ * csa_compress -- overlapped CSA KV compression ([Tricks] "压缩 KV 的具体 trick";
+ * [QbitAI] CSA step one; [Report] section 3).
+ *   out[i, j] = sum_{r in W(i)} softmax_r(logits[r, j] + pos_bias[r-(i-1)m, j]) * cand[r, j]
+ *   W(i) = tokens [(i-1)m, (i+1)m) that exist; bias rows 0..m-1 weight the
+ *   previous block, m..2m-1 the current one; entry 0 pools its own block only.
+ *   Softmax and sum in f32; the result is rounded to bf16.
+ *   cand   [T, c] bf16, row stride ld_cand;   logits [T, c] bf16, row stride ld_logits
+ *   pos_bias [2m, c] f32, row stride ld_bias; out [floor(T/m), c] bf16, row stride ld_out
+ *   A trailing incomplete block produces no entry.  T may be 0 (no-op).
+ *   The same call compresses indexer keys: pass the key candidates as cand,
+ *   the first d_idx channels of the logits/bias (same pointers, same strides)
+ *   and c = d_idx.  c must be a multiple of 8; m in [1, 16].
+ * ------------------------------------------------------------------------- */
+int csa_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int ld_logits,
+                 const float* pos_bias, int ld_bias, int T, int c, int m,
+                 hca_bf16* out, int ld_out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * hca_compress -- HCA KV compression, no overlap ([Tricks] HCA section;
+ * [QbitAI] HCA paragraph; [Report] section 4).
+ *   out[i, j] = sum_{r in [i m', (i+1) m')} softmax_r(logits[r, j] + pos_bias[r - i m', j]) * cand[r, j]
+ *   for B independent sequences: sequence b reads cand + b*seq_stride_in,
+ *   logits + b*seq_stride_in and writes out + b*seq_stride_out.
+ *   cand/logits [T, c] bf16 (row strides ld_cand / ld_logits), pos_bias [m', c]
+ *   f32 (row stride ld_bias, shared by all sequences), out [floor(T/m'), c] bf16.
+ *   Decode use: compress the newest complete block by passing its m' raw
+ *   rows (T = m') and out = the cache row it fills.  m' in [1, 1024].
+ * ------------------------------------------------------------------------- */
+int hca_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int ld_logits,
+                 const float* pos_bias, int ld_bias, int B, long long seq_stride_in, int T, int c,
+                 int m_hca, hca_bf16* out, int ld_out, long long seq_stride_out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * csa_indexer_topk -- lightning-indexer scores and per-query top-k
+ * ([QbitAI] CSA step two; [Tricks] CSA section: 64 heads x 128, top-k 1024).
+ *   I(t, s) = sum_j w_idx[t, j] * ReLU(q_idx[t, j, :] . k_idx[s, :])   (f32 accumulation)
+ *   over the causally complete entries s, (s+1)*cfg->m - 1 <= q_pos[t], s < N.
+ *   topk_idx[t, :] receives the cfg->topk entries with the largest scores
+ *   (ties: lower index first), in no particular order, padded with -1 when
+ *   fewer than topk entries are visible (then all visible ones are taken).
+ *   q_idx  [Tq, H_I, d_I] bf16 (contiguous); w_idx [Tq, H_I] f32 (contiguous)
+ *   k_idx  request r's keys at k_idx + r*k_seq_stride: [N, d_I] bf16 contiguous
+ *   q_pos  [Tq] int32 device: position of each query (0-based)
+ *   mode   HCA_MODE_PREFILL: all queries in request 0 (k_seq_stride ignored);
+ *          HCA_MODE_DECODE: query i reads request i's keys.
+ *   topk_idx [Tq, topk] int32 out.  ws: hca_workspace_size(HCA_OP_INDEXER_TOPK, cfg, Tq, N, mode).
+ * ------------------------------------------------------------------------- */
+int csa_indexer_topk(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* k_idx,
+                     long long k_seq_stride, int N, const int32_t* q_pos, int Tq, int mode,
+                     const hca_layer_cfg* cfg, int32_t* topk_idx, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* ---------------------------------------------------------------------------
+ * sparse_mqa_attend -- core shared-KV multi-query attention over compressed
+ * entries plus the sliding window, one softmax ([QbitAI] CSA step three, the
+ * KV-entry-as-key-and-value remark and the sliding-window paragraph;
+ * [Tricks] HCA and Sliding Window sections).
+ *   For query t and head h, over the row set U(t):
+ *     o[t, h, :] = sum_{u in U(t)} softmax_u(scale * q[t, h, :] . row_u) row_u
+ *   U(t) = { kv[s] : s in idx[t, :], s >= 0 }             (CSA, idx != NULL)
+ *        | { kv[s] : (s+1)*rate - 1 <= q_pos[t], s < N }  (HCA, idx == NULL)
+ *        + window rows of t.
+ *   Window rows: HCA_MODE_PREFILL: win[r] for r in [max(0, t-n_win+1), t]
+ *   (win = the sequence's raw per-token KV rows, row stride cfg->c);
+ *   HCA_MODE_DECODE: the first min(n_win, t+1) rows of request i's block
+ *   win + i*win_seq_stride ([n_win, c]; any order).
+ *   q [Tq, H, c] bf16; kv: request r's entries at kv + r*kv_seq_stride, [N, c];
+ *   idx [Tq, n_idx] int32 (entries < N, visible to the query; -1 = empty slot);
+ *   out [Tq, H, c] bf16.  Logits, softmax and sums in f32.
+ *   ws: hca_workspace_size(HCA_OP_SPARSE_MQA, cfg, Tq, N, mode) (split-K partials).
+ * ------------------------------------------------------------------------- */
+int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N,
+                      const int32_t* idx, int n_idx, int rate, const hca_bf16* win,
+                      long long win_seq_stride, const int32_t* q_pos, int Tq, int mode,
+                      const hca_layer_cfg* cfg, hca_bf16* out, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/* ---------------------------------------------------------------------------
+ * hybrid_attn_decode -- one decode step of a CSA layer and/or an HCA layer for
+ * B requests, one query each at q_pos[b] (device int32 [B]).  Runs, in order:
+ * the HCA compression of the newest complete block (if hca_block_cand), the
+ * indexer + top-k, the CSA sparse attention, the HCA dense attention; split-K
+ * over the context with a combine step.  A layer whose q pointer is NULL is
+ * skipped.  Caches hold entries of request b at base + b*stride.
+ * `events` (optional, may be NULL) is an array of n_events cudaEvent_t handles
+ * that are recorded on `stream` at kernel boundaries, for profiling.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int B;
+  const int32_t* q_pos;
+  /* CSA layer */
+  const hca_bf16* csa_q;      /* [B, H, c] */
+  const hca_bf16* csa_q_idx;  /* [B, H_I, d_I] */
+  const float* csa_w_idx;     /* [B, H_I] */
+  const hca_bf16* csa_kv;     /* [B][csa_N, c] at csa_kv_stride */
+  const hca_bf16* csa_k_idx;  /* [B][csa_N, d_I] at csa_k_stride */
+  int csa_N;
+  long long csa_kv_stride, csa_k_stride;
+  const hca_bf16* csa_win;    /* [B][n_win, c] at csa_win_stride */
+  long long csa_win_stride;
+  int32_t* csa_topk_idx;      /* [B, topk] out */
+  hca_bf16* csa_out;          /* [B, H, c] out */
+  /* HCA layer */
+  const hca_bf16* hca_q;      /* [B, H, c] */
+  hca_bf16* hca_kv;           /* [B][hca_N, c] at hca_kv_stride.  With hca_block_cand, hca_N must equal
+                                 floor((q_pos[b]+1)/m') for every b and row hca_N-1 is written */
+  int hca_N;
+  long long hca_kv_stride;
+  const hca_bf16* hca_block_cand;   /* [B][m', c] newest complete block, or NULL */
+  const hca_bf16* hca_block_logits; /* [B][m', c] */
+  long long hca_block_stride;
+  const float* hca_pos_bias;        /* [m', c] */
+  const hca_bf16* hca_win;    /* [B][n_win, c] at hca_win_stride */
+  long long hca_win_stride;
+  hca_bf16* hca_out;          /* [B, H, c] out */
+  void* const* events;
+  int n_events;
+} hca_decode_args;
+
+int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* args, void* ws,
+                       size_t ws_bytes, void* stream);
+size_t hybrid_attn_decode_workspace(const hca_layer_cfg* cfg, const hca_decode_args* args);
+
+/* ---------------------------------------------------------------------------
+ * hybrid_attn_prefill -- a CSA layer (and optionally an HCA layer) over one
+ * sequence of T raw tokens, every token a query (q_pos = 0..T-1, device).
+ * Runs: CSA compression of KV and indexer keys (indexer-key logits/bias are
+ * the first d_idx channels of logits/bias_csa), indexer + top-k, sparse MQA
+ * with the causal window; then, if hca_kv != NULL, HCA compression and dense
+ * causal MQA with the window.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int T;
+  const int32_t* q_pos;       /* [T] */
+  const hca_bf16* cand;       /* [T, c] raw per-token KV candidates (also the window rows) */
+  const hca_bf16* logits;     /* [T, c] compression weight logits */
+  const hca_bf16* kidx_cand;  /* [T, d_I] per-token indexer-key candidates */
+  const float* bias_csa;      /* [2m, c] */
+  const hca_bf16* q_idx;      /* [T, H_I, d_I] */
+  const float* w_idx;         /* [T, H_I] */
+  const hca_bf16* q;          /* [T, H, c] */
+  hca_bf16* csa_kv;           /* [T/m, c] out */
+  hca_bf16* csa_k_idx;        /* [T/m, d_I] out */
+  int32_t* topk_idx;          /* [T, topk] out */
+  hca_bf16* csa_out;          /* [T, H, c] out */
+  const float* bias_hca;      /* [m', c] */
+  const hca_bf16* hca_q;      /* [T, H, c] */
+  hca_bf16* hca_kv;           /* [T/m', c] out, or NULL: no HCA layer */
+  hca_bf16* hca_out;          /* [T, H, c] out */
+  void* const* events;
+  int n_events;
+} hca_prefill_args;
+
+int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* args, void* ws,
+                        size_t ws_bytes, void* stream);
+size_t hybrid_attn_prefill_workspace(const hca_layer_cfg* cfg, const hca_prefill_args* args);
+
+/* Workspace bytes for one op at Tq queries and N entries per request (mode
+ * as in the calls).  For HCA_OP_SPARSE_MQA the size covers both the sparse
+ * (idx, n_idx = cfg->topk) and the dense (idx = NULL) form.  Returns 0 for
+ * calls that need none, (size_t)-1 for an unsupported configuration. */
+size_t hca_workspace_size(int op, const hca_layer_cfg* cfg, int Tq, int N, int mode);
+
+/* Number of kernels the last successful layer call (hybrid_attn_decode /
+ * hybrid_attn_prefill) on the calling thread launched. */
+int hca_last_launch_count(void);
+
+/* Message describing the last error on the calling thread ("" if none). */
+const char* hca_last_error(void);
+
+/* Library version string. */
+const char* hca_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HCA_H_ */

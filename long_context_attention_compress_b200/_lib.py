@@ -1,0 +1,324 @@
+"""ctypes binding of libhca.so (argument marshalling only).
+
+Every function here takes torch tensors that live on the CUDA device, checks
+their dtype/shape/contiguity, and passes raw device pointers, sizes and the
+current CUDA stream to the C ABI declared in include/hca.h.  All arithmetic
+runs in the library's kernels; there is no other implementation to fall back
+to: if the library is missing, importing this module raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.environ.get("HCA_LIB", os.path.join(_PKG, "libhca.so"))
+
+HCA_MODE_PREFILL = 0
+HCA_MODE_DECODE = 1
+HCA_OP_INDEXER_TOPK = 1
+HCA_OP_SPARSE_MQA = 2
+
+STATUS = {0: "HCA_OK", -1: "HCA_ERR_INVALID_ARG", -2: "HCA_ERR_UNSUPPORTED", -3: "HCA_ERR_WORKSPACE",
+          -4: "HCA_ERR_CUDA", -5: "HCA_ERR_DEVICE_CHECK", -6: "HCA_ERR_INJECTED"}
+
+
+class HcaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libhca.so not built at {LIB_PATH}; run `python -m long_context_attention_compress_b200.build`")
+lib = ctypes.CDLL(LIB_PATH)
+
+c_int, c_ll, c_size, c_float, c_void_p = ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t, ctypes.c_float, ctypes.c_void_p
+
+
+class LayerCfg(ctypes.Structure):
+    _fields_ = [("c", c_int), ("m", c_int), ("m_hca", c_int), ("topk", c_int), ("n_idx_heads", c_int),
+                ("d_idx", c_int), ("n_heads", c_int), ("n_win", c_int), ("scale", c_float)]
+
+
+class DecodeArgs(ctypes.Structure):
+    _fields_ = [("B", c_int), ("q_pos", c_void_p),
+                ("csa_q", c_void_p), ("csa_q_idx", c_void_p), ("csa_w_idx", c_void_p), ("csa_kv", c_void_p),
+                ("csa_k_idx", c_void_p), ("csa_N", c_int), ("csa_kv_stride", c_ll), ("csa_k_stride", c_ll),
+                ("csa_win", c_void_p), ("csa_win_stride", c_ll), ("csa_topk_idx", c_void_p), ("csa_out", c_void_p),
+                ("hca_q", c_void_p), ("hca_kv", c_void_p), ("hca_N", c_int), ("hca_kv_stride", c_ll),
+                ("hca_block_cand", c_void_p), ("hca_block_logits", c_void_p), ("hca_block_stride", c_ll),
+                ("hca_pos_bias", c_void_p), ("hca_win", c_void_p), ("hca_win_stride", c_ll), ("hca_out", c_void_p),
+                ("events", c_void_p), ("n_events", c_int)]
+
+
+class PrefillArgs(ctypes.Structure):
+    _fields_ = [("T", c_int), ("q_pos", c_void_p), ("cand", c_void_p), ("logits", c_void_p),
+                ("kidx_cand", c_void_p), ("bias_csa", c_void_p), ("q_idx", c_void_p), ("w_idx", c_void_p),
+                ("q", c_void_p), ("csa_kv", c_void_p), ("csa_k_idx", c_void_p), ("topk_idx", c_void_p),
+                ("csa_out", c_void_p), ("bias_hca", c_void_p), ("hca_q", c_void_p), ("hca_kv", c_void_p),
+                ("hca_out", c_void_p), ("events", c_void_p), ("n_events", c_int)]
+
+
+def _sig(name, restype, argtypes):
+    f = getattr(lib, name)
+    f.restype = restype
+    f.argtypes = argtypes
+    return f
+
+
+_csa_compress = _sig("csa_compress", c_int, [c_void_p, c_int, c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int,
+                                             c_void_p, c_int, c_void_p])
+_hca_compress = _sig("hca_compress", c_int, [c_void_p, c_int, c_void_p, c_int, c_void_p, c_int, c_int, c_ll, c_int,
+                                             c_int, c_int, c_void_p, c_int, c_ll, c_void_p])
+_indexer = _sig("csa_indexer_topk", c_int, [c_void_p, c_void_p, c_void_p, c_ll, c_int, c_void_p, c_int, c_int,
+                                            ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_size, c_void_p])
+_mqa = _sig("sparse_mqa_attend", c_int, [c_void_p, c_void_p, c_ll, c_int, c_void_p, c_int, c_int, c_void_p, c_ll,
+                                         c_void_p, c_int, c_int, ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_size,
+                                         c_void_p])
+_decode = _sig("hybrid_attn_decode", c_int, [ctypes.POINTER(LayerCfg), ctypes.POINTER(DecodeArgs), c_void_p, c_size,
+                                             c_void_p])
+_decode_ws = _sig("hybrid_attn_decode_workspace", c_size, [ctypes.POINTER(LayerCfg), ctypes.POINTER(DecodeArgs)])
+_prefill = _sig("hybrid_attn_prefill", c_int, [ctypes.POINTER(LayerCfg), ctypes.POINTER(PrefillArgs), c_void_p,
+                                               c_size, c_void_p])
+_prefill_ws = _sig("hybrid_attn_prefill_workspace", c_size, [ctypes.POINTER(LayerCfg), ctypes.POINTER(PrefillArgs)])
+_ws_size = _sig("hca_workspace_size", c_size, [c_int, ctypes.POINTER(LayerCfg), c_int, c_int, c_int])
+_last_error = _sig("hca_last_error", ctypes.c_char_p, [])
+_version = _sig("hca_version", ctypes.c_char_p, [])
+
+SIZE_MAX = (1 << (8 * ctypes.sizeof(c_size))) - 1
+
+
+def version() -> str:
+    return _version().decode()
+
+
+def last_error() -> str:
+    return _last_error().decode()
+
+
+def _check(status: int):
+    if status != 0:
+        raise HcaError(status, last_error())
+
+
+def make_cfg(shape) -> LayerCfg:
+    """LayerCfg from a workloads.LayerShape (or any object with the same fields)."""
+    return LayerCfg(shape.c, shape.m, shape.m_hca, shape.topk, shape.n_idx_heads, shape.d_idx, shape.n_heads,
+                    shape.n_win, float(shape.scale))
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _workspace(nbytes: int, ws, device):
+    if nbytes == SIZE_MAX:
+        raise HcaError(-2, "unsupported configuration (workspace query)")
+    if nbytes == 0:
+        return None, 0
+    if ws is None or ws.numel() * ws.element_size() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws, ws.numel() * ws.element_size()
+
+
+BF16, F32, I32 = torch.bfloat16, torch.float32, torch.int32
+
+
+# ----------------------------------------------------------------------------
+# entry points
+# ----------------------------------------------------------------------------
+def csa_compress(cand, logits, pos_bias, m, out=None, stream=None):
+    """Overlapped CSA compression of [T, c] candidates -> [T // m, c] (bf16).
+    ``logits``/``pos_bias`` may be wider than cand (their first c channels are used)."""
+    T, c = cand.shape
+    if out is None:
+        out = torch.empty((T // m, c), dtype=BF16, device=cand.device)
+    _check(_csa_compress(_ptr(cand, BF16, "cand"), cand.stride(0), _ptr(logits, BF16, "logits"), logits.stride(0),
+                         _ptr(pos_bias, F32, "pos_bias"), pos_bias.stride(0), T, c, m, _ptr(out, BF16, "out"),
+                         out.stride(0), _stream(stream)))
+    return out
+
+
+def hca_compress(cand, logits, pos_bias, m_hca, out=None, stream=None):
+    """HCA compression of [T, c] or [B, T, c] candidates -> [(B,) T // m', c]."""
+    batched = cand.dim() == 3
+    c3 = cand if batched else cand.unsqueeze(0)
+    l3 = logits if batched else logits.unsqueeze(0)
+    B, T, c = c3.shape
+    if out is None:
+        out = torch.empty((B, T // m_hca, c), dtype=BF16, device=cand.device)
+        ret = out if batched else out[0]
+    else:
+        ret = out
+        out = out if out.dim() == 3 else out.unsqueeze(0)
+    _check(_hca_compress(_ptr(c3, BF16, "cand"), c3.stride(1), _ptr(l3, BF16, "logits"), l3.stride(1),
+                         _ptr(pos_bias, F32, "pos_bias"), pos_bias.stride(0), B, c3.stride(0), T, c, m_hca,
+                         _ptr(out, BF16, "out"), out.stride(1), out.stride(0), _stream(stream)))
+    return ret
+
+
+def workspace_size(op, cfg: LayerCfg, Tq: int, N: int, mode: int) -> int:
+    return int(_ws_size(op, ctypes.byref(cfg), Tq, N, mode))
+
+
+def csa_indexer_topk(q_idx, w_idx, k_idx, q_pos, cfg: LayerCfg, mode=HCA_MODE_PREFILL, out=None, ws=None,
+                     stream=None):
+    """Top-k entry indices [Tq, topk] (int32, -1 padded) by lightning-indexer score.
+    k_idx: [N, d_I] (prefill) or [B, N, d_I] (decode, one query per request)."""
+    Tq = q_idx.shape[0]
+    N = k_idx.shape[-2]
+    kstride = k_idx.stride(0) if k_idx.dim() == 3 else 0
+    if out is None:
+        out = torch.empty((Tq, cfg.topk), dtype=I32, device=q_idx.device)
+    ws, nb = _workspace(workspace_size(HCA_OP_INDEXER_TOPK, cfg, Tq, N, mode), ws, q_idx.device)
+    _check(_indexer(_ptr(q_idx, BF16, "q_idx"), _ptr(w_idx, F32, "w_idx"), _ptr(k_idx, BF16, "k_idx"), kstride, N,
+                    _ptr(q_pos, I32, "q_pos"), Tq, mode, ctypes.byref(cfg), _ptr(out, I32, "out"),
+                    None if ws is None else ws.data_ptr(), nb, _stream(stream)))
+    return out
+
+
+def sparse_mqa_attend(q, kv, win, q_pos, cfg: LayerCfg, idx=None, rate=None, mode=HCA_MODE_PREFILL, out=None,
+                      ws=None, stream=None):
+    """Shared-KV MQA over selected (idx) or all visible (idx=None) entries plus the window.
+    kv: [N, c] (prefill) or [B, N, c] (decode); win: raw rows [T, c] (prefill) or [B, n_win, c] (decode)."""
+    Tq = q.shape[0]
+    N = kv.shape[-2]
+    kvs = kv.stride(0) if kv.dim() == 3 else 0
+    ws_stride = win.stride(0) if win.dim() == 3 else 0
+    if rate is None:
+        rate = cfg.m if idx is not None else cfg.m_hca
+    n_idx = idx.shape[1] if idx is not None else 0
+    if out is None:
+        out = torch.empty_like(q)
+    ws, nb = _workspace(workspace_size(HCA_OP_SPARSE_MQA, cfg, Tq, N, mode), ws, q.device)
+    _check(_mqa(_ptr(q, BF16, "q"), _ptr(kv, BF16, "kv"), kvs, N, _ptr(idx, I32, "idx"), n_idx, rate,
+                _ptr(win, BF16, "win"), ws_stride, _ptr(q_pos, I32, "q_pos"), Tq, mode, ctypes.byref(cfg),
+                _ptr(out, BF16, "out"), None if ws is None else ws.data_ptr(), nb, _stream(stream)))
+    return out
+
+
+def _events_array(events):
+    if not events:
+        return None, 0, None
+    handles = []
+    for e in events:
+        if isinstance(e, torch.cuda.Event):
+            if e.cuda_event == 0:
+                e.record()  # creates the event lazily
+            handles.append(e.cuda_event)
+        else:
+            handles.append(int(e))
+    arr = (c_void_p * len(handles))(*handles)
+    return ctypes.cast(arr, c_void_p), len(handles), arr
+
+
+def make_decode_args(B, q_pos, csa=None, hca=None, csa_topk_idx=None, csa_out=None, hca_out=None, events=None):
+    """Build DecodeArgs from dicts of tensors (see workloads.csa_decode_inputs /
+    hca_decode_inputs).  Returns (args, keepalive)."""
+    a = DecodeArgs()
+    a.B = B
+    a.q_pos = _ptr(q_pos, I32, "q_pos")
+    keep = [q_pos]
+    if csa is not None:
+        a.csa_q = _ptr(csa["q"], BF16, "csa.q")
+        a.csa_q_idx = _ptr(csa["q_idx"], BF16, "csa.q_idx")
+        a.csa_w_idx = _ptr(csa["w_idx"], F32, "csa.w_idx")
+        a.csa_kv = _ptr(csa["E"], BF16, "csa.E")
+        a.csa_k_idx = _ptr(csa["K_I"], BF16, "csa.K_I")
+        a.csa_N = csa["E"].shape[1]
+        a.csa_kv_stride = csa["E"].stride(0)
+        a.csa_k_stride = csa["K_I"].stride(0)
+        a.csa_win = _ptr(csa["win"], BF16, "csa.win")
+        a.csa_win_stride = csa["win"].stride(0)
+        a.csa_topk_idx = _ptr(csa_topk_idx, I32, "csa_topk_idx")
+        a.csa_out = _ptr(csa_out, BF16, "csa_out")
+    if hca is not None:
+        a.hca_q = _ptr(hca["q"], BF16, "hca.q")
+        a.hca_kv = _ptr(hca["E_h"], BF16, "hca.E_h")
+        a.hca_N = hca["E_h"].shape[1]
+        a.hca_kv_stride = hca["E_h"].stride(0)
+        if hca.get("block_cand") is not None:
+            a.hca_block_cand = _ptr(hca["block_cand"], BF16, "hca.block_cand")
+            a.hca_block_logits = _ptr(hca["block_logits"], BF16, "hca.block_logits")
+            a.hca_block_stride = hca["block_cand"].stride(0)
+            a.hca_pos_bias = _ptr(hca["bias_hca"], F32, "hca.bias_hca")
+        a.hca_win = _ptr(hca["win"], BF16, "hca.win")
+        a.hca_win_stride = hca["win"].stride(0)
+        a.hca_out = _ptr(hca_out, BF16, "hca_out")
+    ev, n, arr = _events_array(events)
+    a.events = ev
+    a.n_events = n
+    keep.append(arr)
+    return a, keep
+
+
+def hybrid_attn_decode_workspace(cfg: LayerCfg, args: DecodeArgs) -> int:
+    return int(_decode_ws(ctypes.byref(cfg), ctypes.byref(args)))
+
+
+def hybrid_attn_decode(cfg: LayerCfg, args: DecodeArgs, ws=None, stream=None, device=None):
+    """Run one decode step (see include/hca.h).  ``ws`` may be a preallocated uint8 tensor."""
+    need = hybrid_attn_decode_workspace(cfg, args)
+    ws, nb = _workspace(need, ws, device or torch.device("cuda"))
+    _check(_decode(ctypes.byref(cfg), ctypes.byref(args), None if ws is None else ws.data_ptr(), nb, _stream(stream)))
+    return ws
+
+
+def make_prefill_args(inp, csa_kv, csa_k_idx, topk_idx, csa_out, hca_kv=None, hca_q=None, hca_out=None,
+                      events=None):
+    """PrefillArgs from a workloads.prefill_inputs dict (on the device) and output tensors."""
+    a = PrefillArgs()
+    a.T = inp["cand"].shape[0]
+    a.q_pos = _ptr(inp["q_pos"], I32, "q_pos")
+    a.cand = _ptr(inp["cand"], BF16, "cand")
+    a.logits = _ptr(inp["logits"], BF16, "logits")
+    a.kidx_cand = _ptr(inp["kidx_cand"], BF16, "kidx_cand")
+    a.bias_csa = _ptr(inp["bias_csa"], F32, "bias_csa")
+    a.q_idx = _ptr(inp["q_idx"], BF16, "q_idx")
+    a.w_idx = _ptr(inp["w_idx"], F32, "w_idx")
+    a.q = _ptr(inp["q"], BF16, "q")
+    a.csa_kv = _ptr(csa_kv, BF16, "csa_kv")
+    a.csa_k_idx = _ptr(csa_k_idx, BF16, "csa_k_idx")
+    a.topk_idx = _ptr(topk_idx, I32, "topk_idx")
+    a.csa_out = _ptr(csa_out, BF16, "csa_out")
+    if hca_kv is not None:
+        a.bias_hca = _ptr(inp["bias_hca"], F32, "bias_hca")
+        a.hca_q = _ptr(hca_q, BF16, "hca_q")
+        a.hca_kv = _ptr(hca_kv, BF16, "hca_kv")
+        a.hca_out = _ptr(hca_out, BF16, "hca_out")
+    ev, n, arr = _events_array(events)
+    a.events = ev
+    a.n_events = n
+    return a, [arr]
+
+
+def hybrid_attn_prefill_workspace(cfg: LayerCfg, args: PrefillArgs) -> int:
+    return int(_prefill_ws(ctypes.byref(cfg), ctypes.byref(args)))
+
+
+def hybrid_attn_prefill(cfg: LayerCfg, args: PrefillArgs, ws=None, stream=None, device=None):
+    need = hybrid_attn_prefill_workspace(cfg, args)
+    ws, nb = _workspace(need, ws, device or torch.device("cuda"))
+    _check(_prefill(ctypes.byref(cfg), ctypes.byref(args), None if ws is None else ws.data_ptr(), nb,
+                    _stream(stream)))
+    return ws

@@ -1,0 +1,518 @@
+// C ABI of libhca.so: argument checking, workspace planning and launch order.
+// The operations are documented in include/hca.h.
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hca {
+thread_local int g_launch_counter = 0;
+}
+
+using namespace hca;
+
+namespace {
+
+thread_local std::string g_err;
+thread_local int g_last_launches = 0;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return HCA_OK;
+  return fail(HCA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool injected(const char* name) {
+  const char* v = getenv("HCA_INJECT_FAULT");
+  if (!v || !*v) return false;
+  return strcmp(v, "all") == 0 || strcmp(v, name) == 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define CHECK_PTR(p, name)                                                          \
+  do {                                                                              \
+    if (!(p)) return fail(HCA_ERR_INVALID_ARG, "%s: null pointer", name);           \
+    if (!aligned16(p)) return fail(HCA_ERR_INVALID_ARG, "%s: not 16-byte aligned", name); \
+  } while (0)
+
+#define CHECK(cond, code, ...) \
+  do {                         \
+    if (!(cond)) return fail(code, __VA_ARGS__); \
+  } while (0)
+
+#define CUDA_TRY(expr, where)                      \
+  do {                                             \
+    int _s = cuda_status((expr), where);           \
+    if (_s != HCA_OK) return _s;                   \
+  } while (0)
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int check_cfg(const hca_layer_cfg* cfg) {
+  if (!cfg) return fail(HCA_ERR_INVALID_ARG, "cfg: null");
+  CHECK(cfg->c > 0 && cfg->m > 0 && cfg->m_hca > 0 && cfg->topk > 0 && cfg->n_idx_heads > 0 &&
+            cfg->d_idx > 0 && cfg->n_heads > 0 && cfg->n_win > 0,
+        HCA_ERR_INVALID_ARG, "cfg: sizes must be positive");
+  CHECK(cfg->scale > 0.f, HCA_ERR_INVALID_ARG, "cfg: scale must be positive");
+  CHECK((cfg->c == 512 && cfg->n_heads == 64) || (cfg->c == 64 && cfg->n_heads == 4), HCA_ERR_UNSUPPORTED,
+        "cfg: (c=%d, n_heads=%d) not specialised; supported (512, 64) and (64, 4)", cfg->c, cfg->n_heads);
+  CHECK(cfg->d_idx == 128 || cfg->d_idx == 32, HCA_ERR_UNSUPPORTED, "cfg: d_idx=%d not in {32, 128}", cfg->d_idx);
+  CHECK(cfg->n_idx_heads <= 64 && cfg->n_idx_heads % 4 == 0, HCA_ERR_UNSUPPORTED,
+        "cfg: n_idx_heads=%d (need <= 64, multiple of 4)", cfg->n_idx_heads);
+  CHECK(cfg->topk <= 2048, HCA_ERR_UNSUPPORTED, "cfg: topk=%d > 2048", cfg->topk);
+  CHECK(cfg->n_win <= 256, HCA_ERR_UNSUPPORTED, "cfg: n_win=%d > 256", cfg->n_win);
+  CHECK(cfg->m <= 16, HCA_ERR_UNSUPPORTED, "cfg: m=%d > 16", cfg->m);
+  CHECK(cfg->m_hca <= 1024, HCA_ERR_UNSUPPORTED, "cfg: m_hca=%d > 1024", cfg->m_hca);
+  return HCA_OK;
+}
+
+// ---- indexer workspace: score matrix [Tq, ldN] f32 + chunk candidates -------
+struct IndexerPlan {
+  long long ld;   // score row stride
+  int chunk, chunks;
+  size_t cand_off, bytes;
+};
+
+IndexerPlan plan_indexer(int Tq, int N, int k) {
+  IndexerPlan p;
+  p.ld = ((long long)N + 3) / 4 * 4;
+  if (N <= kSelectMaxN) {
+    p.chunk = N > 0 ? N : 1;
+    p.chunks = 1;
+  } else {
+    p.chunk = 16384;
+    p.chunks = (N + p.chunk - 1) / p.chunk;
+  }
+  const size_t score_bytes = (size_t)Tq * (size_t)p.ld * sizeof(float);
+  p.cand_off = (score_bytes + 255) / 256 * 256;
+  const size_t cand_bytes = p.chunks > 1 ? (size_t)Tq * p.chunks * k * sizeof(uint64_t) : 0;
+  p.bytes = p.cand_off + cand_bytes;
+  return p;
+}
+
+int indexer_ok(int N, int k) {
+  const IndexerPlan p = plan_indexer(1, N, k);
+  CHECK((long long)p.chunks * k <= kSelectMaxN, HCA_ERR_UNSUPPORTED,
+        "indexer: N=%d with topk=%d needs %d chunks (max merge %d candidates)", N, k, p.chunks, kSelectMaxN);
+  return HCA_OK;
+}
+
+int run_indexer_topk(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride, int N,
+                     const int32_t* q_pos, int Tq, int mode, const hca_layer_cfg* cfg, int32_t* topk_idx,
+                     void* ws, cudaStream_t st, void* const* ev, int n_ev, int& ev_i) {
+  const IndexerPlan p = plan_indexer(Tq, N, cfg->topk);
+  float* scores = reinterpret_cast<float*>(ws);
+  CUDA_TRY(launch_indexer_scores(q_idx, w_idx, k_idx, k_seq_stride, N, q_pos, Tq, mode, cfg->m, cfg->n_idx_heads,
+                                 cfg->d_idx, scores, p.ld, st),
+           "indexer scores");
+  if (ev && ev_i < n_ev) CUDA_TRY(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
+  SelectRows rows;
+  rows.chunks = p.chunks;
+  rows.chunk = p.chunk;
+  rows.n_rows = Tq * p.chunks;
+  rows.rate = cfg->m;
+  rows.N = N;
+  rows.q_pos = q_pos;
+  rows.ld_scores = p.ld;
+  if (p.chunks == 1) {
+    CUDA_TRY(launch_select_from_scores(scores, rows, cfg->topk, topk_idx, nullptr, st), "select");
+  } else {
+    uint64_t* cand = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(ws) + p.cand_off);
+    CUDA_TRY(launch_select_from_scores(scores, rows, cfg->topk, nullptr, cand, st), "select chunks");
+    CUDA_TRY(launch_select_merge(cand, Tq, p.chunks * cfg->topk, cfg->topk, topk_idx, st), "select merge");
+  }
+  if (ev && ev_i < n_ev) CUDA_TRY(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
+  return HCA_OK;
+}
+
+MqaProblem make_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N,
+                    const int32_t* idx, int n_idx, int rate, const hca_bf16* win, long long win_seq_stride,
+                    const int32_t* q_pos, int Tq, int mode, hca_bf16* out) {
+  MqaProblem p;
+  p.q = reinterpret_cast<const bf16*>(q);
+  p.kv = reinterpret_cast<const bf16*>(kv);
+  p.kv_seq_stride = kv_seq_stride;
+  p.N = N;
+  p.idx = idx;
+  p.n_idx = n_idx;
+  p.rate = rate;
+  p.win = reinterpret_cast<const bf16*>(win);
+  p.win_seq_stride = win_seq_stride;
+  p.q_pos = q_pos;
+  p.Tq = Tq;
+  p.mode = mode;
+  p.H = cfg->n_heads;
+  p.c = cfg->c;
+  p.n_win = cfg->n_win;
+  p.scale = cfg->scale;
+  p.out = reinterpret_cast<bf16*>(out);
+  return p;
+}
+
+size_t mqa_ws_bound(const hca_layer_cfg* cfg, int Tq, int N, int n_idx) {
+  MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, N > n_idx ? N : n_idx, nullptr, 0, 1, nullptr, 0, nullptr, Tq,
+                          HCA_MODE_DECODE, nullptr);
+  return plan_mqa(p).ws_bytes;
+}
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" {
+
+const char* hca_last_error(void) { return g_err.c_str(); }
+
+int hca_last_launch_count(void) { return g_last_launches; }
+
+const char* hca_version(void) { return "hca-b200 0.1 (sm_100a)"; }
+
+int csa_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int ld_logits, const float* pos_bias,
+                 int ld_bias, int T, int c, int m, hca_bf16* out, int ld_out, void* stream) {
+  g_err.clear();
+  CHECK(T >= 0 && c > 0 && m >= 1 && m <= 16, HCA_ERR_INVALID_ARG, "csa_compress: T=%d c=%d m=%d", T, c, m);
+  CHECK(c % 8 == 0, HCA_ERR_UNSUPPORTED, "csa_compress: c=%d not a multiple of 8", c);
+  CHECK(ld_cand >= c && ld_logits >= c && ld_bias >= c && ld_out >= c && ld_cand % 8 == 0 && ld_logits % 8 == 0 &&
+            ld_out % 8 == 0 && ld_bias % 4 == 0,
+        HCA_ERR_INVALID_ARG, "csa_compress: bad row strides");
+  if (T / m == 0) return injected("csa_compress") ? fail(HCA_ERR_INJECTED, "csa_compress: injected") : HCA_OK;
+  CHECK_PTR(cand, "csa_compress: cand");
+  CHECK_PTR(logits, "csa_compress: logits");
+  CHECK_PTR(pos_bias, "csa_compress: pos_bias");
+  CHECK_PTR(out, "csa_compress: out");
+  if (injected("csa_compress")) return fail(HCA_ERR_INJECTED, "csa_compress: injected");
+  CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(cand), ld_cand, reinterpret_cast<const bf16*>(logits),
+                           ld_logits, pos_bias, ld_bias, 1, 0, T, c, m, true, reinterpret_cast<bf16*>(out), ld_out, 0,
+                           as_stream(stream)),
+           "csa_compress");
+  return HCA_OK;
+}
+
+int hca_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int ld_logits, const float* pos_bias,
+                 int ld_bias, int B, long long seq_stride_in, int T, int c, int m_hca, hca_bf16* out, int ld_out,
+                 long long seq_stride_out, void* stream) {
+  g_err.clear();
+  CHECK(B >= 0 && B <= 65535 && T >= 0 && c > 0 && m_hca >= 1 && m_hca <= 1024, HCA_ERR_INVALID_ARG,
+        "hca_compress: B=%d T=%d c=%d m'=%d", B, T, c, m_hca);
+  CHECK(c % 8 == 0, HCA_ERR_UNSUPPORTED, "hca_compress: c=%d not a multiple of 8", c);
+  CHECK(ld_cand >= c && ld_logits >= c && ld_bias >= c && ld_out >= c && ld_cand % 8 == 0 && ld_logits % 8 == 0 &&
+            ld_out % 8 == 0 && ld_bias % 4 == 0 && seq_stride_in % 8 == 0 && seq_stride_out % 8 == 0,
+        HCA_ERR_INVALID_ARG, "hca_compress: bad strides");
+  if (T / m_hca == 0 || B == 0) return injected("hca_compress") ? fail(HCA_ERR_INJECTED, "hca_compress: injected") : HCA_OK;
+  CHECK_PTR(cand, "hca_compress: cand");
+  CHECK_PTR(logits, "hca_compress: logits");
+  CHECK_PTR(pos_bias, "hca_compress: pos_bias");
+  CHECK_PTR(out, "hca_compress: out");
+  if (injected("hca_compress")) return fail(HCA_ERR_INJECTED, "hca_compress: injected");
+  CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(cand), ld_cand, reinterpret_cast<const bf16*>(logits),
+                           ld_logits, pos_bias, ld_bias, B, seq_stride_in, T, c, m_hca, false,
+                           reinterpret_cast<bf16*>(out), ld_out, seq_stride_out, as_stream(stream)),
+           "hca_compress");
+  return HCA_OK;
+}
+
+size_t hca_workspace_size(int op, const hca_layer_cfg* cfg, int Tq, int N, int mode) {
+  (void)mode;
+  if (check_cfg(cfg) != HCA_OK || Tq < 0 || N < 0) return (size_t)-1;
+  switch (op) {
+    case HCA_OP_INDEXER_TOPK:
+      if (indexer_ok(N, cfg->topk) != HCA_OK) return (size_t)-1;
+      return plan_indexer(Tq, N, cfg->topk).bytes;
+    case HCA_OP_SPARSE_MQA:
+      return mqa_ws_bound(cfg, Tq, N, cfg->topk);
+    default:
+      return (size_t)-1;
+  }
+}
+
+int csa_indexer_topk(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* k_idx, long long k_seq_stride, int N,
+                     const int32_t* q_pos, int Tq, int mode, const hca_layer_cfg* cfg, int32_t* topk_idx, void* ws,
+                     size_t ws_bytes, void* stream) {
+  g_err.clear();
+  int s = check_cfg(cfg);
+  if (s != HCA_OK) return s;
+  CHECK(Tq >= 0 && N >= 0, HCA_ERR_INVALID_ARG, "csa_indexer_topk: Tq=%d N=%d", Tq, N);
+  CHECK(mode == HCA_MODE_PREFILL || mode == HCA_MODE_DECODE, HCA_ERR_INVALID_ARG, "csa_indexer_topk: mode=%d", mode);
+  CHECK(mode == HCA_MODE_PREFILL || k_seq_stride % 8 == 0, HCA_ERR_INVALID_ARG, "csa_indexer_topk: k_seq_stride");
+  s = indexer_ok(N, cfg->topk);
+  if (s != HCA_OK) return s;
+  if (Tq == 0) return injected("csa_indexer_topk") ? fail(HCA_ERR_INJECTED, "injected") : HCA_OK;
+  CHECK_PTR(q_idx, "csa_indexer_topk: q_idx");
+  CHECK_PTR(w_idx, "csa_indexer_topk: w_idx");
+  CHECK_PTR(q_pos, "csa_indexer_topk: q_pos");
+  CHECK_PTR(topk_idx, "csa_indexer_topk: topk_idx");
+  if (N > 0) CHECK_PTR(k_idx, "csa_indexer_topk: k_idx");
+  const size_t need = plan_indexer(Tq, N, cfg->topk).bytes;
+  CHECK(ws_bytes >= need, HCA_ERR_WORKSPACE, "csa_indexer_topk: workspace %zu < %zu", ws_bytes, need);
+  if (need) CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
+                  "csa_indexer_topk: ws null or not 256-byte aligned");
+  if (injected("csa_indexer_topk")) return fail(HCA_ERR_INJECTED, "csa_indexer_topk: injected");
+  int ev_i = 0;
+  return run_indexer_topk(reinterpret_cast<const bf16*>(q_idx), w_idx, reinterpret_cast<const bf16*>(k_idx),
+                          k_seq_stride, N, q_pos, Tq, mode, cfg, topk_idx, ws, as_stream(stream), nullptr, 0, ev_i);
+}
+
+static int check_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N,
+                     const int32_t* idx, int n_idx, int rate, const hca_bf16* win, long long win_seq_stride,
+                     const int32_t* q_pos, int Tq, int mode, hca_bf16* out, const char* who) {
+  CHECK(Tq >= 0 && N >= 0 && rate >= 1, HCA_ERR_INVALID_ARG, "%s: Tq=%d N=%d rate=%d", who, Tq, N, rate);
+  CHECK(mode == HCA_MODE_PREFILL || mode == HCA_MODE_DECODE, HCA_ERR_INVALID_ARG, "%s: mode=%d", who, mode);
+  CHECK(!idx || (n_idx > 0 && n_idx <= 4096), HCA_ERR_INVALID_ARG, "%s: n_idx=%d", who, n_idx);
+  CHECK(kv_seq_stride % 8 == 0 && win_seq_stride % 8 == 0, HCA_ERR_INVALID_ARG, "%s: strides", who);
+  if (Tq == 0) return HCA_OK;
+  CHECK_PTR(q, who);
+  CHECK_PTR(win, who);
+  CHECK_PTR(q_pos, who);
+  CHECK_PTR(out, who);
+  if (N > 0) CHECK_PTR(kv, who);
+  if (idx) CHECK_PTR(idx, who);
+  return HCA_OK;
+}
+
+int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N, const int32_t* idx,
+                      int n_idx, int rate, const hca_bf16* win, long long win_seq_stride, const int32_t* q_pos, int Tq,
+                      int mode, const hca_layer_cfg* cfg, hca_bf16* out, void* ws, size_t ws_bytes, void* stream) {
+  g_err.clear();
+  int s = check_cfg(cfg);
+  if (s != HCA_OK) return s;
+  s = check_mqa(cfg, q, kv, kv_seq_stride, N, idx, n_idx, rate, win, win_seq_stride, q_pos, Tq, mode, out,
+                "sparse_mqa_attend");
+  if (s != HCA_OK) return s;
+  MqaProblem p = make_mqa(cfg, q, kv, kv_seq_stride, N, idx, n_idx, rate, win, win_seq_stride, q_pos, Tq, mode, out);
+  const MqaPlan pl = plan_mqa(p);
+  CHECK(ws_bytes >= pl.ws_bytes, HCA_ERR_WORKSPACE, "sparse_mqa_attend: workspace %zu < %zu", ws_bytes, pl.ws_bytes);
+  if (pl.ws_bytes) CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
+                         "sparse_mqa_attend: ws null or not 256-byte aligned");
+  if (injected("sparse_mqa_attend")) return fail(HCA_ERR_INJECTED, "sparse_mqa_attend: injected");
+  if (Tq == 0) return HCA_OK;
+  CUDA_TRY(launch_mqa(p, pl, ws, as_stream(stream)), "sparse_mqa_attend");
+  return HCA_OK;
+}
+
+// ---- decode ------------------------------------------------------------------
+static size_t decode_ws(const hca_layer_cfg* cfg, const hca_decode_args* a) {
+  size_t need = 0;
+  if (a->csa_q) {
+    need = std::max(need, plan_indexer(a->B, a->csa_N, cfg->topk).bytes);
+    MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, a->csa_N, reinterpret_cast<const int32_t*>(1), cfg->topk,
+                            cfg->m, nullptr, 0, nullptr, a->B, HCA_MODE_DECODE, nullptr);
+    need = std::max(need, plan_mqa(p).ws_bytes);
+  }
+  if (a->hca_q) {
+    MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, a->hca_N, nullptr, 0, cfg->m_hca, nullptr, 0, nullptr, a->B,
+                            HCA_MODE_DECODE, nullptr);
+    need = std::max(need, plan_mqa(p).ws_bytes);
+  }
+  return round256(need);
+}
+
+size_t hybrid_attn_decode_workspace(const hca_layer_cfg* cfg, const hca_decode_args* a) {
+  if (check_cfg(cfg) != HCA_OK || !a || a->B < 0) return (size_t)-1;
+  if (a->csa_q && indexer_ok(a->csa_N, cfg->topk) != HCA_OK) return (size_t)-1;
+  return decode_ws(cfg, a);
+}
+
+int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void* ws, size_t ws_bytes, void* stream) {
+  g_err.clear();
+  int s = check_cfg(cfg);
+  if (s != HCA_OK) return s;
+  CHECK(a != nullptr, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: args null");
+  CHECK(a->B >= 0 && a->B <= 65535, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: B=%d", a->B);
+  CHECK(a->csa_q || a->hca_q, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: neither layer given");
+  CHECK(a->n_events >= 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: n_events");
+  if (a->B == 0) return HCA_OK;
+  CHECK_PTR(a->q_pos, "hybrid_attn_decode: q_pos");
+  if (a->csa_q) {
+    s = indexer_ok(a->csa_N, cfg->topk);
+    if (s != HCA_OK) return s;
+    CHECK(a->csa_N > 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: csa_N=%d", a->csa_N);
+    CHECK_PTR(a->csa_q_idx, "hybrid_attn_decode: csa_q_idx");
+    CHECK_PTR(a->csa_w_idx, "hybrid_attn_decode: csa_w_idx");
+    CHECK_PTR(a->csa_k_idx, "hybrid_attn_decode: csa_k_idx");
+    CHECK_PTR(a->csa_topk_idx, "hybrid_attn_decode: csa_topk_idx");
+    CHECK(a->csa_k_stride % 8 == 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: csa_k_stride");
+    s = check_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_N, a->csa_topk_idx, cfg->topk, cfg->m,
+                  a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out, "hybrid_attn_decode: csa");
+    if (s != HCA_OK) return s;
+  }
+  if (a->hca_q) {
+    CHECK(a->hca_N > 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: hca_N=%d", a->hca_N);
+    s = check_mqa(cfg, a->hca_q, a->hca_kv, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, a->hca_win,
+                  a->hca_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->hca_out, "hybrid_attn_decode: hca");
+    if (s != HCA_OK) return s;
+    if (a->hca_block_cand) {
+      CHECK_PTR(a->hca_block_logits, "hybrid_attn_decode: hca_block_logits");
+      CHECK_PTR(a->hca_pos_bias, "hybrid_attn_decode: hca_pos_bias");
+      CHECK(a->hca_block_stride % 8 == 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: hca_block_stride");
+    }
+  }
+  const size_t need = decode_ws(cfg, a);
+  CHECK(ws_bytes >= need, HCA_ERR_WORKSPACE, "hybrid_attn_decode: workspace %zu < %zu", ws_bytes, need);
+  if (need) CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
+                  "hybrid_attn_decode: ws null or not 256-byte aligned");
+  if (injected("hybrid_attn_decode")) return fail(HCA_ERR_INJECTED, "hybrid_attn_decode: injected");
+
+  cudaStream_t st = as_stream(stream);
+  g_launch_counter = 0;
+  g_last_launches = 0;
+  int ev_i = 0;
+  void* const* ev = a->events;
+  const int n_ev = ev ? a->n_events : 0;
+  auto mark = [&]() -> int {
+    if (ev && ev_i < n_ev) return cuda_status(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
+    return HCA_OK;
+  };
+  if ((s = mark()) != HCA_OK) return s;
+  if (a->hca_q && a->hca_block_cand) {
+    // newest complete HCA block of every request -> its cache row.  All
+    // requests share one position here (q_pos is on the device), so the row
+    // is hca_N - 1: the caller passes caches sized to the complete blocks.
+    CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), cfg->c,
+                             reinterpret_cast<const bf16*>(a->hca_block_logits), cfg->c, a->hca_pos_bias, cfg->c, a->B,
+                             a->hca_block_stride, cfg->m_hca, cfg->c, cfg->m_hca, false,
+                             reinterpret_cast<bf16*>(a->hca_kv) + (long long)(a->hca_N - 1) * cfg->c, cfg->c,
+                             a->hca_kv_stride, st),
+             "decode: hca compress");
+    if ((s = mark()) != HCA_OK) return s;
+  }
+  if (a->csa_q) {
+    s = run_indexer_topk(reinterpret_cast<const bf16*>(a->csa_q_idx), a->csa_w_idx,
+                         reinterpret_cast<const bf16*>(a->csa_k_idx), a->csa_k_stride, a->csa_N, a->q_pos, a->B,
+                         HCA_MODE_DECODE, cfg, a->csa_topk_idx, ws, st, ev, n_ev, ev_i);
+    if (s != HCA_OK) return s;
+    MqaProblem p = make_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_N, a->csa_topk_idx, cfg->topk, cfg->m,
+                            a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out);
+    CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "decode: csa attention");
+    if ((s = mark()) != HCA_OK) return s;
+  }
+  if (a->hca_q) {
+    MqaProblem p = make_mqa(cfg, a->hca_q, a->hca_kv, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, a->hca_win,
+                            a->hca_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->hca_out);
+    CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "decode: hca attention");
+    if ((s = mark()) != HCA_OK) return s;
+  }
+  g_last_launches = g_launch_counter;
+  return HCA_OK;
+}
+
+// ---- prefill -----------------------------------------------------------------
+static size_t prefill_ws(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
+  const int T = a->T;
+  const int Nc = T / cfg->m;
+  size_t need = plan_indexer(T, Nc, cfg->topk).bytes;
+  MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, Nc, reinterpret_cast<const int32_t*>(1), cfg->topk, cfg->m,
+                          nullptr, 0, nullptr, T, HCA_MODE_PREFILL, nullptr);
+  need = std::max(need, plan_mqa(p).ws_bytes);
+  if (a->hca_kv) {
+    MqaProblem ph = make_mqa(cfg, nullptr, nullptr, 0, T / cfg->m_hca, nullptr, 0, cfg->m_hca, nullptr, 0, nullptr, T,
+                             HCA_MODE_PREFILL, nullptr);
+    need = std::max(need, plan_mqa(ph).ws_bytes);
+  }
+  return round256(need);
+}
+
+size_t hybrid_attn_prefill_workspace(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
+  if (check_cfg(cfg) != HCA_OK || !a || a->T < 0) return (size_t)-1;
+  if (indexer_ok(a->T / cfg->m, cfg->topk) != HCA_OK) return (size_t)-1;
+  return prefill_ws(cfg, a);
+}
+
+int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, void* ws, size_t ws_bytes, void* stream) {
+  g_err.clear();
+  int s = check_cfg(cfg);
+  if (s != HCA_OK) return s;
+  CHECK(a != nullptr, HCA_ERR_INVALID_ARG, "hybrid_attn_prefill: args null");
+  CHECK(a->T >= 0, HCA_ERR_INVALID_ARG, "hybrid_attn_prefill: T=%d", a->T);
+  CHECK(a->n_events >= 0, HCA_ERR_INVALID_ARG, "hybrid_attn_prefill: n_events");
+  const int T = a->T;
+  if (T == 0) return HCA_OK;
+  const int Nc = T / cfg->m;
+  s = indexer_ok(Nc, cfg->topk);
+  if (s != HCA_OK) return s;
+  CHECK_PTR(a->q_pos, "hybrid_attn_prefill: q_pos");
+  CHECK_PTR(a->cand, "hybrid_attn_prefill: cand");
+  CHECK_PTR(a->logits, "hybrid_attn_prefill: logits");
+  CHECK_PTR(a->kidx_cand, "hybrid_attn_prefill: kidx_cand");
+  CHECK_PTR(a->bias_csa, "hybrid_attn_prefill: bias_csa");
+  CHECK_PTR(a->q_idx, "hybrid_attn_prefill: q_idx");
+  CHECK_PTR(a->w_idx, "hybrid_attn_prefill: w_idx");
+  CHECK_PTR(a->q, "hybrid_attn_prefill: q");
+  CHECK_PTR(a->topk_idx, "hybrid_attn_prefill: topk_idx");
+  CHECK_PTR(a->csa_out, "hybrid_attn_prefill: csa_out");
+  if (Nc > 0) {
+    CHECK_PTR(a->csa_kv, "hybrid_attn_prefill: csa_kv");
+    CHECK_PTR(a->csa_k_idx, "hybrid_attn_prefill: csa_k_idx");
+  }
+  if (a->hca_kv) {
+    CHECK_PTR(a->bias_hca, "hybrid_attn_prefill: bias_hca");
+    CHECK_PTR(a->hca_q, "hybrid_attn_prefill: hca_q");
+    CHECK_PTR(a->hca_out, "hybrid_attn_prefill: hca_out");
+  }
+  const size_t need = prefill_ws(cfg, a);
+  CHECK(ws_bytes >= need, HCA_ERR_WORKSPACE, "hybrid_attn_prefill: workspace %zu < %zu", ws_bytes, need);
+  CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
+        "hybrid_attn_prefill: ws null or not 256-byte aligned");
+  if (injected("hybrid_attn_prefill")) return fail(HCA_ERR_INJECTED, "hybrid_attn_prefill: injected");
+
+  cudaStream_t st = as_stream(stream);
+  g_launch_counter = 0;
+  g_last_launches = 0;
+  int ev_i = 0;
+  void* const* ev = a->events;
+  const int n_ev = ev ? a->n_events : 0;
+  auto mark = [&]() -> int {
+    if (ev && ev_i < n_ev) return cuda_status(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
+    return HCA_OK;
+  };
+  const int c = cfg->c, dI = cfg->d_idx;
+  if ((s = mark()) != HCA_OK) return s;
+  // CSA compression of KV entries and of indexer keys (logits/bias: first d_I channels)
+  CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->cand), c, reinterpret_cast<const bf16*>(a->logits), c,
+                           a->bias_csa, c, 1, 0, T, c, cfg->m, true, reinterpret_cast<bf16*>(a->csa_kv), c, 0, st),
+           "prefill: csa compress");
+  CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->kidx_cand), dI, reinterpret_cast<const bf16*>(a->logits),
+                           c, a->bias_csa, c, 1, 0, T, dI, cfg->m, true, reinterpret_cast<bf16*>(a->csa_k_idx), dI, 0,
+                           st),
+           "prefill: indexer-key compress");
+  if ((s = mark()) != HCA_OK) return s;
+  s = run_indexer_topk(reinterpret_cast<const bf16*>(a->q_idx), a->w_idx, reinterpret_cast<const bf16*>(a->csa_k_idx),
+                       0, Nc, a->q_pos, T, HCA_MODE_PREFILL, cfg, a->topk_idx, ws, st, ev, n_ev, ev_i);
+  if (s != HCA_OK) return s;
+  {
+    MqaProblem p = make_mqa(cfg, a->q, a->csa_kv, 0, Nc, a->topk_idx, cfg->topk, cfg->m, a->cand, 0, a->q_pos, T,
+                            HCA_MODE_PREFILL, a->csa_out);
+    CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "prefill: csa attention");
+    if ((s = mark()) != HCA_OK) return s;
+  }
+  if (a->hca_kv) {
+    const int Nh = T / cfg->m_hca;
+    CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->cand), c, reinterpret_cast<const bf16*>(a->logits), c,
+                             a->bias_hca, c, 1, 0, T, c, cfg->m_hca, false, reinterpret_cast<bf16*>(a->hca_kv), c, 0,
+                             st),
+             "prefill: hca compress");
+    MqaProblem p = make_mqa(cfg, a->hca_q, a->hca_kv, 0, Nh, nullptr, 0, cfg->m_hca, a->cand, 0, a->q_pos, T,
+                            HCA_MODE_PREFILL, a->hca_out);
+    CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "prefill: hca attention");
+    if ((s = mark()) != HCA_OK) return s;
+  }
+  g_last_launches = g_launch_counter;
+  return HCA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,82 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace hca {
+
+// Kernels launched on this thread (incremented by every launch_* below).
+extern thread_local int g_launch_counter;
+
+// ---- compress.cu ----------------------------------------------------------
+cudaError_t launch_compress(const bf16* cand, int ld_cand, const bf16* logits, int ld_logits,
+                            const float* bias, int ld_bias, int B, long long seq_in, int T, int c,
+                            int rate, bool overlap, bf16* out, int ld_out, long long seq_out,
+                            cudaStream_t stream);
+
+// ---- topk.cu ----------------------------------------------------------------
+// Largest candidate-count a single select row may have (smem-resident).
+constexpr int kSelectMaxN = 24576;
+
+// Row r of a score matrix: scores at scores + r*ld_scores (f32), its entry
+// indices are idx_base(r) + position; n(r) elements are candidates.
+// Two ways to describe rows:
+//   by query: row = query q (r = q), n = min(n_visible(q_pos[q]), N) - chunk0
+//   by chunk: row = (q, j), scores + q*ld + j*chunk, n = clamp(nvis - j*chunk, 0, chunk)
+struct SelectRows {
+  int n_rows;       // number of rows
+  int chunks;       // chunks per query (rows = Tq * chunks)
+  int chunk;        // chunk length (elements)
+  int rate;         // compression rate for visibility
+  int N;            // entries per request
+  const int32_t* q_pos;
+  long long ld_scores;  // elements between queries
+};
+// Select the top-k of each row of f32 scores and write either final indices
+// (out_idx [rows, k], -1 padded) or composite candidates (out_cand [rows, k]).
+cudaError_t launch_select_from_scores(const float* scores, const SelectRows& rows, int k,
+                                      int32_t* out_idx, uint64_t* out_cand, cudaStream_t stream);
+// Merge: row q has n_cand composite candidates at cand + q*n_cand; write the
+// top-k indices to out_idx [rows, k].
+cudaError_t launch_select_merge(const uint64_t* cand, int n_rows, int n_cand, int k,
+                                int32_t* out_idx, cudaStream_t stream);
+
+// ---- indexer.cu ---------------------------------------------------------------
+// scores[q, s] = sum_j w[q,j] relu(q_idx[q,j,:] . K[s,:]) for visible s (others untouched).
+cudaError_t launch_indexer_scores(const bf16* q_idx, const float* w_idx, const bf16* k_idx,
+                                  long long k_seq_stride, int N, const int32_t* q_pos, int Tq,
+                                  int mode, int rate, int H_I, int d_I, float* scores,
+                                  long long ld_scores, cudaStream_t stream);
+
+// ---- mqa.cu -----------------------------------------------------------------------
+struct MqaProblem {
+  const bf16* q;            // [Tq, H, c]
+  const bf16* kv;           // compressed entries (request r at kv + r*kv_seq_stride)
+  long long kv_seq_stride;
+  int N;                    // entries per request
+  const int32_t* idx;       // [Tq, n_idx] or nullptr (dense over visible)
+  int n_idx;
+  int rate;
+  const bf16* win;
+  long long win_seq_stride;
+  const int32_t* q_pos;
+  int Tq;
+  int mode;
+  int H, c, n_win;
+  float scale;
+  bf16* out;                // [Tq, H, c]
+};
+// Rows of one split; the workspace layout is decided by plan_mqa().
+struct MqaPlan {
+  int splits;          // splits per query (1 = no combine)
+  int rows_per_split;  // rows of the query's row list per split
+  int max_rows;        // upper bound of the row-list length
+  size_t ws_bytes;
+};
+MqaPlan plan_mqa(const MqaProblem& p);
+cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& plan, void* ws, cudaStream_t stream);
+
+}  // namespace hca

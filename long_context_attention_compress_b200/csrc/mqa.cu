@@ -1,0 +1,270 @@
+// Shared-KV multi-query attention over compressed entries + sliding window
+// (sm_100a), CUDA-core version with split-K and a combine kernel.
+//
+// For query t and head h over the row set U(t) (QbitAI write-up,
+// "混合注意力機制": CSA step three, KV entries serve as both key and value,
+// and the sliding-window branch of the most recent 128 raw tokens;
+// "DeepSeek V4 Architecture Tricks", HCA section: dense over all entries):
+//   o[t,h,:] = sum_u softmax_u(scale * q[t,h,:] . row_u) row_u
+// U(t) = selected CSA entries (idx) or all visible HCA entries, then the
+// window rows.  Each query's row list is cut into `splits` contiguous ranges;
+// one CTA runs an online softmax over its range in tiles of TR rows and
+// writes either the normalised output (one split) or its softmax state
+// (m, l, unnormalised o) for the combine kernel:
+//   o = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i.
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hca {
+
+constexpr int kMqaThreads = 256;
+constexpr int kTR = 16;  // rows per tile
+
+struct RowList {
+  const bf16* kv;       // this request's entries
+  const int32_t* idx;   // this query's selected entries or nullptr
+  int n_first;          // length of the entry part
+  const bf16* win;      // first window row
+  int n_win;            // window rows
+  int c;
+  __device__ __forceinline__ int length() const { return n_first + n_win; }
+  // pointer of list row u, or nullptr for an empty selected slot
+  __device__ __forceinline__ const bf16* row(int u) const {
+    if (u < n_first) {
+      int s = idx ? idx[u] : u;
+      return s < 0 ? nullptr : kv + (long long)s * c;
+    }
+    return win + (long long)(u - n_first) * c;
+  }
+};
+
+__device__ __forceinline__ RowList make_rows(const MqaProblem& p, int q) {
+  RowList L;
+  const int t = p.q_pos[q];
+  const long long rs = p.mode == HCA_MODE_DECODE ? q : 0;
+  L.kv = p.kv + rs * p.kv_seq_stride;
+  L.c = p.c;
+  if (p.idx) {
+    L.idx = p.idx + (long long)q * p.n_idx;
+    L.n_first = p.n_idx;
+  } else {
+    L.idx = nullptr;
+    L.n_first = n_visible(t, p.rate, p.N);
+  }
+  if (p.mode == HCA_MODE_DECODE) {
+    L.win = p.win + rs * p.win_seq_stride;
+    L.n_win = min(p.n_win, t + 1);
+  } else {
+    const int w0 = max(0, t - p.n_win + 1);
+    L.win = p.win + (long long)w0 * p.c;
+    L.n_win = t - w0 + 1;
+  }
+  return L;
+}
+
+template <int H, int C>
+__global__ void __launch_bounds__(kMqaThreads) mqa_split_kernel(MqaProblem p, int splits, int rows_per_split,
+                                                                float* __restrict__ ws_o, float2* __restrict__ ws_ml) {
+  constexpr int CP = C + 8;  // padded smem row stride (bf16 elements)
+  constexpr int DPT = H * C / kMqaThreads;
+  static_assert(H * C % kMqaThreads == 0, "outputs per thread");
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  bf16* s_q = reinterpret_cast<bf16*>(smem_raw);                   // [H][CP]
+  bf16* s_r = s_q + H * CP;                                         // [TR][CP]
+  float* s_s = reinterpret_cast<float*>(s_r + kTR * CP);            // [H][TR] scores
+  float* s_p = s_s + H * kTR;                                       // [TR][H] probabilities
+  float* s_m = s_p + kTR * H;                                       // [H]
+  float* s_l = s_m + H;                                             // [H]
+  float* s_a = s_l + H;                                             // [H] rescale factor
+  __shared__ int s_valid[kTR];
+
+  const int tid = threadIdx.x;
+  const int q = blockIdx.x / splits;
+  const int sp = blockIdx.x % splits;
+  const RowList L = make_rows(p, q);
+  const int u_begin = sp * rows_per_split;
+  const int u_end = min(L.length(), u_begin + rows_per_split);
+
+  // stage q [H][C]
+  const bf16* qp = p.q + (long long)q * H * C;
+  for (int e = tid; e < H * C / 8; e += kMqaThreads) {
+    const int h = e / (C / 8), d = (e % (C / 8)) * 8;
+    *reinterpret_cast<uint4*>(s_q + h * CP + d) = *reinterpret_cast<const uint4*>(qp + h * C + d);
+  }
+  for (int h = tid; h < H; h += kMqaThreads) { s_m[h] = neg_inf(); s_l[h] = 0.f; }
+  float o[DPT];
+#pragma unroll
+  for (int j = 0; j < DPT; ++j) o[j] = 0.f;
+  const float sl2 = p.scale * kLog2e;
+
+  for (int u0 = u_begin; u0 < u_end; u0 += kTR) {
+    __syncthreads();  // previous tile fully consumed
+    // load TR rows (zeros for missing rows)
+    for (int e = tid; e < kTR * (C / 8); e += kMqaThreads) {
+      const int r = e / (C / 8), d = (e % (C / 8)) * 8;
+      const int u = u0 + r;
+      const bf16* rp = u < u_end ? L.row(u) : nullptr;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (rp) v = *reinterpret_cast<const uint4*>(rp + d);
+      *reinterpret_cast<uint4*>(s_r + r * CP + d) = v;
+      if (d == 0) s_valid[r] = rp != nullptr;
+    }
+    __syncthreads();
+    // scores S[h][u] (base-2 scaled)
+    for (int pr = tid; pr < H * kTR; pr += kMqaThreads) {
+      const int h = pr / kTR, r = pr % kTR;
+      const bf16* a = s_q + h * CP;
+      const bf16* b = s_r + r * CP;
+      float acc = 0.f;
+#pragma unroll 4
+      for (int d = 0; d < C; d += 8) {
+        float fa[8], fb[8];
+        unpack8(*reinterpret_cast<const uint4*>(a + d), fa);
+        unpack8(*reinterpret_cast<const uint4*>(b + d), fb);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc = fmaf(fa[k], fb[k], acc);
+      }
+      s_s[h * kTR + r] = s_valid[r] ? acc * sl2 : neg_inf();
+    }
+    __syncthreads();
+    // online softmax per head
+    for (int h = tid; h < H; h += kMqaThreads) {
+      float mx = s_m[h];
+      float tm = neg_inf();
+#pragma unroll
+      for (int r = 0; r < kTR; ++r) tm = fmaxf(tm, s_s[h * kTR + r]);
+      const float mn = fmaxf(mx, tm);
+      float alpha = 1.f, lsum = 0.f;
+      if (mn == neg_inf()) {
+#pragma unroll
+        for (int r = 0; r < kTR; ++r) s_p[r * H + h] = 0.f;
+      } else {
+        alpha = fast_exp2(mx - mn);
+#pragma unroll
+        for (int r = 0; r < kTR; ++r) {
+          const float e = fast_exp2(s_s[h * kTR + r] - mn);
+          s_p[r * H + h] = e;
+          lsum += e;
+        }
+        s_m[h] = mn;
+      }
+      s_l[h] = s_l[h] * alpha + lsum;
+      s_a[h] = alpha;
+    }
+    __syncthreads();
+    // o = o * alpha + P V
+#pragma unroll
+    for (int j = 0; j < DPT; ++j) {
+      const int oi = tid + kMqaThreads * j;
+      o[j] *= s_a[oi / C];
+    }
+#pragma unroll 2
+    for (int r = 0; r < kTR; ++r) {
+      const bf16* rr = s_r + r * CP;
+      const float* pr = s_p + r * H;
+#pragma unroll
+      for (int j = 0; j < DPT; ++j) {
+        const int oi = tid + kMqaThreads * j;
+        const int h = oi / C, d = oi % C;
+        o[j] = fmaf(pr[h], __bfloat162float(rr[d]), o[j]);
+      }
+    }
+  }
+  __syncthreads();
+  if (splits == 1) {
+    bf16* op = p.out + (long long)q * H * C;
+#pragma unroll
+    for (int j = 0; j < DPT; ++j) {
+      const int oi = tid + kMqaThreads * j;
+      const float l = s_l[oi / C];
+      op[oi] = __float2bfloat16_rn(l > 0.f ? o[j] / l : 0.f);
+    }
+  } else {
+    float* wo = ws_o + ((long long)q * splits + sp) * H * C;
+#pragma unroll
+    for (int j = 0; j < DPT; ++j) wo[tid + kMqaThreads * j] = o[j];
+    for (int h = tid; h < H; h += kMqaThreads)
+      ws_ml[((long long)q * splits + sp) * H + h] = make_float2(s_m[h], s_l[h]);
+  }
+}
+
+// combine: grid (Tq, H), block 128 threads over C
+__global__ void __launch_bounds__(128) mqa_combine_kernel(const float* __restrict__ ws_o,
+                                                          const float2* __restrict__ ws_ml, int splits,
+                                                          int H, int C, bf16* __restrict__ out) {
+  const int q = blockIdx.x, h = blockIdx.y;
+  float M = neg_inf();
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, ws_ml[((long long)q * splits + s) * H + h].x);
+  float den = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float2 ml = ws_ml[((long long)q * splits + s) * H + h];
+    if (ml.y > 0.f) den += fast_exp2(ml.x - M) * ml.y;
+  }
+  for (int d = threadIdx.x; d < C; d += 128) {
+    float num = 0.f;
+    for (int s = 0; s < splits; ++s) {
+      const float2 ml = ws_ml[((long long)q * splits + s) * H + h];
+      if (ml.y > 0.f) num += fast_exp2(ml.x - M) * ws_o[(((long long)q * splits + s) * H + h) * C + d];
+    }
+    out[((long long)q * H + h) * C + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+  }
+}
+
+template <int H, int C>
+static size_t mqa_smem() {
+  return (size_t)(H + kTR) * (C + 8) * sizeof(bf16) + (size_t)(2 * H * kTR + 3 * H) * sizeof(float);
+}
+
+MqaPlan plan_mqa(const MqaProblem& p) {
+  MqaPlan pl;
+  const int first = p.idx ? p.n_idx : p.N;
+  pl.max_rows = first + p.n_win;
+  const int target_ctas = 148 * 4;
+  int splits = 1;
+  if (p.Tq < target_ctas) {
+    splits = (target_ctas + p.Tq - 1) / p.Tq;
+    const int max_splits = (pl.max_rows + kTR - 1) / kTR;
+    if (splits > max_splits) splits = max_splits;
+    if (splits < 1) splits = 1;
+  }
+  int rps = (pl.max_rows + splits - 1) / splits;
+  rps = (rps + kTR - 1) / kTR * kTR;
+  splits = (pl.max_rows + rps - 1) / rps;
+  if (splits < 1) splits = 1;
+  pl.splits = splits;
+  pl.rows_per_split = rps;
+  pl.ws_bytes = splits > 1 ? (size_t)p.Tq * splits * p.H * ((size_t)p.c * sizeof(float) + sizeof(float2)) : 0;
+  return pl;
+}
+
+template <int H, int C>
+static cudaError_t launch_mqa_t(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream) {
+  const size_t smem = mqa_smem<H, C>();
+  cudaError_t e = cudaFuncSetAttribute((const void*)mqa_split_kernel<H, C>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  float* ws_o = nullptr;
+  float2* ws_ml = nullptr;
+  if (pl.splits > 1) {
+    ws_o = reinterpret_cast<float*>(ws);
+    ws_ml = reinterpret_cast<float2*>(ws_o + (size_t)p.Tq * pl.splits * H * C);
+  }
+  mqa_split_kernel<H, C><<<p.Tq * pl.splits, kMqaThreads, smem, stream>>>(p, pl.splits, pl.rows_per_split,
+                                                                          ws_o, ws_ml);
+  ++g_launch_counter;
+  e = cudaGetLastError();
+  if (e != cudaSuccess || pl.splits == 1) return e;
+  mqa_combine_kernel<<<dim3(p.Tq, H), 128, 0, stream>>>(ws_o, ws_ml, pl.splits, H, C, p.out);
+  ++g_launch_counter;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream) {
+  if (p.Tq == 0) return cudaSuccess;
+  if (p.H == 64 && p.c == 512) return launch_mqa_t<64, 512>(p, pl, ws, stream);
+  if (p.H == 4 && p.c == 64) return launch_mqa_t<4, 64>(p, pl, ws, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace hca

@@ -1,0 +1,74 @@
+"""Helpers shared by the GPU parity tests: tensor conversion and the
+acceptance rules.
+
+Acceptance (floating point): bf16 inputs, f32 accumulation; an output
+passes when max|gpu - oracle| / rms(oracle) <= 2e-2 over the compared
+elements.  Compressor outputs get a stricter element-wise bound: the GPU's
+bf16 value is within 2^-8 relative (one bf16 rounding of the f32 result plus
+f32 arithmetic error) of the float64 oracle value.
+
+Acceptance (top-k): the GPU's set has exactly min(k, n_visible) distinct,
+visible entries (the rest -1); where it differs from the oracle's set, every
+differing entry's oracle score lies within 1e-3 relative of the oracle's
+k-th score (a near-tie that f32 accumulation may order either way).
+"""
+
+import numpy as np
+import torch
+
+NORM_TOL = 2e-2
+TOPK_BAND = 1e-3
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def to_dev(d, device="cuda"):
+    return {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def norm_err(gpu, ref) -> float:
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = np.sqrt(np.mean(ref ** 2))
+    return float(np.max(np.abs(gpu - ref)) / max(rms, 1e-30))
+
+
+def assert_norm_close(gpu, ref, tol=NORM_TOL, what=""):
+    e = norm_err(gpu, ref)
+    assert e <= tol, f"{what}: normalised max-abs error {e:.3e} > {tol}"
+    return e
+
+
+def assert_bf16_close(gpu, ref64, what=""):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref64 = np.asarray(ref64, dtype=np.float64)
+    scale = np.maximum(np.abs(ref64), 1e-3 * np.sqrt(np.mean(ref64 ** 2)))
+    rel = np.abs(gpu - ref64) / scale
+    worst = float(np.max(rel)) if rel.size else 0.0
+    assert worst <= 2.0 ** -8, f"{what}: worst relative error {worst:.3e} > 2^-8"
+    return worst
+
+
+def check_topk_row(gpu_row, oracle_sel, oracle_scores, k, nvis, band=TOPK_BAND):
+    """Returns the number of near-tie swaps; raises AssertionError on failure."""
+    gpu_row = np.asarray(gpu_row)
+    g = gpu_row[gpu_row >= 0]
+    want = min(k, nvis)
+    assert len(g) == want, f"selected {len(g)} entries, expected {want}"
+    assert np.all(gpu_row[gpu_row < 0] == -1)
+    assert len(np.unique(g)) == len(g), "duplicate entries"
+    assert np.all((g >= 0) & (g < nvis)), "entry not visible"
+    gs, os_ = set(g.tolist()), set(np.asarray(oracle_sel).tolist())
+    if nvis <= k:
+        assert gs == set(range(nvis))
+        return 0
+    diff = gs ^ os_
+    if not diff:
+        return 0
+    kth = oracle_scores[oracle_sel[-1]]
+    tol = band * abs(kth)
+    bad = [s for s in diff if abs(oracle_scores[s] - kth) > tol]
+    assert not bad, f"entries {bad[:5]} differ from the oracle outside the near-tie band (k-th score {kth})"
+    return len(diff) // 2

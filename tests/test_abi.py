@@ -1,0 +1,144 @@
+"""C ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and its host-side argument checking, workspace planning and
+fault injection behave as documented.  No call here reaches a kernel: every
+call fails validation (or is injected) before anything is launched."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HDR = os.path.join(ROOT, "include", "hca.h")
+PKG = os.path.join(ROOT, "long_context_attention_compress_b200")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_attention_compress_b200 import build as b
+    b.build()
+    from long_context_attention_compress_b200 import _lib
+    return _lib
+
+
+def declared_functions():
+    src = open(HDR).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char\s*\*|const char\s*\*)\s*\*?\s*(\w+)\s*\(", src, re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ["csa_compress", "hca_compress", "csa_indexer_topk", "sparse_mqa_attend", "hybrid_attn_decode",
+                 "hybrid_attn_prefill", "hca_workspace_size", "hca_last_error", "hybrid_attn_decode_workspace",
+                 "hybrid_attn_prefill_workspace", "hca_version"]:
+        assert want in names, want
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(lib.lib, n)
+
+
+def test_version(lib):
+    assert "sm_100a" in lib.version()
+
+
+def _cfg(lib, **kw):
+    from long_context_attention_compress_b200 import workloads as wl
+    c = lib.make_cfg(wl.PRO)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+FAKE = 0x10000  # aligned, never dereferenced: every call below stops before a launch
+
+
+def test_unsupported_shapes_rejected(lib):
+    for bad in [dict(c=256), dict(n_heads=32), dict(d_idx=64), dict(topk=4096), dict(n_win=512)]:
+        cfg = _cfg(lib, **bad)
+        assert lib.workspace_size(lib.HCA_OP_INDEXER_TOPK, cfg, 1, 1024, 1) == lib.SIZE_MAX
+        st = lib._indexer(FAKE, FAKE, FAKE, 0, 1024, FAKE, 1, 1, ctypes.byref(cfg), FAKE, FAKE, 1 << 30, None)
+        assert st == -2, (bad, st, lib.last_error())
+    cfg = _cfg(lib, c=0)
+    assert lib._indexer(FAKE, FAKE, FAKE, 0, 1024, FAKE, 1, 1, ctypes.byref(cfg), FAKE, FAKE, 1 << 30, None) == -1
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    cfg = _cfg(lib)
+    st = lib._indexer(None, FAKE, FAKE, 0, 1024, FAKE, 4, 1, ctypes.byref(cfg), FAKE, FAKE, 1 << 30, None)
+    assert st == -1 and "q_idx" in lib.last_error()
+    st = lib._indexer(FAKE + 2, FAKE, FAKE, 0, 1024, FAKE, 4, 1, ctypes.byref(cfg), FAKE, FAKE, 1 << 30, None)
+    assert st == -1 and "aligned" in lib.last_error()
+    st = lib._csa_compress(FAKE, 512, None, 512, FAKE, 512, 64, 512, 4, FAKE, 512, None)
+    assert st == -1
+    st = lib._csa_compress(FAKE, 500, FAKE, 512, FAKE, 512, 64, 512, 4, FAKE, 512, None)
+    assert st == -1  # row stride too small
+    st = lib._mqa(FAKE, FAKE, 0, 100, None, 0, 0, FAKE, 0, FAKE, 4, 0, ctypes.byref(cfg), FAKE, None, 0, None)
+    assert st == -1  # rate 0
+
+
+def test_workspace_too_small(lib):
+    cfg = _cfg(lib)
+    need = lib.workspace_size(lib.HCA_OP_INDEXER_TOPK, cfg, 8, 262144, 1)
+    assert 0 < need < lib.SIZE_MAX
+    st = lib._indexer(FAKE, FAKE, FAKE, 262144 * 128, 262144, FAKE, 8, 1, ctypes.byref(cfg), FAKE, FAKE, need - 1,
+                      None)
+    assert st == -3 and "workspace" in lib.last_error()
+
+
+def test_workspace_sizes_monotone(lib):
+    cfg = _cfg(lib)
+    a = lib.workspace_size(lib.HCA_OP_SPARSE_MQA, cfg, 8, 8192, 1)
+    b = lib.workspace_size(lib.HCA_OP_SPARSE_MQA, cfg, 8, 262144, 1)
+    assert 0 <= a <= b < lib.SIZE_MAX
+    assert lib.workspace_size(99, cfg, 1, 1, 1) == lib.SIZE_MAX
+
+
+def test_decode_workspace_query(lib):
+    cfg = _cfg(lib)
+    a = lib.DecodeArgs()
+    a.B = 8
+    a.csa_q = FAKE
+    a.csa_N = 262144
+    a.hca_q = FAKE
+    a.hca_N = 8192
+    need = lib.hybrid_attn_decode_workspace(cfg, a)
+    assert 0 < need < lib.SIZE_MAX and need % 256 == 0
+    a.csa_N = 1 << 26  # too many chunks to merge
+    assert lib.hybrid_attn_decode_workspace(cfg, a) == lib.SIZE_MAX
+
+
+def test_fault_injection(lib, monkeypatch):
+    cfg = _cfg(lib)
+    monkeypatch.setenv("HCA_INJECT_FAULT", "csa_indexer_topk")
+    need = lib.workspace_size(lib.HCA_OP_INDEXER_TOPK, cfg, 4, 4096, 1)
+    st = lib._indexer(FAKE, FAKE, FAKE, 4096 * 128, 4096, FAKE, 4, 1, ctypes.byref(cfg), FAKE, FAKE, need, None)
+    assert st == -6 and "injected" in lib.last_error()
+    # other entry points are unaffected (this one then fails validation instead)
+    st = lib._csa_compress(FAKE, 512, None, 512, FAKE, 512, 64, 512, 4, FAKE, 512, None)
+    assert st == -1
+    monkeypatch.setenv("HCA_INJECT_FAULT", "all")
+    st = lib._csa_compress(FAKE, 512, FAKE, 512, FAKE, 512, 64, 512, 4, FAKE, 512, None)
+    assert st == -6
+    with pytest.raises(lib.HcaError) as ei:
+        lib._check(st)
+    assert ei.value.status == -6
+
+
+def test_bindings_refuse_cpu_tensors(lib):
+    import torch
+    from long_context_attention_compress_b200 import workloads as wl
+    d = wl.prefill_inputs(wl.TINY, T=16, seed=0)
+    with pytest.raises(ValueError):
+        lib.csa_compress(d["cand"], d["logits"], d["bias_csa"], 4)
+    with pytest.raises(TypeError):
+        lib._ptr([1, 2], torch.int32)
