@@ -90,10 +90,13 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
+        self.first = ""
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            # the timed region starts only once the sampler is producing samples
+            self.first = self.proc.stdout.readline()
         except (FileNotFoundError, OSError):
             self.proc = None
         return self
@@ -407,8 +410,22 @@ def run_ours(a):
         bench.step()
     torch.cuda.synchronize()
     launches = bench.launches_per_step()
+    if a.steps is None:
+        # default K: a timed region of about 2 s (long enough for the clock sampler)
+        t0 = time.perf_counter()
+        for _ in range(3):
+            flush.zero_()
+            bench.step(record=False)
+        torch.cuda.synchronize()
+        per = (time.perf_counter() - t0) / 3
+        a.steps = int(min(20000, max(20, math.ceil(2.0 / max(per, 1e-6)))))
+        if ws > 1:
+            import torch.distributed as dist
+            t = torch.tensor([a.steps], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            a.steps = int(t.item())
     # phase breakdown pass (events between kernels, one sync per step)
-    _, phase_ms = timed_steps(bench, a.steps, flush, rank, ws, device, record=True)
+    _, phase_ms = timed_steps(bench, min(a.steps, 50), flush, rank, ws, device, record=True)
     # headline: K steps without intermediate host syncs
     with ClockSampler(local) as clk:
         total_ms, _ = timed_steps(bench, a.steps, flush, rank, ws, device, record=False)
@@ -529,7 +546,8 @@ def run_reference(a):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: enough for a ~2 s timed region)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="hybrid_decode_b8_1m", choices=[k for k in wl.WORKLOADS
                                                                           if k != "tiny_prefill_1k"])
@@ -541,6 +559,7 @@ def main():
     if a.warmup < 3:
         print("warning: fewer than 3 warm-up steps; the number is not a valid measurement", file=sys.stderr)
     if a.impl == "reference":
+        a.steps = a.steps or 3
         run_reference(a)
     else:
         run_ours(a)
