@@ -137,6 +137,39 @@ int csa_indexer_topk(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* 
                      void* stream);
 
 /* ---------------------------------------------------------------------------
+ * csa_indexer_topk_noalloc -- csa_indexer_topk for callers that cannot
+ * allocate device memory.  (Not an operation of the method: the write-ups
+ * have no counterpart; it is the same indexer + top-k with built-in scratch.)
+ *
+ * Some callers can't call cudaMalloc or hand the library a workspace: for
+ * instance a plugin running inside another runtime that owns all device
+ * memory and gives its plugins no allocator, or a serving loop that forbids
+ * device allocation once it has started.  This entry point takes the same
+ * arguments as csa_indexer_topk minus ws/ws_bytes, computes the same result
+ * with the same kernels, and allocates nothing: its scratch is one static
+ * device array of HCA_NOALLOC_SCRATCH_BYTES (16 MiB) inside libhca.so, which
+ * every GPU that loads the library's device code holds until the process
+ * exits.
+ *   - Limit: calls whose scratch need (the same bytes
+ *     hca_workspace_size(HCA_OP_INDEXER_TOPK, cfg, Tq, N, mode) reports)
+ *     exceeds HCA_NOALLOC_SCRATCH_BYTES return HCA_ERR_WORKSPACE and launch
+ *     nothing.  For the 64 x 128 indexer and top-1024 that is, e.g., up to
+ *     8 requests x 262,144 entries or 32 x 32,768.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.  It allocates nothing.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (nothing in it needs to start at zero: each call writes all it reads).
+ *     Calls whose kernels may overlap on the GPU -- on different streams, or
+ *     from several host threads -- race on the array; order them on one
+ *     stream (or synchronise) instead.
+ * ------------------------------------------------------------------------- */
+#define HCA_NOALLOC_SCRATCH_BYTES (16u << 20)
+int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* k_idx,
+                             long long k_seq_stride, int N, const int32_t* q_pos, int Tq, int mode,
+                             const hca_layer_cfg* cfg, int32_t* topk_idx, void* stream);
+
+/* ---------------------------------------------------------------------------
  * sparse_mqa_attend -- core shared-KV multi-query attention over compressed
  * entries plus the sliding window, one softmax ([QbitAI] CSA step three, the
  * KV-entry-as-key-and-value remark and the sliding-window paragraph;

@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "common.cuh"
@@ -266,6 +267,73 @@ int csa_indexer_topk(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* 
   int ev_i = 0;
   return run_indexer_topk(reinterpret_cast<const bf16*>(q_idx), w_idx, reinterpret_cast<const bf16*>(k_idx),
                           k_seq_stride, N, q_pos, Tq, mode, cfg, topk_idx, ws, as_stream(stream), nullptr, 0, ev_i);
+}
+
+// ---- csa_indexer_topk_noalloc ------------------------------------------------
+// Scratch for callers that cannot allocate device memory: one file-scope
+// device array, present on every GPU that loads this module until the
+// process exits.  Host code only ever sees a stand-in symbol for it; the
+// real device address comes from cudaGetSymbolAddress, taken once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HCA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e, "csa_indexer_topk_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(HCA_ERR_UNSUPPORTED, "csa_indexer_topk_noalloc: device %d beyond %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_status(e, "csa_indexer_topk_noalloc: cudaGetSymbolAddress");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return HCA_OK;
+}
+}  // namespace
+
+int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* k_idx,
+                             long long k_seq_stride, int N, const int32_t* q_pos, int Tq, int mode,
+                             const hca_layer_cfg* cfg, int32_t* topk_idx, void* stream) {
+  g_err.clear();
+  int s = check_cfg(cfg);
+  if (s != HCA_OK) return s;
+  CHECK(Tq >= 0 && N >= 0, HCA_ERR_INVALID_ARG, "csa_indexer_topk_noalloc: Tq=%d N=%d", Tq, N);
+  CHECK(mode == HCA_MODE_PREFILL || mode == HCA_MODE_DECODE, HCA_ERR_INVALID_ARG,
+        "csa_indexer_topk_noalloc: mode=%d", mode);
+  CHECK(mode == HCA_MODE_PREFILL || k_seq_stride % 8 == 0, HCA_ERR_INVALID_ARG,
+        "csa_indexer_topk_noalloc: k_seq_stride");
+  s = indexer_ok(N, cfg->topk);
+  if (s != HCA_OK) return s;
+  const size_t need = plan_indexer(Tq, N, cfg->topk).bytes;
+  CHECK(need <= (size_t)HCA_NOALLOC_SCRATCH_BYTES, HCA_ERR_WORKSPACE,
+        "csa_indexer_topk_noalloc: Tq=%d x N=%d needs %zu bytes of scratch, more than the built-in %zu; "
+        "use csa_indexer_topk with a workspace",
+        Tq, N, need, (size_t)HCA_NOALLOC_SCRATCH_BYTES);
+  if (Tq == 0) return HCA_OK;
+  CHECK_PTR(q_idx, "csa_indexer_topk_noalloc: q_idx");
+  CHECK_PTR(w_idx, "csa_indexer_topk_noalloc: w_idx");
+  CHECK_PTR(q_pos, "csa_indexer_topk_noalloc: q_pos");
+  CHECK_PTR(topk_idx, "csa_indexer_topk_noalloc: topk_idx");
+  if (N > 0) CHECK_PTR(k_idx, "csa_indexer_topk_noalloc: k_idx");
+  if (injected("csa_indexer_topk_noalloc")) return fail(HCA_ERR_INJECTED, "csa_indexer_topk_noalloc: injected");
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != HCA_OK) return s;
+  // Nothing in the scratch needs to start at zero: every score the select
+  // reads and every chunk candidate the merge reads is written earlier in the
+  // same call, so the previous call's contents are never observed.
+  int ev_i = 0;
+  return run_indexer_topk(reinterpret_cast<const bf16*>(q_idx), w_idx, reinterpret_cast<const bf16*>(k_idx),
+                          k_seq_stride, N, q_pos, Tq, mode, cfg, topk_idx, scratch, as_stream(stream), nullptr, 0,
+                          ev_i);
 }
 
 static int check_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N,
