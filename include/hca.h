@@ -284,6 +284,11 @@ size_t hca_workspace_size(int op, const hca_layer_cfg* cfg, int Tq, int N, int m
  * hybrid_attn_prefill) on the calling thread launched. */
 int hca_last_launch_count(void);
 
+/* Synchronise the current device and report kernels that gave up a bounded
+ * wait since the last check (HCA_ERR_DEVICE_CHECK; the record is cleared).
+ * The only entry point that synchronises; meant for tests and diagnostics. */
+int hca_check_device(void);
+
 /* Message describing the last error on the calling thread ("" if none). */
 const char* hca_last_error(void);
 

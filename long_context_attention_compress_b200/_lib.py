@@ -88,6 +88,8 @@ _prefill_ws = _sig("hybrid_attn_prefill_workspace", c_size, [ctypes.POINTER(Laye
 _ws_size = _sig("hca_workspace_size", c_size, [c_int, ctypes.POINTER(LayerCfg), c_int, c_int, c_int])
 _last_error = _sig("hca_last_error", ctypes.c_char_p, [])
 _version = _sig("hca_version", ctypes.c_char_p, [])
+_check_device = _sig("hca_check_device", c_int, [])
+_last_launches = _sig("hca_last_launch_count", c_int, [])
 
 SIZE_MAX = (1 << (8 * ctypes.sizeof(c_size))) - 1
 

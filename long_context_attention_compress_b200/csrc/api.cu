@@ -14,6 +14,18 @@
 
 namespace hca {
 thread_local int g_launch_counter = 0;
+
+int device_sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
 }
 
 using namespace hca;
@@ -119,9 +131,15 @@ int run_indexer_topk(const bf16* q_idx, const float* w_idx, const bf16* k_idx, l
                      void* ws, cudaStream_t st, void* const* ev, int n_ev, int& ev_i) {
   const IndexerPlan p = plan_indexer(Tq, N, cfg->topk);
   float* scores = reinterpret_cast<float*>(ws);
-  CUDA_TRY(launch_indexer_scores(q_idx, w_idx, k_idx, k_seq_stride, N, q_pos, Tq, mode, cfg->m, cfg->n_idx_heads,
-                                 cfg->d_idx, scores, p.ld, st),
-           "indexer scores");
+  if (mode == HCA_MODE_DECODE && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx)) {
+    CUDA_TRY(launch_indexer_decode_tc(q_idx, w_idx, k_idx, k_seq_stride, N, q_pos, Tq, cfg->m, scores, p.ld,
+                                      device_sm_count(), st),
+             "indexer scores (tcgen05)");
+  } else {
+    CUDA_TRY(launch_indexer_scores(q_idx, w_idx, k_idx, k_seq_stride, N, q_pos, Tq, mode, cfg->m,
+                                   cfg->n_idx_heads, cfg->d_idx, scores, p.ld, st),
+             "indexer scores");
+  }
   if (ev && ev_i < n_ev) CUDA_TRY(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
   SelectRows rows;
   rows.chunks = p.chunks;
@@ -183,6 +201,16 @@ const char* hca_last_error(void) { return g_err.c_str(); }
 int hca_last_launch_count(void) { return g_last_launches; }
 
 const char* hca_version(void) { return "hca-b200 0.1 (sm_100a)"; }
+
+int hca_check_device(void) {
+  g_err.clear();
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_status(e, "hca_check_device");
+  const unsigned int w = read_and_clear_indexer_tc_error();
+  if (w == 0xffffffffu) return fail(HCA_ERR_CUDA, "hca_check_device: cannot read the device error word");
+  if (w) return fail(HCA_ERR_DEVICE_CHECK, "hca_check_device: a kernel gave up waiting (error word 0x%x)", w);
+  return HCA_OK;
+}
 
 int csa_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int ld_logits, const float* pos_bias,
                  int ld_bias, int T, int c, int m, hca_bf16* out, int ld_out, void* stream) {

@@ -1,0 +1,269 @@
+// Lightning-indexer scores on the 5th-generation tensor cores (sm_100a).
+//
+//   I(t, s) = sum_j w[t, j] * ReLU(q_I[t, j, :] . K_I[s, :])
+// (QbitAI write-up, "混合注意力機制", CSA step two; "DeepSeek V4 Architecture
+// Tricks", CSA section: 64 indexer heads of dim 128.)
+//
+// Decode shape: one query per request, the request's whole key cache
+// streamed once.  The (request, 128-entry tile) space is split evenly over a
+// persistent grid (one CTA per SM).  Per CTA:
+//   warp 0      TMA producer: key tiles [128 entries x 128 dims] bf16 (two
+//               64-dim 128B-swizzled boxes, 32 KiB) into a ring of stages;
+//               the request's q_I [64 heads x 128] when the request changes.
+//   warp 1      MMA issuer (one thread): S^T[128 entries, 64 heads] =
+//               K_tile . q_I^T with eight M=128 N=64 K=16 tcgen05.mma into one
+//               of four TMEM accumulators (64 f32 columns each).
+//   warps 2..5  epilogue: each thread owns one TMEM lane = one entry, loads
+//               its 64 head dot products, applies ReLU and the head weights
+//               and writes the entry's score (4 bytes per 256-byte key row).
+// The entry is the MMA's M dimension, so the head sum needs no shuffles.
+// Every wait is bounded; a CTA that runs out of budget records an error,
+// lets its own copies and MMAs drain, frees its TMEM and returns.
+
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace hca {
+
+namespace {
+constexpr int kStages = 5;
+constexpr int kTile = 128;   // entries per tile (MMA M)
+constexpr int kHeads = 64;   // indexer heads (MMA N)
+constexpr int kDim = 128;    // key dim (MMA K)
+constexpr int kAcc = 4;      // TMEM accumulators
+constexpr int kTmemCols = kAcc * kHeads;  // 256
+constexpr uint32_t kTileBytes = kTile * kDim * 2;   // 32 KiB
+constexpr uint32_t kChunkBytes = kTile * 128;       // 16 KiB (64 dims)
+constexpr uint32_t kQBytes = kHeads * kDim * 2;     // 16 KiB
+constexpr uint32_t kQChunkBytes = kHeads * 128;     // 8 KiB
+constexpr int kThreads = 192;
+
+struct __align__(8) Bars {
+  uint64_t full[kStages], empty[kStages];
+  uint64_t tfull[kAcc], tempty[kAcc];
+  uint64_t qfull[2], qempty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStages * kTileBytes + 2 * kQBytes + sizeof(Bars);
+}  // namespace
+
+__device__ unsigned int g_indexer_tc_error = 0;
+
+__global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+    const float* __restrict__ w_idx, const int32_t* __restrict__ q_pos, int B, int N, int rate,
+    int tiles_per_req, float* __restrict__ scores, long long ld_scores) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* k_smem = base;                              // [stages][2][128][128 B]
+  unsigned char* q_smem = base + kStages * kTileBytes;        // [2][2][64][128 B]
+  Bars* bars = reinterpret_cast<Bars*>(q_smem + 2 * kQBytes);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long total = (long long)B * tiles_per_req;
+  const long long g0 = total * blockIdx.x / gridDim.x;
+  const long long g1 = total * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { tc::mbar_init(&bars->full[s], 1); tc::mbar_init(&bars->empty[s], 1); }
+    for (int a = 0; a < kAcc; ++a) { tc::mbar_init(&bars->tfull[a], 1); tc::mbar_init(&bars->tempty[a], 4); }
+    for (int b = 0; b < 2; ++b) { tc::mbar_init(&bars->qfull[b], 1); tc::mbar_init(&bars->qempty[b], 1); }
+    tc::mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tm_k);
+      tc::tma_prefetch_desc(&tm_q);
+      int it = 0, rq = 0, cur_r = -1;
+      for (long long g = g0; g < g1; ++g) {
+        const int r = (int)(g / tiles_per_req);
+        const int row0 = (int)(g % tiles_per_req) * kTile;
+        if (row0 >= n_visible(q_pos[r], rate, N)) continue;
+        if (r != cur_r) {
+          const int qb = rq & 1;
+          if (!tc::mbar_wait(&bars->qempty[qb], ((rq >> 1) & 1) ^ 1, abort)) break;
+          tc::mbar_arrive_expect_tx(&bars->qfull[qb], kQBytes);
+          tc::tma_load_2d(q_smem + qb * kQBytes, &tm_q, &bars->qfull[qb], 0, r * kHeads);
+          tc::tma_load_2d(q_smem + qb * kQBytes + kQChunkBytes, &tm_q, &bars->qfull[qb], 64, r * kHeads);
+          cur_r = r;
+          ++rq;
+        }
+        const int s = it % kStages;
+        if (!tc::mbar_wait(&bars->empty[s], ((it / kStages) & 1) ^ 1, abort)) break;
+        tc::mbar_arrive_expect_tx(&bars->full[s], kTileBytes);
+        tc::tma_load_3d(k_smem + s * kTileBytes, &tm_k, &bars->full[s], 0, row0, r);
+        tc::tma_load_3d(k_smem + s * kTileBytes + kChunkBytes, &tm_k, &bars->full[s], 64, row0, r);
+        ++it;
+      }
+      // make sure no copy of ours is still landing in shared memory
+      for (int j = (it > kStages ? it - kStages : 0); j < it; ++j) {
+        for (uint32_t i = 0; i < tc::kSpinLimit && !tc::mbar_try_wait(&bars->full[j % kStages], (j / kStages) & 1); ++i)
+          __nanosleep(64);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16_f32(kTile, kHeads, false, false);
+      const uint32_t k_base = tc::smem_u32(k_smem), q_base = tc::smem_u32(q_smem);
+      int it = 0, rq = 0, cur_r = -1, qb = 0;
+      for (long long g = g0; g < g1; ++g) {
+        const int r = (int)(g / tiles_per_req);
+        const int row0 = (int)(g % tiles_per_req) * kTile;
+        if (row0 >= n_visible(q_pos[r], rate, N)) continue;
+        if (r != cur_r) {
+          if (cur_r >= 0) tc::mma_commit(&bars->qempty[qb]);  // previous q buffer free once its MMAs finish
+          qb = rq & 1;
+          if (!tc::mbar_wait(&bars->qfull[qb], (rq >> 1) & 1, abort)) break;
+          tc::fence_after_sync();
+          cur_r = r;
+          ++rq;
+        }
+        const int s = it % kStages;
+        const int a = it % kAcc;
+        if (!tc::mbar_wait(&bars->full[s], (it / kStages) & 1, abort)) break;
+        if (!tc::mbar_wait(&bars->tempty[a], ((it / kAcc) & 1) ^ 1, abort)) break;
+        tc::fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < kDim / 16; ++k) {
+          const uint32_t koff = (k >> 2) * kChunkBytes + (k & 3) * 32;
+          const uint32_t qoff = (k >> 2) * kQChunkBytes + (k & 3) * 32;
+          const uint64_t ad = tc::sdesc_sw128(k_base + s * kTileBytes + koff, 16, 1024);
+          const uint64_t bd = tc::sdesc_sw128(q_base + qb * kQBytes + qoff, 16, 1024);
+          tc::mma_bf16(tmem + a * kHeads, ad, bd, idesc, k > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&bars->empty[s]);
+        tc::mma_commit(&bars->tfull[a]);
+        ++it;
+      }
+      // wait for every MMA of ours before the TMEM is freed
+      tc::mma_commit(&bars->drain);
+      for (uint32_t i = 0; i < tc::kSpinLimit && !tc::mbar_try_wait(&bars->drain, 0); ++i) __nanosleep(64);
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int lq = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = lq * 32 + lane;
+    float w[kHeads];
+    int it = 0, cur_r = -1;
+    for (long long g = g0; g < g1; ++g) {
+      const int r = (int)(g / tiles_per_req);
+      const int row0 = (int)(g % tiles_per_req) * kTile;
+      const int nvis = n_visible(q_pos[r], rate, N);
+      if (row0 >= nvis) continue;
+      if (r != cur_r) {
+#pragma unroll
+        for (int j = 0; j < kHeads; ++j) w[j] = w_idx[(long long)r * kHeads + j];
+        cur_r = r;
+      }
+      const int a = it % kAcc;
+      if (!tc::mbar_wait(&bars->tfull[a], (it / kAcc) & 1, abort)) break;
+      tc::fence_after_sync();
+      uint32_t v[kHeads];
+      const uint32_t taddr = tmem + ((uint32_t)(lq * 32) << 16) + a * kHeads;
+      tc::tmem_ld32(taddr, v);
+      tc::tmem_ld32(taddr + 32, v + 32);
+      tc::tmem_ld_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->tempty[a]);
+      float sc0 = 0.f, sc1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < kHeads; j += 2) {
+        sc0 = fmaf(w[j], fmaxf(__uint_as_float(v[j]), 0.f), sc0);
+        sc1 = fmaf(w[j + 1], fmaxf(__uint_as_float(v[j + 1]), 0.f), sc1);
+      }
+      const int e = row0 + row_in_tile;
+      if (e < nvis) scores[(long long)r * ld_scores + e] = sc0 + sc1;
+      ++it;
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (threadIdx.x == 0 && bars->abort) atomicOr(&g_indexer_tc_error, 1u);
+  if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---- host side ------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor map, 128B swizzle, box = {64, box_rows, 1}; dims innermost first.
+cudaError_t make_tmap_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+                           const uint64_t* strides_bytes, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t gdim[3], gstride[2];
+  cuuint32_t box[3], estr[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) gdim[i] = dims[i];
+  for (int i = 0; i < rank - 1; ++i) gstride[i] = strides_bytes[i];
+  box[0] = 64;
+  box[1] = box_rows;
+  box[2] = 1;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), gdim, gstride, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+bool indexer_tc_supported(int H_I, int d_I) { return H_I == kHeads && d_I == kDim; }
+
+cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride,
+                                     int N, const int32_t* q_pos, int B, int rate, float* scores, long long ld_scores,
+                                     int num_sms, cudaStream_t stream) {
+  if (B == 0 || N == 0) return cudaSuccess;
+  CUtensorMap tm_k, tm_q;
+  const uint64_t kd[3] = {(uint64_t)kDim, (uint64_t)N, (uint64_t)B};
+  const uint64_t ks[2] = {(uint64_t)kDim * 2, (uint64_t)(B > 1 ? k_seq_stride : (long long)N * kDim) * 2};
+  cudaError_t e = make_tmap_bf16(&tm_k, k_idx, 3, kd, ks, kTile);
+  if (e != cudaSuccess) return e;
+  const uint64_t qd[2] = {(uint64_t)kDim, (uint64_t)B * kHeads};
+  const uint64_t qs[1] = {(uint64_t)kDim * 2};
+  e = make_tmap_bf16(&tm_q, q_idx, 2, qd, qs, kHeads);
+  if (e != cudaSuccess) return e;
+  const int tiles_per_req = (N + kTile - 1) / kTile;
+  const long long total = (long long)B * tiles_per_req;
+  const int grid = (int)(total < num_sms ? total : num_sms);
+  e = cudaFuncSetAttribute((const void*)indexer_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  indexer_decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_k, tm_q, w_idx, q_pos, B, N, rate,
+                                                                   tiles_per_req, scores, ld_scores);
+  ++g_launch_counter;
+  return cudaGetLastError();
+}
+
+unsigned int read_and_clear_indexer_tc_error() {
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_indexer_tc_error, sizeof(v)) != cudaSuccess) return 0xffffffffu;
+  if (v) cudaMemcpyToSymbol(g_indexer_tc_error, &zero, sizeof(zero));
+  return v;
+}
+
+}  // namespace hca

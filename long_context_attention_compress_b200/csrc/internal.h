@@ -51,6 +51,17 @@ cudaError_t launch_indexer_scores(const bf16* q_idx, const float* w_idx, const b
                                   int mode, int rate, int H_I, int d_I, float* scores,
                                   long long ld_scores, cudaStream_t stream);
 
+// ---- indexer_tc.cu (tcgen05) -------------------------------------------------------
+bool indexer_tc_supported(int H_I, int d_I);
+// Decode: query r scores request r's keys (k_idx + r*k_seq_stride), scores[r*ld + s].
+cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride,
+                                     int N, const int32_t* q_pos, int B, int rate, float* scores, long long ld_scores,
+                                     int num_sms, cudaStream_t stream);
+unsigned int read_and_clear_indexer_tc_error();
+
+// SM count of the current device (cached per device).
+int device_sm_count();
+
 // ---- mqa.cu -----------------------------------------------------------------------
 struct MqaProblem {
   const bf16* q;            // [Tq, H, c]

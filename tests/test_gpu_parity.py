@@ -136,6 +136,23 @@ def test_indexer_topk_decode_csa_128k(hca):
     assert swaps <= 32 * 8
 
 
+@pytest.mark.parametrize("B,ctx", [(300, 4 * 2048), (5, 4 * 1000 + 3), (7, 4 * 128 * 3 - 1)])
+def test_indexer_topk_decode_many_requests_ragged(hca, B, ctx):
+    """Many short requests per CTA (the q_I buffer switches mid-range), ragged last tiles,
+    and a position whose newest block is still incomplete."""
+    s = wl.PRO
+    d = wl.csa_decode_inputs(s, B=B, ctx=ctx, seed=B)
+    g = to_dev(d)
+    cfg = hca.make_cfg(s)
+    idx = hca.csa_indexer_topk(g["q_idx"], g["w_idx"], g["K_I"], g["q_pos"], cfg, mode=hca.HCA_MODE_DECODE)
+    idx = idx.cpu().numpy()
+    N = d["K_I"].shape[1]
+    for b in range(B):
+        nv = oracle.n_visible(ctx - 1, s.m, N)
+        sc = oracle.indexer_scores(to64(d["q_idx"][b]), d["w_idx"][b].double().numpy(), to64(d["K_I"][b])[:nv])
+        check_topk_row(idx[b], oracle.topk_select(sc, s.topk), sc, s.topk, nv)
+
+
 # ----------------------------------------------------------------------------
 # attention
 # ----------------------------------------------------------------------------
@@ -332,3 +349,8 @@ def test_decode_short_context_window_partial(hca):
         assert_norm_close(to64(co[b]), r["O"], what="short CSA decode")
         o = oracle.mqa_attend(to64(d["hca"]["q"][b]), to64(d["hca"]["win"][b])[:ctx], s.scale)
         assert_norm_close(to64(ho[b]), o, what="short HCA decode (window only)")
+
+
+def test_no_kernel_gave_up_waiting(hca):
+    """After everything above, no kernel recorded an exhausted bounded wait."""
+    assert hca.lib.hca_check_device() == 0, hca.last_error()
