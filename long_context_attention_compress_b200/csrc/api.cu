@@ -187,7 +187,7 @@ MqaProblem make_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16*
 size_t mqa_ws_bound(const hca_layer_cfg* cfg, int Tq, int N, int n_idx) {
   MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, N > n_idx ? N : n_idx, nullptr, 0, 1, nullptr, 0, nullptr, Tq,
                           HCA_MODE_DECODE, nullptr);
-  return plan_mqa(p).ws_bytes;
+  return mqa_ws_upper_bound(p);
 }
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
@@ -206,8 +206,11 @@ int hca_check_device(void) {
   g_err.clear();
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_status(e, "hca_check_device");
-  const unsigned int w = read_and_clear_indexer_tc_error();
-  if (w == 0xffffffffu) return fail(HCA_ERR_CUDA, "hca_check_device: cannot read the device error word");
+  const unsigned int w1 = read_and_clear_indexer_tc_error();
+  const unsigned int w2 = read_and_clear_mqa_tc_error();
+  if (w1 == 0xffffffffu || w2 == 0xffffffffu)
+    return fail(HCA_ERR_CUDA, "hca_check_device: cannot read the device error word");
+  const unsigned int w = w1 | (w2 << 1);
   if (w) return fail(HCA_ERR_DEVICE_CHECK, "hca_check_device: a kernel gave up waiting (error word 0x%x)", w);
   return HCA_OK;
 }
@@ -406,13 +409,14 @@ static size_t decode_ws(const hca_layer_cfg* cfg, const hca_decode_args* a) {
   size_t need = 0;
   if (a->csa_q) {
     need = std::max(need, plan_indexer(a->B, a->csa_N, cfg->topk).bytes);
-    MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, a->csa_N, reinterpret_cast<const int32_t*>(1), cfg->topk,
-                            cfg->m, nullptr, 0, nullptr, a->B, HCA_MODE_DECODE, nullptr);
+    // same problem (strides included) as the call will plan, so the size is exact
+    MqaProblem p = make_mqa(cfg, nullptr, nullptr, a->csa_kv_stride, a->csa_N, reinterpret_cast<const int32_t*>(1),
+                            cfg->topk, cfg->m, nullptr, a->csa_win_stride, nullptr, a->B, HCA_MODE_DECODE, nullptr);
     need = std::max(need, plan_mqa(p).ws_bytes);
   }
   if (a->hca_q) {
-    MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, a->hca_N, nullptr, 0, cfg->m_hca, nullptr, 0, nullptr, a->B,
-                            HCA_MODE_DECODE, nullptr);
+    MqaProblem p = make_mqa(cfg, nullptr, nullptr, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, nullptr,
+                            a->hca_win_stride, nullptr, a->B, HCA_MODE_DECODE, nullptr);
     need = std::max(need, plan_mqa(p).ws_bytes);
   }
   return round256(need);

@@ -87,7 +87,18 @@ struct MqaPlan {
   int max_rows;        // upper bound of the row-list length
   size_t ws_bytes;
 };
+// plan_mqa / launch_mqa pick the tensor-core kernel when it supports the problem.
 MqaPlan plan_mqa(const MqaProblem& p);
+MqaPlan plan_mqa_cuda_cores(const MqaProblem& p);
+size_t mqa_ws_upper_bound(const MqaProblem& p);  // any idx / stride / mode, rows up to max(N, n_idx)
 cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& plan, void* ws, cudaStream_t stream);
+cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out,
+                               cudaStream_t stream);
+
+// ---- mqa_tc.cu (tcgen05) -------------------------------------------------------------
+bool mqa_tc_supported(const MqaProblem& p);
+MqaPlan plan_mqa_tc(const MqaProblem& p, int num_sms);
+cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream);
+unsigned int read_and_clear_mqa_tc_error();
 
 }  // namespace hca

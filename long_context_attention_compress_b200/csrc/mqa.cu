@@ -216,7 +216,32 @@ static size_t mqa_smem() {
   return (size_t)(H + kTR) * (C + 8) * sizeof(bf16) + (size_t)(2 * H * kTR + 3 * H) * sizeof(float);
 }
 
+cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out,
+                               cudaStream_t stream) {
+  mqa_combine_kernel<<<dim3(Tq, H), 128, 0, stream>>>(ws_o, ws_ml, splits, H, C, out);
+  ++g_launch_counter;
+  return cudaGetLastError();
+}
+
+size_t mqa_ws_upper_bound(const MqaProblem& p) {
+  MqaProblem v0 = p;
+  v0.mode = HCA_MODE_PREFILL;  // the CUDA-core plan, for any row count up to max(N, n_idx)
+  size_t b = plan_mqa_cuda_cores(v0).ws_bytes;
+  const int sms = device_sm_count();
+  const long long smax = p.Tq > 0 ? std::max(1, (2 * sms) / p.Tq) : 1;
+  const size_t tc_bound = (size_t)p.Tq * smax * p.H * ((size_t)p.c * sizeof(float) + sizeof(float2));
+  MqaProblem d = p;
+  d.mode = HCA_MODE_DECODE;
+  const size_t v0d = plan_mqa_cuda_cores(d).ws_bytes;
+  return std::max(b, std::max(tc_bound, v0d));
+}
+
 MqaPlan plan_mqa(const MqaProblem& p) {
+  if (mqa_tc_supported(p)) return plan_mqa_tc(p, device_sm_count());
+  return plan_mqa_cuda_cores(p);
+}
+
+MqaPlan plan_mqa_cuda_cores(const MqaProblem& p) {
   MqaPlan pl;
   const int first = p.idx ? p.n_idx : p.N;
   pl.max_rows = first + p.n_win;
@@ -262,6 +287,7 @@ static cudaError_t launch_mqa_t(const MqaProblem& p, const MqaPlan& pl, void* ws
 
 cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream) {
   if (p.Tq == 0) return cudaSuccess;
+  if (mqa_tc_supported(p)) return launch_mqa_decode_tc(p, pl, ws, stream);
   if (p.H == 64 && p.c == 512) return launch_mqa_t<64, 512>(p, pl, ws, stream);
   if (p.H == 4 && p.c == 64) return launch_mqa_t<4, 64>(p, pl, ws, stream);
   return cudaErrorInvalidValue;
