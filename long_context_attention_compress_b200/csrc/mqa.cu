@@ -189,25 +189,77 @@ __global__ void __launch_bounds__(kMqaThreads) mqa_split_kernel(MqaProblem p, in
   }
 }
 
-// combine: grid (Tq, H), block 128 threads over C
-__global__ void __launch_bounds__(128) mqa_combine_kernel(const float* __restrict__ ws_o,
+// combine: o = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i per (query, head).
+// grid (Tq, ceil(H/4)), 256 threads: one CTA merges 4 heads; the per-split
+// weights are computed once into shared memory, then every thread owns a
+// float4 of one head's output and loads that float4 from all splits with
+// independent loads (the split loop is unrolled by 4).
+constexpr int kCombHeads = 4;
+constexpr int kCombMaxSplits = 1024;  // planners never exceed this
+__global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restrict__ ws_o,
                                                           const float2* __restrict__ ws_ml, int splits,
                                                           int H, int C, bf16* __restrict__ out) {
-  const int q = blockIdx.x, h = blockIdx.y;
-  float M = neg_inf();
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, ws_ml[((long long)q * splits + s) * H + h].x);
-  float den = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float2 ml = ws_ml[((long long)q * splits + s) * H + h];
-    if (ml.y > 0.f) den += fast_exp2(ml.x - M) * ml.y;
-  }
-  for (int d = threadIdx.x; d < C; d += 128) {
-    float num = 0.f;
-    for (int s = 0; s < splits; ++s) {
+  __shared__ float s_w[kCombHeads][kCombMaxSplits];
+  const int q = blockIdx.x, h0 = blockIdx.y * kCombHeads;
+  const int nh = min(kCombHeads, H - h0);
+  // weights: thread hh*64 + lane-group handles head hh
+  for (int hh = threadIdx.x >> 6; hh < nh; hh += 4) {
+    const int h = h0 + hh;
+    const int t = threadIdx.x & 63;
+    float M = neg_inf();
+    for (int s = t; s < splits; s += 64) M = fmaxf(M, ws_ml[((long long)q * splits + s) * H + h].x);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    __shared__ float s_red[4][2];
+    if ((t & 31) == 0) s_red[hh & 3][t >> 5] = M;
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + (hh & 3)) : "memory");
+    M = fmaxf(s_red[hh & 3][0], s_red[hh & 3][1]);
+    float den = 0.f;
+    for (int s = t; s < splits; s += 64) {
       const float2 ml = ws_ml[((long long)q * splits + s) * H + h];
-      if (ml.y > 0.f) num += fast_exp2(ml.x - M) * ws_o[(((long long)q * splits + s) * H + h) * C + d];
+      const float w = ml.y > 0.f ? fast_exp2(ml.x - M) : 0.f;
+      s_w[hh][s] = w;
+      den += w * ml.y;
     }
-    out[((long long)q * H + h) * C + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + (hh & 3)) : "memory");
+    if ((t & 31) == 0) s_red[hh & 3][t >> 5] = den;
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + (hh & 3)) : "memory");
+    den = s_red[hh & 3][0] + s_red[hh & 3][1];
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (int s = t; s < splits; s += 64) s_w[hh][s] *= inv;
+  }
+  __syncthreads();
+  const int per_head = C / 4;  // float4 per head
+  for (int e = threadIdx.x; e < nh * per_head; e += 256) {
+    const int hh = e / per_head, d4 = e % per_head;
+    const int h = h0 + hh;
+    const float4* src = reinterpret_cast<const float4*>(ws_o + ((long long)q * splits * H + h) * C) + d4;
+    const long long sstride = (long long)H * C / 4;  // float4s between splits
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s = 0;
+    for (; s + 4 <= splits; s += 4) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = src[(s + u) * sstride];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float w = s_w[hh][s + u];
+        acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
+        acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
+      }
+    }
+    for (; s < splits; ++s) {
+      const float4 v = src[s * sstride];
+      const float w = s_w[hh][s];
+      acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+    }
+    uint2 pk;
+    pk.x = pack_bf16x2(acc.x, acc.y);
+    pk.y = pack_bf16x2(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(out + ((long long)q * H + h) * C + d4 * 4) = pk;
   }
 }
 
@@ -218,7 +270,7 @@ static size_t mqa_smem() {
 
 cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out,
                                cudaStream_t stream) {
-  mqa_combine_kernel<<<dim3(Tq, H), 128, 0, stream>>>(ws_o, ws_ml, splits, H, C, out);
+  mqa_combine_kernel<<<dim3(Tq, (H + kCombHeads - 1) / kCombHeads), 256, 0, stream>>>(ws_o, ws_ml, splits, H, C, out);
   ++g_launch_counter;
   return cudaGetLastError();
 }
@@ -251,6 +303,7 @@ MqaPlan plan_mqa_cuda_cores(const MqaProblem& p) {
     splits = (target_ctas + p.Tq - 1) / p.Tq;
     const int max_splits = (pl.max_rows + kTR - 1) / kTR;
     if (splits > max_splits) splits = max_splits;
+    if (splits > kCombMaxSplits) splits = kCombMaxSplits;
     if (splits < 1) splits = 1;
   }
   int rps = (pl.max_rows + splits - 1) / splits;
@@ -280,7 +333,8 @@ static cudaError_t launch_mqa_t(const MqaProblem& p, const MqaPlan& pl, void* ws
   ++g_launch_counter;
   e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;
-  mqa_combine_kernel<<<dim3(p.Tq, H), 128, 0, stream>>>(ws_o, ws_ml, pl.splits, H, C, p.out);
+  mqa_combine_kernel<<<dim3(p.Tq, (H + kCombHeads - 1) / kCombHeads), 256, 0, stream>>>(ws_o, ws_ml, pl.splits, H, C,
+                                                                                      p.out);
   ++g_launch_counter;
   return cudaGetLastError();
 }

@@ -489,7 +489,7 @@ MqaPlan plan_mqa_tc(const MqaProblem& p, int num_sms) {
   const int tiles = (first + kRows - 1) / kRows + (p.n_win + kRows - 1) / kRows;
   int best_s = 1;
   long long best_cost = -1;
-  const int smax = p.Tq > 0 ? max(1, (2 * num_sms) / p.Tq) : 1;
+  const int smax = p.Tq > 0 ? min(1024, max(1, (2 * num_sms) / p.Tq)) : 1;  // combine handles <= 1024
   for (int s = 1; s <= smax && s <= tiles; ++s) {
     const int tpc = (tiles + s - 1) / s;
     const int s_eff = (tiles + tpc - 1) / tpc;
