@@ -182,7 +182,9 @@ int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hc
  *   Window rows: HCA_MODE_PREFILL: win[r] for r in [max(0, t-n_win+1), t]
  *   (win = the sequence's raw per-token KV rows, row stride cfg->c);
  *   HCA_MODE_DECODE: the first min(n_win, t+1) rows of request i's block
- *   win + i*win_seq_stride ([n_win, c]; any order).
+ *   win + i*win_seq_stride ([n_win, c]; any order).  In HCA_MODE_PREFILL
+ *   win_seq_stride instead gives the number of rows in win (T >= 1 + every
+ *   q_pos), so that no window tile reads past the sequence.
  *   q [Tq, H, c] bf16; kv: request r's entries at kv + r*kv_seq_stride, [N, c];
  *   idx [Tq, n_idx] int32 (entries < N, visible to the query; -1 = empty slot);
  *   out [Tq, H, c] bf16.  Logits, softmax and sums in f32.

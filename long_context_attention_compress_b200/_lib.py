@@ -206,7 +206,8 @@ def sparse_mqa_attend(q, kv, win, q_pos, cfg: LayerCfg, idx=None, rate=None, mod
     Tq = q.shape[0]
     N = kv.shape[-2]
     kvs = kv.stride(0) if kv.dim() == 3 else 0
-    ws_stride = win.stride(0) if win.dim() == 3 else 0
+    # decode: elements between request windows; prefill: the raw rows' count
+    ws_stride = win.stride(0) if win.dim() == 3 else win.shape[0]
     if rate is None:
         rate = cfg.m if idx is not None else cfg.m_hca
     n_idx = idx.shape[1] if idx is not None else 0

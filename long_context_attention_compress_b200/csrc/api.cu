@@ -2,6 +2,7 @@
 // The operations are documented in include/hca.h.
 
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -128,13 +129,17 @@ int indexer_ok(int N, int k) {
 
 int run_indexer_topk(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride, int N,
                      const int32_t* q_pos, int Tq, int mode, const hca_layer_cfg* cfg, int32_t* topk_idx,
-                     void* ws, cudaStream_t st, void* const* ev, int n_ev, int& ev_i) {
+                     void* ws, cudaStream_t st, void* const* ev, int n_ev, int& ev_i, int grid_sms = 0) {
   const IndexerPlan p = plan_indexer(Tq, N, cfg->topk);
   float* scores = reinterpret_cast<float*>(ws);
   if (mode == HCA_MODE_DECODE && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx)) {
     CUDA_TRY(launch_indexer_decode_tc(q_idx, w_idx, k_idx, k_seq_stride, N, q_pos, Tq, cfg->m, scores, p.ld,
-                                      device_sm_count(), st),
+                                      grid_sms > 0 ? grid_sms : device_sm_count(), st),
              "indexer scores (tcgen05)");
+  } else if (mode == HCA_MODE_PREFILL && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx)) {
+    CUDA_TRY(launch_indexer_prefill_tc(q_idx, w_idx, k_idx, N, q_pos, Tq, cfg->m, scores, p.ld,
+                                       grid_sms > 0 ? grid_sms : device_sm_count(), st),
+             "indexer scores (tcgen05, prefill)");
   } else {
     CUDA_TRY(launch_indexer_scores(q_idx, w_idx, k_idx, k_seq_stride, N, q_pos, Tq, mode, cfg->m,
                                    cfg->n_idx_heads, cfg->d_idx, scores, p.ld, st),
@@ -172,7 +177,9 @@ MqaProblem make_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16*
   p.n_idx = n_idx;
   p.rate = rate;
   p.win = reinterpret_cast<const bf16*>(win);
-  p.win_seq_stride = win_seq_stride;
+  // the same argument carries the window's row count in prefill mode
+  p.win_seq_stride = mode == HCA_MODE_DECODE ? win_seq_stride : 0;
+  p.win_rows = mode == HCA_MODE_PREFILL ? win_seq_stride : 0;
   p.q_pos = q_pos;
   p.Tq = Tq;
   p.mode = mode;
@@ -373,7 +380,11 @@ static int check_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16
   CHECK(Tq >= 0 && N >= 0 && rate >= 1, HCA_ERR_INVALID_ARG, "%s: Tq=%d N=%d rate=%d", who, Tq, N, rate);
   CHECK(mode == HCA_MODE_PREFILL || mode == HCA_MODE_DECODE, HCA_ERR_INVALID_ARG, "%s: mode=%d", who, mode);
   CHECK(!idx || (n_idx > 0 && n_idx <= 4096), HCA_ERR_INVALID_ARG, "%s: n_idx=%d", who, n_idx);
-  CHECK(kv_seq_stride % 8 == 0 && win_seq_stride % 8 == 0, HCA_ERR_INVALID_ARG, "%s: strides", who);
+  CHECK(kv_seq_stride % 8 == 0 && (mode == HCA_MODE_PREFILL || win_seq_stride % 8 == 0), HCA_ERR_INVALID_ARG,
+        "%s: strides", who);
+  // prefill: the same argument is the window's row count (at least one row per query position)
+  CHECK(mode == HCA_MODE_DECODE || win_seq_stride >= 1, HCA_ERR_INVALID_ARG, "%s: window row count %lld", who,
+        win_seq_stride);
   if (Tq == 0) return HCA_OK;
   CHECK_PTR(q, who);
   CHECK_PTR(win, who);
@@ -405,21 +416,99 @@ int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_st
 }
 
 // ---- decode ------------------------------------------------------------------
-static size_t decode_ws(const hca_layer_cfg* cfg, const hca_decode_args* a) {
-  size_t need = 0;
-  if (a->csa_q) {
-    need = std::max(need, plan_indexer(a->B, a->csa_N, cfg->topk).bytes);
-    // same problem (strides included) as the call will plan, so the size is exact
-    MqaProblem p = make_mqa(cfg, nullptr, nullptr, a->csa_kv_stride, a->csa_N, reinterpret_cast<const int32_t*>(1),
-                            cfg->topk, cfg->m, nullptr, a->csa_win_stride, nullptr, a->B, HCA_MODE_DECODE, nullptr);
-    need = std::max(need, plan_mqa(p).ws_bytes);
+// When both layers are present, the HCA layer (its block compression and dense
+// attention) runs on a side stream, concurrently with the CSA indexer, on a
+// share of the SMs proportional to its bytes; the indexer's persistent grid
+// leaves those SMs free.  The two then join before the call returns.  The HCA
+// attention partials get their own workspace region.
+struct DecodeSched {
+  bool overlap = false;
+  int sms = 0, r_hca = 0;
+  MqaPlan csa_pl{}, hca_pl{};
+  size_t main_bytes = 0, hca_off = 0, total = 0;
+};
+
+static MqaProblem decode_csa_problem(const hca_layer_cfg* cfg, const hca_decode_args* a) {
+  return make_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_N,
+                  a->csa_topk_idx ? a->csa_topk_idx : reinterpret_cast<const int32_t*>(1), cfg->topk, cfg->m,
+                  a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out);
+}
+static MqaProblem decode_hca_problem(const hca_layer_cfg* cfg, const hca_decode_args* a) {
+  return make_mqa(cfg, a->hca_q, a->hca_kv, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, a->hca_win,
+                  a->hca_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->hca_out);
+}
+
+static DecodeSched decode_schedule(const hca_layer_cfg* cfg, const hca_decode_args* a) {
+  DecodeSched d;
+  d.sms = device_sm_count();
+  const bool csa = a->csa_q != nullptr, hcl = a->hca_q != nullptr;
+  MqaProblem pc, ph;
+  if (csa) pc = decode_csa_problem(cfg, a);
+  if (hcl) ph = decode_hca_problem(cfg, a);
+  d.overlap = csa && hcl && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx) && mqa_tc_supported(ph) && d.sms >= 16;
+  if (d.overlap) {
+    // Balance the two sides' SM-time: the attention costs about kAttnTileUs per
+    // 64-row tile on one SM, the indexer streams about kIdxBytesPerSmUs bytes
+    // per microsecond per SM (measured on B200).  The HCA share is a whole
+    // number of splits per request so that it runs as a single wave.
+    constexpr double kAttnTileUs = 4.5, kIdxBytesPerSmUs = 35e3;
+    const double hca_tiles = (double)a->B * std::ceil(((double)a->hca_N + cfg->n_win) / 64.0);
+    const double hca_us = hca_tiles * kAttnTileUs;
+    const double idx_us = (double)a->B * a->csa_N * cfg->d_idx * 2.0 / kIdxBytesPerSmUs;
+    int r = (int)(d.sms * hca_us / (hca_us + idx_us) + 0.5);
+    r = std::min(r, d.sms / 2);
+    r = std::max(1, r / a->B) * a->B;
+    if (r > d.sms / 2) {
+      d.overlap = false;  // too many requests to share the machine this way
+    } else {
+      d.r_hca = r;
+      d.hca_pl = plan_mqa_sms(ph, r);
+    }
   }
-  if (a->hca_q) {
-    MqaProblem p = make_mqa(cfg, nullptr, nullptr, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, nullptr,
-                            a->hca_win_stride, nullptr, a->B, HCA_MODE_DECODE, nullptr);
-    need = std::max(need, plan_mqa(p).ws_bytes);
+  if (!d.overlap && hcl) {
+    d.hca_pl = plan_mqa(ph);
   }
-  return round256(need);
+  if (csa) {
+    d.csa_pl = plan_mqa(pc);
+    d.main_bytes = std::max(plan_indexer(a->B, a->csa_N, cfg->topk).bytes, d.csa_pl.ws_bytes);
+  }
+  if (d.overlap) {
+    d.hca_off = round256(d.main_bytes);
+    d.total = round256(d.hca_off + d.hca_pl.ws_bytes);
+  } else {
+    d.hca_off = 0;
+    d.total = round256(std::max(d.main_bytes, hcl ? d.hca_pl.ws_bytes : (size_t)0));
+  }
+  return d;
+}
+
+static size_t decode_ws(const hca_layer_cfg* cfg, const hca_decode_args* a) { return decode_schedule(cfg, a).total; }
+
+// Side stream and fork/join events of the calling host thread on the current
+// device (created on first use, kept for the thread's lifetime).
+struct SideStream {
+  int dev = -1;
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+static int side_stream(SideStream** out) {
+  static thread_local SideStream cache[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e, "side stream: cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(HCA_ERR_UNSUPPORTED, "side stream: device %d", dev);
+  SideStream& ss = cache[dev];
+  if (!ss.s) {
+    if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_status(e, "side stream: create");
+    if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_status(e, "side stream: event");
+    if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess)
+      return cuda_status(e, "side stream: event");
+    ss.dev = dev;
+  }
+  *out = &ss;
+  return HCA_OK;
 }
 
 size_t hybrid_attn_decode_workspace(const hca_layer_cfg* cfg, const hca_decode_args* a) {
@@ -478,34 +567,64 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
     if (ev && ev_i < n_ev) return cuda_status(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
     return HCA_OK;
   };
+  const DecodeSched sched = decode_schedule(cfg, a);
+  SideStream* side = nullptr;
+  if (sched.overlap) {
+    if ((s = side_stream(&side)) != HCA_OK) return s;
+  }
+  cudaStream_t hst = sched.overlap ? side->s : st;  // stream of the HCA layer
+  void* hws = reinterpret_cast<char*>(ws) + sched.hca_off;
   if ((s = mark()) != HCA_OK) return s;
-  if (a->hca_q && a->hca_block_cand) {
-    // newest complete HCA block of every request -> its cache row.  All
-    // requests share one position here (q_pos is on the device), so the row
-    // is hca_N - 1: the caller passes caches sized to the complete blocks.
-    CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), cfg->c,
-                             reinterpret_cast<const bf16*>(a->hca_block_logits), cfg->c, a->hca_pos_bias, cfg->c, a->B,
-                             a->hca_block_stride, cfg->m_hca, cfg->c, cfg->m_hca, false,
-                             reinterpret_cast<bf16*>(a->hca_kv) + (long long)(a->hca_N - 1) * cfg->c, cfg->c,
-                             a->hca_kv_stride, st),
-             "decode: hca compress");
+  if (sched.overlap) {
+    CUDA_TRY(cudaEventRecord(side->fork, st), "decode: fork");
+    CUDA_TRY(cudaStreamWaitEvent(side->s, side->fork, 0), "decode: fork wait");
+  }
+  auto run_hca = [&]() -> int {
+    if (a->hca_block_cand) {
+      // newest complete HCA block of every request -> its cache row.  All
+      // requests share one position here (q_pos is on the device), so the row
+      // is hca_N - 1: the caller passes caches sized to the complete blocks.
+      CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), cfg->c,
+                               reinterpret_cast<const bf16*>(a->hca_block_logits), cfg->c, a->hca_pos_bias, cfg->c,
+                               a->B, a->hca_block_stride, cfg->m_hca, cfg->c, cfg->m_hca, false,
+                               reinterpret_cast<bf16*>(a->hca_kv) + (long long)(a->hca_N - 1) * cfg->c, cfg->c,
+                               a->hca_kv_stride, hst),
+               "decode: hca compress");
+    }
+    MqaProblem p = decode_hca_problem(cfg, a);
+    CUDA_TRY(launch_mqa(p, sched.hca_pl, hws, hst), "decode: hca attention");
+    return HCA_OK;
+  };
+  if (a->hca_q && sched.overlap) {
+    // launched first so that its CTAs take their SMs before the indexer's persistent grid
+    if ((s = run_hca()) != HCA_OK) return s;
+    CUDA_TRY(cudaEventRecord(side->join, side->s), "decode: join");
+  } else if (a->hca_q && a->hca_block_cand) {
+    // sequential: the block compression first (marked as its own phase)
+    if ((s = run_hca()) != HCA_OK) return s;
     if ((s = mark()) != HCA_OK) return s;
   }
   if (a->csa_q) {
     s = run_indexer_topk(reinterpret_cast<const bf16*>(a->csa_q_idx), a->csa_w_idx,
                          reinterpret_cast<const bf16*>(a->csa_k_idx), a->csa_k_stride, a->csa_N, a->q_pos, a->B,
-                         HCA_MODE_DECODE, cfg, a->csa_topk_idx, ws, st, ev, n_ev, ev_i);
+                         HCA_MODE_DECODE, cfg, a->csa_topk_idx, ws, st, ev, n_ev, ev_i,
+                         sched.overlap ? sched.sms - sched.r_hca : 0);
     if (s != HCA_OK) return s;
-    MqaProblem p = make_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_N, a->csa_topk_idx, cfg->topk, cfg->m,
-                            a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out);
-    CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "decode: csa attention");
+    MqaProblem p = decode_csa_problem(cfg, a);
+    CUDA_TRY(launch_mqa(p, sched.csa_pl, ws, st), "decode: csa attention");
     if ((s = mark()) != HCA_OK) return s;
   }
   if (a->hca_q) {
-    MqaProblem p = make_mqa(cfg, a->hca_q, a->hca_kv, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, a->hca_win,
-                            a->hca_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->hca_out);
-    CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "decode: hca attention");
-    if ((s = mark()) != HCA_OK) return s;
+    if (sched.overlap) {
+      CUDA_TRY(cudaStreamWaitEvent(st, side->join, 0), "decode: join wait");
+    } else if (!a->hca_block_cand) {
+      if ((s = run_hca()) != HCA_OK) return s;
+    } else {
+      // already run above, before the CSA layer
+    }
+    if (!(a->hca_block_cand && !sched.overlap)) {
+      if ((s = mark()) != HCA_OK) return s;
+    }
   }
   g_last_launches = g_launch_counter;
   return HCA_OK;
@@ -517,10 +636,10 @@ static size_t prefill_ws(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
   const int Nc = T / cfg->m;
   size_t need = plan_indexer(T, Nc, cfg->topk).bytes;
   MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, Nc, reinterpret_cast<const int32_t*>(1), cfg->topk, cfg->m,
-                          nullptr, 0, nullptr, T, HCA_MODE_PREFILL, nullptr);
+                          nullptr, T, nullptr, T, HCA_MODE_PREFILL, nullptr);
   need = std::max(need, plan_mqa(p).ws_bytes);
   if (a->hca_kv) {
-    MqaProblem ph = make_mqa(cfg, nullptr, nullptr, 0, T / cfg->m_hca, nullptr, 0, cfg->m_hca, nullptr, 0, nullptr, T,
+    MqaProblem ph = make_mqa(cfg, nullptr, nullptr, 0, T / cfg->m_hca, nullptr, 0, cfg->m_hca, nullptr, T, nullptr, T,
                              HCA_MODE_PREFILL, nullptr);
     need = std::max(need, plan_mqa(ph).ws_bytes);
   }
@@ -595,7 +714,7 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
                        0, Nc, a->q_pos, T, HCA_MODE_PREFILL, cfg, a->topk_idx, ws, st, ev, n_ev, ev_i);
   if (s != HCA_OK) return s;
   {
-    MqaProblem p = make_mqa(cfg, a->q, a->csa_kv, 0, Nc, a->topk_idx, cfg->topk, cfg->m, a->cand, 0, a->q_pos, T,
+    MqaProblem p = make_mqa(cfg, a->q, a->csa_kv, 0, Nc, a->topk_idx, cfg->topk, cfg->m, a->cand, T, a->q_pos, T,
                             HCA_MODE_PREFILL, a->csa_out);
     CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "prefill: csa attention");
     if ((s = mark()) != HCA_OK) return s;
@@ -606,7 +725,7 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
                              a->bias_hca, c, 1, 0, T, c, cfg->m_hca, false, reinterpret_cast<bf16*>(a->hca_kv), c, 0,
                              st),
              "prefill: hca compress");
-    MqaProblem p = make_mqa(cfg, a->hca_q, a->hca_kv, 0, Nh, nullptr, 0, cfg->m_hca, a->cand, 0, a->q_pos, T,
+    MqaProblem p = make_mqa(cfg, a->hca_q, a->hca_kv, 0, Nh, nullptr, 0, cfg->m_hca, a->cand, T, a->q_pos, T,
                             HCA_MODE_PREFILL, a->hca_out);
     CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "prefill: hca attention");
     if ((s = mark()) != HCA_OK) return s;

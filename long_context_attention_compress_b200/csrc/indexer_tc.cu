@@ -201,6 +201,198 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
   if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
+// ---- prefill: groups of 4 queries (N = 4 x 64 heads = 256) ---------------------
+// One sequence: query t sees entries s < n_visible(q_pos[t]).  A CTA owns
+// groups of four consecutive queries (their q_I rows form the 256-row B
+// operand, 64 KiB) and streams the key tiles visible to the group's last
+// query through a 4-stage ring; two 256-column TMEM accumulators let the
+// epilogue of one tile overlap the MMAs of the next.  Groups are dealt to the
+// persistent grid largest first, interleaved, which balances the causal
+// triangle.  Epilogue: per query, ReLU of 64 head dot products weighted by the
+// f32 head weights (staged in shared memory per group).
+namespace {
+constexpr int kPStages = 4;
+constexpr int kPQ = 4;                       // queries per group
+constexpr int kPN = kPQ * kHeads;            // 256 = MMA N
+constexpr uint32_t kPQBytes = kPN * kDim * 2;        // 64 KiB
+constexpr uint32_t kPQChunkBytes = kPN * 128;        // 32 KiB
+constexpr int kPAcc = 2;
+constexpr int kPThreads = 192;
+struct __align__(8) PBars {
+  uint64_t full[kPStages], empty[kPStages];
+  uint64_t tfull[kPAcc], tempty[kPAcc];
+  uint64_t qfull, qempty, drain;
+  uint32_t tmem_base;
+  int abort;
+  float w[kPN];
+  int nvis[kPQ];
+};
+constexpr size_t kPSmemBytes = 1024 + kPStages * kTileBytes + kPQBytes + sizeof(PBars);
+}  // namespace
+
+__global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+    const float* __restrict__ w_idx, const int32_t* __restrict__ q_pos, int Tq, int N, int rate,
+    float* __restrict__ scores, long long ld_scores) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* k_smem = base;                           // [stages][2][128][128 B]
+  unsigned char* q_smem = base + kPStages * kTileBytes;   // [2][256][128 B]
+  PBars* bars = reinterpret_cast<PBars*>(q_smem + kPQBytes);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_groups = (Tq + kPQ - 1) / kPQ;
+  // tiles of group g: entries visible to its queries (q_pos is non-decreasing within a group
+  // in the layer call; the maximum over the group is used in general)
+  auto group_tiles = [&](int g) -> int {
+    int nv = 0;
+    for (int j = 0; j < kPQ; ++j) {
+      const int q = g * kPQ + j;
+      if (q < Tq) nv = max(nv, n_visible(q_pos[q], rate, N));
+    }
+    return (nv + kTile - 1) / kTile;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) { tc::mbar_init(&bars->full[s], 1); tc::mbar_init(&bars->empty[s], 1); }
+    for (int a = 0; a < kPAcc; ++a) { tc::mbar_init(&bars->tfull[a], 1); tc::mbar_init(&bars->tempty[a], 4); }
+    tc::mbar_init(&bars->qfull, 1);
+    tc::mbar_init(&bars->qempty, 1);
+    tc::mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kPAcc * kPN);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tm_k);
+      tc::tma_prefetch_desc(&tm_q);
+      int it = 0, gi = 0;  // gi counts the groups actually processed (one q-buffer phase each)
+      bool ok = true;
+      for (int g = n_groups - 1 - (int)blockIdx.x; ok && g >= 0; g -= (int)gridDim.x) {
+        const int nt = group_tiles(g);
+        if (nt == 0) continue;
+        if (!tc::mbar_wait(&bars->qempty, (gi++ & 1) ^ 1, abort)) break;
+        tc::mbar_arrive_expect_tx(&bars->qfull, kPQBytes);
+        tc::tma_load_2d(q_smem, &tm_q, &bars->qfull, 0, g * kPN);
+        tc::tma_load_2d(q_smem + kPQChunkBytes, &tm_q, &bars->qfull, 64, g * kPN);
+        for (int t = 0; t < nt; ++t, ++it) {
+          const int s = it % kPStages;
+          if (!tc::mbar_wait(&bars->empty[s], ((it / kPStages) & 1) ^ 1, abort)) { ok = false; break; }
+          tc::mbar_arrive_expect_tx(&bars->full[s], kTileBytes);
+          tc::tma_load_3d(k_smem + s * kTileBytes, &tm_k, &bars->full[s], 0, t * kTile, 0);
+          tc::tma_load_3d(k_smem + s * kTileBytes + kChunkBytes, &tm_k, &bars->full[s], 64, t * kTile, 0);
+        }
+      }
+      for (int j = (it > kPStages ? it - kPStages : 0); j < it; ++j)
+        for (uint32_t i = 0; i < tc::kSpinLimit && !tc::mbar_try_wait(&bars->full[j % kPStages], (j / kPStages) & 1); ++i)
+          __nanosleep(64);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = tc::idesc_bf16_f32(kTile, kPN, false, false);
+      const uint64_t qd0 = tc::sdesc_sw128(tc::smem_u32(q_smem), 16, 1024);
+      const uint32_t k_base = tc::smem_u32(k_smem);
+      int it = 0, gi = 0;
+      bool ok = true;
+      for (int g = n_groups - 1 - (int)blockIdx.x; ok && g >= 0; g -= (int)gridDim.x) {
+        const int nt = group_tiles(g);
+        if (nt == 0) continue;
+        if (!tc::mbar_wait(&bars->qfull, gi++ & 1, abort)) break;
+        tc::fence_after_sync();
+        for (int t = 0; t < nt; ++t, ++it) {
+          const int s = it % kPStages, a = it % kPAcc;
+          if (!tc::mbar_wait(&bars->full[s], (it / kPStages) & 1, abort)) { ok = false; break; }
+          if (!tc::mbar_wait(&bars->tempty[a], ((it / kPAcc) & 1) ^ 1, abort)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint64_t ad0 = tc::sdesc_sw128(k_base + s * kTileBytes, 16, 1024);
+#pragma unroll
+          for (int k = 0; k < kDim / 16; ++k) {
+            const uint32_t aoff = ((k >> 2) * kChunkBytes + (k & 3) * 32) >> 4;
+            const uint32_t boff = ((k >> 2) * kPQChunkBytes + (k & 3) * 32) >> 4;
+            tc::mma_bf16(tmem + a * kPN, ad0 + aoff, qd0 + boff, idesc, k > 0 ? 1u : 0u);
+          }
+          tc::mma_commit(&bars->empty[s]);
+          tc::mma_commit(&bars->tfull[a]);
+        }
+        tc::mma_commit(&bars->qempty);  // q buffer free once this group's MMAs finish
+      }
+      tc::mma_commit(&bars->drain);
+      for (uint32_t i = 0; i < tc::kSpinLimit && !tc::mbar_try_wait(&bars->drain, 0); ++i) __nanosleep(64);
+    }
+    __syncwarp();
+  } else {
+    // epilogue: warps 2..5, one TMEM lane (= entry) per thread
+    const int lq = warp & 3;
+    const int row_in_tile = lq * 32 + lane;
+    const int et = threadIdx.x - 64;  // 0..127
+    int it = 0;
+    bool failed = false;
+    for (int g = n_groups - 1 - (int)blockIdx.x; g >= 0; g -= (int)gridDim.x) {
+      const int nt = group_tiles(g);
+      if (nt == 0) continue;
+      // stage this group's weights and visible counts (the previous group's readers are done)
+      tc::named_bar(1, 128);
+      for (int e = et; e < kPN; e += 128) {
+        const int q = g * kPQ + e / kHeads;
+        bars->w[e] = q < Tq ? w_idx[(long long)q * kHeads + (e % kHeads)] : 0.f;
+      }
+      if (et < kPQ) {
+        const int q = g * kPQ + et;
+        bars->nvis[et] = q < Tq ? n_visible(q_pos[q], rate, N) : 0;
+      }
+      tc::named_bar(1, 128);
+      for (int t = 0; t < nt; ++t, ++it) {
+        const int a = it % kPAcc;
+        if (!failed) failed = !tc::warp_wait(&bars->tfull[a], (it / kPAcc) & 1, abort);
+        if (failed) continue;
+        tc::fence_after_sync();
+        const int e = t * kTile + row_in_tile;
+        float sc[kPQ];
+#pragma unroll
+        for (int j = 0; j < kPQ; ++j) {
+          uint32_t v[kHeads];
+          const uint32_t taddr = tmem + ((uint32_t)(lq * 32) << 16) + a * kPN + j * kHeads;
+          tc::tmem_ld32(taddr, v);
+          tc::tmem_ld32(taddr + 32, v + 32);
+          tc::tmem_ld_wait();
+          const float* w = bars->w + j * kHeads;
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int h = 0; h < kHeads; h += 4) {
+            const float4 wv = *reinterpret_cast<const float4*>(w + h);
+            s0 = fmaf(wv.x, fmaxf(__uint_as_float(v[h]), 0.f), s0);
+            s1 = fmaf(wv.y, fmaxf(__uint_as_float(v[h + 1]), 0.f), s1);
+            s0 = fmaf(wv.z, fmaxf(__uint_as_float(v[h + 2]), 0.f), s0);
+            s1 = fmaf(wv.w, fmaxf(__uint_as_float(v[h + 3]), 0.f), s1);
+          }
+          sc[j] = s0 + s1;
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars->tempty[a]);
+#pragma unroll
+        for (int j = 0; j < kPQ; ++j) {
+          const int q = g * kPQ + j;
+          if (q < Tq && e < bars->nvis[j]) scores[(long long)q * ld_scores + e] = sc[j];
+        }
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (threadIdx.x == 0 && bars->abort) atomicOr(&g_indexer_tc_error, 2u);
+  if (warp == 1) tc::tmem_dealloc(tmem, kPAcc * kPN);
+}
+
 // ---- host side ------------------------------------------------------------------
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -255,6 +447,30 @@ cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, cons
   if (e != cudaSuccess) return e;
   indexer_decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_k, tm_q, w_idx, q_pos, B, N, rate,
                                                                    tiles_per_req, scores, ld_scores);
+  ++g_launch_counter;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_indexer_prefill_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, int N,
+                                      const int32_t* q_pos, int Tq, int rate, float* scores, long long ld_scores,
+                                      int num_sms, cudaStream_t stream) {
+  if (Tq == 0 || N == 0) return cudaSuccess;
+  CUtensorMap tm_k, tm_q;
+  const uint64_t kd[3] = {(uint64_t)kDim, (uint64_t)N, 1};
+  const uint64_t ks[2] = {(uint64_t)kDim * 2, (uint64_t)N * kDim * 2};
+  cudaError_t e = make_tmap_bf16(&tm_k, k_idx, 3, kd, ks, kTile);
+  if (e != cudaSuccess) return e;
+  const uint64_t qd[2] = {(uint64_t)kDim, (uint64_t)Tq * kHeads};
+  const uint64_t qs[1] = {(uint64_t)kDim * 2};
+  e = make_tmap_bf16(&tm_q, q_idx, 2, qd, qs, kPN);
+  if (e != cudaSuccess) return e;
+  const int n_groups = (Tq + kPQ - 1) / kPQ;
+  const int grid = n_groups < num_sms ? n_groups : num_sms;
+  e = cudaFuncSetAttribute((const void*)indexer_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kPSmemBytes);
+  if (e != cudaSuccess) return e;
+  indexer_prefill_tc_kernel<<<grid, kPThreads, kPSmemBytes, stream>>>(tm_k, tm_q, w_idx, q_pos, Tq, N, rate, scores,
+                                                                      ld_scores);
   ++g_launch_counter;
   return cudaGetLastError();
 }

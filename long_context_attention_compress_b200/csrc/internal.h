@@ -57,6 +57,10 @@ bool indexer_tc_supported(int H_I, int d_I);
 cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride,
                                      int N, const int32_t* q_pos, int B, int rate, float* scores, long long ld_scores,
                                      int num_sms, cudaStream_t stream);
+// Prefill: queries of one sequence against its keys [N, d_I]; scores[q*ld + s] for visible s.
+cudaError_t launch_indexer_prefill_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, int N,
+                                      const int32_t* q_pos, int Tq, int rate, float* scores, long long ld_scores,
+                                      int num_sms, cudaStream_t stream);
 unsigned int read_and_clear_indexer_tc_error();
 
 // SM count of the current device (cached per device).
@@ -72,7 +76,8 @@ struct MqaProblem {
   int n_idx;
   int rate;
   const bf16* win;
-  long long win_seq_stride;
+  long long win_seq_stride;  // decode: elements between requests' window blocks
+  long long win_rows;        // prefill: raw token rows in win (>= 1 + every q_pos)
   const int32_t* q_pos;
   int Tq;
   int mode;
@@ -89,6 +94,7 @@ struct MqaPlan {
 };
 // plan_mqa / launch_mqa pick the tensor-core kernel when it supports the problem.
 MqaPlan plan_mqa(const MqaProblem& p);
+MqaPlan plan_mqa_sms(const MqaProblem& p, int sms);  // one wave of at most `sms` CTAs
 MqaPlan plan_mqa_cuda_cores(const MqaProblem& p);
 size_t mqa_ws_upper_bound(const MqaProblem& p);  // any idx / stride / mode, rows up to max(N, n_idx)
 cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& plan, void* ws, cudaStream_t stream);

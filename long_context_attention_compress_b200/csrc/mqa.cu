@@ -288,8 +288,10 @@ size_t mqa_ws_upper_bound(const MqaProblem& p) {
   return std::max(b, std::max(tc_bound, v0d));
 }
 
-MqaPlan plan_mqa(const MqaProblem& p) {
-  if (mqa_tc_supported(p)) return plan_mqa_tc(p, device_sm_count());
+MqaPlan plan_mqa(const MqaProblem& p) { return plan_mqa_sms(p, device_sm_count()); }
+
+MqaPlan plan_mqa_sms(const MqaProblem& p, int sms) {
+  if (mqa_tc_supported(p)) return plan_mqa_tc(p, sms);
   return plan_mqa_cuda_cores(p);
 }
 

@@ -137,6 +137,7 @@ struct MqaTcParams {
   int n_idx;
   const int32_t* q_pos;
   int rate, N, n_win;
+  int prefill;                // one sequence (window = raw token rows) rather than per-request blocks
   long long kv_rows_stride;   // rows between requests in the kv map
   long long win_rows_stride;  // rows between requests in the window map
   float scale_log2;
@@ -201,8 +202,11 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       tc::mbar_arrive_expect_tx(&bars->qfull, kQBytes);
       for (int c = 0; c < kChunks; ++c) tc::tma_load_2d(base + kOffQ + c * kQChunk, &tm_q, &bars->qfull, c * 64, q * kH);
     }
-    const long long kv_row_base = (long long)q * p.kv_rows_stride;
-    const long long win_row_base = (long long)q * p.win_rows_stride;
+    // decode: request q's cache and window block; prefill: one sequence whose
+    // window is the raw token rows [max(0, t - n_win + 1), t]
+    const long long kv_row_base = p.prefill ? 0ll : (long long)q * p.kv_rows_stride;
+    const long long win_row_base = p.prefill ? (long long)max(0, t_pos - p.n_win + 1)
+                                             : (long long)q * p.win_rows_stride;
     int i = 0;
     for (; i < nt; ++i) {
       const Tile t = tiles.get(i);
@@ -254,43 +258,68 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       constexpr uint32_t id_l = tc::idesc_bf16_f32(128, kH, false, true);
       const uint32_t q_base = tc::smem_u32(base + kOffQ), kv_base = tc::smem_u32(base + kOffKv),
                      p_base = tc::smem_u32(base + kOffP), ones = tc::smem_u32(base + kOffOnes);
+      const uint64_t q_desc0 = tc::sdesc_sw128(q_base, 16, 1024);
+      const uint64_t p_hi_desc0 = tc::sdesc_sw128(p_base, kPBytes, 1024);
+      const uint64_t p_lo_desc0 = tc::sdesc_sw128(p_base + kPBytes, kPBytes, 1024);
+      const uint64_t ones_desc = tc::sdesc_noswz(ones, 128, 256);
       bool ok = tc::mbar_wait(&bars->qfull, 0, abort);
       auto issue_qk = [&](int j) -> bool {
         const int s = j & 1;
         if (!tc::mbar_wait(&bars->kvfull[s], (j >> 1) & 1, abort)) return false;
         if (!tc::mbar_wait(&bars->sempty[s], ((j >> 1) & 1) ^ 1, abort)) return false;
         tc::fence_after_sync();
-#pragma unroll 4
+        // Descriptors are built once; each K-step only adds a compile-time
+        // offset (>> 4) to the start-address field, which keeps the single
+        // issuing thread from becoming the bottleneck.
+        const uint64_t a0 = tc::sdesc_sw128(kv_base + s * kStageOff, 16, 1024);
+        const uint32_t d_s = tmem + kColS + s * kH;
+#pragma unroll
         for (int k = 0; k < kC / 16; ++k) {
-          const uint32_t off = (k >> 2) * kKvChunk + (k & 3) * 32;
-          const uint64_t ad = tc::sdesc_sw128(kv_base + s * kStageOff + off, 16, 1024);
-          const uint64_t bd = tc::sdesc_sw128(q_base + (k >> 2) * kQChunk + (k & 3) * 32, 16, 1024);
-          tc::mma_bf16(tmem + kColS + s * kH, ad, bd, id_qk, k > 0 ? 1u : 0u);
+          const uint32_t aoff = ((k >> 2) * kKvChunk + (k & 3) * 32) >> 4;
+          const uint32_t boff = ((k >> 2) * kQChunk + (k & 3) * 32) >> 4;
+          tc::mma_bf16(d_s, a0 + aoff, q_desc0 + boff, id_qk, k > 0 ? 1u : 0u);
         }
         tc::mma_commit(&bars->sfull[s]);
         return true;
       };
       if (ok && nt > 0) ok = issue_qk(0);
+      // Issue whichever is ready first: QK^T of the next tile (its rows have
+      // landed and its S buffer is free) or PV of the oldest tile whose P is
+      // published.  QK(j) runs at most one tile ahead of PV, so every barrier
+      // is waited on at most one phase ahead.
+      int next_qk = 1;
       for (int i = 0; ok && i < nt; ++i) {
-        if (i + 1 < nt && !issue_qk(i + 1)) break;
         const int s = i & 1;
-        // P(i) is published once per tile and is never more than one tile ahead
-        if (!tc::mbar_wait(&bars->pfull[0], i & 1, abort)) break;
+        uint32_t spins = 0;
+        for (;;) {
+          if (next_qk < nt && next_qk <= i + 1 && tc::mbar_try_wait(&bars->kvfull[next_qk & 1], (next_qk >> 1) & 1) &&
+              tc::mbar_try_wait(&bars->sempty[next_qk & 1], ((next_qk >> 1) & 1) ^ 1)) {
+            ok = issue_qk(next_qk);  // both waits inside succeed at once
+            ++next_qk;
+            if (!ok) break;
+            continue;
+          }
+          if (tc::mbar_try_wait(&bars->pfull[0], i & 1)) break;  // P(i) ready
+          if (++spins > tc::kSpinLimit || *abort) { *abort = 1; ok = false; break; }
+          if ((spins & 255u) == 0) __nanosleep(64);
+        }
+        if (!ok) break;
         tc::fence_after_sync();
+        const uint64_t va0 = tc::sdesc_sw128(kv_base + s * kStageOff, kKvChunk, 1024);
+        const uint32_t acc0 = i > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kRows / 16; ++kk) {
-          const uint64_t bhi = tc::sdesc_sw128(p_base + kk * 2048, kPBytes, 1024);
-          const uint64_t blo = tc::sdesc_sw128(p_base + kPBytes + kk * 2048, kPBytes, 1024);
-          const uint32_t first = (i > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t bhi = p_hi_desc0 + ((kk * 2048) >> 4);
+          const uint64_t blo = p_lo_desc0 + ((kk * 2048) >> 4);
+          const uint32_t first = kk > 0 ? 1u : acc0;
 #pragma unroll
           for (int mb = 0; mb < 4; ++mb) {
-            const uint64_t ad = tc::sdesc_sw128(kv_base + (2 * mb) * kKvChunk + s * kStageOff + kk * 2048, kKvChunk, 1024);
+            const uint64_t ad = va0 + (((2 * mb) * kKvChunk + kk * 2048) >> 4);
             tc::mma_bf16(tmem + kColO + mb * kH, ad, bhi, id_pv, first);
             tc::mma_bf16(tmem + kColO + mb * kH, ad, blo, id_pv, 1u);
           }
-          const uint64_t od = tc::sdesc_noswz(ones, 128, 256);
-          tc::mma_bf16(tmem + kColL, od, bhi, id_l, first);
-          tc::mma_bf16(tmem + kColL, od, blo, id_l, 1u);
+          tc::mma_bf16(tmem + kColL, ones_desc, bhi, id_l, first);
+          tc::mma_bf16(tmem + kColL, ones_desc, blo, id_l, 1u);
         }
         tc::mma_commit(&bars->kvempty[s]);
         tc::mma_commit(&bars->odone);
@@ -477,8 +506,9 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
 
 // ---- host side ------------------------------------------------------------------
 bool mqa_tc_supported(const MqaProblem& p) {
-  return p.mode == HCA_MODE_DECODE && p.H == kH && p.c == kC && p.kv_seq_stride % kC == 0 &&
-         p.win_seq_stride % kC == 0 && p.n_win <= 256;
+  if (p.H != kH || p.c != kC || p.n_win > 256) return false;
+  if (p.mode == HCA_MODE_PREFILL) return p.win_rows > 0;
+  return p.mode == HCA_MODE_DECODE && p.kv_seq_stride % kC == 0 && p.win_seq_stride % kC == 0;
 }
 
 // Splits per query: one wave of at most num_sms CTAs, fewest tiles per CTA.
@@ -518,14 +548,16 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   const uint64_t qd[2] = {(uint64_t)kC, (uint64_t)p.Tq * kH};
   cudaError_t e = make_tmap_bf16(&tm_q, p.q, 2, qd, rstride, 64);
   if (e != cudaSuccess) return e;
-  const long long kv_rs = p.kv_seq_stride / kC;
+  const long long kv_rs = p.mode == HCA_MODE_PREFILL ? 0 : p.kv_seq_stride / kC;
   const uint64_t kvd[2] = {(uint64_t)kC, (uint64_t)((long long)(p.Tq - 1) * kv_rs + (p.N > 0 ? p.N : 1))};
   e = make_tmap_bf16(&tm_kv, p.kv, 2, kvd, rstride, 64);
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16(&tm_kvg, p.kv, 2, kvd, rstride, 1);
   if (e != cudaSuccess) return e;
-  const long long win_rs = p.win_seq_stride / kC;
-  const uint64_t wd[2] = {(uint64_t)kC, (uint64_t)((long long)(p.Tq - 1) * win_rs + p.n_win)};
+  const bool prefill = p.mode == HCA_MODE_PREFILL;
+  const long long win_rs = prefill ? 0 : p.win_seq_stride / kC;
+  const uint64_t wd[2] = {(uint64_t)kC,
+                          prefill ? (uint64_t)p.win_rows : (uint64_t)((long long)(p.Tq - 1) * win_rs + p.n_win)};
   e = make_tmap_bf16(&tm_win, p.win, 2, wd, rstride, 64);
   if (e != cudaSuccess) return e;
   MqaTcParams a;
@@ -535,7 +567,8 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   a.rate = p.rate;
   a.N = p.N;
   a.n_win = p.n_win;
-  a.kv_rows_stride = kv_rs;
+  a.kv_rows_stride = prefill ? 0 : kv_rs;
+  a.prefill = prefill ? 1 : 0;
   a.win_rows_stride = win_rs;
   a.scale_log2 = p.scale * kLog2e;
   a.splits = pl.splits;
