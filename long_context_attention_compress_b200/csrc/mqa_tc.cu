@@ -1,6 +1,7 @@
 // Shared-KV multi-query attention on the 5th-generation tensor cores (sm_100a),
-// decode shape: one query (64 heads x 512) per request, split over CTAs along
-// its row list, partial softmax states merged by the combine kernel.
+// for decode (one query of 64 heads x 512 per request, split over CTAs along
+// its row list, partial softmax states merged by the combine kernel) and for
+// prefill (one CTA per query of one sequence).
 //
 // What it computes (QbitAI write-up, "混合注意力機制": CSA step three, KV
 // entries act as both key and value, sliding-window branch; "DeepSeek V4
@@ -10,27 +11,32 @@
 // window rows.
 //
 // Design.  Rows are the MMA's M dimension and heads its N dimension, so one
-// 64-row KV tile staged in shared memory (128B-swizzled, eight 64-dim
-// chunks) serves as the K-major A operand of S^T = R . Q^T and, read
-// MN-major, as the A operand of O^T += V^T . P^T.  Shared memory holds Q
-// (64 KiB) and two 64-row stages interleaved per chunk (128 KiB); the
-// QK^T MMA runs with M = 128 and reads the other stage's rows as its upper
-// 64 rows, whose results are ignored (decode is bandwidth-bound; the MMA
-// has time to spare).  Dense rows arrive as TMA tiles, selected rows as
-// tile::gather4 loads of four 1 KiB rows per 64-dim chunk.
-//   warp 0     producer (all lanes issue loads)
-//   warp 1     MMA issuer; QK^T of tile i+1 overlaps the softmax of tile i
-//   warps 4,5  softmax of the 64 rows (TMEM lanes 0..63): per-head tile
-//              maximum by a warp reduce-scatter, P = 2^(s - m) written to
-//              shared memory as two bf16 terms P_hi + P_lo (MN-major B
-//              operands of PV; two MMAs give P ~16 significant bits)
-//   warps 2..5 lazy rescale of the TMEM accumulators (only when a head's
-//              maximum grows by more than 2^8) and the final epilogue
-// Row sums l_h come from a small MMA of a ones matrix with P^T, so they use
-// exactly the bf16 P that the PV product uses.
-// TMEM: S^T 2 x 64 columns, O^T 4 blocks x 64, l 64.
+// 128-row KV tile in shared memory (128B-swizzled, eight 64-dim chunks of
+// [128 rows x 128 B]) is the K-major A operand of S^T = R . Q^T (M = 128) and,
+// read MN-major, the A operand of O^T += V^T . P^T (M = 128 dims per block,
+// K = rows).  The tile is tracked as four 128-dim column blocks (two chunks
+// each) with their own full/empty barriers: PV runs block by block and
+// releases each block as soon as its MMAs finish, so the next tile's loads of
+// that block, and its QK^T over it, start while PV is still running.
+// Dense rows arrive as 2-D TMA tiles.  Selected rows arrive as tile::gather4
+// loads (four 128-byte row pieces each), issued by two lanes of each of the
+// eight compute warps: the TMA issue rate is per warp, and sixteen issuers in
+// eight warps gather about three times faster than one warp.
+//   warp 0     MMA issuer (and TMEM owner)
+//   warps 1-8  two per TMEM lane quarter (32 rows of S^T), each owning 32 of
+//              the 64 heads: per-head tile maxima by a warp reduce-scatter plus
+//              a 4-way shared-memory step; P = 2^(s - m) written as two bf16
+//              terms P_hi + P_lo (MN-major B operands of PV, so P keeps ~16
+//              significant bits); lazy rescale of the TMEM accumulators (only
+//              when a head's maximum grows by more than 2^8); the loads of the
+//              next tile; the final epilogue.
+// Row sums l_h come from an MMA of a ones matrix (held in TMEM as the A
+// operand) with P^T, so they use exactly the P that PV uses.
+// TMEM: S^T 64 columns, O^T 4 blocks x 64, l 64, ones 32.
 
 #include <cudaTypedefs.h>
+
+#include <cstddef>
 
 #include "common.cuh"
 #include "internal.h"
@@ -39,34 +45,41 @@
 namespace hca {
 
 namespace {
-constexpr int kThreads = 192;
-constexpr int kRows = 64;
+constexpr int kCompute = 8;                          // compute warps
+constexpr int kThreads = 32 * (1 + kCompute);
+constexpr int kRows = 128;                           // rows per tile
 constexpr int kC = 512;
 constexpr int kH = 64;
 constexpr int kChunks = kC / 64;
+constexpr int kBlocks = 4;                           // 128-dim column blocks
+constexpr int kIssueLanes = 2;                       // gather issuers per compute warp
+constexpr int kGroupsPerIssuer = kRows / 4 / (kCompute * kIssueLanes);  // 4-row groups per issuer
 constexpr uint32_t kQBytes = kH * kC * 2;            // 64 KiB
 constexpr uint32_t kQChunk = kH * 128;               // 8 KiB
-constexpr uint32_t kStageOff = kRows * 128;          // 8 KiB (stage within a chunk)
-constexpr uint32_t kKvChunk = 2 * kStageOff;         // 16 KiB (both stages of a chunk)
+constexpr uint32_t kKvChunk = kRows * 128;           // 16 KiB
 constexpr uint32_t kKvBytes = kChunks * kKvChunk;    // 128 KiB
-constexpr uint32_t kTileBytes = kRows * kC * 2;      // 64 KiB per stage
-constexpr uint32_t kPBytes = kRows * kH * 2;         // 8 KiB
-constexpr uint32_t kOnesBytes = 128 * 16 * 2;        // 4 KiB
-constexpr uint32_t kOffQ = 0, kOffKv = kQBytes, kOffP = kOffKv + kKvBytes, kOffOnes = kOffP + 2 * kPBytes,
-                   kOffBars = kOffOnes + kOnesBytes;
-constexpr uint32_t kColS = 0, kColO = 128, kColL = 384, kTmemCols = 512;
+constexpr uint32_t kBlockBytes = 2 * kKvChunk;       // 32 KiB
+constexpr uint32_t kPBytes = kRows * kH * 2;         // 16 KiB per P term
+constexpr uint32_t kOffQ = 0, kOffKv = kQBytes, kOffP = kOffKv + kKvBytes, kOffBars = kOffP + 2 * kPBytes;
+constexpr uint32_t kColS = 0, kColO = 64, kColL = 320, kColOnes = 384, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
+static_assert(kGroupsPerIssuer * kCompute * kIssueLanes * 4 == kRows, "issuers cover the tile");
 
-struct __align__(8) Bars {
-  uint64_t qfull, kvfull[2], kvempty[2], sfull[2], sempty[2], pfull[2], odone, drain;
+struct __align__(16) Bars {
+  // float arrays first: mref is read with 16-byte vector loads
+  float red[4][kH];
+  float mref[kH];
+  float alpha[kH];
+  uint64_t qfull, kvfull[kBlocks], kvempty[kBlocks], sfull, sempty, pfull, odone, drain;
   uint32_t tmem_base;
   int abort;
   int rescale;
-  float red[2][kH];
-  float mref[kH];
-  float alpha[kH];
 };
+static_assert(offsetof(Bars, mref) % 16 == 0 && offsetof(Bars, red) % 16 == 0, "vector-loaded arrays");
+static_assert(offsetof(Bars, qfull) % 8 == 0, "mbarriers are 8-byte aligned");
+static_assert(kOffBars % 1024 == 0, "operand buffers keep 1024-byte alignment");
 constexpr size_t kSmemBytes = 1024 + kOffBars + sizeof(Bars);
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Tile {
   int seg;    // 0: entries, 1: window
@@ -75,7 +88,7 @@ struct Tile {
 };
 
 // Tiles of one split: the split's range of the row list cut at the
-// entries/window boundary, 64 rows per tile.
+// entries/window boundary, 128 rows per tile.
 struct SplitTiles {
   int a0, a1, b0, b1, na, nb;
   __device__ __forceinline__ SplitTiles(int n_first, int n_win, int ub, int ue) {
@@ -106,10 +119,10 @@ struct SplitTiles {
   }
 };
 
-// One reduce-scatter step over lane bit O: of the n values held, keep the
+// One reduce-scatter step over lane bit O: of the NV values held, keep the
 // half selected by the bit and fold in the partner's copy of that half.
 template <int O, int NV>
-__device__ __forceinline__ void rs_max_step(float (&a)[kH], int lane) {
+__device__ __forceinline__ void rs_max_step(float (&a)[32], int lane) {
   const bool hi = (lane & O) != 0;
 #pragma unroll
   for (int j = 0; j < NV / 2; ++j) {
@@ -118,22 +131,21 @@ __device__ __forceinline__ void rs_max_step(float (&a)[kH], int lane) {
     a[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, O));
   }
 }
-// Afterwards lane l holds the warp-wide maxima of heads 2l and 2l+1 (62 shuffles).
-__device__ __forceinline__ void warp_max2(float (&a)[kH], int lane, float (&out)[2]) {
-  rs_max_step<16, 64>(a, lane);
-  rs_max_step<8, 32>(a, lane);
-  rs_max_step<4, 16>(a, lane);
-  rs_max_step<2, 8>(a, lane);
-  rs_max_step<1, 4>(a, lane);
-  out[0] = a[0];
-  out[1] = a[1];
+// Afterwards lane l holds the warp-wide maximum of value l (31 shuffles).
+__device__ __forceinline__ float warp_max32(float (&a)[32], int lane) {
+  rs_max_step<16, 32>(a, lane);
+  rs_max_step<8, 16>(a, lane);
+  rs_max_step<4, 8>(a, lane);
+  rs_max_step<2, 4>(a, lane);
+  rs_max_step<1, 2>(a, lane);
+  return a[0];
 }
 }  // namespace
 
 __device__ unsigned int g_mqa_tc_error = 0;
 
 struct MqaTcParams {
-  const int32_t* idx;      // [Tq, n_idx] or nullptr
+  const int32_t* idx;         // [Tq, n_idx] or nullptr
   int n_idx;
   const int32_t* q_pos;
   int rate, N, n_win;
@@ -171,272 +183,268 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
 
   if (threadIdx.x == 0) {
     tc::mbar_init(&bars->qfull, 1);
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&bars->kvfull[s], 1);
-      tc::mbar_init(&bars->kvempty[s], 1);
-      tc::mbar_init(&bars->sfull[s], 1);
-      tc::mbar_init(&bars->sempty[s], 2);
-      tc::mbar_init(&bars->pfull[s], 2);
+    for (int b = 0; b < kBlocks; ++b) {
+      tc::mbar_init(&bars->kvfull[b], 1);
+      tc::mbar_init(&bars->kvempty[b], 1);
     }
+    tc::mbar_init(&bars->sfull, 1);
+    tc::mbar_init(&bars->sempty, kCompute);
+    tc::mbar_init(&bars->pfull, kCompute);
     tc::mbar_init(&bars->odone, 1);
     tc::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     bars->rescale = 0;
     tc::fence_mbar_init();
   }
-  // ones matrix for the row-sum MMA (4 KiB of bf16 1.0)
-  for (int i = threadIdx.x; i < (int)(kOnesBytes / 16); i += kThreads)
-    reinterpret_cast<uint4*>(base + kOffOnes)[i] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
   for (int h = threadIdx.x; h < kH; h += kThreads) { bars->mref[h] = neg_inf(); bars->alpha[h] = 1.f; }
-  tc::fence_proxy_async_smem();
-  if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
+  if (warp == 0) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
+  if (warp >= 1 && warp <= 4) {
+    // ones matrix (A operand of the row-sum MMA) in TMEM: every lane, 32 columns of bf16 pairs 1.0
+    uint32_t ones[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) ones[j] = 0x3f803f80u;
+    tc::tmem_st32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + kColOnes, ones);
+    tc::tmem_st_wait();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
 
   if (warp == 0) {
-    // ------------------------------ producer ------------------------------
-    if (lane == 0) {
-      tc::tma_prefetch_desc(&tm_kv);
-      tc::mbar_arrive_expect_tx(&bars->qfull, kQBytes);
-      for (int c = 0; c < kChunks; ++c) tc::tma_load_2d(base + kOffQ + c * kQChunk, &tm_q, &bars->qfull, c * 64, q * kH);
-    }
-    // decode: request q's cache and window block; prefill: one sequence whose
-    // window is the raw token rows [max(0, t - n_win + 1), t]
-    const long long kv_row_base = p.prefill ? 0ll : (long long)q * p.kv_rows_stride;
-    const long long win_row_base = p.prefill ? (long long)max(0, t_pos - p.n_win + 1)
-                                             : (long long)q * p.win_rows_stride;
-    int i = 0;
-    for (; i < nt; ++i) {
-      const Tile t = tiles.get(i);
-      const int s = i & 1;
-      bool ok = true;
-      if (lane == 0) {
-        ok = tc::mbar_wait(&bars->kvempty[s], ((i >> 1) & 1) ^ 1, abort);
-        if (ok) tc::mbar_arrive_expect_tx(&bars->kvfull[s], kTileBytes);
-      }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      unsigned char* st = base + kOffKv + s * kStageOff;
-      if (t.seg == 0 && idx_q != nullptr) {
-        // gathered rows: lane g < 16 loads rows 4g..4g+3 (invalid slots read row 0, masked later)
-        if (lane < 16) {
-          int y[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int r = 4 * lane + j;
-            int e = r < t.nrows ? idx_q[t.row0 + r] : 0;
-            if (e < 0 || e >= p.N) e = 0;
-            y[j] = (int)(kv_row_base + e);
-          }
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c)
-            tc::tma_gather4(st + c * kKvChunk + lane * 512, &tm_kvg, &bars->kvfull[s], c * 64, y[0], y[1], y[2], y[3]);
-        }
-      } else if (lane < kChunks) {
-        const int c = lane;
-        if (t.seg == 0)
-          tc::tma_load_2d(st + c * kKvChunk, &tm_kv, &bars->kvfull[s], c * 64, (int)(kv_row_base + t.row0));
-        else
-          tc::tma_load_2d(st + c * kKvChunk, &tm_win, &bars->kvfull[s], c * 64, (int)(win_row_base + t.row0));
-      }
-      __syncwarp();
-    }
-    // drain: every stage we filled has landed before the CTA may exit
-    if (lane == 0) {
-      for (int j = (i > 2 ? i - 2 : 0); j < i; ++j)
-        for (uint32_t k = 0; k < tc::kSpinLimit && !tc::mbar_try_wait(&bars->kvfull[j & 1], (j >> 1) & 1); ++k)
-          __nanosleep(64);
-      for (uint32_t k = 0; k < tc::kSpinLimit && !tc::mbar_try_wait(&bars->qfull, 0); ++k) __nanosleep(64);
-    }
-  } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
-      constexpr uint32_t id_qk = tc::idesc_bf16_f32(128, kH, false, false);
+      tc::mbar_arrive_expect_tx(&bars->qfull, kQBytes);
+      for (int c = 0; c < kChunks; ++c) tc::tma_load_2d(base + kOffQ + c * kQChunk, &tm_q, &bars->qfull, c * 64, q * kH);
+      constexpr uint32_t id_qk = tc::idesc_bf16_f32(kRows, kH, false, false);
       constexpr uint32_t id_pv = tc::idesc_bf16_f32(128, kH, true, true);
       constexpr uint32_t id_l = tc::idesc_bf16_f32(128, kH, false, true);
       const uint32_t q_base = tc::smem_u32(base + kOffQ), kv_base = tc::smem_u32(base + kOffKv),
-                     p_base = tc::smem_u32(base + kOffP), ones = tc::smem_u32(base + kOffOnes);
-      const uint64_t q_desc0 = tc::sdesc_sw128(q_base, 16, 1024);
-      const uint64_t p_hi_desc0 = tc::sdesc_sw128(p_base, kPBytes, 1024);
-      const uint64_t p_lo_desc0 = tc::sdesc_sw128(p_base + kPBytes, kPBytes, 1024);
-      const uint64_t ones_desc = tc::sdesc_noswz(ones, 128, 256);
+                     p_base = tc::smem_u32(base + kOffP);
+      // Descriptors are built once; each K-step only adds a compile-time
+      // offset (>> 4) to the start-address field.
+      uint64_t q_desc0 = tc::sdesc_sw128(q_base, 16, 1024);
+      uint64_t k_desc0 = tc::sdesc_sw128(kv_base, 16, 1024);
+      uint64_t v_desc0 = tc::sdesc_sw128(kv_base, kKvChunk, 1024);
+      uint64_t p_hi0 = tc::sdesc_sw128(p_base, kPBytes, 1024);
+      uint64_t p_lo0 = tc::sdesc_sw128(p_base + kPBytes, kPBytes, 1024);
+      const uint32_t ones = tmem + kColOnes;
       bool ok = tc::mbar_wait(&bars->qfull, 0, abort);
-      auto issue_qk = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!tc::mbar_wait(&bars->kvfull[s], (j >> 1) & 1, abort)) return false;
-        if (!tc::mbar_wait(&bars->sempty[s], ((j >> 1) & 1) ^ 1, abort)) return false;
-        tc::fence_after_sync();
-        // Descriptors are built once; each K-step only adds a compile-time
-        // offset (>> 4) to the start-address field, which keeps the single
-        // issuing thread from becoming the bottleneck.
-        const uint64_t a0 = tc::sdesc_sw128(kv_base + s * kStageOff, 16, 1024);
-        const uint32_t d_s = tmem + kColS + s * kH;
-#pragma unroll
-        for (int k = 0; k < kC / 16; ++k) {
-          const uint32_t aoff = ((k >> 2) * kKvChunk + (k & 3) * 32) >> 4;
-          const uint32_t boff = ((k >> 2) * kQChunk + (k & 3) * 32) >> 4;
-          tc::mma_bf16(d_s, a0 + aoff, q_desc0 + boff, id_qk, k > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(&bars->sfull[s]);
-        return true;
-      };
-      if (ok && nt > 0) ok = issue_qk(0);
-      // Issue whichever is ready first: QK^T of the next tile (its rows have
-      // landed and its S buffer is free) or PV of the oldest tile whose P is
-      // published.  QK(j) runs at most one tile ahead of PV, so every barrier
-      // is waited on at most one phase ahead.
-      int next_qk = 1;
       for (int i = 0; ok && i < nt; ++i) {
-        const int s = i & 1;
-        uint32_t spins = 0;
-        for (;;) {
-          if (next_qk < nt && next_qk <= i + 1 && tc::mbar_try_wait(&bars->kvfull[next_qk & 1], (next_qk >> 1) & 1) &&
-              tc::mbar_try_wait(&bars->sempty[next_qk & 1], ((next_qk >> 1) & 1) ^ 1)) {
-            ok = issue_qk(next_qk);  // both waits inside succeed at once
-            ++next_qk;
-            if (!ok) break;
-            continue;
+        const uint32_t ph = i & 1;
+        // keep the per-step descriptors from being hoisted out of the loop (96 live 64-bit values)
+        asm volatile("" : "+l"(q_desc0), "+l"(k_desc0), "+l"(v_desc0), "+l"(p_hi0), "+l"(p_lo0));
+        if (!tc::mbar_wait(&bars->sempty, ph ^ 1, abort)) { ok = false; break; }
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b) {
+          if (!tc::mbar_wait(&bars->kvfull[b], ph, abort)) { ok = false; break; }
+          tc::fence_after_sync();
+#pragma unroll
+          for (int k = 8 * b; k < 8 * b + 8; ++k) {
+            const uint32_t aoff = ((k >> 2) * kKvChunk + (k & 3) * 32) >> 4;
+            const uint32_t boff = ((k >> 2) * kQChunk + (k & 3) * 32) >> 4;
+            tc::mma_bf16(tmem + kColS, k_desc0 + aoff, q_desc0 + boff, id_qk, k > 0 ? 1u : 0u);
           }
-          if (tc::mbar_try_wait(&bars->pfull[0], i & 1)) break;  // P(i) ready
-          if (++spins > tc::kSpinLimit || *abort) { *abort = 1; ok = false; break; }
-          if ((spins & 255u) == 0) __nanosleep(64);
         }
         if (!ok) break;
+        tc::mma_commit(&bars->sfull);
+        if (!tc::mbar_wait(&bars->pfull, ph, abort)) { ok = false; break; }
         tc::fence_after_sync();
-        const uint64_t va0 = tc::sdesc_sw128(kv_base + s * kStageOff, kKvChunk, 1024);
         const uint32_t acc0 = i > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk) {
-          const uint64_t bhi = p_hi_desc0 + ((kk * 2048) >> 4);
-          const uint64_t blo = p_lo_desc0 + ((kk * 2048) >> 4);
-          const uint32_t first = kk > 0 ? 1u : acc0;
+        for (int b = 0; b < kBlocks; ++b) {
 #pragma unroll
-          for (int mb = 0; mb < 4; ++mb) {
-            const uint64_t ad = va0 + (((2 * mb) * kKvChunk + kk * 2048) >> 4);
-            tc::mma_bf16(tmem + kColO + mb * kH, ad, bhi, id_pv, first);
-            tc::mma_bf16(tmem + kColO + mb * kH, ad, blo, id_pv, 1u);
+          for (int kk = 0; kk < kRows / 16; ++kk) {
+            const uint32_t koff = (kk * 2048) >> 4;
+            const uint32_t first = kk > 0 ? 1u : acc0;
+            const uint64_t ad = v_desc0 + (((2 * b) * kKvChunk) >> 4) + koff;
+            tc::mma_bf16(tmem + kColO + b * kH, ad, p_hi0 + koff, id_pv, first);
+            tc::mma_bf16(tmem + kColO + b * kH, ad, p_lo0 + koff, id_pv, 1u);
+            if (b == 0) {
+              tc::mma_bf16_ta(tmem + kColL, ones, p_hi0 + koff, id_l, first);
+              tc::mma_bf16_ta(tmem + kColL, ones, p_lo0 + koff, id_l, 1u);
+            }
           }
-          tc::mma_bf16(tmem + kColL, ones_desc, bhi, id_l, first);
-          tc::mma_bf16(tmem + kColL, ones_desc, blo, id_l, 1u);
+          tc::mma_commit(&bars->kvempty[b]);  // this block's columns of the tile may be reloaded
         }
-        tc::mma_commit(&bars->kvempty[s]);
         tc::mma_commit(&bars->odone);
       }
       tc::mma_commit(&bars->drain);
       for (uint32_t k = 0; k < tc::kSpinLimit && !tc::mbar_try_wait(&bars->drain, 0); ++k) __nanosleep(64);
+      for (uint32_t k = 0; k < tc::kSpinLimit && !tc::mbar_try_wait(&bars->qfull, 0); ++k) __nanosleep(64);
     }
   } else {
-    // ------------------------------ softmax / correction / epilogue ------------------------------
+    // --------------------- loads, softmax / correction / epilogue ---------------------
+    const int cw = warp - 1;                       // compute warp 0..7
     const int quarter = warp & 3;                  // TMEM lane quarter
-    const bool smx = quarter < 2;                  // warps 4, 5: rows 0..63
-    const int row = quarter * 32 + lane;           // S^T lane (softmax) / O^T lane
-    const int st = (warp - 2) * 32 + lane;         // 0..127 within the compute group
-    const int sm_t = row;                          // 0..63 for the softmax threads
-    // Every named barrier below is reached by all of its participants on every
+    const int hsel = cw >> 2;                      // heads [32 hsel, 32 hsel + 32)
+    const int row = quarter * 32 + lane;           // S^T row (tile row) / O^T lane
+    const int st = cw * 32 + lane;                 // 0..255 within the compute group
+    const uint32_t lanebase = (uint32_t)(quarter * 32) << 16;
+    const bool issuer = lane < kIssueLanes;
+    const int g0 = cw * kIssueLanes + lane;        // first 4-row group of this issuer
+    // decode: request q's cache and window block; prefill: one sequence whose
+    // window is the raw token rows [max(0, t - n_win + 1), t]
+    const long long kv_row_base = p.prefill ? 0ll : (long long)q * p.kv_rows_stride;
+    const int req = p.prefill ? 0 : q;
+    const int win_row0 = p.prefill ? max(0, t_pos - p.n_win + 1) : 0;
+    int loaded = 0;  // tiles whose loads were issued (thread st == 0 drains them)
+
+    // Rows of tile j this issuer gathers (map rows; invalid slots read the request's row 0,
+    // masked by the softmax).
+    auto gather_rows = [&](int j, int (&y)[4 * kGroupsPerIssuer]) {
+      const Tile t = tiles.get(j);
+#pragma unroll
+      for (int gg = 0; gg < kGroupsPerIssuer; ++gg) {
+#pragma unroll
+        for (int r4 = 0; r4 < 4; ++r4) {
+          const int r = 4 * (g0 + gg * kCompute * kIssueLanes) + r4;
+          int e = (t.seg == 0 && idx_q != nullptr && r < t.nrows) ? idx_q[t.row0 + r] : 0;
+          if (e < 0 || e >= p.N) e = 0;
+          y[4 * gg + r4] = (int)(kv_row_base + e);
+        }
+      }
+    };
+    // Issue the loads of tile j, block by block, each once PV of the previous
+    // tile has released it.  Returns false on a failed wait (warp-uniform).
+    auto issue_tile = [&](int j, const int (&y)[4 * kGroupsPerIssuer]) -> bool {
+      const Tile t = tiles.get(j);
+      const bool gathered = t.seg == 0 && idx_q != nullptr;
+      for (int b = 0; b < kBlocks; ++b) {
+        if (!tc::warp_wait(&bars->kvempty[b], (j & 1) ^ 1, abort)) return false;
+        if (st == 0) tc::mbar_arrive_expect_tx(&bars->kvfull[b], kBlockBytes);
+        unsigned char* dst = base + kOffKv + 2 * b * kKvChunk;
+        if (gathered) {
+          if (issuer) {
+#pragma unroll
+            for (int gg = 0; gg < kGroupsPerIssuer; ++gg) {
+              const int g = g0 + gg * kCompute * kIssueLanes;
+#pragma unroll
+              for (int c = 0; c < 2; ++c)
+                tc::tma_gather4(dst + c * kKvChunk + g * 512, &tm_kvg, &bars->kvfull[b], (2 * b + c) * 64,
+                                y[4 * gg], y[4 * gg + 1], y[4 * gg + 2], y[4 * gg + 3]);
+            }
+          }
+        } else if (st == 0) {
+          // 3-D maps (dims, rows, request): rows past the request's own extent read as zeros
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            if (t.seg == 0)
+              tc::tma_load_3d(dst + c * kKvChunk, &tm_kv, &bars->kvfull[b], (2 * b + c) * 64, t.row0, req);
+            else
+              tc::tma_load_3d(dst + c * kKvChunk, &tm_win, &bars->kvfull[b], (2 * b + c) * 64,
+                              (int)(win_row0 + t.row0), req);
+          }
+        }
+        __syncwarp();
+      }
+      return true;
+    };
+
+    // Every named barrier below is reached by all compute threads on every
     // iteration; failures are agreed through bar.red.or before anyone leaves.
     bool failed = false;
+    int y[4 * kGroupsPerIssuer];
+    if (nt > 0) {
+      gather_rows(0, y);
+      failed = !issue_tile(0, y);
+      if (!failed) loaded = 1;
+    }
     for (int i = 0; i < nt; ++i) {
       const Tile t = tiles.get(i);
-      const int s = i & 1;
-      float sv[kH];
-      if (smx) {
-        if (!failed) failed = !tc::warp_wait(&bars->sfull[s], (i >> 1) & 1, abort);
-        if (!failed) {
-          tc::fence_after_sync();
-          uint32_t v[kH];
-          const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + kColS + s * kH;
-          tc::tmem_ld32(ta, v);
-          tc::tmem_ld32(ta + 32, v + 32);
-          tc::tmem_ld_wait();
-          tc::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&bars->sempty[s]);
-          bool valid = row < t.nrows;
-          if (valid && t.seg == 0 && idx_q != nullptr) {
-            const int e = idx_q[t.row0 + row];
-            valid = e >= 0 && e < p.N;
-          }
-#pragma unroll
-          for (int h = 0; h < kH; ++h) sv[h] = valid ? __uint_as_float(v[h]) * p.scale_log2 : neg_inf();
-          float tmp[kH];
-#pragma unroll
-          for (int h = 0; h < kH; ++h) tmp[h] = sv[h];
-          float m2[2];
-          warp_max2(tmp, lane, m2);
-          bars->red[quarter][2 * lane] = m2[0];
-          bars->red[quarter][2 * lane + 1] = m2[1];
-        }
-        tc::named_bar(1, 64);
-        if (!failed) {
-          const int h = sm_t;
-          const float mt = fmaxf(bars->red[0][h], bars->red[1][h]);
-          const float mo = bars->mref[h];
-          if (mt > mo + kRescaleLog2 || (mo == neg_inf() && mt != neg_inf())) {
-            bars->alpha[h] = (mo == neg_inf()) ? 0.f : fast_exp2(mo - mt);
-            bars->mref[h] = mt;
-            bars->rescale = 1;
-          } else {
-            bars->alpha[h] = 1.f;
-          }
-        }
+      const uint32_t ph = i & 1;
+      bool valid = row < t.nrows;
+      if (valid && t.seg == 0 && idx_q != nullptr) {
+        const int e = idx_q[t.row0 + row];
+        valid = e >= 0 && e < p.N;
       }
-      if (tc::named_bar_or(2, 128, failed || *abort)) { failed = true; break; }
-      if (i > 0) {
-        // Wait for PV(i-1) on every tile, in order: the odone barrier completes once per
-        // tile, and a parity wait is only unambiguous while the waiter is at most one
-        // phase behind (PV(i) cannot complete before this group publishes P(i)).
-        if (!tc::warp_wait(&bars->odone, (i - 1) & 1, abort)) failed = true;
-      }
-      if (bars->rescale && i > 0) {
-        // O^T and l hold the sums up to tile i-1: scale column h by alpha[h]
-        if (!failed) {
-          tc::fence_after_sync();
-          const uint32_t lanebase = (uint32_t)(quarter * 32) << 16;
-#pragma unroll 1
-          for (int blk = 0; blk < 5; ++blk) {
-            const uint32_t ta = tmem + lanebase + (blk < 4 ? kColO + blk * kH : kColL);
-            uint32_t v[kH];
-            tc::tmem_ld32(ta, v);
-            tc::tmem_ld32(ta + 32, v + 32);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int h = 0; h < kH; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * bars->alpha[h]);
-            tc::tmem_st32(ta, v);
-            tc::tmem_st32(ta + 32, v + 32);
-          }
-          tc::tmem_st_wait();
-          tc::fence_before_sync();
-        }
-      }
-      if (tc::named_bar_or(2, 128, failed || *abort)) { failed = true; break; }
-      if (smx) {
-        if (sm_t == 0) bars->rescale = 0;
-        // PV(i-1), the last reader of the P buffer, has completed (waited above).
-        // P = P_hi + P_lo, both bf16: the PV and row-sum MMAs run on both halves,
-        // so the probabilities carry ~16 significant bits instead of 8.
-        unsigned char* phi = base + kOffP + row * 128;
-        unsigned char* plo = phi + kPBytes;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t wh[4], wl[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int h = c * 8 + 2 * j;
-            const float m0 = bars->mref[h], m1 = bars->mref[h + 1];
-            const float p0 = (m0 == neg_inf()) ? 0.f : fast_exp2(sv[h] - m0);
-            const float p1 = (m1 == neg_inf()) ? 0.f : fast_exp2(sv[h + 1] - m1);
-            wh[j] = pack_bf16x2(p0, p1);
-            wl[j] = pack_bf16x2(p0 - bf16_lo(wh[j]), p1 - bf16_hi(wh[j]));
-          }
-          const uint32_t sw = (uint32_t)((c ^ (row & 7)) << 4);
-          *reinterpret_cast<uint4*>(phi + sw) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-          *reinterpret_cast<uint4*>(plo + sw) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-        }
-        tc::fence_proxy_async_smem();
+      if (i + 1 < nt) gather_rows(i + 1, y);  // index loads overlap the wait below
+      float sv[32];
+      if (!failed) failed = !tc::warp_wait(&bars->sfull, ph, abort);
+      if (!failed) {
+        tc::fence_after_sync();
+        uint32_t v[32];
+        tc::tmem_ld32(tmem + lanebase + kColS + 32 * hsel, v);
+        tc::tmem_ld_wait();
+        tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars->pfull[0]);
+        if (lane == 0) tc::mbar_arrive(&bars->sempty);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) sv[h] = valid ? __uint_as_float(v[h]) * p.scale_log2 : neg_inf();
+        float tmp[32];
+#pragma unroll
+        for (int h = 0; h < 32; ++h) tmp[h] = sv[h];
+        bars->red[quarter][32 * hsel + lane] = warp_max32(tmp, lane);
+      }
+      if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
+      if (st < kH) {
+        const int h = st;
+        const float mt = fmaxf(fmaxf(bars->red[0][h], bars->red[1][h]), fmaxf(bars->red[2][h], bars->red[3][h]));
+        const float mo = bars->mref[h];
+        if (mt > mo + kRescaleLog2 || (mo == neg_inf() && mt != neg_inf())) {
+          bars->alpha[h] = (mo == neg_inf()) ? 0.f : fast_exp2(mo - mt);
+          bars->mref[h] = mt;
+          bars->rescale = 1;
+        } else {
+          bars->alpha[h] = 1.f;
+        }
+      }
+      if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
+      // Wait for PV(i-1) on every tile, in order: the odone barrier completes once per
+      // tile, and a parity wait is only unambiguous while the waiter is at most one
+      // phase behind (PV(i) cannot complete before this group publishes P(i)).
+      if (i > 0 && !tc::warp_wait(&bars->odone, (i - 1) & 1, abort)) failed = true;
+      if (!failed && bars->rescale && i > 0) {
+        // O^T and l hold the sums up to tile i-1: scale column h by alpha[h]
+        tc::fence_after_sync();
+#pragma unroll 1
+        for (int blk = 0; blk < 5; ++blk) {
+          const uint32_t ta = tmem + lanebase + (blk < 4 ? kColO + blk * kH : kColL) + 32 * hsel;
+          uint32_t v[32];
+          tc::tmem_ld32(ta, v);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int h = 0; h < 32; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * bars->alpha[32 * hsel + h]);
+          tc::tmem_st32(ta, v);
+        }
+        tc::tmem_st_wait();
+        tc::fence_before_sync();
+      }
+      if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
+      if (st == 0) bars->rescale = 0;  // every reader has passed the barrier above
+      // P = P_hi + P_lo, both bf16 (PV(i-1), the last reader of the P buffers, has completed)
+      unsigned char* phi = base + kOffP + row * 128;
+      unsigned char* plo = phi + kPBytes;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * hsel + cc;  // 16-byte unit of the row: heads 8c .. 8c+7
+        const float4 ma = *reinterpret_cast<const float4*>(bars->mref + c * 8);
+        const float4 mb = *reinterpret_cast<const float4*>(bars->mref + c * 8 + 4);
+        const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+        uint32_t wh[4], wl[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int h = cc * 8 + 2 * j;
+          const float m0 = mm[2 * j], m1 = mm[2 * j + 1];
+          const float p0 = (m0 == neg_inf()) ? 0.f : fast_exp2(sv[h] - m0);
+          const float p1 = (m1 == neg_inf()) ? 0.f : fast_exp2(sv[h + 1] - m1);
+          wh[j] = pack_bf16x2(p0, p1);
+          wl[j] = pack_bf16x2(p0 - bf16_lo(wh[j]), p1 - bf16_hi(wh[j]));
+        }
+        const uint32_t sw = (uint32_t)((c ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(phi + sw) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        *reinterpret_cast<uint4*>(plo + sw) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+      }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bars->pfull);
+      // next tile's rows, block by block as PV(i) releases them
+      if (!failed && i + 1 < nt) {
+        if (issue_tile(i + 1, y)) loaded = i + 2;
+        else failed = true;
       }
     }
     // ---- epilogue: O^T (dims x heads) and l ----
@@ -444,56 +452,60 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     if (ok && nt > 0) ok = tc::warp_wait(&bars->odone, (nt - 1) & 1, abort);
     if (ok) {
       tc::fence_after_sync();
-      const uint32_t lanebase = (uint32_t)(quarter * 32) << 16;
-      uint32_t lv[kH];
+      uint32_t lv[32];
       if (nt > 0) {
-        tc::tmem_ld32(tmem + lanebase + kColL, lv);
-        tc::tmem_ld32(tmem + lanebase + kColL + 32, lv + 32);
+        tc::tmem_ld32(tmem + lanebase + kColL + 32 * hsel, lv);
         tc::tmem_ld_wait();
       } else {
 #pragma unroll
-        for (int h = 0; h < kH; ++h) lv[h] = 0u;
+        for (int h = 0; h < 32; ++h) lv[h] = 0u;
       }
       const int dim_lane = quarter * 32 + lane;
       if (p.splits == 1) {
-        bf16* op = p.out + (long long)q * kH * kC;
+        bf16* op = p.out + (long long)q * kH * kC + (long long)(32 * hsel) * kC;
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
-          uint32_t v[kH];
+          uint32_t v[32];
           if (nt > 0) {
-            tc::tmem_ld32(tmem + lanebase + kColO + mb * kH, v);
-            tc::tmem_ld32(tmem + lanebase + kColO + mb * kH + 32, v + 32);
+            tc::tmem_ld32(tmem + lanebase + kColO + mb * kH + 32 * hsel, v);
             tc::tmem_ld_wait();
           }
           const int d = mb * 128 + dim_lane;
 #pragma unroll
-          for (int h = 0; h < kH; ++h) {
+          for (int h = 0; h < 32; ++h) {
             const float l = __uint_as_float(lv[h]);
             const float o = (nt > 0 && l > 0.f) ? __uint_as_float(v[h]) / l : 0.f;
             op[h * kC + d] = __float2bfloat16_rn(o);
           }
         }
       } else {
-        float* wo = p.ws_o + ((long long)q * p.splits + sp) * kH * kC;
+        float* wo = p.ws_o + ((long long)q * p.splits + sp) * kH * kC + (long long)(32 * hsel) * kC;
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
-          uint32_t v[kH];
+          uint32_t v[32];
           if (nt > 0) {
-            tc::tmem_ld32(tmem + lanebase + kColO + mb * kH, v);
-            tc::tmem_ld32(tmem + lanebase + kColO + mb * kH + 32, v + 32);
+            tc::tmem_ld32(tmem + lanebase + kColO + mb * kH + 32 * hsel, v);
             tc::tmem_ld_wait();
           }
           const int d = mb * 128 + dim_lane;
 #pragma unroll
-          for (int h = 0; h < kH; ++h) wo[h * kC + d] = nt > 0 ? __uint_as_float(v[h]) : 0.f;
+          for (int h = 0; h < 32; ++h) wo[h * kC + d] = nt > 0 ? __uint_as_float(v[h]) : 0.f;
         }
-        if (st < kH) {
-          float l = 0.f;  // lv[st] without a dynamically indexed register array
+        if (quarter == 0) {
+          // lane l of the quarter-0 warps: head 32 hsel + l (l is the same in every TMEM lane)
+          float l = 0.f;  // lv[lane] without a dynamically indexed register array
 #pragma unroll
-          for (int h = 0; h < kH; ++h) l = (h == st && nt > 0) ? __uint_as_float(lv[h]) : l;
-          p.ws_ml[((long long)q * p.splits + sp) * kH + st] = make_float2(l > 0.f ? bars->mref[st] : neg_inf(), l);
+          for (int h = 0; h < 32; ++h) l = (h == lane && nt > 0) ? __uint_as_float(lv[h]) : l;
+          const int hh = 32 * hsel + lane;
+          p.ws_ml[((long long)q * p.splits + sp) * kH + hh] = make_float2(l > 0.f ? bars->mref[hh] : neg_inf(), l);
         }
       }
+    }
+    // drain: every block load issued has landed before the CTA may exit
+    if (st == 0 && loaded > 0) {
+      const int j = loaded - 1;
+      for (int b = 0; b < kBlocks; ++b)
+        for (uint32_t k = 0; k < tc::kSpinLimit && !tc::mbar_try_wait(&bars->kvfull[b], j & 1); ++k) __nanosleep(64);
     }
   }
 
@@ -501,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
   __syncthreads();
   tc::fence_after_sync();
   if (threadIdx.x == 0 && bars->abort) atomicOr(&g_mqa_tc_error, 1u);
-  if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
+  if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---- host side ------------------------------------------------------------------
@@ -511,7 +523,7 @@ bool mqa_tc_supported(const MqaProblem& p) {
   return p.mode == HCA_MODE_DECODE && p.kv_seq_stride % kC == 0 && p.win_seq_stride % kC == 0;
 }
 
-// Splits per query: one wave of at most num_sms CTAs, fewest tiles per CTA.
+// Splits per query: at most num_sms CTAs per wave, fewest tiles on the critical path.
 MqaPlan plan_mqa_tc(const MqaProblem& p, int num_sms) {
   MqaPlan pl;
   const int first = p.idx ? p.n_idx : p.N;
@@ -525,15 +537,14 @@ MqaPlan plan_mqa_tc(const MqaProblem& p, int num_sms) {
     const int s_eff = (tiles + tpc - 1) / tpc;
     const long long ctas = (long long)p.Tq * s_eff;
     const long long waves = (ctas + num_sms - 1) / num_sms;
-    const long long cost = waves * tpc * 4 + (s_eff > 1 ? 1 : 0);  // tiles on the critical path, + combine
+    const long long cost = waves * (tpc * 4 + 3) + (s_eff > 1 ? 2 : 0);  // tiles + per-CTA setup, + combine
     if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_s = s_eff; }
   }
   const int tpc = (tiles + best_s - 1) / best_s;
   pl.splits = best_s;
+  // Splits start on tile boundaries of the entries segment (rows_per_split is a
+  // multiple of the tile height and each segment is tiled from its own start).
   pl.rows_per_split = tpc * kRows;
-  // A split boundary must not cut a tile of the window segment out of step with
-  // the entries segment: rows_per_split is a multiple of 64 and the first
-  // segment is tiled from its own start, so splits only ever start on a tile.
   pl.ws_bytes = best_s > 1 ? (size_t)p.Tq * best_s * kH * ((size_t)kC * sizeof(float) + sizeof(float2)) : 0;
   return pl;
 }
@@ -548,17 +559,26 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   const uint64_t qd[2] = {(uint64_t)kC, (uint64_t)p.Tq * kH};
   cudaError_t e = make_tmap_bf16(&tm_q, p.q, 2, qd, rstride, 64);
   if (e != cudaSuccess) return e;
-  const long long kv_rs = p.mode == HCA_MODE_PREFILL ? 0 : p.kv_seq_stride / kC;
-  const uint64_t kvd[2] = {(uint64_t)kC, (uint64_t)((long long)(p.Tq - 1) * kv_rs + (p.N > 0 ? p.N : 1))};
-  e = make_tmap_bf16(&tm_kv, p.kv, 2, kvd, rstride, 64);
+  const bool prefill = p.mode == HCA_MODE_PREFILL;
+  const long long kv_rs = prefill ? 0 : p.kv_seq_stride / kC;
+  const uint64_t n_kv = (uint64_t)(p.N > 0 ? p.N : 1);
+  // dense tiles: (dims, rows of one request, request), so a tile never reads
+  // another request's rows or the unused capacity behind a request's entries
+  const uint64_t kvd3[3] = {(uint64_t)kC, n_kv, prefill ? 1ull : (uint64_t)p.Tq};
+  const long long kv_req_elems = (prefill || p.Tq == 1) ? (long long)n_kv * kC : p.kv_seq_stride;
+  const uint64_t kvs3[2] = {(uint64_t)kC * 2, (uint64_t)kv_req_elems * 2};
+  e = make_tmap_bf16(&tm_kv, p.kv, 3, kvd3, kvs3, kRows);
   if (e != cudaSuccess) return e;
+  // gathered rows: one 2-D map over every request's rows
+  const uint64_t kvd[2] = {(uint64_t)kC, (uint64_t)((long long)(p.Tq - 1) * kv_rs) + n_kv};
   e = make_tmap_bf16(&tm_kvg, p.kv, 2, kvd, rstride, 1);
   if (e != cudaSuccess) return e;
-  const bool prefill = p.mode == HCA_MODE_PREFILL;
   const long long win_rs = prefill ? 0 : p.win_seq_stride / kC;
-  const uint64_t wd[2] = {(uint64_t)kC,
-                          prefill ? (uint64_t)p.win_rows : (uint64_t)((long long)(p.Tq - 1) * win_rs + p.n_win)};
-  e = make_tmap_bf16(&tm_win, p.win, 2, wd, rstride, 64);
+  const uint64_t wd3[3] = {(uint64_t)kC, prefill ? (uint64_t)p.win_rows : (uint64_t)p.n_win,
+                           prefill ? 1ull : (uint64_t)p.Tq};
+  const long long win_req_elems = prefill ? p.win_rows * kC : (p.Tq == 1 ? (long long)p.n_win * kC : p.win_seq_stride);
+  const uint64_t ws3[2] = {(uint64_t)kC * 2, (uint64_t)win_req_elems * 2};
+  e = make_tmap_bf16(&tm_win, p.win, 3, wd3, ws3, kRows);
   if (e != cudaSuccess) return e;
   MqaTcParams a;
   a.idx = p.idx;
@@ -567,8 +587,8 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   a.rate = p.rate;
   a.N = p.N;
   a.n_win = p.n_win;
-  a.kv_rows_stride = prefill ? 0 : kv_rs;
   a.prefill = prefill ? 1 : 0;
+  a.kv_rows_stride = kv_rs;
   a.win_rows_stride = win_rs;
   a.scale_log2 = p.scale * kLog2e;
   a.splits = pl.splits;

@@ -65,12 +65,13 @@ def assert_bf16_close(gpu, ref64, what=""):
     return worst
 
 
-def assert_bf16_ulps(a, b, ulps=1, what=""):
-    """Two bf16-valued arrays agree to within `ulps` bf16 ulps element-wise."""
+def assert_bf16_ulps(a, b, ulps=1, what="", rms_slack=2.0 ** -20):
+    """Two bf16-valued arrays agree to within `ulps` bf16 ulps element-wise, plus
+    `rms_slack` times the RMS of b (for elements that come out of cancellation)."""
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     rms = np.sqrt(np.mean(b ** 2)) if b.size else 0.0
-    bound = ulps * 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)) + 2.0 ** -20 * rms
+    bound = ulps * 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)) + rms_slack * rms
     bad = np.abs(a - b) > bound
     assert not np.any(bad), f"{what}: {int(bad.sum())} elements differ by more than {ulps} bf16 ulp"
 

@@ -215,13 +215,15 @@ def test_sparse_mqa_permutation_invariant(hca):
     # A permutation moves rows between tiles and splits, which changes the f32
     # summation order and which running maximum each probability is rounded
     # against; both orders must meet the parity bar, and agree with each other
-    # to well within it.
+    # to one bf16 rounding of the output (a flat softmax over ~1,150 rows moves
+    # the output by ~3% of its RMS for a dropped or doubled row, far above the
+    # 2^-10 RMS slack for cancelling elements).
     ref = np.stack([oracle.mqa_attend(to64(d["q"][b]),
                                       np.concatenate([to64(d["E"][b])[idx[b]], to64(d["win"][b])]), s.scale)
                     for b in range(4)])
     assert_norm_close(to64(o1), ref, what="sparse MQA decode")
     assert_norm_close(to64(o2), ref, what="sparse MQA decode, permuted")
-    assert_norm_close(to64(o1), to64(o2), tol=1e-2, what="permutation")
+    assert_bf16_ulps(to64(o1), to64(o2), ulps=1, rms_slack=2.0 ** -10, what="permutation")
 
 
 def test_mqa_decode_rescale_path(hca):
