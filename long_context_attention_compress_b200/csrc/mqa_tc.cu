@@ -74,6 +74,7 @@ struct __align__(16) Bars {
   uint32_t tmem_base;
   int abort;
   int rescale;
+  int need[3];  // per tile (mod 3): some score exceeds its head's running maximum by > 2^8
 };
 static_assert(offsetof(Bars, mref) % 16 == 0 && offsetof(Bars, red) % 16 == 0, "vector-loaded arrays");
 static_assert(offsetof(Bars, qfull) % 8 == 0, "mbarriers are 8-byte aligned");
@@ -167,6 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(base + kOffBars);
   volatile int* abort = &bars->abort;
+  volatile int* need_flag = bars->need;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = blockIdx.x / p.splits;
   const int sp = blockIdx.x % p.splits;
@@ -194,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     tc::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     bars->rescale = 0;
+    for (int k = 0; k < 3; ++k) bars->need[k] = 0;
     tc::fence_mbar_init();
   }
   for (int h = threadIdx.x; h < kH; h += kThreads) { bars->mref[h] = neg_inf(); bars->alpha[h] = 1.f; }
@@ -363,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       }
       if (i + 1 < nt) gather_rows(i + 1, y);  // index loads overlap the wait below
       float sv[32];
+      bool need = false;  // a score above its head's running maximum + 2^8 (or the first valid one)
       if (!failed) failed = !tc::warp_wait(&bars->sfull, ph, abort);
       if (!failed) {
         tc::fence_after_sync();
@@ -373,48 +377,70 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&bars->sempty);
 #pragma unroll
-        for (int h = 0; h < 32; ++h) sv[h] = valid ? __uint_as_float(v[h]) * p.scale_log2 : neg_inf();
+        for (int c = 0; c < 8; ++c) {
+          const float4 m4 = *reinterpret_cast<const float4*>(bars->mref + 32 * hsel + 4 * c);
+          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int h = 4 * c + j;
+            sv[h] = valid ? __uint_as_float(v[h]) * p.scale_log2 : neg_inf();
+            need |= sv[h] > mm[j] + kRescaleLog2;  // -inf + 2^8 = -inf: any valid score of an empty head
+          }
+        }
+        if (need) need_flag[i % 3] = 1;
+      }
+      if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
+      // The flag of tile i+2 is cleared here: its writers are past the next barrier,
+      // which this thread reaches first, and its last readers (tile i-1) are past this one.
+      if (st == 0) need_flag[(i + 2) % 3] = 0;
+      // Full path, only when some head's maximum grew by more than 2^8: exact tile
+      // maxima, new running maxima and the rescale of the accumulators.  Otherwise
+      // every head keeps its running maximum, exactly as the full path would decide.
+      const bool full = need_flag[i % 3] != 0;
+      if (full) {
         float tmp[32];
 #pragma unroll
         for (int h = 0; h < 32; ++h) tmp[h] = sv[h];
         bars->red[quarter][32 * hsel + lane] = warp_max32(tmp, lane);
-      }
-      if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
-      if (st < kH) {
-        const int h = st;
-        const float mt = fmaxf(fmaxf(bars->red[0][h], bars->red[1][h]), fmaxf(bars->red[2][h], bars->red[3][h]));
-        const float mo = bars->mref[h];
-        if (mt > mo + kRescaleLog2 || (mo == neg_inf() && mt != neg_inf())) {
-          bars->alpha[h] = (mo == neg_inf()) ? 0.f : fast_exp2(mo - mt);
-          bars->mref[h] = mt;
-          bars->rescale = 1;
-        } else {
-          bars->alpha[h] = 1.f;
+        if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
+        if (st < kH) {
+          const int h = st;
+          const float mt = fmaxf(fmaxf(bars->red[0][h], bars->red[1][h]), fmaxf(bars->red[2][h], bars->red[3][h]));
+          const float mo = bars->mref[h];
+          if (mt > mo + kRescaleLog2 || (mo == neg_inf() && mt != neg_inf())) {
+            bars->alpha[h] = (mo == neg_inf()) ? 0.f : fast_exp2(mo - mt);
+            bars->mref[h] = mt;
+            bars->rescale = 1;
+          } else {
+            bars->alpha[h] = 1.f;
+          }
         }
+        if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
       }
-      if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
       // Wait for PV(i-1) on every tile, in order: the odone barrier completes once per
       // tile, and a parity wait is only unambiguous while the waiter is at most one
       // phase behind (PV(i) cannot complete before this group publishes P(i)).
       if (i > 0 && !tc::warp_wait(&bars->odone, (i - 1) & 1, abort)) failed = true;
-      if (!failed && bars->rescale && i > 0) {
-        // O^T and l hold the sums up to tile i-1: scale column h by alpha[h]
-        tc::fence_after_sync();
+      if (full) {
+        if (!failed && bars->rescale && i > 0) {
+          // O^T and l hold the sums up to tile i-1: scale column h by alpha[h]
+          tc::fence_after_sync();
 #pragma unroll 1
-        for (int blk = 0; blk < 5; ++blk) {
-          const uint32_t ta = tmem + lanebase + (blk < 4 ? kColO + blk * kH : kColL) + 32 * hsel;
-          uint32_t v[32];
-          tc::tmem_ld32(ta, v);
-          tc::tmem_ld_wait();
+          for (int blk = 0; blk < 5; ++blk) {
+            const uint32_t ta = tmem + lanebase + (blk < 4 ? kColO + blk * kH : kColL) + 32 * hsel;
+            uint32_t v[32];
+            tc::tmem_ld32(ta, v);
+            tc::tmem_ld_wait();
 #pragma unroll
-          for (int h = 0; h < 32; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * bars->alpha[32 * hsel + h]);
-          tc::tmem_st32(ta, v);
+            for (int h = 0; h < 32; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * bars->alpha[32 * hsel + h]);
+            tc::tmem_st32(ta, v);
+          }
+          tc::tmem_st_wait();
+          tc::fence_before_sync();
         }
-        tc::tmem_st_wait();
-        tc::fence_before_sync();
+        if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
+        if (st == 0) bars->rescale = 0;  // every reader has passed the barrier above
       }
-      if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
-      if (st == 0) bars->rescale = 0;  // every reader has passed the barrier above
       // P = P_hi + P_lo, both bf16 (PV(i-1), the last reader of the P buffers, has completed)
       unsigned char* phi = base + kOffP + row * 128;
       unsigned char* plo = phi + kPBytes;
