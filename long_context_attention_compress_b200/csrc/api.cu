@@ -100,9 +100,17 @@ int check_cfg(const hca_layer_cfg* cfg) {
 struct IndexerPlan {
   long long ld;   // score row stride
   int chunk, chunks;
-  size_t cand_off, bytes;
+  size_t cand_off;  // chunked select: [Tq][chunks][k] composites
+  // decode select from the indexer's score histogram (N > kSelectMaxN):
+  int hist_ctas;    // select CTAs per request (kHistSlice entries each)
+  size_t hist_off, done_off, cnt_off, above_off, eq_off;
+  size_t bytes;
 };
 
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Workspace: the f32 score rows, then either select layout (they share the space;
+// only one is used per call).
 IndexerPlan plan_indexer(int Tq, int N, int k) {
   IndexerPlan p;
   p.ld = ((long long)N + 3) / 4 * 4;
@@ -114,14 +122,32 @@ IndexerPlan plan_indexer(int Tq, int N, int k) {
     p.chunks = (N + p.chunk - 1) / p.chunk;
   }
   const size_t score_bytes = (size_t)Tq * (size_t)p.ld * sizeof(float);
-  p.cand_off = (score_bytes + 255) / 256 * 256;
+  p.cand_off = align256(score_bytes);
   const size_t cand_bytes = p.chunks > 1 ? (size_t)Tq * p.chunks * k * sizeof(uint64_t) : 0;
-  p.bytes = p.cand_off + cand_bytes;
+  size_t end = p.cand_off + cand_bytes;
+  p.hist_ctas = N > kSelectMaxN ? (N + kHistSlice - 1) / kHistSlice : 0;
+  p.hist_off = p.done_off = p.cnt_off = p.above_off = p.eq_off = 0;
+  if (p.hist_ctas > 0) {
+    const size_t C = (size_t)p.hist_ctas;
+    p.hist_off = align256(score_bytes);
+    p.done_off = p.hist_off + 2 * (size_t)Tq * kHistBins * sizeof(int);  // zeroed together with the histograms
+    p.cnt_off = align256(p.done_off + (size_t)Tq * sizeof(int));
+    p.above_off = align256(p.cnt_off + (size_t)Tq * C * sizeof(int2));
+    p.eq_off = align256(p.above_off + (size_t)Tq * C * k * sizeof(int32_t));
+    const size_t hist_end = p.eq_off + (size_t)Tq * C * kHistSlice * sizeof(uint64_t);
+    end = end > hist_end ? end : hist_end;
+  }
+  p.bytes = end;
   return p;
 }
 
-int indexer_ok(int N, int k) {
+int indexer_ok(int N, int k, int mode) {
   const IndexerPlan p = plan_indexer(1, N, k);
+  if (mode == HCA_MODE_DECODE) {
+    CHECK(p.hist_ctas <= kHistMaxCtas, HCA_ERR_UNSUPPORTED, "indexer: N=%d exceeds %d entries per request", N,
+          kHistMaxCtas * kHistSlice);
+    return HCA_OK;
+  }
   CHECK((long long)p.chunks * k <= kSelectMaxN, HCA_ERR_UNSUPPORTED,
         "indexer: N=%d with topk=%d needs %d chunks (max merge %d candidates)", N, k, p.chunks, kSelectMaxN);
   return HCA_OK;
@@ -132,9 +158,17 @@ int run_indexer_topk(const bf16* q_idx, const float* w_idx, const bf16* k_idx, l
                      void* ws, cudaStream_t st, void* const* ev, int n_ev, int& ev_i, int grid_sms = 0) {
   const IndexerPlan p = plan_indexer(Tq, N, cfg->topk);
   float* scores = reinterpret_cast<float*>(ws);
+  // decode with more entries than one select CTA holds: the indexer also builds
+  // each request's score-key histogram, and one threshold select follows
+  const bool hist = mode == HCA_MODE_DECODE && p.hist_ctas > 0 && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx);
+  char* wsb = reinterpret_cast<char*>(ws);
+  if (hist)
+    CUDA_TRY(cudaMemsetAsync(wsb + p.hist_off, 0, (size_t)Tq * (2 * kHistBins + 1) * sizeof(int), st),
+             "histogram reset");
   if (mode == HCA_MODE_DECODE && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx)) {
     CUDA_TRY(launch_indexer_decode_tc(q_idx, w_idx, k_idx, k_seq_stride, N, q_pos, Tq, cfg->m, scores, p.ld,
-                                      grid_sms > 0 ? grid_sms : device_sm_count(), st),
+                                      grid_sms > 0 ? grid_sms : device_sm_count(), st,
+                                      hist ? reinterpret_cast<int*>(wsb + p.hist_off) : nullptr),
              "indexer scores (tcgen05)");
   } else if (mode == HCA_MODE_PREFILL && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx)) {
     CUDA_TRY(launch_indexer_prefill_tc(q_idx, w_idx, k_idx, N, q_pos, Tq, cfg->m, scores, p.ld,
@@ -146,6 +180,27 @@ int run_indexer_topk(const bf16* q_idx, const float* w_idx, const bf16* k_idx, l
              "indexer scores");
   }
   if (ev && ev_i < n_ev) CUDA_TRY(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
+  if (hist) {
+    HistSelect a;
+    a.scores = scores;
+    a.ld = p.ld;
+    a.q_pos = q_pos;
+    a.rate = cfg->m;
+    a.N = N;
+    a.k = cfg->topk;
+    a.hist = reinterpret_cast<int*>(wsb + p.hist_off);
+    a.B = Tq;
+    a.done = reinterpret_cast<int*>(wsb + p.done_off);
+    a.cnt = reinterpret_cast<int2*>(wsb + p.cnt_off);
+    a.above = reinterpret_cast<int32_t*>(wsb + p.above_off);
+    a.eq = reinterpret_cast<uint64_t*>(wsb + p.eq_off);
+    a.C = p.hist_ctas;
+    a.slice = kHistSlice;
+    a.out = topk_idx;
+    CUDA_TRY(launch_select_hist(a, Tq, st), "select (histogram threshold)");
+    if (ev && ev_i < n_ev) CUDA_TRY(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
+    return HCA_OK;
+  }
   SelectRows rows;
   rows.chunks = p.chunks;
   rows.chunk = p.chunk;
@@ -215,10 +270,12 @@ int hca_check_device(void) {
   if (e != cudaSuccess) return cuda_status(e, "hca_check_device");
   const unsigned int w1 = read_and_clear_indexer_tc_error();
   const unsigned int w2 = read_and_clear_mqa_tc_error();
-  if (w1 == 0xffffffffu || w2 == 0xffffffffu)
+  const unsigned int w3 = read_and_clear_select_error();
+  if (w1 == 0xffffffffu || w2 == 0xffffffffu || w3 == 0xffffffffu)
     return fail(HCA_ERR_CUDA, "hca_check_device: cannot read the device error word");
   const unsigned int w = w1 | (w2 << 1);
   if (w) return fail(HCA_ERR_DEVICE_CHECK, "hca_check_device: a kernel gave up waiting (error word 0x%x)", w);
+  if (w3) return fail(HCA_ERR_DEVICE_CHECK, "hca_check_device: a top-k histogram disagreed with its scores");
   return HCA_OK;
 }
 
@@ -267,11 +324,10 @@ int hca_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int 
 }
 
 size_t hca_workspace_size(int op, const hca_layer_cfg* cfg, int Tq, int N, int mode) {
-  (void)mode;
   if (check_cfg(cfg) != HCA_OK || Tq < 0 || N < 0) return (size_t)-1;
   switch (op) {
     case HCA_OP_INDEXER_TOPK:
-      if (indexer_ok(N, cfg->topk) != HCA_OK) return (size_t)-1;
+      if (indexer_ok(N, cfg->topk, mode) != HCA_OK) return (size_t)-1;
       return plan_indexer(Tq, N, cfg->topk).bytes;
     case HCA_OP_SPARSE_MQA:
       return mqa_ws_bound(cfg, Tq, N, cfg->topk);
@@ -289,7 +345,7 @@ int csa_indexer_topk(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* 
   CHECK(Tq >= 0 && N >= 0, HCA_ERR_INVALID_ARG, "csa_indexer_topk: Tq=%d N=%d", Tq, N);
   CHECK(mode == HCA_MODE_PREFILL || mode == HCA_MODE_DECODE, HCA_ERR_INVALID_ARG, "csa_indexer_topk: mode=%d", mode);
   CHECK(mode == HCA_MODE_PREFILL || k_seq_stride % 8 == 0, HCA_ERR_INVALID_ARG, "csa_indexer_topk: k_seq_stride");
-  s = indexer_ok(N, cfg->topk);
+  s = indexer_ok(N, cfg->topk, mode);
   if (s != HCA_OK) return s;
   if (Tq == 0) return injected("csa_indexer_topk") ? fail(HCA_ERR_INJECTED, "injected") : HCA_OK;
   CHECK_PTR(q_idx, "csa_indexer_topk: q_idx");
@@ -348,7 +404,7 @@ int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hc
         "csa_indexer_topk_noalloc: mode=%d", mode);
   CHECK(mode == HCA_MODE_PREFILL || k_seq_stride % 8 == 0, HCA_ERR_INVALID_ARG,
         "csa_indexer_topk_noalloc: k_seq_stride");
-  s = indexer_ok(N, cfg->topk);
+  s = indexer_ok(N, cfg->topk, mode);
   if (s != HCA_OK) return s;
   const size_t need = plan_indexer(Tq, N, cfg->topk).bytes;
   CHECK(need <= (size_t)HCA_NOALLOC_SCRATCH_BYTES, HCA_ERR_WORKSPACE,
@@ -513,7 +569,7 @@ static int side_stream(SideStream** out) {
 
 size_t hybrid_attn_decode_workspace(const hca_layer_cfg* cfg, const hca_decode_args* a) {
   if (check_cfg(cfg) != HCA_OK || !a || a->B < 0) return (size_t)-1;
-  if (a->csa_q && indexer_ok(a->csa_N, cfg->topk) != HCA_OK) return (size_t)-1;
+  if (a->csa_q && indexer_ok(a->csa_N, cfg->topk, HCA_MODE_DECODE) != HCA_OK) return (size_t)-1;
   return decode_ws(cfg, a);
 }
 
@@ -528,7 +584,7 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
   if (a->B == 0) return HCA_OK;
   CHECK_PTR(a->q_pos, "hybrid_attn_decode: q_pos");
   if (a->csa_q) {
-    s = indexer_ok(a->csa_N, cfg->topk);
+    s = indexer_ok(a->csa_N, cfg->topk, HCA_MODE_DECODE);
     if (s != HCA_OK) return s;
     CHECK(a->csa_N > 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: csa_N=%d", a->csa_N);
     CHECK_PTR(a->csa_q_idx, "hybrid_attn_decode: csa_q_idx");
@@ -648,7 +704,7 @@ static size_t prefill_ws(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
 
 size_t hybrid_attn_prefill_workspace(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
   if (check_cfg(cfg) != HCA_OK || !a || a->T < 0) return (size_t)-1;
-  if (indexer_ok(a->T / cfg->m, cfg->topk) != HCA_OK) return (size_t)-1;
+  if (indexer_ok(a->T / cfg->m, cfg->topk, HCA_MODE_PREFILL) != HCA_OK) return (size_t)-1;
   return prefill_ws(cfg, a);
 }
 
@@ -662,7 +718,7 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
   const int T = a->T;
   if (T == 0) return HCA_OK;
   const int Nc = T / cfg->m;
-  s = indexer_ok(Nc, cfg->topk);
+  s = indexer_ok(Nc, cfg->topk, HCA_MODE_PREFILL);
   if (s != HCA_OK) return s;
   CHECK_PTR(a->q_pos, "hybrid_attn_prefill: q_pos");
   CHECK_PTR(a->cand, "hybrid_attn_prefill: cand");

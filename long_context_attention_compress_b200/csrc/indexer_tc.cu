@@ -49,7 +49,8 @@ struct __align__(8) Bars {
   uint32_t tmem_base;
   int abort;
 };
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStages * kTileBytes + 2 * kQBytes + sizeof(Bars);
+constexpr size_t kSmemBytes =
+    1024 /*align slack*/ + kStages * kTileBytes + 2 * kQBytes + sizeof(Bars) + kHistBins * sizeof(int);
 }  // namespace
 
 __device__ unsigned int g_indexer_tc_error = 0;
@@ -57,12 +58,13 @@ __device__ unsigned int g_indexer_tc_error = 0;
 __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
     const float* __restrict__ w_idx, const int32_t* __restrict__ q_pos, int B, int N, int rate,
-    int tiles_per_req, float* __restrict__ scores, long long ld_scores) {
+    int tiles_per_req, float* __restrict__ scores, long long ld_scores, int* __restrict__ hist_g) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* k_smem = base;                              // [stages][2][128][128 B]
   unsigned char* q_smem = base + kStages * kTileBytes;        // [2][2][64][128 B]
   Bars* bars = reinterpret_cast<Bars*>(q_smem + 2 * kQBytes);
+  int* s_hist = reinterpret_cast<int*>(bars + 1);             // [kHistBins] score-key histogram
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -78,6 +80,8 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
     bars->abort = 0;
     tc::fence_mbar_init();
   }
+  if (hist_g)
+    for (int i = threadIdx.x; i < kHistBins; i += kThreads) s_hist[i] = 0;
   if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
@@ -159,20 +163,40 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
     // ------------------------------ epilogue ------------------------------
     const int lq = warp & 3;  // TMEM lane quarter this warp may access
     const int row_in_tile = lq * 32 + lane;
+    const int et = (warp - 2) * 32 + lane;  // 0..127 within the epilogue warps
     float w[kHeads];
     int it = 0, cur_r = -1;
+    // A failed wait does not leave the loop: every epilogue thread still reaches
+    // the histogram flushes, whose barriers agree on the failure first.
+    bool failed = false;
+    // Add this CTA's counts for request r to the request's global histogram.
+    auto flush = [&](int r) {
+      if (tc::named_bar_or(1, 128, failed || *abort)) { failed = true; return; }
+#pragma unroll 4
+      for (int b = et * (kHistBins / 128); b < (et + 1) * (kHistBins / 128); ++b) {
+        const int c = s_hist[b];
+        if (c) {
+          atomicAdd(hist_g + (long long)r * kHistBins + b, c);
+          s_hist[b] = 0;
+        }
+      }
+      tc::named_bar(1, 128);
+    };
     for (long long g = g0; g < g1; ++g) {
       const int r = (int)(g / tiles_per_req);
       const int row0 = (int)(g % tiles_per_req) * kTile;
       const int nvis = n_visible(q_pos[r], rate, N);
       if (row0 >= nvis) continue;
       if (r != cur_r) {
+        if (hist_g && cur_r >= 0) flush(cur_r);
 #pragma unroll
         for (int j = 0; j < kHeads; ++j) w[j] = w_idx[(long long)r * kHeads + j];
         cur_r = r;
       }
       const int a = it % kAcc;
-      if (!tc::mbar_wait(&bars->tfull[a], (it / kAcc) & 1, abort)) break;
+      ++it;
+      if (!failed) failed = !tc::mbar_wait(&bars->tfull[a], ((it - 1) / kAcc) & 1, abort);
+      if (failed) continue;
       tc::fence_after_sync();
       uint32_t v[kHeads];
       const uint32_t taddr = tmem + ((uint32_t)(lq * 32) << 16) + a * kHeads;
@@ -189,9 +213,16 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
         sc1 = fmaf(w[j + 1], fmaxf(__uint_as_float(v[j + 1]), 0.f), sc1);
       }
       const int e = row0 + row_in_tile;
-      if (e < nvis) scores[(long long)r * ld_scores + e] = sc0 + sc1;
-      ++it;
+      const float sc = sc0 + sc1;
+      if (e < nvis) scores[(long long)r * ld_scores + e] = sc;
+      if (hist_g) {
+        // neighbouring entries share few bins: one shared-memory atomic per distinct bin of the warp
+        const uint32_t bin = e < nvis ? float_key(sc) >> 20 : 0xffffffffu;
+        const unsigned same = __match_any_sync(0xffffffffu, bin);
+        if (e < nvis && (int)(__ffs(same) - 1) == lane) atomicAdd(s_hist + bin, __popc(same));
+      }
     }
+    if (hist_g && cur_r >= 0) flush(cur_r);
   }
 
   tc::fence_before_sync();
@@ -428,7 +459,7 @@ bool indexer_tc_supported(int H_I, int d_I) { return H_I == kHeads && d_I == kDi
 
 cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride,
                                      int N, const int32_t* q_pos, int B, int rate, float* scores, long long ld_scores,
-                                     int num_sms, cudaStream_t stream) {
+                                     int num_sms, cudaStream_t stream, int* hist) {
   if (B == 0 || N == 0) return cudaSuccess;
   CUtensorMap tm_k, tm_q;
   const uint64_t kd[3] = {(uint64_t)kDim, (uint64_t)N, (uint64_t)B};
@@ -446,7 +477,7 @@ cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, cons
                            (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   indexer_decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_k, tm_q, w_idx, q_pos, B, N, rate,
-                                                                   tiles_per_req, scores, ld_scores);
+                                                                   tiles_per_req, scores, ld_scores, hist);
   ++g_launch_counter;
   return cudaGetLastError();
 }

@@ -43,6 +43,27 @@ cudaError_t launch_select_from_scores(const float* scores, const SelectRows& row
 // top-k indices to out_idx [rows, k].
 cudaError_t launch_select_merge(const uint64_t* cand, int n_rows, int n_cand, int k,
                                 int32_t* out_idx, cudaStream_t stream);
+// Decode top-k from a per-request histogram of score keys (bins: key >> 20),
+// built by the indexer.  Workspace regions as laid out by plan_indexer.
+constexpr int kHistBins = 4096;
+constexpr int kHistMaxCtas = 128;
+constexpr int kHistSlice = 16384;  // entries per select CTA
+struct HistSelect {
+  const float* scores;
+  long long ld;          // elements between requests' score rows
+  const int32_t* q_pos;
+  int rate, N, k;
+  int* hist;             // [2][B][kHistBins]: level 1 by the indexer, level 2 here (zeroed before the indexer)
+  int* done;             // [B] arrival tickets (zeroed with hist)
+  int B;
+  int2* cnt;             // [B][C] per-CTA (above, bin-T) counts
+  int32_t* above;        // [B][C][k]
+  uint64_t* eq;          // [B][C][slice] composites
+  int C, slice;
+  int32_t* out;          // [B][k]
+};
+cudaError_t launch_select_hist(const HistSelect& a, int B, cudaStream_t stream);
+unsigned int read_and_clear_select_error();
 
 // ---- indexer.cu ---------------------------------------------------------------
 // scores[q, s] = sum_j w[q,j] relu(q_idx[q,j,:] . K[s,:]) for visible s (others untouched).
@@ -56,7 +77,8 @@ bool indexer_tc_supported(int H_I, int d_I);
 // Decode: query r scores request r's keys (k_idx + r*k_seq_stride), scores[r*ld + s].
 cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride,
                                      int N, const int32_t* q_pos, int B, int rate, float* scores, long long ld_scores,
-                                     int num_sms, cudaStream_t stream);
+                                     int num_sms, cudaStream_t stream,
+                                     int* hist = nullptr);
 // Prefill: queries of one sequence against its keys [N, d_I]; scores[q*ld + s] for visible s.
 cudaError_t launch_indexer_prefill_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, int N,
                                       const int32_t* q_pos, int Tq, int rate, float* scores, long long ld_scores,

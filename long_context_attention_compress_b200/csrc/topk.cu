@@ -19,6 +19,7 @@
 namespace hca {
 
 constexpr int kSelThreads = 1024;
+__device__ unsigned int g_select_error = 0;
 
 // Block-wide exclusive scan of two counters (NT threads, NT % 32 == 0).
 template <int NT>
@@ -239,6 +240,227 @@ __global__ void __launch_bounds__(kSelThreads) select_merge_kernel(const uint64_
   select_core<kSelThreads>(s_c, n, k, out_idx + (long long)r * k, nullptr);
 }
 
+// ---- decode: threshold select from a per-request score histogram ------------------
+// The indexer counts each request's visible scores into 4096 bins of the top 12
+// bits of their order-preserving key.  Bin T holding the k-th largest score splits
+// every entry into three classes: above T (always selected), in T (candidates for
+// the remaining k - above places) and below (never).  C CTAs per request scan
+// slices of the scores and compact both classes in entry order; the last CTA to
+// finish concatenates the "above" lists in slice order and runs the exact radix
+// select over the bin-T candidates only.  The output is deterministic: the
+// entries above T in index order, then the chosen bin-T entries in index order.
+// Threshold over a 4096-bin histogram read from global memory: the bin holding the
+// `k`-th largest entry, and the number of entries in higher bins.  All NT threads.
+template <int NT>
+__device__ void hist_threshold(const int* h, int k, int* s_bin, int* s_higher, int2* s_warp) {
+  static_assert(NT * 4 == kHistBins, "four bins per thread");
+  const int tid = threadIdx.x;
+  if (tid == 0) { *s_bin = -1; *s_higher = 0; }
+  const int4 h4 = __ldcg(reinterpret_cast<const int4*>(h + kHistBins - 4 * (tid + 1)));
+  const int hv[4] = {h4.w, h4.z, h4.y, h4.x};  // bins 4095 - 4t, 4094 - 4t, ...
+  int ex, dummy, tot, tdummy;
+  block_scan2<NT>(hv[0] + hv[1] + hv[2] + hv[3], 0, ex, dummy, tot, tdummy, s_warp);
+  int run = ex;  // entries in higher bins
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    if (run < k && run + hv[u] >= k) { *s_bin = kHistBins - 1 - (4 * tid + u); *s_higher = run; }
+    run += hv[u];
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_hist_kernel(HistSelect a) {
+  extern __shared__ uint64_t s_c[];
+  __shared__ int2 s_warp[kSelThreads / 32 + 1];
+  __shared__ int s_T, s_above, s_T2, s_above2, s_last;
+  __shared__ int2 s_cnt[kHistMaxCtas];
+  __shared__ int2 s_off[kHistMaxCtas + 1];
+  __shared__ uint64_t s_tie[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r = blockIdx.x / a.C, c = blockIdx.x % a.C;
+  const int k = a.k;
+  const int nvis = n_visible(a.q_pos[r], a.rate, a.N);
+  int32_t* out = a.out + (long long)r * k;
+  if (nvis <= k) {  // every visible entry (no histogram needed)
+    if (c == 0)
+      for (int e = tid; e < k; e += kSelThreads) out[e] = e < nvis ? e : -1;
+    return;
+  }
+  // this CTA's slice, thread t owning 16 consecutive entries: loads issued first,
+  // so their latency overlaps the threshold search
+  const int e0 = c * a.slice + 16 * tid;
+  const float* sp = a.scores + (long long)r * a.ld;
+  float v[16];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int e = e0 + 4 * u;
+    const float4 f = (e + 3 < nvis) ? __ldcg(reinterpret_cast<const float4*>(sp + e))
+                                    : make_float4(e < nvis ? sp[e] : 0.f, e + 1 < nvis ? sp[e + 1] : 0.f,
+                                                  e + 2 < nvis ? sp[e + 2] : 0.f, 0.f);
+    v[4 * u] = f.x; v[4 * u + 1] = f.y; v[4 * u + 2] = f.z; v[4 * u + 3] = f.w;
+  }
+  // level 1: bin of the top 12 key bits holding the k-th largest score
+  hist_threshold<kSelThreads>(a.hist + (long long)r * kHistBins, k, &s_T, &s_above, s_warp);
+  if (s_T < 0) {  // fewer counted entries than visible ones: the histogram is not this call's
+    if (tid == 0) atomicOr(&g_select_error, 1u);
+    return;
+  }
+  const uint32_t T = (uint32_t)s_T;
+  const int above_total = s_above;
+  int* hist2 = a.hist + (long long)(a.B + r) * kHistBins;  // level-2 histograms follow the B level-1 ones
+  int na = 0, ne = 0;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    if (e0 + u < nvis) {
+      const uint32_t key = float_key(v[u]);
+      na += (key >> 20) > T;
+      if ((key >> 20) == T) {
+        ++ne;
+        atomicAdd(hist2 + ((key >> 8) & (kHistBins - 1)), 1);  // level 2: the next 12 key bits
+      }
+    }
+  }
+  int oa, oe, ta, te;
+  block_scan2<kSelThreads>(na, ne, oa, oe, ta, te, s_warp);
+  int32_t* above = a.above + ((long long)r * a.C + c) * k;
+  uint64_t* eq = a.eq + ((long long)r * a.C + c) * a.slice;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int e = e0 + u;
+    if (e < nvis) {
+      const uint32_t b = float_key(v[u]) >> 20;
+      // (a CTA never holds more than k - 1 entries above T; the bound only guards the
+      // region if the histogram were not this call's -- the merge then reports it)
+      if (b > T) { if (oa < k) above[oa] = e; ++oa; }
+      else if (b == T) eq[oe++] = make_cand(v[u], e);
+    }
+  }
+  // the last CTA of the request to finish merges
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    a.cnt[(long long)r * a.C + c] = make_int2(ta, te);
+    __threadfence();
+    s_last = atomicAdd(a.done + r, 1) == a.C - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // every CTA's counts (written by other CTAs: read from L2), exclusive offsets by warp 0
+  if (tid < a.C) s_cnt[tid] = __ldcg(a.cnt + (long long)r * a.C + tid);
+  __syncthreads();
+  if (warp == 0) {
+    int ca = 0, ce = 0;
+    for (int j0 = 0; j0 < a.C; j0 += 32) {
+      const int j = j0 + lane;
+      const int2 n2 = j < a.C ? s_cnt[j] : make_int2(0, 0);
+      int xa = n2.x, xe = n2.y;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ya = __shfl_up_sync(0xffffffffu, xa, o), ye = __shfl_up_sync(0xffffffffu, xe, o);
+        if (lane >= o) { xa += ya; xe += ye; }
+      }
+      if (j < a.C) s_off[j] = make_int2(ca + xa - n2.x, ce + xe - n2.y);
+      ca += __shfl_sync(0xffffffffu, xa, 31);
+      ce += __shfl_sync(0xffffffffu, xe, 31);
+    }
+    if (lane == 0) s_off[a.C] = make_int2(ca, ce);
+  }
+  __syncthreads();
+  const int n_above = s_off[a.C].x, n_eq = s_off[a.C].y;
+  if (n_above != above_total || n_above >= k || n_eq < k - n_above) {
+    // the histogram disagrees with the scores: report instead of selecting wrongly
+    if (tid == 0) atomicOr(&g_select_error, 1u);
+    return;
+  }
+  const int need = k - n_above;
+  // one warp per slice list: the "above" entries go straight to the output
+  for (int j = warp; j < a.C; j += kSelThreads / 32) {
+    const int32_t* src_a = a.above + ((long long)r * a.C + j) * k;
+    for (int t = lane; t < s_cnt[j].x; t += 32) out[s_off[j].x + t] = __ldcg(src_a + t);
+  }
+  if (n_eq <= kSelectMaxN) {
+    // bin-T candidates staged in shared memory in entry order
+    for (int j = warp; j < a.C; j += kSelThreads / 32) {
+      const uint64_t* src_e = a.eq + ((long long)r * a.C + j) * a.slice;
+      for (int t = lane; t < s_cnt[j].y; t += 32) s_c[s_off[j].y + t] = __ldcg(src_e + t);
+    }
+    // level 2 threshold among them (the histogram's total is n_eq)
+    hist_threshold<kSelThreads>(hist2, need, &s_T2, &s_above2, s_warp);
+    const int T2 = s_T2, above2 = s_above2;
+    if (T2 < 0) {
+      if (tid == 0) atomicOr(&g_select_error, 1u);
+      return;
+    }
+    // one pass in entry order: level-2 bins above T2 are selected, bin T2 ties collected
+    const int per = (n_eq + kSelThreads - 1) / kSelThreads;
+    const int t0 = tid * per, t1 = min(n_eq, t0 + per);
+    int ng = 0, nq = 0;
+    for (int t = t0; t < t1; ++t) {
+      const int b2 = (int)((s_c[t] >> 40) & (kHistBins - 1));
+      ng += b2 > T2;
+      nq += b2 == T2;
+    }
+    int og, oq, tg, tq;
+    block_scan2<kSelThreads>(ng, nq, og, oq, tg, tq, s_warp);
+    if (tg != above2) {
+      if (tid == 0) atomicOr(&g_select_error, 1u);
+      return;
+    }
+    const int need2 = need - above2;
+    if (tq < need2) {
+      if (tid == 0) atomicOr(&g_select_error, 1u);
+      return;
+    }
+    // The level-2 ties go to a shared array when there are few (the usual case),
+    // else to this request's candidate region in global memory, free now that its
+    // lists are staged in shared memory.
+    const bool few = tq <= 32;
+    uint64_t* gties = a.eq + (long long)r * a.C * a.slice;
+    for (int t = t0; t < t1; ++t) {
+      const uint64_t cnd = s_c[t];
+      const int b2 = (int)((cnd >> 40) & (kHistBins - 1));
+      if (b2 > T2) {
+        out[n_above + og++] = cand_index(cnd);
+      } else if (b2 == T2) {
+        if (few) s_tie[oq] = cnd;
+        else gties[oq] = cnd;
+        ++oq;
+      }
+    }
+    __threadfence_block();
+    __syncthreads();
+    if (few) {
+      // rank the ties within one warp (composites are distinct)
+      if (warp == 0) {
+        const uint64_t mine = lane < tq ? s_tie[lane] : 0ull;
+        int rank = 0;
+        for (int j = 0; j < tq; ++j) rank += s_tie[j] > mine;
+        if (lane < tq && rank < need2) out[n_above + above2 + rank] = cand_index(mine);
+      }
+    } else {
+      select_core<kSelThreads>(gties, tq, need2, out + n_above + above2, nullptr);
+    }
+  } else {
+    // Many ties around the threshold: gather the candidates to the front of this
+    // request's region (a left shift, chunk by chunk) and select from global memory.
+    uint64_t* gdst = a.eq + (long long)r * a.C * a.slice;
+    for (int j = 0; j < a.C; ++j) {
+      const uint64_t* src = a.eq + ((long long)r * a.C + j) * a.slice;
+      for (int t0 = 0; t0 < s_cnt[j].y; t0 += kSelThreads) {
+        const int t = t0 + tid;
+        const uint64_t x = t < s_cnt[j].y ? __ldcg(src + t) : 0ull;
+        __syncthreads();
+        if (t < s_cnt[j].y) gdst[s_off[j].y + t] = x;
+        __syncthreads();
+      }
+    }
+    __threadfence_block();
+    __syncthreads();
+    select_core<kSelThreads>(gdst, n_eq, need, out + n_above, nullptr);
+  }
+}
+
 static cudaError_t set_smem(const void* fn, size_t bytes) {
   return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
@@ -263,6 +485,24 @@ cudaError_t launch_select_merge(const uint64_t* cand, int n_rows, int n_cand, in
   select_merge_kernel<<<n_rows, kSelThreads, smem, stream>>>(cand, n_cand, k, out_idx);
   ++g_launch_counter;
   return cudaGetLastError();
+}
+
+cudaError_t launch_select_hist(const HistSelect& a, int B, cudaStream_t stream) {
+  if (B == 0) return cudaSuccess;
+  if (a.C > kHistMaxCtas || a.slice != 16 * kSelThreads) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)kSelectMaxN * sizeof(uint64_t);
+  cudaError_t e = set_smem((const void*)select_hist_kernel, smem);
+  if (e != cudaSuccess) return e;
+  select_hist_kernel<<<B * a.C, kSelThreads, smem, stream>>>(a);
+  ++g_launch_counter;
+  return cudaGetLastError();
+}
+
+unsigned int read_and_clear_select_error() {
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_select_error, sizeof(v)) != cudaSuccess) return 0xffffffffu;
+  if (v) cudaMemcpyToSymbol(g_select_error, &zero, sizeof(zero));
+  return v;
 }
 
 }  // namespace hca

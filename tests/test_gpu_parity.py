@@ -136,6 +136,38 @@ def test_indexer_topk_decode_csa_128k(hca):
     assert swaps <= 32 * 8
 
 
+def test_indexer_topk_decode_threshold_ties(hca):
+    """Decode top-k when thousands of scores tie at the threshold.  Request 0: every
+    third key is the same vector and the rest are zero, so ~13,300 equal scores
+    compete for the 1024 places (ties go to the lower index).  Request 1: all keys
+    zero, so all 40,000 scores are equal -- more threshold candidates than one CTA
+    stages in shared memory.  Request 2: ordinary random keys."""
+    s = wl.PRO
+    d = wl.csa_decode_inputs(s, B=3, ctx=4 * 40000, seed=11)
+    K = d["K_I"].clone()
+    N = K.shape[1]
+    K[0] = 0
+    K[0, ::3] = d["K_I"][0, 7]
+    K[1] = 0
+    d["K_I"] = K
+    g = to_dev(d)
+    cfg = hca.make_cfg(s)
+    idx = hca.csa_indexer_topk(g["q_idx"], g["w_idx"], g["K_I"], g["q_pos"], cfg, mode=hca.HCA_MODE_DECODE)
+    torch.cuda.synchronize()
+    assert hca.lib.hca_check_device() == 0, hca.last_error()
+    idx = idx.cpu().numpy()
+    for b in range(3):
+        sc = oracle.indexer_scores(to64(d["q_idx"][b]), d["w_idx"][b].double().numpy(), to64(d["K_I"][b]))
+        sel = oracle.topk_select(sc, s.topk)
+        if b < 2:
+            # exactly tied scores: the lower indices win, on both sides
+            assert sorted(idx[b].tolist()) == sorted(sel.tolist())
+        else:
+            check_topk_row(idx[b], sel, sc, s.topk, N)
+    assert sorted(idx[0].tolist()) == list(range(0, 3 * s.topk, 3))
+    assert sorted(idx[1].tolist()) == list(range(s.topk))
+
+
 @pytest.mark.parametrize("B,ctx", [(300, 4 * 2048), (5, 4 * 1000 + 3), (7, 4 * 128 * 3 - 1)])
 def test_indexer_topk_decode_many_requests_ragged(hca, B, ctx):
     """Many short requests per CTA (the q_I buffer switches mid-range), ragged last tiles,
