@@ -367,9 +367,13 @@ class PrefillBench:
         return time.perf_counter() - t0
 
 
-def make_bench(name, seed, device):
+def make_bench(name, seed, device, tokens=None):
     spec = wl.WORKLOADS[name]
     if spec["kind"] == "prefill":
+        if tokens:
+            # a shorter sequence of the same shape (profiling captures): not the headline workload
+            spec = dict(spec, T=int(tokens))
+            name = f"{name}_T{int(tokens)}"
         return PrefillBench(name, spec, seed, device)
     return DecodeBench(name, spec, seed, device)
 
@@ -404,7 +408,7 @@ def run_ours(a):
     rank, local, ws = init_dist("nccl")
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    bench = make_bench(a.workload, shard_seed(a.seed, rank), device)
+    bench = make_bench(a.workload, shard_seed(a.seed, rank), device, tokens=a.tokens)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     for _ in range(a.warmup):
         bench.step()
@@ -555,6 +559,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-sample", type=int, default=4, help="requests (decode) / queries (prefill) for the oracle")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="prefill workloads: a shorter sequence of the same shape (for profiler captures)")
     a = ap.parse_args()
     if a.warmup < 3:
         print("warning: fewer than 3 warm-up steps; the number is not a valid measurement", file=sys.stderr)
