@@ -504,10 +504,11 @@ static DecodeSched decode_schedule(const hca_layer_cfg* cfg, const hca_decode_ar
   d.overlap = csa && hcl && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx) && mqa_tc_supported(ph) && d.sms >= 16;
   if (d.overlap) {
     // Balance the two sides' SM-time: the attention costs about kAttnTileUs per
-    // 64-row tile on one SM, the indexer streams about kIdxBytesPerSmUs bytes
-    // per microsecond per SM (measured on B200).  The HCA share is a whole
-    // number of splits per request so that it runs as a single wave.
-    constexpr double kAttnTileUs = 4.5, kIdxBytesPerSmUs = 35e3;
+    // 64 rows on one SM, the indexer streams about kIdxBytesPerSmUs bytes per
+    // microsecond per SM (calibrated on B200 by sweeping the HCA share of the
+    // 8-request 1M-context step: 24 of 148 SMs is best there).  The HCA share is
+    // a whole number of splits per request so that it runs as a single wave.
+    constexpr double kAttnTileUs = 3.0, kIdxBytesPerSmUs = 35e3;
     const double hca_tiles = (double)a->B * std::ceil(((double)a->hca_N + cfg->n_win) / 64.0);
     const double hca_us = hca_tiles * kAttnTileUs;
     const double idx_us = (double)a->B * a->csa_N * cfg->d_idx * 2.0 / kIdxBytesPerSmUs;
@@ -635,29 +636,32 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
     CUDA_TRY(cudaEventRecord(side->fork, st), "decode: fork");
     CUDA_TRY(cudaStreamWaitEvent(side->s, side->fork, 0), "decode: fork wait");
   }
-  auto run_hca = [&]() -> int {
-    if (a->hca_block_cand) {
-      // newest complete HCA block of every request -> its cache row.  All
-      // requests share one position here (q_pos is on the device), so the row
-      // is hca_N - 1: the caller passes caches sized to the complete blocks.
-      CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), cfg->c,
-                               reinterpret_cast<const bf16*>(a->hca_block_logits), cfg->c, a->hca_pos_bias, cfg->c,
-                               a->B, a->hca_block_stride, cfg->m_hca, cfg->c, cfg->m_hca, false,
-                               reinterpret_cast<bf16*>(a->hca_kv) + (long long)(a->hca_N - 1) * cfg->c, cfg->c,
-                               a->hca_kv_stride, hst),
-               "decode: hca compress");
-    }
+  // newest complete HCA block of every request -> its cache row.  All requests
+  // share one position here (q_pos is on the device), so the row is hca_N - 1:
+  // the caller passes caches sized to the complete blocks.
+  auto run_hca_compress = [&]() -> int {
+    CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), cfg->c,
+                             reinterpret_cast<const bf16*>(a->hca_block_logits), cfg->c, a->hca_pos_bias, cfg->c,
+                             a->B, a->hca_block_stride, cfg->m_hca, cfg->c, cfg->m_hca, false,
+                             reinterpret_cast<bf16*>(a->hca_kv) + (long long)(a->hca_N - 1) * cfg->c, cfg->c,
+                             a->hca_kv_stride, hst),
+             "decode: hca compress");
+    return HCA_OK;
+  };
+  auto run_hca_attention = [&]() -> int {
     MqaProblem p = decode_hca_problem(cfg, a);
     CUDA_TRY(launch_mqa(p, sched.hca_pl, hws, hst), "decode: hca attention");
     return HCA_OK;
   };
+  // Phase marks, in order: [hca compress] [indexer, top-k, csa attention] [hca attention].
   if (a->hca_q && sched.overlap) {
     // launched first so that its CTAs take their SMs before the indexer's persistent grid
-    if ((s = run_hca()) != HCA_OK) return s;
+    if (a->hca_block_cand && (s = run_hca_compress()) != HCA_OK) return s;
+    if ((s = run_hca_attention()) != HCA_OK) return s;
     CUDA_TRY(cudaEventRecord(side->join, side->s), "decode: join");
+    if (a->hca_block_cand && (s = mark()) != HCA_OK) return s;  // (the compression overlaps the rest)
   } else if (a->hca_q && a->hca_block_cand) {
-    // sequential: the block compression first (marked as its own phase)
-    if ((s = run_hca()) != HCA_OK) return s;
+    if ((s = run_hca_compress()) != HCA_OK) return s;
     if ((s = mark()) != HCA_OK) return s;
   }
   if (a->csa_q) {
@@ -673,14 +677,10 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
   if (a->hca_q) {
     if (sched.overlap) {
       CUDA_TRY(cudaStreamWaitEvent(st, side->join, 0), "decode: join wait");
-    } else if (!a->hca_block_cand) {
-      if ((s = run_hca()) != HCA_OK) return s;
-    } else {
-      // already run above, before the CSA layer
+    } else if ((s = run_hca_attention()) != HCA_OK) {
+      return s;
     }
-    if (!(a->hca_block_cand && !sched.overlap)) {
-      if ((s = mark()) != HCA_OK) return s;
-    }
+    if ((s = mark()) != HCA_OK) return s;
   }
   g_last_launches = g_launch_counter;
   return HCA_OK;
