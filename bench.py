@@ -238,27 +238,42 @@ class DecodeBench:
 
     # --- end to end: per-step inputs from pinned host memory, outputs back ---
     def e2e_setup(self):
-        self.h_in, self.d_in, self.h_out, self.d_out = [], [], [], []
+        """Two device buffer sets of the per-step inputs and outputs (set 0 is the
+        bench's own), so that one step's copies overlap the neighbouring steps'
+        compute; the caches and the workspace are shared (compute is serial)."""
+        in_keys = ("q", "q_idx", "w_idx", "win", "block_cand", "block_logits")
+        self.h_in = []
         for d in (self.csa, self.hcad):
             if d is None:
                 continue
-            for k in ("q", "q_idx", "w_idx", "win", "block_cand", "block_logits"):
+            for k in in_keys:
                 if k in d:
-                    self.d_in.append(d[k])
                     self.h_in.append(torch.empty(d[k].shape, dtype=d[k].dtype, pin_memory=True).copy_(d[k].cpu()))
-        for t in (self.idx, self.csa_out, self.hca_out):
-            if t is not None:
-                self.d_out.append(t)
-                self.h_out.append(torch.empty(t.shape, dtype=t.dtype, pin_memory=True))
+        self.sets = []
+        for b in range(2):
+            csa = dict(self.csa) if self.csa is not None else None
+            hcad = dict(self.hcad) if self.hcad is not None else None
+            if b == 0:
+                outs = (self.idx, self.csa_out, self.hca_out)
+            else:
+                for d in (csa, hcad):
+                    if d is not None:
+                        for k in in_keys:
+                            if k in d:
+                                d[k] = d[k].clone()
+                outs = tuple(None if t is None else torch.empty_like(t) for t in (self.idx, self.csa_out, self.hca_out))
+            d_in = [d[k] for d in (csa, hcad) if d is not None for k in in_keys if k in d]
+            d_out = [t for t in outs if t is not None]
+            args, keep = self.hca.make_decode_args(self.B, self.q_pos, csa=csa, hca=hcad, csa_topk_idx=outs[0],
+                                                   csa_out=outs[1], hca_out=outs[2])
+            h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]
+            self.sets.append({"args": args, "keep": (keep, csa, hcad, outs), "d_in": d_in, "d_out": d_out,
+                              "h_out": h_out})
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
-        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.sets[0]["h_out"])
 
-    def e2e_step(self):
-        for h, d in zip(self.h_in, self.d_in):
-            d.copy_(h, non_blocking=True)
-        self.step(record=False)
-        for h, d in zip(self.h_out, self.d_out):
-            h.copy_(d, non_blocking=True)
+    def run_set(self, b):
+        self.hca.hybrid_attn_decode(self.cfg, self.sets[b]["args"], ws=self.ws)
 
     # --- CPU oracle on a bounded sample of requests ---
     def oracle_sample(self, n_req):
@@ -338,20 +353,23 @@ class PrefillBench:
                 "indexer": f"{s.n_idx_heads}x{s.d_idx}", "n_win": s.n_win}
 
     def e2e_setup(self):
+        """Two device buffer sets of the per-step inputs and outputs (see DecodeBench)."""
         keys = ("cand", "logits", "kidx_cand", "q_idx", "w_idx", "q")
-        self.d_in = [self.inp[k] for k in keys]
-        self.h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu()) for t in self.d_in]
-        self.d_out = [self.topk, self.out]
-        self.h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in self.d_out]
+        self.h_in = [torch.empty(self.inp[k].shape, dtype=self.inp[k].dtype, pin_memory=True).copy_(self.inp[k].cpu())
+                     for k in keys]
+        self.sets = []
+        for b in range(2):
+            inp = dict(self.inp) if b == 0 else {k: (v.clone() if k in keys else v) for k, v in self.inp.items()}
+            topk, out = (self.topk, self.out) if b == 0 else (torch.empty_like(self.topk), torch.empty_like(self.out))
+            args, keep = self.hca.make_prefill_args(inp, self.csa_kv, self.csa_k, topk, out)
+            d_out = [topk, out]
+            self.sets.append({"args": args, "keep": (keep, inp), "d_in": [inp[k] for k in keys], "d_out": d_out,
+                              "h_out": [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]})
         self.h2d = sum(t.numel() * t.element_size() for t in self.h_in)
-        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.sets[0]["h_out"])
 
-    def e2e_step(self):
-        for h, d in zip(self.h_in, self.d_in):
-            d.copy_(h, non_blocking=True)
-        self.step(record=False)
-        for h, d in zip(self.h_out, self.d_out):
-            h.copy_(d, non_blocking=True)
+    def run_set(self, b):
+        self.hca.hybrid_attn_prefill(self.cfg, self.sets[b]["args"], ws=self.ws)
 
     def oracle_sample(self, n_q):
         import oracle
@@ -404,6 +422,54 @@ def timed_steps(bench, K, flush, rank, ws, device, record=True):
     return total, {p: v / K for p, v in phase_ms.items()}
 
 
+def e2e_pipelined(bench, K, device):
+    """K steps through the C ABI, each with the host->device copy of its inputs
+    from pinned memory and the device->host copy of its results, as a serving
+    loop runs them: copies on their own streams (one per direction), two device
+    buffer sets, so that step s+1's inputs arrive and step s-1's results leave
+    while step s computes.  Returns device ms per step (first copy to last copy,
+    CUDA events).  No L2 flush between steps: a step streams far more than the
+    L2 holds (the indexer keys alone are 512 MiB at 1M context)."""
+    main = torch.cuda.current_stream(device)
+    h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def load(s):
+        b = s % 2
+        with torch.cuda.stream(h2d):
+            if s >= 2:
+                h2d.wait_event(done[b])  # step s-2 has consumed this set's inputs
+            for h, d in zip(bench.h_in, bench.sets[b]["d_in"]):
+                d.copy_(h, non_blocking=True)
+            in_ready[b].record(h2d)
+
+    torch.cuda.synchronize(device)
+    start.record(main)
+    h2d.wait_event(start)
+    load(0)
+    for s in range(K):
+        b = s % 2
+        if s + 1 < K:
+            load(s + 1)
+        main.wait_event(in_ready[b])
+        if s >= 2:
+            main.wait_event(out_done[b])  # step s-2's results have left this set's outputs
+        bench.run_set(b)
+        done[b].record(main)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(done[b])
+            for h, d in zip(bench.sets[b]["h_out"], bench.sets[b]["d_out"]):
+                h.copy_(d, non_blocking=True)
+            out_done[b].record(d2h)
+    main.wait_stream(d2h)
+    main.wait_stream(h2d)
+    end.record(main)
+    torch.cuda.synchronize(device)
+    return start.elapsed_time(end) / K
+
+
 def run_ours(a):
     rank, local, ws = init_dist("nccl")
     torch.cuda.set_device(local)
@@ -439,19 +505,8 @@ def run_ours(a):
 
     # end to end through the C ABI with host buffers
     bench.e2e_setup()
-    for _ in range(2):
-        bench.e2e_step()
-    torch.cuda.synchronize()
-    s_ev = [torch.cuda.Event(enable_timing=True) for _ in range(a.steps)]
-    e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(a.steps)]
-    barrier(ws)
-    for i in range(a.steps):
-        flush.zero_()
-        s_ev[i].record()
-        bench.e2e_step()
-        e_ev[i].record()
-    torch.cuda.synchronize()
-    e2e_ms = reduce_max(sum(x.elapsed_time(y) for x, y in zip(s_ev, e_ev)), ws, device) / a.steps
+    e2e_ms = e2e_pipelined(bench, 2, device)  # warm-up
+    e2e_ms = reduce_max(e2e_pipelined(bench, a.steps, device), ws, device)
     e2e_value = bench.units * ws / (e2e_ms / 1e3)
 
     # roofline of the dominant kernel
@@ -487,8 +542,10 @@ def run_ours(a):
                           l2="flushed before every timed step (256 MiB write, outside the step's events)"),
            "e2e": {"value": round(e2e_value, 2), "unit": bench.unit, "h2d_bytes_per_step": bench.h2d,
                    "d2h_bytes_per_step": bench.d2h, "ms_per_step": round(e2e_ms, 4),
-                   "note": "per-step inputs (queries, windows, new block) from pinned host memory and outputs back; "
-                           "KV caches resident on the device"},
+                   "note": "every step copies its inputs (queries, indexer queries and weights, windows, new block) "
+                           "from pinned host memory and its outputs back, on copy streams that overlap the "
+                           "neighbouring steps' compute (two device buffer sets; no L2 flush: a step streams more "
+                           "than the L2 holds); KV caches resident on the device"},
            "gpu_launches": launches * a.steps,
            "phase_ms": {k: round(v, 4) for k, v in phase_ms.items()},
            "roofline": roof,
