@@ -101,7 +101,7 @@ struct IndexerPlan {
   long long ld;   // score row stride
   int chunk, chunks;
   size_t cand_off;  // chunked select: [Tq][chunks][k] composites
-  // decode select from the indexer's score histogram (N > kSelectMaxN):
+  // decode select from the indexer's score histogram (N > kSelectRowMaxN):
   int hist_ctas;    // select CTAs per request (kHistSlice entries each)
   size_t hist_off, done_off, cnt_off, above_off, eq_off;
   size_t bytes;
@@ -114,7 +114,7 @@ static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 IndexerPlan plan_indexer(int Tq, int N, int k) {
   IndexerPlan p;
   p.ld = ((long long)N + 3) / 4 * 4;
-  if (N <= kSelectMaxN) {
+  if (N <= kSelectRowMaxN) {
     p.chunk = N > 0 ? N : 1;
     p.chunks = 1;
   } else {
@@ -125,7 +125,7 @@ IndexerPlan plan_indexer(int Tq, int N, int k) {
   p.cand_off = align256(score_bytes);
   const size_t cand_bytes = p.chunks > 1 ? (size_t)Tq * p.chunks * k * sizeof(uint64_t) : 0;
   size_t end = p.cand_off + cand_bytes;
-  p.hist_ctas = N > kSelectMaxN ? (N + kHistSlice - 1) / kHistSlice : 0;
+  p.hist_ctas = N > kSelectRowMaxN ? (N + kHistSlice - 1) / kHistSlice : 0;
   p.hist_off = p.done_off = p.cnt_off = p.above_off = p.eq_off = 0;
   if (p.hist_ctas > 0) {
     const size_t C = (size_t)p.hist_ctas;
@@ -210,7 +210,7 @@ int run_indexer_topk(const bf16* q_idx, const float* w_idx, const bf16* k_idx, l
   rows.q_pos = q_pos;
   rows.ld_scores = p.ld;
   if (p.chunks == 1) {
-    CUDA_TRY(launch_select_from_scores(scores, rows, cfg->topk, topk_idx, nullptr, st), "select");
+    CUDA_TRY(launch_select_rows(scores, rows, cfg->topk, topk_idx, st), "select");
   } else {
     uint64_t* cand = reinterpret_cast<uint64_t*>(reinterpret_cast<char*>(ws) + p.cand_off);
     CUDA_TRY(launch_select_from_scores(scores, rows, cfg->topk, nullptr, cand, st), "select chunks");

@@ -19,7 +19,8 @@ cudaError_t launch_compress(const bf16* cand, int ld_cand, const bf16* logits, i
 
 // ---- topk.cu ----------------------------------------------------------------
 // Largest candidate-count a single select row may have (smem-resident).
-constexpr int kSelectMaxN = 24576;
+constexpr int kSelectMaxN = 24576;     // 64-bit composites staged in shared memory
+constexpr int kSelectRowMaxN = 49152;  // 32-bit score keys staged in shared memory (one row per CTA)
 
 // Row r of a score matrix: scores at scores + r*ld_scores (f32), its entry
 // indices are idx_base(r) + position; n(r) elements are candidates.
@@ -39,6 +40,10 @@ struct SelectRows {
 // (out_idx [rows, k], -1 padded) or composite candidates (out_cand [rows, k]).
 cudaError_t launch_select_from_scores(const float* scores, const SelectRows& rows, int k,
                                       int32_t* out_idx, uint64_t* out_cand, cudaStream_t stream);
+// Rows of at most kSelectRowMaxN visible entries, one CTA each (rows.chunks == 1):
+// final indices to out_idx [rows, k].
+cudaError_t launch_select_rows(const float* scores, const SelectRows& rows, int k, int32_t* out_idx,
+                               cudaStream_t stream);
 // Merge: row q has n_cand composite candidates at cand + q*n_cand; write the
 // top-k indices to out_idx [rows, k].
 cudaError_t launch_select_merge(const uint64_t* cand, int n_rows, int n_cand, int k,

@@ -186,6 +186,126 @@ __device__ void select_core(const uint64_t* s_c, int n, int k, int32_t* out_idx,
   }
 }
 
+// The same selection over 32-bit score keys staged in index order (the index is
+// the position): half the shared memory and at most four 8-bit passes.  Equal
+// keys keep index order, so ties still go to the lower index.
+template <int NT>
+__device__ void select_core32(const uint32_t* s_c, int n, int k, int idx_base, int32_t* out_idx) {
+  __shared__ int s_hist[256];
+  __shared__ int s_wsum[8];
+  __shared__ int s_bucket, s_greater;
+  __shared__ unsigned int s_min, s_max;
+  __shared__ int2 s_warp[NT / 32 + 1];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (n <= k) {
+    for (int e = tid; e < k; e += NT) out_idx[e] = e < n ? idx_base + e : -1;
+    return;
+  }
+
+  // range of the composites -> highest differing bit
+  unsigned int mn = ~0u, mx = 0u;
+  for (int e = tid; e < n; e += NT) {
+    const unsigned int c = s_c[e];
+    mn = c < mn ? c : mn;
+    mx = c > mx ? c : mx;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const unsigned int a = __shfl_xor_sync(0xffffffffu, mn, o);
+    const unsigned int b = __shfl_xor_sync(0xffffffffu, mx, o);
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
+  }
+  if (tid == 0) { s_min = ~0u; s_max = 0u; }
+  __syncthreads();
+  if (lane == 0) { atomicMin(&s_min, mn); atomicMax(&s_max, mx); }
+  __syncthreads();
+  const unsigned int cmin = s_min, cmax = s_max;
+  // n > k >= 1 distinct composites except for empty slots: cmin < cmax unless
+  // all are empty (then every slot is equal and any k of them will do)
+  int hi = cmin == cmax ? -1 : 31 - __clz((int)(cmin ^ cmax));
+  uint32_t prefix = hi >= 31 ? 0u : (cmin >> (hi + 1)) << (hi + 1);
+  int lo = hi + 1;  // lowest bit decided so far
+  int remaining = k;
+  while (hi >= 0) {
+    lo = hi >= 7 ? hi - 7 : 0;
+    const int width = hi - lo + 1;
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int b = tid; b < 256; b += NT) s_hist[b] = 0;
+    __syncthreads();
+    for (int e = tid; e < n; e += NT) {
+      const uint32_t c = s_c[e];
+      if (hi >= 31 || (c >> (hi + 1)) == (prefix >> (hi + 1))) atomicAdd(&s_hist[(int)((c >> lo) & dmask)], 1);
+    }
+    __syncthreads();
+    // suffix sums over the 256 bins: warps 0..7 hold 32 bins each
+    if (tid < 256) {
+      const int v = s_hist[tid];
+      int suf = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += y;
+      }
+      if (lane == 0) s_wsum[warp] = suf;
+      // publish after every warp wrote its total
+      asm volatile("bar.sync 3, 256;" ::: "memory");
+      int above = 0;
+      for (int w = warp + 1; w < 8; ++w) above += s_wsum[w];
+      suf += above;
+      const int nxt = suf - v;  // suffix of bin tid + 1
+      if (suf >= remaining && nxt < remaining) { s_bucket = tid; s_greater = nxt; }
+    }
+    __syncthreads();
+    const int b = s_bucket;
+    remaining -= s_greater;
+    prefix |= (uint32_t)b << lo;
+    const int cnt = s_hist[b];
+    __syncthreads();
+    hi = lo - 1;
+    if (cnt == remaining) break;
+  }
+  const int shift = lo;
+
+  // Output in candidate order: all above the threshold prefix, then the first
+  // `remaining` equal to it (only duplicates -- empty slots -- can tie here).
+  // Warp w owns the contiguous range [w*seg, (w+1)*seg); lanes read it 32
+  // consecutive candidates at a time (no bank conflicts), ranks come from
+  // ballots, warp offsets from a scan of the 32 warp totals.
+  const uint32_t P = prefix >> shift;
+  constexpr int NW = NT / 32;
+  const int seg = ((n + NW - 1) / NW + 31) / 32 * 32;
+  const int w0 = warp * seg, w1 = min(n, w0 + seg);
+  const unsigned lt = (1u << lane) - 1u;
+  int ng = 0, ne = 0;
+  for (int e = w0 + lane; e - lane < w1; e += 32) {
+    const uint32_t v = e < w1 ? (s_c[e] >> shift) : 0u;
+    ng += __popc(__ballot_sync(0xffffffffu, e < w1 && v > P));
+    ne += __popc(__ballot_sync(0xffffffffu, e < w1 && v == P));
+  }
+  int og, oe, tg, te;
+  // one thread per warp carries the warp's totals into the block scan
+  block_scan2<NT>(lane == 0 ? ng : 0, lane == 0 ? ne : 0, og, oe, tg, te, s_warp);
+  og = __shfl_sync(0xffffffffu, og, 0);
+  oe = __shfl_sync(0xffffffffu, oe, 0);
+  for (int e = w0 + lane; e - lane < w1; e += 32) {
+    const bool in = e < w1;
+    const uint32_t v = in ? (s_c[e] >> shift) : 0u;
+    const bool g = in && v > P, q = in && v == P;
+    const unsigned bg = __ballot_sync(0xffffffffu, g), bq = __ballot_sync(0xffffffffu, q);
+    int slot = -1;
+    if (g) slot = og + __popc(bg & lt);
+    if (q) {
+      const int r = oe + __popc(bq & lt);
+      if (r < remaining) slot = tg + r;
+    }
+    if (slot >= 0) out_idx[slot] = idx_base + e;
+    og += __popc(bg);
+    oe += __popc(bq);
+  }
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_scores_kernel(const float* __restrict__ scores,
                                                                     SelectRows rows, int k,
                                                                     int32_t* out_idx, uint64_t* out_cand) {
@@ -215,6 +335,32 @@ __global__ void __launch_bounds__(kSelThreads) select_scores_kernel(const float*
   __syncthreads();
   select_core<kSelThreads>(s_c, n, k, out_idx ? out_idx + (long long)r * k : nullptr,
                            out_cand ? out_cand + (long long)r * k : nullptr);
+}
+
+// One row per CTA with at most kSelectRowMaxN visible entries: stage the score
+// keys, select, write the final indices.
+__global__ void __launch_bounds__(kSelThreads) select_row_kernel(const float* __restrict__ scores, SelectRows rows,
+                                                                 int k, int32_t* out_idx) {
+  extern __shared__ uint32_t s_k[];
+  const int q = blockIdx.x;
+  const int n = n_visible(rows.q_pos[q], rows.rate, rows.N);
+  const float* sp = scores + (long long)q * rows.ld_scores;
+  // 8 independent loads in flight per thread before the shared-memory stores
+  for (int b0 = 0; b0 < n; b0 += 8 * kSelThreads) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = b0 + u * kSelThreads + (int)threadIdx.x;
+      v[u] = e < n ? sp[e] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = b0 + u * kSelThreads + (int)threadIdx.x;
+      if (e < n) s_k[e] = float_key(v[u]);
+    }
+  }
+  __syncthreads();
+  select_core32<kSelThreads>(s_k, n, k, 0, out_idx + (long long)q * k);
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_merge_kernel(const uint64_t* __restrict__ cand, int n_cand,
@@ -472,6 +618,17 @@ cudaError_t launch_select_from_scores(const float* scores, const SelectRows& row
   cudaError_t e = set_smem((const void*)select_scores_kernel, smem);
   if (e != cudaSuccess) return e;
   select_scores_kernel<<<rows.n_rows, kSelThreads, smem, stream>>>(scores, rows, k, out_idx, out_cand);
+  ++g_launch_counter;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_rows(const float* scores, const SelectRows& rows, int k, int32_t* out_idx,
+                               cudaStream_t stream) {
+  if (rows.n_rows == 0) return cudaSuccess;
+  const size_t smem = (size_t)(rows.N < kSelectRowMaxN ? rows.N : kSelectRowMaxN) * sizeof(uint32_t) + 16;
+  cudaError_t e = set_smem((const void*)select_row_kernel, smem);
+  if (e != cudaSuccess) return e;
+  select_row_kernel<<<rows.n_rows, kSelThreads, smem, stream>>>(scores, rows, k, out_idx);
   ++g_launch_counter;
   return cudaGetLastError();
 }

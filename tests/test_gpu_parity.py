@@ -136,16 +136,19 @@ def test_indexer_topk_decode_csa_128k(hca):
     assert swaps <= 32 * 8
 
 
-def test_indexer_topk_decode_threshold_ties(hca):
-    """Decode top-k when thousands of scores tie at the threshold.  Request 0: every
-    third key is the same vector and the rest are zero, so ~13,300 equal scores
-    compete for the 1024 places (ties go to the lower index).  Request 1: all keys
-    zero, so all 40,000 scores are equal -- more threshold candidates than one CTA
-    stages in shared memory.  Request 2: ordinary random keys."""
+@pytest.mark.parametrize("N", [40000, 60000])
+def test_indexer_topk_decode_threshold_ties(hca, N):
+    """Decode top-k when thousands of scores tie at the threshold, for a row that one
+    CTA selects from shared memory (40,000 entries) and for the histogram path
+    (60,000).  Request 0: every third key is the same vector and the rest are zero,
+    so N/3 equal scores compete for the 1024 places (ties go to the lower index).
+    Request 1: all keys zero, so all N scores are equal (on the histogram path, more
+    threshold candidates than one CTA stages in shared memory).  Request 2: ordinary
+    random keys."""
     s = wl.PRO
-    d = wl.csa_decode_inputs(s, B=3, ctx=4 * 40000, seed=11)
+    d = wl.csa_decode_inputs(s, B=3, ctx=4 * N, seed=11)
     K = d["K_I"].clone()
-    N = K.shape[1]
+    assert K.shape[1] == N
     K[0] = 0
     K[0, ::3] = d["K_I"][0, 7]
     K[1] = 0
