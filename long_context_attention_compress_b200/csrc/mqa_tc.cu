@@ -30,9 +30,9 @@
 //              significant bits); lazy rescale of the TMEM accumulators (only
 //              when a head's maximum grows by more than 2^8); the loads of the
 //              next tile; the final epilogue.
-// Row sums l_h come from an MMA of a ones matrix (held in TMEM as the A
-// operand) with P^T, so they use exactly the P that PV uses.
-// TMEM: S^T 64 columns, O^T 4 blocks x 64, l 64, ones 32.
+// Row sums l_h are warp reduce-scatter sums of exactly the bf16 P_hi + P_lo
+// that PV multiplies (kept per warp across tiles, rescaled with O).
+// TMEM: S^T 64 columns, O^T 4 blocks x 64.
 
 #include <cudaTypedefs.h>
 
@@ -61,7 +61,7 @@ constexpr uint32_t kKvBytes = kChunks * kKvChunk;    // 128 KiB
 constexpr uint32_t kBlockBytes = 2 * kKvChunk;       // 32 KiB
 constexpr uint32_t kPBytes = kRows * kH * 2;         // 16 KiB per P term
 constexpr uint32_t kOffQ = 0, kOffKv = kQBytes, kOffP = kOffKv + kKvBytes, kOffBars = kOffP + 2 * kPBytes;
-constexpr uint32_t kColS = 0, kColO = 64, kColL = 320, kColOnes = 384, kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColO = 64, kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.f;
 static_assert(kGroupsPerIssuer * kCompute * kIssueLanes * 4 == kRows, "issuers cover the tile");
 
@@ -131,6 +131,25 @@ __device__ __forceinline__ void rs_max_step(float (&a)[32], int lane) {
     const float keep = hi ? a[j + NV / 2] : a[j];
     a[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, O));
   }
+}
+template <int O, int NV>
+__device__ __forceinline__ void rs_sum_step(float (&a)[32], int lane) {
+  const bool hi = (lane & O) != 0;
+#pragma unroll
+  for (int j = 0; j < NV / 2; ++j) {
+    const float send = hi ? a[j] : a[j + NV / 2];
+    const float keep = hi ? a[j + NV / 2] : a[j];
+    a[j] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+  }
+}
+// Afterwards lane l holds the warp-wide sum of value l (31 shuffles).
+__device__ __forceinline__ float warp_sum32(float (&a)[32], int lane) {
+  rs_sum_step<16, 32>(a, lane);
+  rs_sum_step<8, 16>(a, lane);
+  rs_sum_step<4, 8>(a, lane);
+  rs_sum_step<2, 4>(a, lane);
+  rs_sum_step<1, 2>(a, lane);
+  return a[0];
 }
 // Afterwards lane l holds the warp-wide maximum of value l (31 shuffles).
 __device__ __forceinline__ float warp_max32(float (&a)[32], int lane) {
@@ -205,17 +224,6 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
-  if (warp >= 1 && warp <= 4) {
-    // ones matrix (A operand of the row-sum MMA) in TMEM: every lane, 32 columns of bf16 pairs 1.0
-    uint32_t ones[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) ones[j] = 0x3f803f80u;
-    tc::tmem_st32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + kColOnes, ones);
-    tc::tmem_st_wait();
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
 
   if (warp == 0) {
     // ------------------------------ MMA issuer ------------------------------
@@ -224,7 +232,6 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       for (int c = 0; c < kChunks; ++c) tc::tma_load_2d(base + kOffQ + c * kQChunk, &tm_q, &bars->qfull, c * 64, q * kH);
       constexpr uint32_t id_qk = tc::idesc_bf16_f32(kRows, kH, false, false);
       constexpr uint32_t id_pv = tc::idesc_bf16_f32(128, kH, true, true);
-      constexpr uint32_t id_l = tc::idesc_bf16_f32(128, kH, false, true);
       const uint32_t q_base = tc::smem_u32(base + kOffQ), kv_base = tc::smem_u32(base + kOffKv),
                      p_base = tc::smem_u32(base + kOffP);
       // Descriptors are built once; each K-step only adds a compile-time
@@ -234,7 +241,6 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       uint64_t v_desc0 = tc::sdesc_sw128(kv_base, kKvChunk, 1024);
       uint64_t p_hi0 = tc::sdesc_sw128(p_base, kPBytes, 1024);
       uint64_t p_lo0 = tc::sdesc_sw128(p_base + kPBytes, kPBytes, 1024);
-      const uint32_t ones = tmem + kColOnes;
       bool ok = tc::mbar_wait(&bars->qfull, 0, abort);
       for (int i = 0; ok && i < nt; ++i) {
         const uint32_t ph = i & 1;
@@ -266,10 +272,6 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
             const uint64_t ad = v_desc0 + (((2 * b) * kKvChunk) >> 4) + koff;
             tc::mma_bf16(tmem + kColO + b * kH, ad, p_hi0 + koff, id_pv, first);
             tc::mma_bf16(tmem + kColO + b * kH, ad, p_lo0 + koff, id_pv, 1u);
-            if (b == 0) {
-              tc::mma_bf16_ta(tmem + kColL, ones, p_hi0 + koff, id_l, first);
-              tc::mma_bf16_ta(tmem + kColL, ones, p_lo0 + koff, id_l, 1u);
-            }
           }
           tc::mma_commit(&bars->kvempty[b]);  // this block's columns of the tile may be reloaded
         }
@@ -350,6 +352,10 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     // Every named barrier below is reached by all compute threads on every
     // iteration; failures are agreed through bar.red.or before anyone leaves.
     bool failed = false;
+    // Row sums: lane l of this warp carries the sum over its quarter's rows of
+    // P[row, 32 hsel + l] (exactly the bf16 P_hi + P_lo that PV multiplies), over
+    // all tiles so far, relative to the running maxima.
+    float lw = 0.f;
     int y[4 * kGroupsPerIssuer];
     if (nt > 0) {
       gather_rows(0, y);
@@ -422,12 +428,13 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       // phase behind (PV(i) cannot complete before this group publishes P(i)).
       if (i > 0 && !tc::warp_wait(&bars->odone, (i - 1) & 1, abort)) failed = true;
       if (full) {
+        lw *= bars->alpha[32 * hsel + lane];
         if (!failed && bars->rescale && i > 0) {
-          // O^T and l hold the sums up to tile i-1: scale column h by alpha[h]
+          // O^T holds the sums up to tile i-1: scale column h by alpha[h]
           tc::fence_after_sync();
 #pragma unroll 1
-          for (int blk = 0; blk < 5; ++blk) {
-            const uint32_t ta = tmem + lanebase + (blk < 4 ? kColO + blk * kH : kColL) + 32 * hsel;
+          for (int blk = 0; blk < 4; ++blk) {
+            const uint32_t ta = tmem + lanebase + kColO + blk * kH + 32 * hsel;
             uint32_t v[32];
             tc::tmem_ld32(ta, v);
             tc::tmem_ld_wait();
@@ -459,6 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
           const float p1 = (m1 == neg_inf()) ? 0.f : fast_exp2(sv[h + 1] - m1);
           wh[j] = pack_bf16x2(p0, p1);
           wl[j] = pack_bf16x2(p0 - bf16_lo(wh[j]), p1 - bf16_hi(wh[j]));
+          sv[h] = bf16_lo(wh[j]) + bf16_lo(wl[j]);  // the probability PV uses (exact in f32)
+          sv[h + 1] = bf16_hi(wh[j]) + bf16_hi(wl[j]);
         }
         const uint32_t sw = (uint32_t)((c ^ (row & 7)) << 4);
         *reinterpret_cast<uint4*>(phi + sw) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
@@ -467,6 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&bars->pfull);
+      lw += warp_sum32(sv, lane);
       // next tile's rows, block by block as PV(i) releases them
       if (!failed && i + 1 < nt) {
         if (issue_tile(i + 1, y)) loaded = i + 2;
@@ -474,17 +484,19 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       }
     }
     // ---- epilogue: O^T (dims x heads) and l ----
-    bool ok = !failed;
+    // The four quarters' row-sum partials meet in shared memory.  Every compute
+    // thread reaches this barrier (the loop only ends together or normally) and
+    // it also settles, for all of them, whether a wait failed on the last tile.
+    bars->red[quarter][32 * hsel + lane] = lw;
+    bool ok = !tc::named_bar_or(1, 32 * kCompute, failed || *abort);
     if (ok && nt > 0) ok = tc::warp_wait(&bars->odone, (nt - 1) & 1, abort);
     if (ok) {
       tc::fence_after_sync();
       uint32_t lv[32];
-      if (nt > 0) {
-        tc::tmem_ld32(tmem + lanebase + kColL + 32 * hsel, lv);
-        tc::tmem_ld_wait();
-      } else {
 #pragma unroll
-        for (int h = 0; h < 32; ++h) lv[h] = 0u;
+      for (int h = 0; h < 32; ++h) {
+        const int hh = 32 * hsel + h;
+        lv[h] = __float_as_uint((bars->red[0][hh] + bars->red[1][hh]) + (bars->red[2][hh] + bars->red[3][hh]));
       }
       const int dim_lane = quarter * 32 + lane;
       if (p.splits == 1) {
