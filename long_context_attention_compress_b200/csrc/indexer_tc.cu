@@ -22,6 +22,8 @@
 
 #include <cudaTypedefs.h>
 
+#include <cstddef>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -248,16 +250,18 @@ constexpr int kPN = kPQ * kHeads;            // 256 = MMA N
 constexpr uint32_t kPQBytes = kPN * kDim * 2;        // 64 KiB
 constexpr uint32_t kPQChunkBytes = kPN * 128;        // 32 KiB
 constexpr int kPAcc = 2;
-constexpr int kPThreads = 192;
-struct __align__(8) PBars {
+constexpr int kPThreads = 320;  // producer, MMA, 8 epilogue warps (two per TMEM lane quarter)
+struct __align__(16) PBars {
+  float w[kPN];  // first: read with 16-byte vector loads
+  int nvis[kPQ];
   uint64_t full[kPStages], empty[kPStages];
   uint64_t tfull[kPAcc], tempty[kPAcc];
   uint64_t qfull, qempty, drain;
   uint32_t tmem_base;
   int abort;
-  float w[kPN];
-  int nvis[kPQ];
 };
+static_assert(offsetof(PBars, w) % 16 == 0 && offsetof(PBars, full) % 8 == 0, "PBars alignment");
+static_assert((kPStages * kTileBytes + kPQBytes) % 16 == 0, "PBars starts 16-byte aligned");
 constexpr size_t kPSmemBytes = 1024 + kPStages * kTileBytes + kPQBytes + sizeof(PBars);
 }  // namespace
 
@@ -286,7 +290,7 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPStages; ++s) { tc::mbar_init(&bars->full[s], 1); tc::mbar_init(&bars->empty[s], 1); }
-    for (int a = 0; a < kPAcc; ++a) { tc::mbar_init(&bars->tfull[a], 1); tc::mbar_init(&bars->tempty[a], 4); }
+    for (int a = 0; a < kPAcc; ++a) { tc::mbar_init(&bars->tfull[a], 1); tc::mbar_init(&bars->tempty[a], 8); }
     tc::mbar_init(&bars->qfull, 1);
     tc::mbar_init(&bars->qempty, 1);
     tc::mbar_init(&bars->drain, 1);
@@ -359,18 +363,20 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
     }
     __syncwarp();
   } else {
-    // epilogue: warps 2..5, one TMEM lane (= entry) per thread
+    // epilogue: warps 2..9, one TMEM lane (= entry) per thread; the two warps of a
+    // lane quarter score two of the group's four queries each
     const int lq = warp & 3;
     const int row_in_tile = lq * 32 + lane;
-    const int et = threadIdx.x - 64;  // 0..127
+    const int et = threadIdx.x - 64;  // 0..255
+    const int j0 = 2 * ((warp - 2) >> 2);
     int it = 0;
     bool failed = false;
     for (int g = n_groups - 1 - (int)blockIdx.x; g >= 0; g -= (int)gridDim.x) {
       const int nt = group_tiles(g);
       if (nt == 0) continue;
       // stage this group's weights and visible counts (the previous group's readers are done)
-      tc::named_bar(1, 128);
-      for (int e = et; e < kPN; e += 128) {
+      tc::named_bar(1, 256);
+      for (int e = et; e < kPN; e += 256) {
         const int q = g * kPQ + e / kHeads;
         bars->w[e] = q < Tq ? w_idx[(long long)q * kHeads + (e % kHeads)] : 0.f;
       }
@@ -378,16 +384,17 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
         const int q = g * kPQ + et;
         bars->nvis[et] = q < Tq ? n_visible(q_pos[q], rate, N) : 0;
       }
-      tc::named_bar(1, 128);
+      tc::named_bar(1, 256);
       for (int t = 0; t < nt; ++t, ++it) {
         const int a = it % kPAcc;
         if (!failed) failed = !tc::warp_wait(&bars->tfull[a], (it / kPAcc) & 1, abort);
         if (failed) continue;
         tc::fence_after_sync();
         const int e = t * kTile + row_in_tile;
-        float sc[kPQ];
+        float sc[2];
 #pragma unroll
-        for (int j = 0; j < kPQ; ++j) {
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = j0 + jj;
           uint32_t v[kHeads];
           const uint32_t taddr = tmem + ((uint32_t)(lq * 32) << 16) + a * kPN + j * kHeads;
           tc::tmem_ld32(taddr, v);
@@ -403,15 +410,15 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
             s0 = fmaf(wv.z, fmaxf(__uint_as_float(v[h + 2]), 0.f), s0);
             s1 = fmaf(wv.w, fmaxf(__uint_as_float(v[h + 3]), 0.f), s1);
           }
-          sc[j] = s0 + s1;
+          sc[jj] = s0 + s1;
         }
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&bars->tempty[a]);
 #pragma unroll
-        for (int j = 0; j < kPQ; ++j) {
-          const int q = g * kPQ + j;
-          if (q < Tq && e < bars->nvis[j]) scores[(long long)q * ld_scores + e] = sc[j];
+        for (int jj = 0; jj < 2; ++jj) {
+          const int q = g * kPQ + j0 + jj;
+          if (q < Tq && e < bars->nvis[j0 + jj]) scores[(long long)q * ld_scores + e] = sc[jj];
         }
       }
     }
