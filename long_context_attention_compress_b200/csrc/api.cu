@@ -671,7 +671,7 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
                          sched.overlap ? sched.sms - sched.r_hca : 0);
     if (s != HCA_OK) return s;
     MqaProblem p = decode_csa_problem(cfg, a);
-    CUDA_TRY(launch_mqa(p, sched.csa_pl, ws, st), "decode: csa attention");
+    CUDA_TRY(launch_mqa(p, sched.csa_pl, ws, st, true), "decode: csa attention");
     if ((s = mark()) != HCA_OK) return s;
   }
   if (a->hca_q) {
@@ -772,7 +772,7 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
   {
     MqaProblem p = make_mqa(cfg, a->q, a->csa_kv, 0, Nc, a->topk_idx, cfg->topk, cfg->m, a->cand, T, a->q_pos, T,
                             HCA_MODE_PREFILL, a->csa_out);
-    CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "prefill: csa attention");
+    CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st, true), "prefill: csa attention");
     if ((s = mark()) != HCA_OK) return s;
   }
   if (a->hca_kv) {

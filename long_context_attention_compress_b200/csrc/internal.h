@@ -27,6 +27,25 @@ constexpr int kSelectRowMaxN = 49152;  // 32-bit score keys staged in shared mem
 // Two ways to describe rows:
 //   by query: row = query q (r = q), n = min(n_visible(q_pos[q]), N) - chunk0
 //   by chunk: row = (q, j), scores + q*ld + j*chunk, n = clamp(nvis - j*chunk, 0, chunk)
+// Launch, optionally with programmatic stream serialisation: the kernel may then
+// start while the previous kernel of the stream finishes; it must call
+// griddep_wait() (tc.cuh) before touching anything an earlier kernel writes or reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(bool pdl, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 struct SelectRows {
   int n_rows;       // number of rows
   int chunks;       // chunks per query (rows = Tq * chunks)
@@ -120,18 +139,21 @@ struct MqaPlan {
   size_t ws_bytes;
 };
 // plan_mqa / launch_mqa pick the tensor-core kernel when it supports the problem.
+// pdl: launch it (and its combine) as programmatic dependents of the previous
+// kernel of the stream (the caller's top-k); off for work started from events.
 MqaPlan plan_mqa(const MqaProblem& p);
 MqaPlan plan_mqa_sms(const MqaProblem& p, int sms);  // one wave of at most `sms` CTAs
 MqaPlan plan_mqa_cuda_cores(const MqaProblem& p);
 size_t mqa_ws_upper_bound(const MqaProblem& p);  // any idx / stride / mode, rows up to max(N, n_idx)
-cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& plan, void* ws, cudaStream_t stream);
+cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& plan, void* ws, cudaStream_t stream, bool pdl = false);
 cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out,
-                               cudaStream_t stream);
+                               cudaStream_t stream,
+                               bool pdl = false);
 
 // ---- mqa_tc.cu (tcgen05) -------------------------------------------------------------
 bool mqa_tc_supported(const MqaProblem& p);
 MqaPlan plan_mqa_tc(const MqaProblem& p, int num_sms);
-cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream);
+cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream, bool pdl);
 unsigned int read_and_clear_mqa_tc_error();
 
 }  // namespace hca

@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace hca {
 
@@ -200,6 +201,7 @@ __global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restric
                                                           const float2* __restrict__ ws_ml, int splits,
                                                           int H, int C, bf16* __restrict__ out) {
   __shared__ float s_w[kCombHeads][kCombMaxSplits];
+  tc::griddep_wait();  // the partial states come from the attention kernel
   const int q = blockIdx.x, h0 = blockIdx.y * kCombHeads;
   const int nh = min(kCombHeads, H - h0);
   // weights: thread hh*64 + lane-group handles head hh
@@ -269,8 +271,10 @@ static size_t mqa_smem() {
 }
 
 cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out,
-                               cudaStream_t stream) {
-  mqa_combine_kernel<<<dim3(Tq, (H + kCombHeads - 1) / kCombHeads), 256, 0, stream>>>(ws_o, ws_ml, splits, H, C, out);
+                               cudaStream_t stream, bool pdl) {
+  cudaError_t e = launch_pdl(pdl, mqa_combine_kernel, dim3(Tq, (H + kCombHeads - 1) / kCombHeads), dim3(256), 0,
+                             stream, ws_o, ws_ml, splits, H, C, out);
+  if (e != cudaSuccess) return e;
   ++g_launch_counter;
   return cudaGetLastError();
 }
@@ -341,9 +345,9 @@ static cudaError_t launch_mqa_t(const MqaProblem& p, const MqaPlan& pl, void* ws
   return cudaGetLastError();
 }
 
-cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream) {
+cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream, bool pdl) {
   if (p.Tq == 0) return cudaSuccess;
-  if (mqa_tc_supported(p)) return launch_mqa_decode_tc(p, pl, ws, stream);
+  if (mqa_tc_supported(p)) return launch_mqa_decode_tc(p, pl, ws, stream, pdl);
   if (p.H == 64 && p.c == 512) return launch_mqa_t<64, 512>(p, pl, ws, stream);
   if (p.H == 4 && p.c == 64) return launch_mqa_t<4, 64>(p, pl, ws, stream);
   return cudaErrorInvalidValue;

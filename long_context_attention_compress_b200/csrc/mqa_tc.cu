@@ -224,12 +224,18 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
+  tc::griddep_launch_dependents();
+  // The queries are a call input: their load may start before the previous kernel
+  // (the top-k) has finished; everything else waits for it.
+  if (warp == 0 && lane == 0) {
+    tc::mbar_arrive_expect_tx(&bars->qfull, kQBytes);
+    for (int c = 0; c < kChunks; ++c) tc::tma_load_2d(base + kOffQ + c * kQChunk, &tm_q, &bars->qfull, c * 64, q * kH);
+  }
+  tc::griddep_wait();
 
   if (warp == 0) {
     // ------------------------------ MMA issuer ------------------------------
     if (lane == 0) {
-      tc::mbar_arrive_expect_tx(&bars->qfull, kQBytes);
-      for (int c = 0; c < kChunks; ++c) tc::tma_load_2d(base + kOffQ + c * kQChunk, &tm_q, &bars->qfull, c * 64, q * kH);
       constexpr uint32_t id_qk = tc::idesc_bf16_f32(kRows, kH, false, false);
       constexpr uint32_t id_pv = tc::idesc_bf16_f32(128, kH, true, true);
       const uint32_t q_base = tc::smem_u32(base + kOffQ), kv_base = tc::smem_u32(base + kOffKv),
@@ -590,7 +596,7 @@ MqaPlan plan_mqa_tc(const MqaProblem& p, int num_sms) {
 extern cudaError_t make_tmap_bf16(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
                                   const uint64_t* strides_bytes, uint32_t box_rows);
 
-cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream) {
+cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream, bool pdl) {
   if (p.Tq == 0) return cudaSuccess;
   CUtensorMap tm_q, tm_kv, tm_kvg, tm_win;
   const uint64_t rstride[1] = {(uint64_t)kC * 2};
@@ -638,11 +644,12 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   e = cudaFuncSetAttribute((const void*)mqa_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  mqa_decode_tc_kernel<<<p.Tq * pl.splits, kThreads, kSmemBytes, stream>>>(tm_q, tm_kv, tm_kvg, tm_win, a);
+  e = launch_pdl(pdl, mqa_decode_tc_kernel, dim3(p.Tq * pl.splits), dim3(kThreads), kSmemBytes, stream, tm_q, tm_kv,
+                 tm_kvg, tm_win, a);
   ++g_launch_counter;
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;
-  return launch_mqa_combine(a.ws_o, a.ws_ml, p.Tq, pl.splits, kH, kC, p.out, stream);
+  return launch_mqa_combine(a.ws_o, a.ws_ml, p.Tq, pl.splits, kH, kC, p.out, stream, pdl);
 }
 
 unsigned int read_and_clear_mqa_tc_error() {

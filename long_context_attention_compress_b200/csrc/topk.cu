@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace hca {
 
@@ -310,6 +311,8 @@ __global__ void __launch_bounds__(kSelThreads) select_scores_kernel(const float*
                                                                     SelectRows rows, int k,
                                                                     int32_t* out_idx, uint64_t* out_cand) {
   extern __shared__ uint64_t s_c[];
+  tc::griddep_launch_dependents();
+  tc::griddep_wait();  // the scores come from the previous kernel
   const int r = blockIdx.x;
   const int q = r / rows.chunks;
   const int j = r % rows.chunks;
@@ -342,6 +345,8 @@ __global__ void __launch_bounds__(kSelThreads) select_scores_kernel(const float*
 __global__ void __launch_bounds__(kSelThreads) select_row_kernel(const float* __restrict__ scores, SelectRows rows,
                                                                  int k, int32_t* out_idx) {
   extern __shared__ uint32_t s_k[];
+  tc::griddep_launch_dependents();
+  tc::griddep_wait();  // the scores come from the previous kernel
   const int q = blockIdx.x;
   const int n = n_visible(rows.q_pos[q], rows.rate, rows.N);
   const float* sp = scores + (long long)q * rows.ld_scores;
@@ -366,6 +371,8 @@ __global__ void __launch_bounds__(kSelThreads) select_row_kernel(const float* __
 __global__ void __launch_bounds__(kSelThreads) select_merge_kernel(const uint64_t* __restrict__ cand, int n_cand,
                                                                    int k, int32_t* out_idx) {
   extern __shared__ uint64_t s_c[];
+  tc::griddep_launch_dependents();
+  tc::griddep_wait();  // the candidates come from the previous kernel
   const int r = blockIdx.x;
   const uint64_t* cp = cand + (long long)r * n_cand;
   for (int b0 = 0; b0 < n_cand; b0 += 8 * kSelThreads) {
@@ -422,6 +429,8 @@ __global__ void __launch_bounds__(kSelThreads) select_hist_kernel(HistSelect a) 
   __shared__ int2 s_cnt[kHistMaxCtas];
   __shared__ int2 s_off[kHistMaxCtas + 1];
   __shared__ uint64_t s_tie[32];
+  tc::griddep_launch_dependents();
+  tc::griddep_wait();  // scores and histograms come from the indexer
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = blockIdx.x / a.C, c = blockIdx.x % a.C;
   const int k = a.k;
@@ -617,7 +626,9 @@ cudaError_t launch_select_from_scores(const float* scores, const SelectRows& row
   const size_t smem = (size_t)rows.chunk * sizeof(uint64_t);
   cudaError_t e = set_smem((const void*)select_scores_kernel, smem);
   if (e != cudaSuccess) return e;
-  select_scores_kernel<<<rows.n_rows, kSelThreads, smem, stream>>>(scores, rows, k, out_idx, out_cand);
+  e = launch_pdl(true, select_scores_kernel, dim3(rows.n_rows), dim3(kSelThreads), smem, stream, scores, rows, k,
+                 out_idx, out_cand);
+  if (e != cudaSuccess) return e;
   ++g_launch_counter;
   return cudaGetLastError();
 }
@@ -628,7 +639,9 @@ cudaError_t launch_select_rows(const float* scores, const SelectRows& rows, int 
   const size_t smem = (size_t)(rows.N < kSelectRowMaxN ? rows.N : kSelectRowMaxN) * sizeof(uint32_t) + 16;
   cudaError_t e = set_smem((const void*)select_row_kernel, smem);
   if (e != cudaSuccess) return e;
-  select_row_kernel<<<rows.n_rows, kSelThreads, smem, stream>>>(scores, rows, k, out_idx);
+  e = launch_pdl(true, select_row_kernel, dim3(rows.n_rows), dim3(kSelThreads), smem, stream, scores, rows, k,
+                 out_idx);
+  if (e != cudaSuccess) return e;
   ++g_launch_counter;
   return cudaGetLastError();
 }
@@ -639,7 +652,8 @@ cudaError_t launch_select_merge(const uint64_t* cand, int n_rows, int n_cand, in
   const size_t smem = (size_t)n_cand * sizeof(uint64_t);
   cudaError_t e = set_smem((const void*)select_merge_kernel, smem);
   if (e != cudaSuccess) return e;
-  select_merge_kernel<<<n_rows, kSelThreads, smem, stream>>>(cand, n_cand, k, out_idx);
+  e = launch_pdl(true, select_merge_kernel, dim3(n_rows), dim3(kSelThreads), smem, stream, cand, n_cand, k, out_idx);
+  if (e != cudaSuccess) return e;
   ++g_launch_counter;
   return cudaGetLastError();
 }
@@ -650,7 +664,8 @@ cudaError_t launch_select_hist(const HistSelect& a, int B, cudaStream_t stream) 
   const size_t smem = (size_t)kSelectMaxN * sizeof(uint64_t);
   cudaError_t e = set_smem((const void*)select_hist_kernel, smem);
   if (e != cudaSuccess) return e;
-  select_hist_kernel<<<B * a.C, kSelThreads, smem, stream>>>(a);
+  e = launch_pdl(true, select_hist_kernel, dim3(B * a.C), dim3(kSelThreads), smem, stream, a);
+  if (e != cudaSuccess) return e;
   ++g_launch_counter;
   return cudaGetLastError();
 }
