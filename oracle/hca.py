@@ -210,19 +210,30 @@ def mqa_partial(q: np.ndarray, rows: np.ndarray, scale: float):
     return mx, np.sum(e, axis=1), e @ rows
 
 
-def mqa_attend(q: np.ndarray, rows: np.ndarray, scale: float) -> np.ndarray:
-    """o_h = sum_u softmax_u(scale * q_h . rows_u) rows_u; q [H, c], rows [U, c]."""
+def mqa_attend(q: np.ndarray, rows: np.ndarray, scale: float, sink=None) -> np.ndarray:
+    """o_h = sum_u softmax_u(scale * q_h . rows_u) rows_u; q [H, c], rows [U, c].
+
+    sink [H] (optional): a learnable logit per head added to the softmax
+    denominator only, so that the weights of the rows may sum to less than one
+    ([QbitAI] "混合注意力機制", attention-sink paragraph; [Tricks] "Partial RoPE
+    和 Attention Sink"):  o_h = sum_u e^{s_hu} rows_u / (e^{z_h} + sum_u e^{s_hu}).
+    """
     mx, l, o = mqa_partial(q, rows, scale)
+    if sink is not None:
+        l = l + np.exp(np.asarray(sink, dtype=np.float64) - mx)
     return o / l[:, None]
 
 
-def combine_partials(parts) -> np.ndarray:
+def combine_partials(parts, sink=None) -> np.ndarray:
     """Merge softmax states of disjoint row subsets:
-    o = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i, M = max_i m_i."""
+    o = sum_i e^{m_i - M} o_i / (sum_i e^{m_i - M} l_i [+ e^{z - M}]), M = max_i m_i
+    (the sink logit z, if any, enters the denominator once, not per subset)."""
     ms = np.stack([p[0] for p in parts])          # [P, H]
     M = np.max(ms, axis=0)
     num = sum(np.exp(p[0] - M)[:, None] * p[2] for p in parts)
     den = sum(np.exp(p[0] - M) * p[1] for p in parts)
+    if sink is not None:
+        den = den + np.exp(np.asarray(sink, dtype=np.float64) - M)
     return num / den[:, None]
 
 
@@ -230,7 +241,7 @@ def combine_partials(parts) -> np.ndarray:
 # whole layers
 # ----------------------------------------------------------------------------
 def csa_layer_prefill(cand, logits, kidx_cand, pos_bias, q_idx, w_idx, q, *,
-                      m, topk, d_idx, n_win, scale, queries=None):
+                      m, topk, d_idx, n_win, scale, queries=None, sink=None):
     """CSA layer over one sequence of T raw tokens, for the given query positions.
 
     cand/logits [T, c]; kidx_cand [T, d_I] (per-token indexer-key candidates,
@@ -256,11 +267,11 @@ def csa_layer_prefill(cand, logits, kidx_cand, pos_bias, q_idx, w_idx, q, *,
         res["idx"][t] = sel
         res["scores"][t] = sc
         res["n_vis"][t] = nv
-        res["O"][t] = mqa_attend(q[t], rows, scale)
+        res["O"][t] = mqa_attend(q[t], rows, scale, sink)
     return res
 
 
-def hca_layer_prefill(cand, logits, pos_bias, q, *, m_hca, n_win, scale, queries=None):
+def hca_layer_prefill(cand, logits, pos_bias, q, *, m_hca, n_win, scale, queries=None, sink=None):
     """HCA layer over one sequence: dense attention over every visible HCA
     entry plus the sliding window ([Tricks] HCA section: no top-k selector)."""
     T = cand.shape[0]
@@ -273,11 +284,11 @@ def hca_layer_prefill(cand, logits, pos_bias, q, *, m_hca, n_win, scale, queries
         nv = n_visible(t, m_hca, N)
         rows = np.concatenate([E[:nv], cand64[window_rows(t, n_win)]], axis=0)
         res["n_vis"][t] = nv
-        res["O"][t] = mqa_attend(q[t], rows, scale)
+        res["O"][t] = mqa_attend(q[t], rows, scale, sink)
     return res
 
 
-def csa_layer_decode(E, K_I, win, q, q_idx, w_idx, t, *, m, topk, n_win, scale):
+def csa_layer_decode(E, K_I, win, q, q_idx, w_idx, t, *, m, topk, n_win, scale, sink=None):
     """One decode query of one request against its CSA cache.
 
     E [N, c] compressed entries, K_I [N, d_I] indexer keys, win [n_win, c]
@@ -290,10 +301,10 @@ def csa_layer_decode(E, K_I, win, q, q_idx, w_idx, t, *, m, topk, n_win, scale):
     nw = min(n_win, t + 1)
     rows = np.concatenate([np.asarray(E, dtype=np.float64)[sel],
                            np.asarray(win, dtype=np.float64)[:nw]], axis=0)
-    return {"idx": sel, "scores": sc, "n_vis": nv, "O": mqa_attend(q, rows, scale)}
+    return {"idx": sel, "scores": sc, "n_vis": nv, "O": mqa_attend(q, rows, scale, sink)}
 
 
-def hca_layer_decode(E_h, block_cand, block_logits, pos_bias, win, q, t, *, m_hca, n_win, scale):
+def hca_layer_decode(E_h, block_cand, block_logits, pos_bias, win, q, t, *, m_hca, n_win, scale, sink=None):
     """One decode query of one request against its HCA cache, including the
     compression of the newest complete block ([Report] section 5 and [Jiedu]
     cache layout: the tail block is kept raw until it completes).
@@ -309,4 +320,4 @@ def hca_layer_decode(E_h, block_cand, block_logits, pos_bias, win, q, t, *, m_hc
     Eh = np.concatenate([np.asarray(E_h, dtype=np.float64)[:n - 1], new], axis=0)
     nw = min(n_win, t + 1)
     rows = np.concatenate([Eh, np.asarray(win, dtype=np.float64)[:nw]], axis=0)
-    return {"new_entry": new[0], "O": mqa_attend(q, rows, scale)}
+    return {"new_entry": new[0], "O": mqa_attend(q, rows, scale, sink)}

@@ -72,3 +72,17 @@ def attend(q_heads, rows, scale):
         tot = sum(es)
         out.append([sum(es[u] / tot * rows[u][d] for u in range(len(rows))) for d in range(len(qh))])
     return out
+
+
+def attend_with_sink_row(q_heads, rows, scale, sink):
+    """The sink as one more row: logit sink[h] for head h and an all-zero value, in
+    an ordinary softmax over U + 1 rows (loops only)."""
+    out = []
+    for h, qh in enumerate(q_heads):
+        logits = [scale * sum(a * b for a, b in zip(qh, r)) for r in rows] + [sink[h]]
+        values = [list(r) for r in rows] + [[0.0] * len(qh)]
+        mx = max(logits)
+        es = [math.exp(x - mx) for x in logits]
+        tot = sum(es)
+        out.append([sum(es[u] / tot * values[u][d] for u in range(len(values))) for d in range(len(qh))])
+    return out

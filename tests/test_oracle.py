@@ -301,6 +301,54 @@ def test_split_combine_equals_unsplit(cuts):
 
 
 # --------------------------------------------------------------------------
+# attention sink: one logit per head in the softmax denominator only
+# ([QbitAI] "混合注意力機制", attention-sink paragraph; [Tricks] "Partial RoPE 和
+# Attention Sink")
+# --------------------------------------------------------------------------
+def test_sink_at_minus_infinity_is_plain_attention():
+    rng = np.random.default_rng(40)
+    q, rows = _rand(rng, 4, 8), _rand(rng, 17, 8)
+    np.testing.assert_array_equal(oracle.mqa_attend(q, rows, 0.5, sink=np.full(4, -np.inf)),
+                                  oracle.mqa_attend(q, rows, 0.5))
+
+
+def test_sink_with_one_row_is_a_sigmoid():
+    from scipy.special import expit
+    rng = np.random.default_rng(41)
+    q, row = _rand(rng, 5, 8) * 2, _rand(rng, 1, 8)
+    z = rng.standard_normal(5)
+    s = 0.5 * (q @ row[0])
+    np.testing.assert_allclose(oracle.mqa_attend(q, row, 0.5, sink=z), expit(s - z)[:, None] * row, atol=1e-14)
+
+
+def test_sink_equals_an_extra_zero_valued_row():
+    rng = np.random.default_rng(42)
+    q, rows = _rand(rng, 3, 6) * 2, _rand(rng, 11, 6)
+    z = rng.standard_normal(3) + 1.0
+    np.testing.assert_allclose(oracle.mqa_attend(q, rows, 0.6, sink=z),
+                               bf.attend_with_sink_row(q.tolist(), rows.tolist(), 0.6, z.tolist()), atol=1e-13)
+
+
+@pytest.mark.parametrize("cuts", [[5], [1, 2, 30]])
+def test_sink_split_combine_equals_unsplit(cuts):
+    rng = np.random.default_rng(43)
+    q, rows = _rand(rng, 4, 8) * 3, _rand(rng, 40, 8)
+    z = rng.standard_normal(4) * 3
+    bounds = [0] + cuts + [40]
+    parts = [oracle.mqa_partial(q, rows[a:b], 0.5) for a, b in zip(bounds[:-1], bounds[1:])]
+    np.testing.assert_allclose(oracle.combine_partials(parts, sink=z), oracle.mqa_attend(q, rows, 0.5, sink=z),
+                               atol=1e-13)
+
+
+def test_a_dominant_sink_silences_the_head():
+    rng = np.random.default_rng(44)
+    q, rows = _rand(rng, 2, 8), _rand(rng, 9, 8)
+    o = oracle.mqa_attend(q, rows, 0.5, sink=np.array([500.0, -np.inf]))
+    assert np.all(np.abs(o[0]) < 1e-200)
+    np.testing.assert_array_equal(o[1], oracle.mqa_attend(q, rows, 0.5)[1])
+
+
+# --------------------------------------------------------------------------
 # whole layers on the tiny shape
 # --------------------------------------------------------------------------
 @pytest.fixture(scope="module")
