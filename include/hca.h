@@ -188,13 +188,18 @@ int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hc
  *   q [Tq, H, c] bf16; kv: request r's entries at kv + r*kv_seq_stride, [N, c];
  *   idx [Tq, n_idx] int32 (entries < N, visible to the query; -1 = empty slot);
  *   out [Tq, H, c] bf16.  Logits, softmax and sums in f32.
+ *   sink: NULL, or [H] f32 (device) learnable sink logits, one per head, in the
+ *   units of scale * q . row: they join the softmax denominator only,
+ *     o[t, h, :] = sum_u e^{s_u} row_u / (e^{sink[h]} + sum_u e^{s_u})
+ *   ([QbitAI] attention-sink paragraph; [Tricks] "Partial RoPE 和 Attention
+ *   Sink"), once per query also when the rows are split over CTAs.
  *   ws: hca_workspace_size(HCA_OP_SPARSE_MQA, cfg, Tq, N, mode) (split-K partials).
  * ------------------------------------------------------------------------- */
 int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N,
                       const int32_t* idx, int n_idx, int rate, const hca_bf16* win,
                       long long win_seq_stride, const int32_t* q_pos, int Tq, int mode,
-                      const hca_layer_cfg* cfg, hca_bf16* out, void* ws, size_t ws_bytes,
-                      void* stream);
+                      const hca_layer_cfg* cfg, const float* sink, hca_bf16* out, void* ws,
+                      size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * hybrid_attn_decode -- one decode step of a CSA layer and/or an HCA layer for
@@ -236,6 +241,8 @@ typedef struct {
   hca_bf16* hca_out;          /* [B, H, c] out */
   void* const* events;
   int n_events;
+  const float* csa_sink;      /* [H] sink logits of the CSA layer, or NULL (see sparse_mqa_attend) */
+  const float* hca_sink;      /* [H] sink logits of the HCA layer, or NULL */
 } hca_decode_args;
 
 int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* args, void* ws,
@@ -270,6 +277,8 @@ typedef struct {
   hca_bf16* hca_out;          /* [T, H, c] out */
   void* const* events;
   int n_events;
+  const float* csa_sink;      /* [H] sink logits of the CSA layer, or NULL (see sparse_mqa_attend) */
+  const float* hca_sink;      /* [H] sink logits of the HCA layer, or NULL */
 } hca_prefill_args;
 
 int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* args, void* ws,

@@ -52,7 +52,7 @@ class DecodeArgs(ctypes.Structure):
                 ("hca_q", c_void_p), ("hca_kv", c_void_p), ("hca_N", c_int), ("hca_kv_stride", c_ll),
                 ("hca_block_cand", c_void_p), ("hca_block_logits", c_void_p), ("hca_block_stride", c_ll),
                 ("hca_pos_bias", c_void_p), ("hca_win", c_void_p), ("hca_win_stride", c_ll), ("hca_out", c_void_p),
-                ("events", c_void_p), ("n_events", c_int)]
+                ("events", c_void_p), ("n_events", c_int), ("csa_sink", c_void_p), ("hca_sink", c_void_p)]
 
 
 class PrefillArgs(ctypes.Structure):
@@ -60,7 +60,8 @@ class PrefillArgs(ctypes.Structure):
                 ("kidx_cand", c_void_p), ("bias_csa", c_void_p), ("q_idx", c_void_p), ("w_idx", c_void_p),
                 ("q", c_void_p), ("csa_kv", c_void_p), ("csa_k_idx", c_void_p), ("topk_idx", c_void_p),
                 ("csa_out", c_void_p), ("bias_hca", c_void_p), ("hca_q", c_void_p), ("hca_kv", c_void_p),
-                ("hca_out", c_void_p), ("events", c_void_p), ("n_events", c_int)]
+                ("hca_out", c_void_p), ("events", c_void_p), ("n_events", c_int), ("csa_sink", c_void_p),
+                ("hca_sink", c_void_p)]
 
 
 def _sig(name, restype, argtypes):
@@ -77,8 +78,8 @@ _hca_compress = _sig("hca_compress", c_int, [c_void_p, c_int, c_void_p, c_int, c
 _indexer = _sig("csa_indexer_topk", c_int, [c_void_p, c_void_p, c_void_p, c_ll, c_int, c_void_p, c_int, c_int,
                                             ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_size, c_void_p])
 _mqa = _sig("sparse_mqa_attend", c_int, [c_void_p, c_void_p, c_ll, c_int, c_void_p, c_int, c_int, c_void_p, c_ll,
-                                         c_void_p, c_int, c_int, ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_size,
-                                         c_void_p])
+                                         c_void_p, c_int, c_int, ctypes.POINTER(LayerCfg), c_void_p, c_void_p,
+                                         c_void_p, c_size, c_void_p])
 _decode = _sig("hybrid_attn_decode", c_int, [ctypes.POINTER(LayerCfg), ctypes.POINTER(DecodeArgs), c_void_p, c_size,
                                              c_void_p])
 _decode_ws = _sig("hybrid_attn_decode_workspace", c_size, [ctypes.POINTER(LayerCfg), ctypes.POINTER(DecodeArgs)])
@@ -200,9 +201,10 @@ def csa_indexer_topk(q_idx, w_idx, k_idx, q_pos, cfg: LayerCfg, mode=HCA_MODE_PR
 
 
 def sparse_mqa_attend(q, kv, win, q_pos, cfg: LayerCfg, idx=None, rate=None, mode=HCA_MODE_PREFILL, out=None,
-                      ws=None, stream=None):
+                      ws=None, stream=None, sink=None):
     """Shared-KV MQA over selected (idx) or all visible (idx=None) entries plus the window.
-    kv: [N, c] (prefill) or [B, N, c] (decode); win: raw rows [T, c] (prefill) or [B, n_win, c] (decode)."""
+    kv: [N, c] (prefill) or [B, N, c] (decode); win: raw rows [T, c] (prefill) or [B, n_win, c] (decode);
+    sink: optional [H] float32 sink logits (one per head, in the denominator only)."""
     Tq = q.shape[0]
     N = kv.shape[-2]
     kvs = kv.stride(0) if kv.dim() == 3 else 0
@@ -216,7 +218,8 @@ def sparse_mqa_attend(q, kv, win, q_pos, cfg: LayerCfg, idx=None, rate=None, mod
     ws, nb = _workspace(workspace_size(HCA_OP_SPARSE_MQA, cfg, Tq, N, mode), ws, q.device)
     _check(_mqa(_ptr(q, BF16, "q"), _ptr(kv, BF16, "kv"), kvs, N, _ptr(idx, I32, "idx"), n_idx, rate,
                 _ptr(win, BF16, "win"), ws_stride, _ptr(q_pos, I32, "q_pos"), Tq, mode, ctypes.byref(cfg),
-                _ptr(out, BF16, "out"), None if ws is None else ws.data_ptr(), nb, _stream(stream)))
+                _ptr(sink, F32, "sink"), _ptr(out, BF16, "out"), None if ws is None else ws.data_ptr(), nb,
+                _stream(stream)))
     return out
 
 
@@ -235,10 +238,14 @@ def _events_array(events):
     return ctypes.cast(arr, c_void_p), len(handles), arr
 
 
-def make_decode_args(B, q_pos, csa=None, hca=None, csa_topk_idx=None, csa_out=None, hca_out=None, events=None):
+def make_decode_args(B, q_pos, csa=None, hca=None, csa_topk_idx=None, csa_out=None, hca_out=None, events=None,
+                     csa_sink=None, hca_sink=None):
     """Build DecodeArgs from dicts of tensors (see workloads.csa_decode_inputs /
-    hca_decode_inputs).  Returns (args, keepalive)."""
+    hca_decode_inputs); csa_sink / hca_sink: optional [H] float32 sink logits.
+    Returns (args, keepalive)."""
     a = DecodeArgs()
+    a.csa_sink = _ptr(csa_sink, F32, "csa_sink")
+    a.hca_sink = _ptr(hca_sink, F32, "hca_sink")
     a.B = B
     a.q_pos = _ptr(q_pos, I32, "q_pos")
     keep = [q_pos]
@@ -288,9 +295,12 @@ def hybrid_attn_decode(cfg: LayerCfg, args: DecodeArgs, ws=None, stream=None, de
 
 
 def make_prefill_args(inp, csa_kv, csa_k_idx, topk_idx, csa_out, hca_kv=None, hca_q=None, hca_out=None,
-                      events=None):
-    """PrefillArgs from a workloads.prefill_inputs dict (on the device) and output tensors."""
+                      events=None, csa_sink=None, hca_sink=None):
+    """PrefillArgs from a workloads.prefill_inputs dict (on the device) and output tensors;
+    csa_sink / hca_sink: optional [H] float32 sink logits."""
     a = PrefillArgs()
+    a.csa_sink = _ptr(csa_sink, F32, "csa_sink")
+    a.hca_sink = _ptr(hca_sink, F32, "hca_sink")
     a.T = inp["cand"].shape[0]
     a.q_pos = _ptr(inp["q_pos"], I32, "q_pos")
     a.cand = _ptr(inp["cand"], BF16, "cand")

@@ -222,7 +222,7 @@ int run_indexer_topk(const bf16* q_idx, const float* w_idx, const bf16* k_idx, l
 
 MqaProblem make_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N,
                     const int32_t* idx, int n_idx, int rate, const hca_bf16* win, long long win_seq_stride,
-                    const int32_t* q_pos, int Tq, int mode, hca_bf16* out) {
+                    const int32_t* q_pos, int Tq, int mode, hca_bf16* out, const float* sink) {
   MqaProblem p;
   p.q = reinterpret_cast<const bf16*>(q);
   p.kv = reinterpret_cast<const bf16*>(kv);
@@ -243,12 +243,13 @@ MqaProblem make_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16*
   p.n_win = cfg->n_win;
   p.scale = cfg->scale;
   p.out = reinterpret_cast<bf16*>(out);
+  p.sink = sink;
   return p;
 }
 
 size_t mqa_ws_bound(const hca_layer_cfg* cfg, int Tq, int N, int n_idx) {
   MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, N > n_idx ? N : n_idx, nullptr, 0, 1, nullptr, 0, nullptr, Tq,
-                          HCA_MODE_DECODE, nullptr);
+                          HCA_MODE_DECODE, nullptr, nullptr);
   return mqa_ws_upper_bound(p);
 }
 
@@ -453,14 +454,16 @@ static int check_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16
 
 int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N, const int32_t* idx,
                       int n_idx, int rate, const hca_bf16* win, long long win_seq_stride, const int32_t* q_pos, int Tq,
-                      int mode, const hca_layer_cfg* cfg, hca_bf16* out, void* ws, size_t ws_bytes, void* stream) {
+                      int mode, const hca_layer_cfg* cfg, const float* sink, hca_bf16* out, void* ws,
+                      size_t ws_bytes, void* stream) {
   g_err.clear();
   int s = check_cfg(cfg);
   if (s != HCA_OK) return s;
   s = check_mqa(cfg, q, kv, kv_seq_stride, N, idx, n_idx, rate, win, win_seq_stride, q_pos, Tq, mode, out,
                 "sparse_mqa_attend");
   if (s != HCA_OK) return s;
-  MqaProblem p = make_mqa(cfg, q, kv, kv_seq_stride, N, idx, n_idx, rate, win, win_seq_stride, q_pos, Tq, mode, out);
+  MqaProblem p = make_mqa(cfg, q, kv, kv_seq_stride, N, idx, n_idx, rate, win, win_seq_stride, q_pos, Tq, mode, out,
+                          sink);
   const MqaPlan pl = plan_mqa(p);
   CHECK(ws_bytes >= pl.ws_bytes, HCA_ERR_WORKSPACE, "sparse_mqa_attend: workspace %zu < %zu", ws_bytes, pl.ws_bytes);
   if (pl.ws_bytes) CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
@@ -487,11 +490,11 @@ struct DecodeSched {
 static MqaProblem decode_csa_problem(const hca_layer_cfg* cfg, const hca_decode_args* a) {
   return make_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_N,
                   a->csa_topk_idx ? a->csa_topk_idx : reinterpret_cast<const int32_t*>(1), cfg->topk, cfg->m,
-                  a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out);
+                  a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out, a->csa_sink);
 }
 static MqaProblem decode_hca_problem(const hca_layer_cfg* cfg, const hca_decode_args* a) {
   return make_mqa(cfg, a->hca_q, a->hca_kv, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, a->hca_win,
-                  a->hca_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->hca_out);
+                  a->hca_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->hca_out, a->hca_sink);
 }
 
 static DecodeSched decode_schedule(const hca_layer_cfg* cfg, const hca_decode_args* a) {
@@ -692,11 +695,11 @@ static size_t prefill_ws(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
   const int Nc = T / cfg->m;
   size_t need = plan_indexer(T, Nc, cfg->topk).bytes;
   MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, Nc, reinterpret_cast<const int32_t*>(1), cfg->topk, cfg->m,
-                          nullptr, T, nullptr, T, HCA_MODE_PREFILL, nullptr);
+                          nullptr, T, nullptr, T, HCA_MODE_PREFILL, nullptr, nullptr);
   need = std::max(need, plan_mqa(p).ws_bytes);
   if (a->hca_kv) {
     MqaProblem ph = make_mqa(cfg, nullptr, nullptr, 0, T / cfg->m_hca, nullptr, 0, cfg->m_hca, nullptr, T, nullptr, T,
-                             HCA_MODE_PREFILL, nullptr);
+                             HCA_MODE_PREFILL, nullptr, nullptr);
     need = std::max(need, plan_mqa(ph).ws_bytes);
   }
   return round256(need);
@@ -771,7 +774,7 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
   if (s != HCA_OK) return s;
   {
     MqaProblem p = make_mqa(cfg, a->q, a->csa_kv, 0, Nc, a->topk_idx, cfg->topk, cfg->m, a->cand, T, a->q_pos, T,
-                            HCA_MODE_PREFILL, a->csa_out);
+                            HCA_MODE_PREFILL, a->csa_out, a->csa_sink);
     CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st, true), "prefill: csa attention");
     if ((s = mark()) != HCA_OK) return s;
   }
@@ -782,7 +785,7 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
                              st),
              "prefill: hca compress");
     MqaProblem p = make_mqa(cfg, a->hca_q, a->hca_kv, 0, Nh, nullptr, 0, cfg->m_hca, a->cand, T, a->q_pos, T,
-                            HCA_MODE_PREFILL, a->hca_out);
+                            HCA_MODE_PREFILL, a->hca_out, a->hca_sink);
     CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "prefill: hca attention");
     if ((s = mark()) != HCA_OK) return s;
   }

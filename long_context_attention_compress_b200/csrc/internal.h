@@ -130,6 +130,7 @@ struct MqaProblem {
   int H, c, n_win;
   float scale;
   bf16* out;                // [Tq, H, c]
+  const float* sink;        // [H] sink logits (natural units, like scale * q . k) or nullptr
 };
 // Rows of one split; the workspace layout is decided by plan_mqa().
 struct MqaPlan {
@@ -146,7 +147,7 @@ MqaPlan plan_mqa_sms(const MqaProblem& p, int sms);  // one wave of at most `sms
 MqaPlan plan_mqa_cuda_cores(const MqaProblem& p);
 size_t mqa_ws_upper_bound(const MqaProblem& p);  // any idx / stride / mode, rows up to max(N, n_idx)
 cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& plan, void* ws, cudaStream_t stream, bool pdl = false);
-cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out,
+cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out, const float* sink,
                                cudaStream_t stream,
                                bool pdl = false);
 

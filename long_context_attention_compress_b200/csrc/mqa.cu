@@ -174,6 +174,11 @@ __global__ void __launch_bounds__(kMqaThreads) mqa_split_kernel(MqaProblem p, in
   }
   __syncthreads();
   if (splits == 1) {
+    if (p.sink) {
+      // the sink joins the denominator (in the base-2 scale of the running maxima)
+      for (int h = tid; h < H; h += kMqaThreads) s_l[h] += fast_exp2(p.sink[h] * kLog2e - s_m[h]);
+      __syncthreads();
+    }
     bf16* op = p.out + (long long)q * H * C;
 #pragma unroll
     for (int j = 0; j < DPT; ++j) {
@@ -199,7 +204,8 @@ constexpr int kCombHeads = 4;
 constexpr int kCombMaxSplits = 1024;  // planners never exceed this
 __global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restrict__ ws_o,
                                                           const float2* __restrict__ ws_ml, int splits,
-                                                          int H, int C, bf16* __restrict__ out) {
+                                                          int H, int C, bf16* __restrict__ out,
+                                                          const float* __restrict__ sink) {
   __shared__ float s_w[kCombHeads][kCombMaxSplits];
   tc::griddep_wait();  // the partial states come from the attention kernel
   const int q = blockIdx.x, h0 = blockIdx.y * kCombHeads;
@@ -216,6 +222,9 @@ __global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restric
     if ((t & 31) == 0) s_red[hh & 3][t >> 5] = M;
     asm volatile("bar.sync %0, 64;" ::"r"(1 + (hh & 3)) : "memory");
     M = fmaxf(s_red[hh & 3][0], s_red[hh & 3][1]);
+    // a sink logit (base-2 scale like the maxima) joins the denominator once per query
+    const float z = sink ? sink[h] * kLog2e : neg_inf();
+    M = fmaxf(M, z);
     float den = 0.f;
     for (int s = t; s < splits; s += 64) {
       const float2 ml = ws_ml[((long long)q * splits + s) * H + h];
@@ -229,6 +238,7 @@ __global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restric
     if ((t & 31) == 0) s_red[hh & 3][t >> 5] = den;
     asm volatile("bar.sync %0, 64;" ::"r"(1 + (hh & 3)) : "memory");
     den = s_red[hh & 3][0] + s_red[hh & 3][1];
+    if (sink) den += fast_exp2(z - M);
     const float inv = den > 0.f ? 1.f / den : 0.f;
     for (int s = t; s < splits; s += 64) s_w[hh][s] *= inv;
   }
@@ -271,9 +281,9 @@ static size_t mqa_smem() {
 }
 
 cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out,
-                               cudaStream_t stream, bool pdl) {
+                               const float* sink, cudaStream_t stream, bool pdl) {
   cudaError_t e = launch_pdl(pdl, mqa_combine_kernel, dim3(Tq, (H + kCombHeads - 1) / kCombHeads), dim3(256), 0,
-                             stream, ws_o, ws_ml, splits, H, C, out);
+                             stream, ws_o, ws_ml, splits, H, C, out, sink);
   if (e != cudaSuccess) return e;
   ++g_launch_counter;
   return cudaGetLastError();
@@ -340,7 +350,7 @@ static cudaError_t launch_mqa_t(const MqaProblem& p, const MqaPlan& pl, void* ws
   e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;
   mqa_combine_kernel<<<dim3(p.Tq, (H + kCombHeads - 1) / kCombHeads), 256, 0, stream>>>(ws_o, ws_ml, pl.splits, H, C,
-                                                                                      p.out);
+                                                                                      p.out, p.sink);
   ++g_launch_counter;
   return cudaGetLastError();
 }

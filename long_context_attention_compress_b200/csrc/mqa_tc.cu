@@ -177,6 +177,8 @@ struct MqaTcParams {
   bf16* out;
   float* ws_o;
   float2* ws_ml;
+  const float* sink;          // [H] sink logits (natural units) or nullptr; unsplit queries add it here,
+                              // split ones in the combine
 };
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
@@ -499,10 +501,15 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     if (ok) {
       tc::fence_after_sync();
       uint32_t lv[32];
+      // an unsplit query's sink logit joins its denominator here (base-2 scale, against the
+      // head's running maximum); split queries leave it to the combine
+      const bool sink_here = p.sink != nullptr && p.splits == 1;
 #pragma unroll
       for (int h = 0; h < 32; ++h) {
         const int hh = 32 * hsel + h;
-        lv[h] = __float_as_uint((bars->red[0][hh] + bars->red[1][hh]) + (bars->red[2][hh] + bars->red[3][hh]));
+        float l = (bars->red[0][hh] + bars->red[1][hh]) + (bars->red[2][hh] + bars->red[3][hh]);
+        if (sink_here) l += fast_exp2(p.sink[hh] * kLog2e - bars->mref[hh]);
+        lv[h] = __float_as_uint(l);
       }
       const int dim_lane = quarter * 32 + lane;
       if (p.splits == 1) {
@@ -638,6 +645,7 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   a.splits = pl.splits;
   a.rows_per_split = pl.rows_per_split;
   a.out = p.out;
+  a.sink = p.sink;
   a.ws_o = pl.splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
   a.ws_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) + (size_t)p.Tq * pl.splits * kH * kC)
                           : nullptr;
@@ -649,7 +657,7 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   ++g_launch_counter;
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;
-  return launch_mqa_combine(a.ws_o, a.ws_ml, p.Tq, pl.splits, kH, kC, p.out, stream, pdl);
+  return launch_mqa_combine(a.ws_o, a.ws_ml, p.Tq, pl.splits, kH, kC, p.out, p.sink, stream, pdl);
 }
 
 unsigned int read_and_clear_mqa_tc_error() {

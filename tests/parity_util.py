@@ -52,6 +52,21 @@ def assert_norm_close(gpu, ref, tol=NORM_TOL, what=""):
     return e
 
 
+def assert_norm_close_per_head(gpu, ref, tol=NORM_TOL, what=""):
+    """max |gpu - ref| / rms(ref) over the c outputs of each (query, head).
+
+    With attention-sink logits every head has its own output scale (the sink
+    takes anything from none to nearly all of a head's mass), so one RMS per
+    query would be set by its largest heads and the bf16 rounding of their
+    largest elements alone could pass the bar; each head is held to its own."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = np.sqrt(np.mean(ref ** 2, axis=-1, keepdims=True))
+    e = float(np.max(np.abs(gpu - ref) / np.maximum(rms, 1e-300)))
+    assert e <= tol, f"{what}: per-head normalised max-abs error {e:.3e} > {tol}"
+    return e
+
+
 def assert_bf16_close(gpu, ref64, what=""):
     """gpu (bf16 values) within one bf16 rounding (half an ulp <= 2^-8 relative)
     of the unrounded float64 reference, plus f32 arithmetic slack."""

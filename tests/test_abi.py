@@ -82,7 +82,7 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert st == -1
     st = lib._csa_compress(FAKE, 500, FAKE, 512, FAKE, 512, 64, 512, 4, FAKE, 512, None)
     assert st == -1  # row stride too small
-    st = lib._mqa(FAKE, FAKE, 0, 100, None, 0, 0, FAKE, 0, FAKE, 4, 0, ctypes.byref(cfg), FAKE, None, 0, None)
+    st = lib._mqa(FAKE, FAKE, 0, 100, None, 0, 0, FAKE, 0, FAKE, 4, 0, ctypes.byref(cfg), None, FAKE, None, 0, None)
     assert st == -1  # rate 0
 
 
