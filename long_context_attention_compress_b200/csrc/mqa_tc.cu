@@ -196,7 +196,9 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
 
   // this query's row list
   const int t_pos = p.q_pos[q];
-  const int n_first = p.idx ? p.n_idx : n_visible(t_pos, p.rate, p.N);
+  // (no entries at all, e.g. a sequence shorter than one block: only the window;
+  // every selected slot is then empty and nothing may be read from the cache)
+  const int n_first = p.N <= 0 ? 0 : (p.idx ? p.n_idx : n_visible(t_pos, p.rate, p.N));
   const int n_win = min(p.n_win, t_pos + 1);
   const int ub = sp * p.rows_per_split;
   const int ue = min(n_first + n_win, ub + p.rows_per_split);
@@ -613,16 +615,19 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   const bool prefill = p.mode == HCA_MODE_PREFILL;
   const long long kv_rs = prefill ? 0 : p.kv_seq_stride / kC;
   const uint64_t n_kv = (uint64_t)(p.N > 0 ? p.N : 1);
+  // With no entries the entry maps are never used (no entry tiles): point them at
+  // the window rows, which exist, instead of a cache that may have no rows.
+  const void* kv_base = p.N > 0 ? (const void*)p.kv : (const void*)p.win;
   // dense tiles: (dims, rows of one request, request), so a tile never reads
   // another request's rows or the unused capacity behind a request's entries
   const uint64_t kvd3[3] = {(uint64_t)kC, n_kv, prefill ? 1ull : (uint64_t)p.Tq};
-  const long long kv_req_elems = (prefill || p.Tq == 1) ? (long long)n_kv * kC : p.kv_seq_stride;
+  const long long kv_req_elems = (prefill || p.Tq == 1 || p.N <= 0) ? (long long)n_kv * kC : p.kv_seq_stride;
   const uint64_t kvs3[2] = {(uint64_t)kC * 2, (uint64_t)kv_req_elems * 2};
-  e = make_tmap_bf16(&tm_kv, p.kv, 3, kvd3, kvs3, kRows);
+  e = make_tmap_bf16(&tm_kv, kv_base, 3, kvd3, kvs3, kRows);
   if (e != cudaSuccess) return e;
   // gathered rows: one 2-D map over every request's rows
   const uint64_t kvd[2] = {(uint64_t)kC, (uint64_t)((long long)(p.Tq - 1) * kv_rs) + n_kv};
-  e = make_tmap_bf16(&tm_kvg, p.kv, 2, kvd, rstride, 1);
+  e = make_tmap_bf16(&tm_kvg, kv_base, 2, kvd, rstride, 1);
   if (e != cudaSuccess) return e;
   const long long win_rs = prefill ? 0 : p.win_seq_stride / kC;
   const uint64_t wd3[3] = {(uint64_t)kC, prefill ? (uint64_t)p.win_rows : (uint64_t)p.n_win,

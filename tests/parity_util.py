@@ -14,6 +14,7 @@ k-th score (a near-tie that f32 accumulation may order either way).
 """
 
 import numpy as np
+import oracle
 import torch
 
 NORM_TOL = 2e-2
@@ -46,10 +47,31 @@ def norm_err(gpu, ref) -> float:
     return float(np.max(err / np.maximum(rms, 1e-30)))
 
 
+def _per_query_norm_err(gpu, ref):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    if ref.ndim < 3:
+        gpu, ref = gpu[None], ref[None]
+    ax = tuple(range(1, ref.ndim))
+    rms = np.maximum(np.sqrt(np.mean(ref ** 2, axis=ax)), 1e-30)
+    return np.max(np.abs(gpu - ref), axis=ax) / rms, ref, rms, ax
+
+
 def assert_norm_close(gpu, ref, tol=NORM_TOL, what=""):
-    e = norm_err(gpu, ref)
-    assert e <= tol, f"{what}: normalised max-abs error {e:.3e} > {tol}"
-    return e
+    """Per-query normalised max-abs error within `tol`, or -- for a query whose
+    exact output cannot be stored in bf16 within `tol` at all -- within 1.5x the
+    error of the correctly rounded exact output (the best any bf16 result can
+    reach, plus room for the f32 accumulation).  That floor only matters for
+    queries with few rows and a heavy-tailed output (short prefills), where one
+    value many times the query's RMS carries a rounding error near 2^-9 of
+    itself."""
+    err, ref64, rms, ax = _per_query_norm_err(gpu, ref)
+    floor = np.max(np.abs(oracle.round_bf16(ref64) - ref64), axis=ax) / rms
+    bar = np.maximum(tol, 1.5 * floor)
+    bad = np.nonzero(err > bar)[0]
+    assert bad.size == 0, (f"{what}: normalised max-abs error {err[bad[0]]:.3e} > {bar[bad[0]]:.3e} "
+                           f"at query {bad[0]} ({bad.size} queries over the bar)")
+    return float(np.max(err))
 
 
 def assert_norm_close_per_head(gpu, ref, tol=NORM_TOL, what=""):
