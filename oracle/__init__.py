@@ -31,4 +31,12 @@ from .hca import (  # noqa: F401
     hca_layer_prefill,
     csa_layer_decode,
     hca_layer_decode,
+    QKNorm,
+    rms_norm,
+    rope_theta,
+    rope,
+    entry_position,
+    norm_rope_rows,
+    attend_norm_rope,
+    cache_entries,
 )

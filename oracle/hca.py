@@ -40,6 +40,17 @@ notes):
   * Compressed entries are stored as bf16 (the cache format); the oracle
     rounds its float64 compressor output to bf16 (round-to-nearest-even, via
     float32) before it is attended or indexed.
+  * Q/KV normalisation and partial RoPE (optional, ``norm=``): RMSNorm over
+    the c channels of every query head and every KV row, with one learned
+    weight vector for the queries and one for the KV rows of a layer, eps
+    1e-6; RoPE then rotates the last rope_dims (64) channels in adjacent
+    pairs (2j, 2j+1) by pos * base^(-2j/rope_dims), base 10000; the
+    attention output is rotated back by -t.  A compressed entry sits at the
+    position of the last token of its own block, (i+1)*rate - 1; a window row
+    at its token's position.  Entries are cached after normalisation and
+    rotation (one bf16 rounding); window rows are kept raw (they are the
+    compressor's input too) and normalised when attended.  The indexer is
+    not core attention and is left as it is.
 """
 
 from __future__ import annotations
@@ -52,6 +63,8 @@ __all__ = [
     "indexer_scores", "topk_select", "window_rows", "mqa_attend",
     "mqa_partial", "combine_partials", "csa_layer_prefill",
     "hca_layer_prefill", "csa_layer_decode", "hca_layer_decode",
+    "rms_norm", "rope_theta", "rope", "entry_position", "QKNorm",
+    "norm_rope_rows", "attend_norm_rope", "cache_entries",
 ]
 
 
@@ -238,10 +251,98 @@ def combine_partials(parts, sink=None) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------
+# (5) Q/KV RMSNorm, partial RoPE and the output's inverse rotation
+#     ([QbitAI] "混合注意力機制": the Q/KV normalisation and partial-RoPE
+#     tricks; [Tricks] "Partial RoPE 和 Attention Sink")
+# ----------------------------------------------------------------------------
+class QKNorm:
+    """Parameters of the Q/KV normalisation of one layer: weight vectors
+    q_gamma [c] and kv_gamma [c], eps, and the rotary part (the last
+    rope_dims channels, frequency base `base`)."""
+
+    def __init__(self, q_gamma, kv_gamma, eps=1e-6, rope_dims=64, base=10000.0):
+        self.q_gamma = np.asarray(q_gamma, dtype=np.float64)
+        self.kv_gamma = np.asarray(kv_gamma, dtype=np.float64)
+        self.eps = float(eps)
+        self.rope_dims = int(rope_dims)
+        self.base = float(base)
+
+
+def rms_norm(x: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * gamma."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * np.asarray(gamma, dtype=np.float64)
+
+
+def rope_theta(rope_dims: int, base: float) -> np.ndarray:
+    """Frequencies of the rotary pairs: theta_j = base^(-2j / rope_dims)."""
+    j = np.arange(rope_dims // 2, dtype=np.float64)
+    return np.power(float(base), -2.0 * j / rope_dims)
+
+
+def rope(x: np.ndarray, pos, rope_dims: int, base: float) -> np.ndarray:
+    """Rotate the last rope_dims channels of x [..., c] at position(s) pos.
+
+    Pair j of the rotary part, channels (c - rope_dims + 2j, c - rope_dims + 2j + 1),
+    turns by the angle pos * theta_j:  (a, b) -> (a cos - b sin, a sin + b cos).
+    `pos` is a scalar or broadcasts against x's leading axes.  The other
+    channels pass through unchanged."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    if rope_dims == 0:
+        return x
+    c = x.shape[-1]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * rope_theta(rope_dims, base)
+    cs, sn = np.cos(ang), np.sin(ang)
+    a = x[..., c - rope_dims::2].copy()
+    b = x[..., c - rope_dims + 1::2].copy()
+    x[..., c - rope_dims::2] = a * cs - b * sn
+    x[..., c - rope_dims + 1::2] = a * sn + b * cs
+    return x
+
+
+def entry_position(i, rate: int):
+    """Position of compressed entry i: the last token of its own block."""
+    return (np.asarray(i) + 1) * rate - 1
+
+
+def norm_rope_rows(rows: np.ndarray, pos, gamma: np.ndarray, nrm: "QKNorm") -> np.ndarray:
+    """RMSNorm with `gamma`, then RoPE at `pos` ([U] or scalar), row by row."""
+    return rope(rms_norm(rows, gamma, nrm.eps), pos, nrm.rope_dims, nrm.base)
+
+
+def attend_norm_rope(q: np.ndarray, t: int, rows: np.ndarray, row_pos, scale: float, nrm: "QKNorm",
+                     sink=None, rows_ready=None) -> np.ndarray:
+    """Core attention of one query at position t with Q/KV normalisation.
+
+    q [H, c] raw query heads; rows [U, c] raw KV rows at positions row_pos [U]
+    (normalised and rotated here), or, for rows already in the cache's form,
+    rows_ready [U', c] appended as they are.  The output is rotated back by -t,
+    which leaves only relative positions in it (a KV row is both key and value,
+    so its own rotation reaches the output)."""
+    qn = norm_rope_rows(q, t, nrm.q_gamma, nrm)
+    kv = norm_rope_rows(rows, np.asarray(row_pos), nrm.kv_gamma, nrm) if len(rows) else np.zeros((0, q.shape[1]))
+    if rows_ready is not None:
+        kv = np.concatenate([np.asarray(rows_ready, dtype=np.float64), kv], axis=0)
+    o = mqa_attend(qn, kv, scale, sink)
+    return rope(o, -t, nrm.rope_dims, nrm.base)
+
+
+def cache_entries(E_exact: np.ndarray, rate: int, nrm: "QKNorm" = None, first: int = 0) -> np.ndarray:
+    """Compressed entries in the cache's form: bf16, after the KV normalisation
+    and rotation at their own positions when `nrm` is given (entry indices
+    start at `first`)."""
+    if nrm is None:
+        return round_bf16(E_exact)
+    pos = entry_position(np.arange(first, first + E_exact.shape[0]), rate)
+    return round_bf16(norm_rope_rows(E_exact, pos, nrm.kv_gamma, nrm))
+
+
+# ----------------------------------------------------------------------------
 # whole layers
 # ----------------------------------------------------------------------------
 def csa_layer_prefill(cand, logits, kidx_cand, pos_bias, q_idx, w_idx, q, *,
-                      m, topk, d_idx, n_win, scale, queries=None, sink=None):
+                      m, topk, d_idx, n_win, scale, queries=None, sink=None, norm=None):
     """CSA layer over one sequence of T raw tokens, for the given query positions.
 
     cand/logits [T, c]; kidx_cand [T, d_I] (per-token indexer-key candidates,
@@ -249,10 +350,11 @@ def csa_layer_prefill(cand, logits, kidx_cand, pos_bias, q_idx, w_idx, q, *,
     pos_bias[:, :d_I]); q_idx [T, H_I, d_I]; w_idx [T, H_I]; q [T, H, c].
     Returns dict with E [N, c] and K_I [N, d_I] (bf16-valued float64), and per
     query: the selected indices (ordered), their scores, the visible count and
-    the output o [H, c].
+    the output o [H, c].  norm (a QKNorm, optional): Q/KV normalisation and
+    partial RoPE; E is then the cache form (normalised and rotated).
     """
     T = cand.shape[0]
-    E = round_bf16(csa_compress(cand, logits, pos_bias, m))
+    E = cache_entries(csa_compress(cand, logits, pos_bias, m), m, norm)
     K_I = round_bf16(csa_compress(kidx_cand, np.asarray(logits)[:, :d_idx],
                                   np.asarray(pos_bias)[:, :d_idx], m))
     N = E.shape[0]
@@ -263,48 +365,62 @@ def csa_layer_prefill(cand, logits, kidx_cand, pos_bias, q_idx, w_idx, q, *,
         nv = n_visible(t, m, N)
         sc = indexer_scores(q_idx[t], w_idx[t], K_I[:nv])
         sel = topk_select(sc, topk)
-        rows = np.concatenate([E[sel], cand64[window_rows(t, n_win)]], axis=0)
+        wr = window_rows(t, n_win)
         res["idx"][t] = sel
         res["scores"][t] = sc
         res["n_vis"][t] = nv
-        res["O"][t] = mqa_attend(q[t], rows, scale, sink)
+        if norm is None:
+            rows = np.concatenate([E[sel], cand64[wr]], axis=0)
+            res["O"][t] = mqa_attend(q[t], rows, scale, sink)
+        else:
+            res["O"][t] = attend_norm_rope(q[t], t, cand64[wr], wr, scale, norm, sink, rows_ready=E[sel])
     return res
 
 
-def hca_layer_prefill(cand, logits, pos_bias, q, *, m_hca, n_win, scale, queries=None, sink=None):
+def hca_layer_prefill(cand, logits, pos_bias, q, *, m_hca, n_win, scale, queries=None, sink=None, norm=None):
     """HCA layer over one sequence: dense attention over every visible HCA
-    entry plus the sliding window ([Tricks] HCA section: no top-k selector)."""
+    entry plus the sliding window ([Tricks] HCA section: no top-k selector).
+    norm: as in csa_layer_prefill."""
     T = cand.shape[0]
-    E = round_bf16(hca_compress(cand, logits, pos_bias, m_hca))
+    E = cache_entries(hca_compress(cand, logits, pos_bias, m_hca), m_hca, norm)
     N = E.shape[0]
     qs = range(T) if queries is None else queries
     cand64 = np.asarray(cand, dtype=np.float64)
     res = {"E": E, "n_vis": {}, "O": {}}
     for t in qs:
         nv = n_visible(t, m_hca, N)
-        rows = np.concatenate([E[:nv], cand64[window_rows(t, n_win)]], axis=0)
+        wr = window_rows(t, n_win)
         res["n_vis"][t] = nv
-        res["O"][t] = mqa_attend(q[t], rows, scale, sink)
+        if norm is None:
+            rows = np.concatenate([E[:nv], cand64[wr]], axis=0)
+            res["O"][t] = mqa_attend(q[t], rows, scale, sink)
+        else:
+            res["O"][t] = attend_norm_rope(q[t], t, cand64[wr], wr, scale, norm, sink, rows_ready=E[:nv])
     return res
 
 
-def csa_layer_decode(E, K_I, win, q, q_idx, w_idx, t, *, m, topk, n_win, scale, sink=None):
+def csa_layer_decode(E, K_I, win, q, q_idx, w_idx, t, *, m, topk, n_win, scale, sink=None, norm=None):
     """One decode query of one request against its CSA cache.
 
-    E [N, c] compressed entries, K_I [N, d_I] indexer keys, win [n_win, c]
-    the raw rows of the last min(n_win, t+1) tokens (first rows valid, any
-    order), q [H, c], q_idx [H_I, d_I], w_idx [H_I].
+    E [N, c] compressed entries (the cache's form), K_I [N, d_I] indexer keys,
+    win [n_win, c] the raw rows of the last min(n_win, t+1) tokens (first rows
+    valid; oldest first, which matters only with `norm`), q [H, c],
+    q_idx [H_I, d_I], w_idx [H_I].
     """
     nv = n_visible(t, m, E.shape[0])
     sc = indexer_scores(q_idx, w_idx, K_I[:nv])
     sel = topk_select(sc, topk)
     nw = min(n_win, t + 1)
-    rows = np.concatenate([np.asarray(E, dtype=np.float64)[sel],
-                           np.asarray(win, dtype=np.float64)[:nw]], axis=0)
-    return {"idx": sel, "scores": sc, "n_vis": nv, "O": mqa_attend(q, rows, scale, sink)}
+    E64, win64 = np.asarray(E, dtype=np.float64), np.asarray(win, dtype=np.float64)
+    if norm is None:
+        O = mqa_attend(q, np.concatenate([E64[sel], win64[:nw]], axis=0), scale, sink)
+    else:
+        O = attend_norm_rope(q, t, win64[:nw], window_rows(t, n_win), scale, norm, sink, rows_ready=E64[sel])
+    return {"idx": sel, "scores": sc, "n_vis": nv, "O": O}
 
 
-def hca_layer_decode(E_h, block_cand, block_logits, pos_bias, win, q, t, *, m_hca, n_win, scale, sink=None):
+def hca_layer_decode(E_h, block_cand, block_logits, pos_bias, win, q, t, *, m_hca, n_win, scale, sink=None,
+                     norm=None):
     """One decode query of one request against its HCA cache, including the
     compression of the newest complete block ([Report] section 5 and [Jiedu]
     cache layout: the tail block is kept raw until it completes).
@@ -316,8 +432,12 @@ def hca_layer_decode(E_h, block_cand, block_logits, pos_bias, win, q, t, *, m_hc
     """
     n = (t + 1) // m_hca
     assert (t + 1) % m_hca == 0, "the newest block completes at t"
-    new = round_bf16(hca_compress(block_cand, block_logits, pos_bias, m_hca))  # [1, c]
+    new = cache_entries(hca_compress(block_cand, block_logits, pos_bias, m_hca), m_hca, norm, first=n - 1)
     Eh = np.concatenate([np.asarray(E_h, dtype=np.float64)[:n - 1], new], axis=0)
     nw = min(n_win, t + 1)
-    rows = np.concatenate([Eh, np.asarray(win, dtype=np.float64)[:nw]], axis=0)
-    return {"new_entry": new[0], "O": mqa_attend(q, rows, scale, sink)}
+    win64 = np.asarray(win, dtype=np.float64)
+    if norm is None:
+        O = mqa_attend(q, np.concatenate([Eh, win64[:nw]], axis=0), scale, sink)
+    else:
+        O = attend_norm_rope(q, t, win64[:nw], window_rows(t, n_win), scale, norm, sink, rows_ready=Eh)
+    return {"new_entry": new[0], "O": O}
