@@ -49,8 +49,9 @@ notes):
     position of the last token of its own block, (i+1)*rate - 1; a window row
     at its token's position.  Entries are cached after normalisation and
     rotation (one bf16 rounding); window rows are kept raw (they are the
-    compressor's input too) and normalised when attended.  The indexer is
-    not core attention and is left as it is.
+    compressor's input too) and normalised when attended.  Normalised queries
+    and window rows enter the attention as bf16 values, like the entries.
+    The indexer is not core attention and is left as it is.
 """
 
 from __future__ import annotations
@@ -312,16 +313,23 @@ def norm_rope_rows(rows: np.ndarray, pos, gamma: np.ndarray, nrm: "QKNorm") -> n
 
 
 def attend_norm_rope(q: np.ndarray, t: int, rows: np.ndarray, row_pos, scale: float, nrm: "QKNorm",
-                     sink=None, rows_ready=None) -> np.ndarray:
+                     sink=None, rows_ready=None, bf16_operands: bool = True) -> np.ndarray:
     """Core attention of one query at position t with Q/KV normalisation.
 
     q [H, c] raw query heads; rows [U, c] raw KV rows at positions row_pos [U]
     (normalised and rotated here), or, for rows already in the cache's form,
     rows_ready [U', c] appended as they are.  The output is rotated back by -t,
     which leaves only relative positions in it (a KV row is both key and value,
-    so its own rotation reaches the output)."""
+    so its own rotation reaches the output).
+
+    bf16_operands: the normalised, rotated queries and rows enter the attention
+    as bf16 values, like the cached entries (the pages keep the rotated KV
+    channels in BF16 in the cache; bf16 is the attention's operand type).
+    False gives the unrounded definition."""
     qn = norm_rope_rows(q, t, nrm.q_gamma, nrm)
     kv = norm_rope_rows(rows, np.asarray(row_pos), nrm.kv_gamma, nrm) if len(rows) else np.zeros((0, q.shape[1]))
+    if bf16_operands:
+        qn, kv = round_bf16(qn), round_bf16(kv)
     if rows_ready is not None:
         kv = np.concatenate([np.asarray(rows_ready, dtype=np.float64), kv], axis=0)
     o = mqa_attend(qn, kv, scale, sink)

@@ -104,7 +104,7 @@ def test_one_row_attention_is_the_row_turned_by_the_offset():
     nrm = _nrm(c, rng)
     q, v = rng.normal(size=(8, c)), rng.normal(size=(1, c))
     t, j = 5000, 4321
-    o = oracle.attend_norm_rope(q, t, v, [j], 1 / math.sqrt(c), nrm)
+    o = oracle.attend_norm_rope(q, t, v, [j], 1 / math.sqrt(c), nrm, bf16_operands=False)
     want = oracle.rope(oracle.rms_norm(v, nrm.kv_gamma, nrm.eps), j - t, 64, 1e4)[0]
     np.testing.assert_allclose(o, np.broadcast_to(want, o.shape), atol=1e-12)
 
@@ -115,10 +115,10 @@ def test_output_depends_only_on_relative_positions():
     nrm = _nrm(c, rng)
     q, rows = rng.normal(size=(8, c)), rng.normal(size=(40, c))
     pos = rng.integers(0, 3000, size=40)
-    o = oracle.attend_norm_rope(q, 3000, rows, pos, 1 / math.sqrt(c), nrm)
+    o = oracle.attend_norm_rope(q, 3000, rows, pos, 1 / math.sqrt(c), nrm, bf16_operands=False)
     for s in (1, 12345):
-        np.testing.assert_allclose(oracle.attend_norm_rope(q, 3000 + s, rows, pos + s, 1 / math.sqrt(c), nrm),
-                                   o, atol=1e-10)
+        np.testing.assert_allclose(oracle.attend_norm_rope(q, 3000 + s, rows, pos + s, 1 / math.sqrt(c), nrm,
+                                                           bf16_operands=False), o, atol=1e-10)
     # without the output rotation the shift would show
     o_plain = oracle.mqa_attend(oracle.norm_rope_rows(q, 3000, nrm.q_gamma, nrm),
                                 oracle.norm_rope_rows(rows, pos, nrm.kv_gamma, nrm), 1 / math.sqrt(c))
@@ -134,6 +134,7 @@ def test_weights_act_on_their_own_side():
     pos, t = np.arange(30) * 7, 250
     one = np.ones(c)
     base = oracle.attend_norm_rope(q, t, rows, pos, 2 * sc, _nrm(c, gq=one, gkv=one))
+    # (a weight of 2 scales by a power of two: the bf16 operands scale exactly too)
     np.testing.assert_allclose(oracle.attend_norm_rope(q, t, rows, pos, sc, _nrm(c, gq=2 * one, gkv=one)),
                                base, atol=1e-12)
     np.testing.assert_allclose(oracle.attend_norm_rope(q, t, rows, pos, sc, _nrm(c, gq=one, gkv=2 * one)),
@@ -147,7 +148,11 @@ def test_without_rope_unit_weights_it_is_attention_over_unit_rms_rows():
     nrm = _nrm(c, rope_dims=0, eps=0.0, gq=np.ones(c), gkv=np.ones(c))
     unit = lambda z: z / (np.linalg.norm(z, axis=1, keepdims=True) / math.sqrt(c))  # noqa: E731
     want = oracle.mqa_attend(unit(q), unit(rows), 0.125)
-    np.testing.assert_allclose(oracle.attend_norm_rope(q, 77, rows, np.arange(9), 0.125, nrm), want, atol=1e-12)
+    np.testing.assert_allclose(oracle.attend_norm_rope(q, 77, rows, np.arange(9), 0.125, nrm, bf16_operands=False),
+                               want, atol=1e-12)
+    # with bf16 operands: the same attention over the rounded unit-RMS rows
+    want16 = oracle.mqa_attend(oracle.round_bf16(unit(q)), oracle.round_bf16(unit(rows)), 0.125)
+    np.testing.assert_allclose(oracle.attend_norm_rope(q, 77, rows, np.arange(9), 0.125, nrm), want16, atol=1e-12)
 
 
 # --------------------------------------------------------------------------
