@@ -162,13 +162,18 @@ def source_hash(files):
 class DecodeBench:
     """Hybrid / CSA / HCA decode.  Per step: one hybrid_attn_decode call."""
 
-    def __init__(self, name, spec, seed, device):
+    def __init__(self, name, spec, seed, device, qk_norm=False):
         import long_context_attention_compress_b200 as hca
         self.hca = hca
         self.name = name
         self.spec = spec
         s = self.shape = spec["shape"]
         B, ctx = spec["B"], spec["ctx"]
+        # Q/KV normalisation + partial RoPE: synthetic weights per layer
+        self.norm_kw = {}
+        if qk_norm:
+            self.norm_kw = {"csa_norm": wl.norm_weights(s, seed=seed, device=device),
+                            "hca_norm": wl.norm_weights(s, seed=seed + 1, device=device)}
         self.B, self.ctx = B, ctx
         kind = spec["kind"]
         std = spec["cache_std"]
@@ -194,9 +199,11 @@ class DecodeBench:
         if self.hcad is not None:
             self.phases.append("hca_attention")
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
+        self.norm_kw = {k: v for k, v in self.norm_kw.items()
+                        if (k == "csa_norm" and self.csa is not None) or (k == "hca_norm" and self.hcad is not None)}
         self.args, self._keep = hca.make_decode_args(B, self.q_pos, csa=self.csa, hca=self.hcad,
                                                      csa_topk_idx=self.idx, csa_out=self.csa_out,
-                                                     hca_out=self.hca_out, events=self.events)
+                                                     hca_out=self.hca_out, events=self.events, **self.norm_kw)
         self.ws = torch.empty(max(1, hca.hybrid_attn_decode_workspace(self.cfg, self.args)), dtype=torch.uint8,
                               device=dev)
         self.units = B
@@ -265,7 +272,7 @@ class DecodeBench:
             d_in = [d[k] for d in (csa, hcad) if d is not None for k in in_keys if k in d]
             d_out = [t for t in outs if t is not None]
             args, keep = self.hca.make_decode_args(self.B, self.q_pos, csa=csa, hca=hcad, csa_topk_idx=outs[0],
-                                                   csa_out=outs[1], hca_out=outs[2])
+                                                   csa_out=outs[1], hca_out=outs[2], **self.norm_kw)
             h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]
             self.sets.append({"args": args, "keep": (keep, csa, hcad, outs), "d_in": d_in, "d_out": d_out,
                               "h_out": h_out})
@@ -305,12 +312,13 @@ class DecodeBench:
 class PrefillBench:
     """CSA prefill of one 65,536-token sequence (compress, indexer + top-k, sparse MQA)."""
 
-    def __init__(self, name, spec, seed, device):
+    def __init__(self, name, spec, seed, device, qk_norm=False):
         import long_context_attention_compress_b200 as hca
         self.hca = hca
         self.name = name
         s = self.shape = spec["shape"]
         T = self.T = spec["T"]
+        self.norm_kw = {"csa_norm": wl.norm_weights(s, seed=seed, device=device)} if qk_norm else {}
         self.inp = wl.prefill_inputs(s, T, seed=seed, device=device, with_hca=False)
         dev = device
         Nc = T // s.m
@@ -322,7 +330,7 @@ class PrefillBench:
         self.phases = ["compress", "indexer_scores", "topk_select", "csa_attention"]
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
         self.args, self._keep = hca.make_prefill_args(self.inp, self.csa_kv, self.csa_k, self.topk, self.out,
-                                                      events=self.events)
+                                                      events=self.events, **self.norm_kw)
         self.ws = torch.empty(max(1, hca.hybrid_attn_prefill_workspace(self.cfg, self.args)), dtype=torch.uint8,
                               device=dev)
         self.units = T
@@ -361,7 +369,7 @@ class PrefillBench:
         for b in range(2):
             inp = dict(self.inp) if b == 0 else {k: (v.clone() if k in keys else v) for k, v in self.inp.items()}
             topk, out = (self.topk, self.out) if b == 0 else (torch.empty_like(self.topk), torch.empty_like(self.out))
-            args, keep = self.hca.make_prefill_args(inp, self.csa_kv, self.csa_k, topk, out)
+            args, keep = self.hca.make_prefill_args(inp, self.csa_kv, self.csa_k, topk, out, **self.norm_kw)
             d_out = [topk, out]
             self.sets.append({"args": args, "keep": (keep, inp), "d_in": [inp[k] for k in keys], "d_out": d_out,
                               "h_out": [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]})
@@ -385,15 +393,42 @@ class PrefillBench:
         return time.perf_counter() - t0
 
 
-def make_bench(name, seed, device, tokens=None):
+def make_bench(name, seed, device, tokens=None, qk_norm=False):
     spec = wl.WORKLOADS[name]
+    if qk_norm:
+        name = f"{name}+qk_norm"  # the layer with Q/KV RMSNorm + partial RoPE (not the headline workload)
     if spec["kind"] == "prefill":
         if tokens:
             # a shorter sequence of the same shape (profiling captures): not the headline workload
             spec = dict(spec, T=int(tokens))
             name = f"{name}_T{int(tokens)}"
-        return PrefillBench(name, spec, seed, device)
-    return DecodeBench(name, spec, seed, device)
+        return PrefillBench(name, spec, seed, device, qk_norm)
+    return DecodeBench(name, spec, seed, device, qk_norm)
+
+
+def norm_prologue_roofline(bench, flush, pk, reps=20):
+    """The Q/KV normaliser timed alone on the prefill's queries [T, H, c] (its
+    largest launch): algorithmic bytes = one bf16 read and one bf16 write per element."""
+    q = bench.inp["q"]
+    w = bench.norm_kw["csa_norm"][0]
+    out = torch.empty_like(q)
+    st = torch.cuda.current_stream()
+    ms = []
+    for i in range(reps + 3):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        bench.hca.rms_norm_rope(q, w, bench.cfg, pos=bench.inp["q_pos"], out=out)
+        e1.record(st)
+        torch.cuda.synchronize()
+        if i >= 3:
+            ms.append(e0.elapsed_time(e1))
+    avg = sum(ms) / len(ms)
+    nbytes = 2 * q.numel() * 2
+    ach = nbytes / (avg / 1e3) / 1e9
+    return {"kernel": "norm_rope_kernel", "rows": int(q.shape[0] * q.shape[1]), "ms": round(avg, 4),
+            "bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / pk["hbm_gbs"], 4)}
 
 
 # ----------------------------------------------------------------------------
@@ -474,7 +509,7 @@ def run_ours(a):
     rank, local, ws = init_dist("nccl")
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    bench = make_bench(a.workload, shard_seed(a.seed, rank), device, tokens=a.tokens)
+    bench = make_bench(a.workload, shard_seed(a.seed, rank), device, tokens=a.tokens, qk_norm=a.qk_norm)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     for _ in range(a.warmup):
         bench.step()
@@ -550,6 +585,8 @@ def run_ours(a):
            "phase_ms": {k: round(v, 4) for k, v in phase_ms.items()},
            "roofline": roof,
            "clocks": clk.summary()}
+    if a.qk_norm and isinstance(bench, PrefillBench):
+        out["qk_norm_prologue"] = norm_prologue_roofline(bench, flush, pk)
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
         import oracle  # noqa: F401  (timed baseline only)
         cores = len(os.sched_getaffinity(0))
@@ -616,6 +653,8 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--cpu-sample", type=int, default=4, help="requests (decode) / queries (prefill) for the oracle")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--qk-norm", action="store_true",
+                    help="the layer with Q/KV RMSNorm + partial RoPE (synthetic weights)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="prefill workloads: a shorter sequence of the same shape (for profiler captures)")
     a = ap.parse_args()

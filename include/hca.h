@@ -62,10 +62,22 @@ typedef enum {
  *   n_idx_heads  lightning-indexer heads H_I (64), d_idx their dim (128)
  *   n_heads      query heads sharing the single KV head (MQA)
  *   n_win        sliding-window length (128, [Tricks] Sliding Window Branch)
- *   scale        attention logit scale (1/sqrt(c)) */
+ *   scale        attention logit scale (1/sqrt(c))
+ * Q/KV normalisation and partial RoPE ([QbitAI] "混合注意力機制", the Q/KV
+ * normalisation and partial-RoPE tricks; [Tricks] "Partial RoPE 和 Attention
+ * Sink"); read only by calls that are given normalisation weights or asked to
+ * rotate their output:
+ *   rope_dims    rotated channels at the end of every row (64); pair j =
+ *                channels (c - rope_dims + 2j, +1) turns by pos * rope_base^(-2j/rope_dims).
+ *                0 = no rotation; else even, a multiple of 8 and <= min(c, 256)
+ *   rope_base    frequency base (10000); > 0 when rope_dims > 0
+ *   norm_eps     RMSNorm epsilon (1e-6), >= 0 */
 typedef struct {
   int c, m, m_hca, topk, n_idx_heads, d_idx, n_heads, n_win;
   float scale;
+  int rope_dims;
+  float rope_base;
+  float norm_eps;
 } hca_layer_cfg;
 
 /* Query modes of the indexer and attention calls. */
@@ -115,6 +127,32 @@ int csa_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int 
 int hca_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int ld_logits,
                  const float* pos_bias, int ld_bias, int B, long long seq_stride_in, int T, int c,
                  int m_hca, hca_bf16* out, int ld_out, long long seq_stride_out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * rms_norm_rope -- Q/KV RMSNorm followed by partial RoPE, row by row
+ * ([QbitAI] "混合注意力機制": queries and KV entries are RMS-normalised before
+ * core attention, and only their last 64 channels carry a rotary position;
+ * [Tricks] "Partial RoPE 和 Attention Sink").
+ *   y = rms_norm(x) with weights gamma: x / sqrt(mean_j x_j^2 + cfg->norm_eps) * gamma,
+ *   then pair j of the last cfg->rope_dims channels turns by pos * theta_j,
+ *   theta_j = cfg->rope_base^(-2j / rope_dims):  (a, b) -> (a cos - b sin, a sin + b cos).
+ *   f32 arithmetic (the angle is reduced in f64); y is rounded to bf16.
+ *   Rows come in n_seq sequences of rows_per_seq rows: row r of sequence s is
+ *     x + s*seq_stride_x + r*ld_x   ->   y + s*seq_stride_y + r*ld_y
+ *   and sits at position max((pos ? pos[s] : 0) + pos_add, 0) + r*pos_step.
+ *   Examples: queries [Tq, H, c] -> n_seq = Tq, rows_per_seq = H, pos = q_pos,
+ *   pos_step = 0; compressed entries -> pos = NULL, pos_add = rate-1,
+ *   pos_step = rate; a decode window block [n_win, c] ending at q_pos[s] ->
+ *   pos = q_pos, pos_add = -(n_win-1), pos_step = 1.
+ *   x: bf16 (x_is_f32 = 0) or f32 (x_is_f32 = 1), cfg->c channels per row;
+ *   gamma [c] f32; pos [n_seq] int32 or NULL; y bf16.  Strides in elements
+ *   (multiples of 8 for bf16, 4 for f32).  x and y may be the same rows
+ *   (in place, bf16 only).  n_seq or rows_per_seq 0: no-op.
+ * ------------------------------------------------------------------------- */
+int rms_norm_rope(const void* x, int x_is_f32, long long ld_x, long long seq_stride_x, int n_seq,
+                  int rows_per_seq, const int32_t* pos, int pos_add, int pos_step, const float* gamma,
+                  const hca_layer_cfg* cfg, hca_bf16* y, long long ld_y, long long seq_stride_y,
+                  void* stream);
 
 /* ---------------------------------------------------------------------------
  * csa_indexer_topk -- lightning-indexer scores and per-query top-k
@@ -193,13 +231,16 @@ int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hc
  *     o[t, h, :] = sum_u e^{s_u} row_u / (e^{sink[h]} + sum_u e^{s_u})
  *   ([QbitAI] attention-sink paragraph; [Tricks] "Partial RoPE 和 Attention
  *   Sink"), once per query also when the rows are split over CTAs.
+ *   rotate_out: nonzero -> the last cfg->rope_dims channels of every output
+ *   head are turned back by -q_pos[t] (the partial-RoPE output rotation, see
+ *   rms_norm_rope; with shared K = V it leaves only relative positions).
  *   ws: hca_workspace_size(HCA_OP_SPARSE_MQA, cfg, Tq, N, mode) (split-K partials).
  * ------------------------------------------------------------------------- */
 int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N,
                       const int32_t* idx, int n_idx, int rate, const hca_bf16* win,
                       long long win_seq_stride, const int32_t* q_pos, int Tq, int mode,
-                      const hca_layer_cfg* cfg, const float* sink, hca_bf16* out, void* ws,
-                      size_t ws_bytes, void* stream);
+                      const hca_layer_cfg* cfg, const float* sink, int rotate_out, hca_bf16* out,
+                      void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * hybrid_attn_decode -- one decode step of a CSA layer and/or an HCA layer for
@@ -210,6 +251,14 @@ int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_st
  * skipped.  Caches hold entries of request b at base + b*stride.
  * `events` (optional, may be NULL) is an array of n_events cudaEvent_t handles
  * that are recorded on `stream` at kernel boundaries, for profiling.
+ * Q/KV normalisation (csa_norm / hca_norm = [2, c] f32: query weights, then KV
+ * weights; NULL = none): the layer's queries and window rows are normalised
+ * and rotated (rms_norm_rope) before its attention, its output is rotated
+ * back (rotate_out), and the HCA entry compressed here is normalised and
+ * rotated at its position, (hca_N-1)*m' + m'-1, before it is stored.  The
+ * caches (csa_kv, hca_kv rows < hca_N-1) already hold entries in that form;
+ * window blocks hold raw rows, oldest first (row w = token
+ * max(0, q_pos-n_win+1) + w).
  * ------------------------------------------------------------------------- */
 typedef struct {
   int B;
@@ -243,6 +292,8 @@ typedef struct {
   int n_events;
   const float* csa_sink;      /* [H] sink logits of the CSA layer, or NULL (see sparse_mqa_attend) */
   const float* hca_sink;      /* [H] sink logits of the HCA layer, or NULL */
+  const float* csa_norm;      /* [2, c] Q/KV normalisation weights of the CSA layer, or NULL */
+  const float* hca_norm;      /* [2, c] of the HCA layer, or NULL */
 } hca_decode_args;
 
 int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* args, void* ws,
@@ -256,6 +307,11 @@ size_t hybrid_attn_decode_workspace(const hca_layer_cfg* cfg, const hca_decode_a
  * the first d_idx channels of logits/bias_csa), indexer + top-k, sparse MQA
  * with the causal window; then, if hca_kv != NULL, HCA compression and dense
  * causal MQA with the window.
+ * Q/KV normalisation (csa_norm / hca_norm, as in hybrid_attn_decode): the
+ * compressed entries are normalised and rotated at their positions
+ * ((i+1)*rate - 1) before they are stored in csa_kv / hca_kv (one bf16
+ * rounding), the queries and the window rows (cand) before the attention,
+ * and the output is rotated back.  Indexer keys are not normalised.
  * ------------------------------------------------------------------------- */
 typedef struct {
   int T;
@@ -279,6 +335,8 @@ typedef struct {
   int n_events;
   const float* csa_sink;      /* [H] sink logits of the CSA layer, or NULL (see sparse_mqa_attend) */
   const float* hca_sink;      /* [H] sink logits of the HCA layer, or NULL */
+  const float* csa_norm;      /* [2, c] Q/KV normalisation weights of the CSA layer, or NULL */
+  const float* hca_norm;      /* [2, c] of the HCA layer, or NULL */
 } hca_prefill_args;
 
 int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* args, void* ws,

@@ -41,7 +41,8 @@ c_int, c_ll, c_size, c_float, c_void_p = ctypes.c_int, ctypes.c_longlong, ctypes
 
 class LayerCfg(ctypes.Structure):
     _fields_ = [("c", c_int), ("m", c_int), ("m_hca", c_int), ("topk", c_int), ("n_idx_heads", c_int),
-                ("d_idx", c_int), ("n_heads", c_int), ("n_win", c_int), ("scale", c_float)]
+                ("d_idx", c_int), ("n_heads", c_int), ("n_win", c_int), ("scale", c_float),
+                ("rope_dims", c_int), ("rope_base", c_float), ("norm_eps", c_float)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -52,7 +53,8 @@ class DecodeArgs(ctypes.Structure):
                 ("hca_q", c_void_p), ("hca_kv", c_void_p), ("hca_N", c_int), ("hca_kv_stride", c_ll),
                 ("hca_block_cand", c_void_p), ("hca_block_logits", c_void_p), ("hca_block_stride", c_ll),
                 ("hca_pos_bias", c_void_p), ("hca_win", c_void_p), ("hca_win_stride", c_ll), ("hca_out", c_void_p),
-                ("events", c_void_p), ("n_events", c_int), ("csa_sink", c_void_p), ("hca_sink", c_void_p)]
+                ("events", c_void_p), ("n_events", c_int), ("csa_sink", c_void_p), ("hca_sink", c_void_p),
+                ("csa_norm", c_void_p), ("hca_norm", c_void_p)]
 
 
 class PrefillArgs(ctypes.Structure):
@@ -61,7 +63,7 @@ class PrefillArgs(ctypes.Structure):
                 ("q", c_void_p), ("csa_kv", c_void_p), ("csa_k_idx", c_void_p), ("topk_idx", c_void_p),
                 ("csa_out", c_void_p), ("bias_hca", c_void_p), ("hca_q", c_void_p), ("hca_kv", c_void_p),
                 ("hca_out", c_void_p), ("events", c_void_p), ("n_events", c_int), ("csa_sink", c_void_p),
-                ("hca_sink", c_void_p)]
+                ("hca_sink", c_void_p), ("csa_norm", c_void_p), ("hca_norm", c_void_p)]
 
 
 def _sig(name, restype, argtypes):
@@ -78,8 +80,10 @@ _hca_compress = _sig("hca_compress", c_int, [c_void_p, c_int, c_void_p, c_int, c
 _indexer = _sig("csa_indexer_topk", c_int, [c_void_p, c_void_p, c_void_p, c_ll, c_int, c_void_p, c_int, c_int,
                                             ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_size, c_void_p])
 _mqa = _sig("sparse_mqa_attend", c_int, [c_void_p, c_void_p, c_ll, c_int, c_void_p, c_int, c_int, c_void_p, c_ll,
-                                         c_void_p, c_int, c_int, ctypes.POINTER(LayerCfg), c_void_p, c_void_p,
+                                         c_void_p, c_int, c_int, ctypes.POINTER(LayerCfg), c_void_p, c_int, c_void_p,
                                          c_void_p, c_size, c_void_p])
+_norm_rope = _sig("rms_norm_rope", c_int, [c_void_p, c_int, c_ll, c_ll, c_int, c_int, c_void_p, c_int, c_int,
+                                          c_void_p, ctypes.POINTER(LayerCfg), c_void_p, c_ll, c_ll, c_void_p])
 _decode = _sig("hybrid_attn_decode", c_int, [ctypes.POINTER(LayerCfg), ctypes.POINTER(DecodeArgs), c_void_p, c_size,
                                              c_void_p])
 _decode_ws = _sig("hybrid_attn_decode_workspace", c_size, [ctypes.POINTER(LayerCfg), ctypes.POINTER(DecodeArgs)])
@@ -111,7 +115,8 @@ def _check(status: int):
 def make_cfg(shape) -> LayerCfg:
     """LayerCfg from a workloads.LayerShape (or any object with the same fields)."""
     return LayerCfg(shape.c, shape.m, shape.m_hca, shape.topk, shape.n_idx_heads, shape.d_idx, shape.n_heads,
-                    shape.n_win, float(shape.scale))
+                    shape.n_win, float(shape.scale), int(shape.rope_dims), float(shape.rope_base),
+                    float(shape.norm_eps))
 
 
 def _ptr(t, dtype=None, name="tensor"):
@@ -200,11 +205,29 @@ def csa_indexer_topk(q_idx, w_idx, k_idx, q_pos, cfg: LayerCfg, mode=HCA_MODE_PR
     return out
 
 
+def rms_norm_rope(x, gamma, cfg: LayerCfg, pos=None, pos_add=0, pos_step=0, out=None, stream=None):
+    """Q/KV RMSNorm + partial RoPE of the rows of x ([n_seq, rows_per_seq, c] or [rows, c]; bf16 or
+    float32), row r of sequence s at position max((pos[s] if pos else 0) + pos_add, 0) + r*pos_step.
+    Returns bf16 rows of x's shape (out may be x itself for bf16 x)."""
+    x3 = x if x.dim() == 3 else x.unsqueeze(0)
+    n_seq, rps, c = x3.shape
+    if x.dtype not in (BF16, F32):
+        raise TypeError(f"x: dtype {x.dtype}")
+    if out is None:
+        out = torch.empty(x.shape, dtype=BF16, device=x.device)
+    o3 = out if out.dim() == 3 else out.unsqueeze(0)
+    _check(_norm_rope(_ptr(x, None, "x"), 1 if x.dtype == F32 else 0, x3.stride(1), x3.stride(0), n_seq, rps,
+                      _ptr(pos, I32, "pos"), int(pos_add), int(pos_step), _ptr(gamma, F32, "gamma"),
+                      ctypes.byref(cfg), _ptr(out, BF16, "out"), o3.stride(1), o3.stride(0), _stream(stream)))
+    return out
+
+
 def sparse_mqa_attend(q, kv, win, q_pos, cfg: LayerCfg, idx=None, rate=None, mode=HCA_MODE_PREFILL, out=None,
-                      ws=None, stream=None, sink=None):
+                      ws=None, stream=None, sink=None, rotate_out=False):
     """Shared-KV MQA over selected (idx) or all visible (idx=None) entries plus the window.
     kv: [N, c] (prefill) or [B, N, c] (decode); win: raw rows [T, c] (prefill) or [B, n_win, c] (decode);
-    sink: optional [H] float32 sink logits (one per head, in the denominator only)."""
+    sink: optional [H] float32 sink logits (one per head, in the denominator only);
+    rotate_out: turn the last cfg.rope_dims channels of each output head back by -q_pos."""
     Tq = q.shape[0]
     N = kv.shape[-2]
     kvs = kv.stride(0) if kv.dim() == 3 else 0
@@ -218,7 +241,8 @@ def sparse_mqa_attend(q, kv, win, q_pos, cfg: LayerCfg, idx=None, rate=None, mod
     ws, nb = _workspace(workspace_size(HCA_OP_SPARSE_MQA, cfg, Tq, N, mode), ws, q.device)
     _check(_mqa(_ptr(q, BF16, "q"), _ptr(kv, BF16, "kv"), kvs, N, _ptr(idx, I32, "idx"), n_idx, rate,
                 _ptr(win, BF16, "win"), ws_stride, _ptr(q_pos, I32, "q_pos"), Tq, mode, ctypes.byref(cfg),
-                _ptr(sink, F32, "sink"), _ptr(out, BF16, "out"), None if ws is None else ws.data_ptr(), nb,
+                _ptr(sink, F32, "sink"), 1 if rotate_out else 0, _ptr(out, BF16, "out"),
+                None if ws is None else ws.data_ptr(), nb,
                 _stream(stream)))
     return out
 
@@ -239,16 +263,20 @@ def _events_array(events):
 
 
 def make_decode_args(B, q_pos, csa=None, hca=None, csa_topk_idx=None, csa_out=None, hca_out=None, events=None,
-                     csa_sink=None, hca_sink=None):
+                     csa_sink=None, hca_sink=None, csa_norm=None, hca_norm=None):
     """Build DecodeArgs from dicts of tensors (see workloads.csa_decode_inputs /
-    hca_decode_inputs); csa_sink / hca_sink: optional [H] float32 sink logits.
+    hca_decode_inputs); csa_sink / hca_sink: optional [H] float32 sink logits;
+    csa_norm / hca_norm: optional [2, c] float32 Q/KV normalisation weights.
     Returns (args, keepalive)."""
     a = DecodeArgs()
     a.csa_sink = _ptr(csa_sink, F32, "csa_sink")
     a.hca_sink = _ptr(hca_sink, F32, "hca_sink")
+    a.csa_norm = _ptr(csa_norm, F32, "csa_norm")
+    a.hca_norm = _ptr(hca_norm, F32, "hca_norm")
     a.B = B
     a.q_pos = _ptr(q_pos, I32, "q_pos")
-    keep = [q_pos]
+    # every tensor the struct points at stays alive with the returned keepalive
+    keep = [q_pos, csa_sink, hca_sink, csa_norm, hca_norm, csa, hca, csa_topk_idx, csa_out, hca_out]
     if csa is not None:
         a.csa_q = _ptr(csa["q"], BF16, "csa.q")
         a.csa_q_idx = _ptr(csa["q_idx"], BF16, "csa.q_idx")
@@ -295,12 +323,15 @@ def hybrid_attn_decode(cfg: LayerCfg, args: DecodeArgs, ws=None, stream=None, de
 
 
 def make_prefill_args(inp, csa_kv, csa_k_idx, topk_idx, csa_out, hca_kv=None, hca_q=None, hca_out=None,
-                      events=None, csa_sink=None, hca_sink=None):
+                      events=None, csa_sink=None, hca_sink=None, csa_norm=None, hca_norm=None):
     """PrefillArgs from a workloads.prefill_inputs dict (on the device) and output tensors;
-    csa_sink / hca_sink: optional [H] float32 sink logits."""
+    csa_sink / hca_sink: optional [H] float32 sink logits; csa_norm / hca_norm: optional
+    [2, c] float32 Q/KV normalisation weights."""
     a = PrefillArgs()
     a.csa_sink = _ptr(csa_sink, F32, "csa_sink")
     a.hca_sink = _ptr(hca_sink, F32, "hca_sink")
+    a.csa_norm = _ptr(csa_norm, F32, "csa_norm")
+    a.hca_norm = _ptr(hca_norm, F32, "hca_norm")
     a.T = inp["cand"].shape[0]
     a.q_pos = _ptr(inp["q_pos"], I32, "q_pos")
     a.cand = _ptr(inp["cand"], BF16, "cand")
@@ -322,7 +353,9 @@ def make_prefill_args(inp, csa_kv, csa_k_idx, topk_idx, csa_out, hca_kv=None, hc
     ev, n, arr = _events_array(events)
     a.events = ev
     a.n_events = n
-    return a, [arr]
+    # every tensor the struct points at stays alive with the returned keepalive
+    return a, [arr, inp, csa_kv, csa_k_idx, topk_idx, csa_out, hca_kv, hca_q, hca_out, csa_sink, hca_sink, csa_norm,
+               hca_norm]
 
 
 def hybrid_attn_prefill_workspace(cfg: LayerCfg, args: PrefillArgs) -> int:

@@ -93,7 +93,36 @@ int check_cfg(const hca_layer_cfg* cfg) {
   CHECK(cfg->n_win <= 256, HCA_ERR_UNSUPPORTED, "cfg: n_win=%d > 256", cfg->n_win);
   CHECK(cfg->m <= 16, HCA_ERR_UNSUPPORTED, "cfg: m=%d > 16", cfg->m);
   CHECK(cfg->m_hca <= 1024, HCA_ERR_UNSUPPORTED, "cfg: m_hca=%d > 1024", cfg->m_hca);
+  CHECK(cfg->rope_dims >= 0 && cfg->rope_dims % 8 == 0 && cfg->rope_dims <= cfg->c && cfg->rope_dims <= 256,
+        HCA_ERR_UNSUPPORTED, "cfg: rope_dims=%d (need a multiple of 8, <= min(c, 256))", cfg->rope_dims);
+  CHECK(cfg->rope_dims == 0 || cfg->rope_base > 0.f, HCA_ERR_INVALID_ARG, "cfg: rope_base must be positive");
+  CHECK(cfg->norm_eps >= 0.f, HCA_ERR_INVALID_ARG, "cfg: norm_eps must be >= 0");
   return HCA_OK;
+}
+
+// Q/KV normalisation of rows (see rms_norm_rope in hca.h).
+NormRope norm_rows(const hca_layer_cfg* cfg, const void* x, bool x_f32, long long ld_x, long long seq_x, int n_seq,
+                   int rows_per_seq, const int32_t* pos, int pos_add, int pos_step, const float* gamma, void* y,
+                   long long ld_y, long long seq_y) {
+  NormRope r;
+  r.x = x;
+  r.x_f32 = x_f32;
+  r.ld_x = ld_x;
+  r.seq_x = seq_x;
+  r.n_seq = n_seq;
+  r.rows_per_seq = rows_per_seq;
+  r.pos = pos;
+  r.pos_add = pos_add;
+  r.pos_step = pos_step;
+  r.gamma = gamma;
+  r.c = cfg->c;
+  r.rope_dims = cfg->rope_dims;
+  r.eps = cfg->norm_eps;
+  r.rope_base = cfg->rope_base;
+  r.y = reinterpret_cast<bf16*>(y);
+  r.ld_y = ld_y;
+  r.seq_y = seq_y;
+  return r;
 }
 
 // ---- indexer workspace: score matrix [Tq, ldN] f32 + chunk candidates -------
@@ -244,7 +273,18 @@ MqaProblem make_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16*
   p.scale = cfg->scale;
   p.out = reinterpret_cast<bf16*>(out);
   p.sink = sink;
+  p.rope_dims = 0;
+  p.rope_base = cfg->rope_base;
   return p;
+}
+
+// The attention of a normalised layer reads its normalised queries and window
+// rows from the workspace and rotates its output back.
+void use_normalised(MqaProblem& p, const hca_layer_cfg* cfg, const void* qn, const void* wn, bool decode) {
+  p.q = reinterpret_cast<const bf16*>(qn);
+  p.win = reinterpret_cast<const bf16*>(wn);
+  if (decode) p.win_seq_stride = (long long)cfg->n_win * cfg->c;
+  p.rope_dims = cfg->rope_dims;
 }
 
 size_t mqa_ws_bound(const hca_layer_cfg* cfg, int Tq, int N, int n_idx) {
@@ -431,6 +471,33 @@ int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hc
                           ev_i);
 }
 
+int rms_norm_rope(const void* x, int x_is_f32, long long ld_x, long long seq_stride_x, int n_seq, int rows_per_seq,
+                  const int32_t* pos, int pos_add, int pos_step, const float* gamma, const hca_layer_cfg* cfg,
+                  hca_bf16* y, long long ld_y, long long seq_stride_y, void* stream) {
+  g_err.clear();
+  int s = check_cfg(cfg);
+  if (s != HCA_OK) return s;
+  CHECK(n_seq >= 0 && rows_per_seq >= 0, HCA_ERR_INVALID_ARG, "rms_norm_rope: n_seq=%d rows_per_seq=%d", n_seq,
+        rows_per_seq);
+  const long long al = x_is_f32 ? 4 : 8;
+  CHECK(ld_x >= cfg->c && ld_x % al == 0 && seq_stride_x >= 0 && seq_stride_x % al == 0, HCA_ERR_INVALID_ARG,
+        "rms_norm_rope: x strides (%lld, %lld)", ld_x, seq_stride_x);
+  CHECK(ld_y >= cfg->c && ld_y % 8 == 0 && seq_stride_y >= 0 && seq_stride_y % 8 == 0, HCA_ERR_INVALID_ARG,
+        "rms_norm_rope: y strides (%lld, %lld)", ld_y, seq_stride_y);
+  CHECK(!(x_is_f32 && (const void*)x == (const void*)y), HCA_ERR_INVALID_ARG,
+        "rms_norm_rope: in place needs bf16 rows");
+  if (n_seq == 0 || rows_per_seq == 0) return HCA_OK;
+  CHECK_PTR(x, "rms_norm_rope: x");
+  CHECK_PTR(gamma, "rms_norm_rope: gamma");
+  CHECK_PTR(y, "rms_norm_rope: y");
+  if (injected("rms_norm_rope")) return fail(HCA_ERR_INJECTED, "rms_norm_rope: injected");
+  CUDA_TRY(launch_norm_rope(norm_rows(cfg, x, x_is_f32 != 0, ld_x, seq_stride_x, n_seq, rows_per_seq, pos, pos_add,
+                                      pos_step, gamma, y, ld_y, seq_stride_y),
+                            as_stream(stream)),
+           "rms_norm_rope");
+  return HCA_OK;
+}
+
 static int check_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N,
                      const int32_t* idx, int n_idx, int rate, const hca_bf16* win, long long win_seq_stride,
                      const int32_t* q_pos, int Tq, int mode, hca_bf16* out, const char* who) {
@@ -454,8 +521,8 @@ static int check_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16
 
 int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_stride, int N, const int32_t* idx,
                       int n_idx, int rate, const hca_bf16* win, long long win_seq_stride, const int32_t* q_pos, int Tq,
-                      int mode, const hca_layer_cfg* cfg, const float* sink, hca_bf16* out, void* ws,
-                      size_t ws_bytes, void* stream) {
+                      int mode, const hca_layer_cfg* cfg, const float* sink, int rotate_out, hca_bf16* out,
+                      void* ws, size_t ws_bytes, void* stream) {
   g_err.clear();
   int s = check_cfg(cfg);
   if (s != HCA_OK) return s;
@@ -464,6 +531,7 @@ int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_st
   if (s != HCA_OK) return s;
   MqaProblem p = make_mqa(cfg, q, kv, kv_seq_stride, N, idx, n_idx, rate, win, win_seq_stride, q_pos, Tq, mode, out,
                           sink);
+  if (rotate_out) p.rope_dims = cfg->rope_dims;
   const MqaPlan pl = plan_mqa(p);
   CHECK(ws_bytes >= pl.ws_bytes, HCA_ERR_WORKSPACE, "sparse_mqa_attend: workspace %zu < %zu", ws_bytes, pl.ws_bytes);
   if (pl.ws_bytes) CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
@@ -485,6 +553,9 @@ struct DecodeSched {
   int sms = 0, r_hca = 0;
   MqaPlan csa_pl{}, hca_pl{};
   size_t main_bytes = 0, hca_off = 0, total = 0;
+  // Q/KV normalisation: normalised queries [B, H, c] and window blocks [B, n_win, c]
+  // (bf16) of each normalised layer, and the HCA entries in f32 [B, c] before theirs
+  size_t csa_qn = 0, csa_wn = 0, hca_qn = 0, hca_wn = 0, hca_ef = 0;
 };
 
 static MqaProblem decode_csa_problem(const hca_layer_cfg* cfg, const hca_decode_args* a) {
@@ -538,6 +609,19 @@ static DecodeSched decode_schedule(const hca_layer_cfg* cfg, const hca_decode_ar
   } else {
     d.hca_off = 0;
     d.total = round256(std::max(d.main_bytes, hcl ? d.hca_pl.ws_bytes : (size_t)0));
+  }
+  const size_t qbytes = round256((size_t)a->B * cfg->n_heads * cfg->c * 2);
+  const size_t wbytes = round256((size_t)a->B * cfg->n_win * cfg->c * 2);
+  if (csa && a->csa_norm) {
+    d.csa_qn = d.total;
+    d.csa_wn = d.csa_qn + qbytes;
+    d.total = d.csa_wn + wbytes;
+  }
+  if (hcl && a->hca_norm) {
+    d.hca_qn = d.total;
+    d.hca_wn = d.hca_qn + qbytes;
+    d.hca_ef = d.hca_wn + wbytes;
+    d.total = d.hca_ef + round256((size_t)a->B * cfg->c * 4);
   }
   return d;
 }
@@ -599,12 +683,14 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
     s = check_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_N, a->csa_topk_idx, cfg->topk, cfg->m,
                   a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out, "hybrid_attn_decode: csa");
     if (s != HCA_OK) return s;
+    if (a->csa_norm) CHECK_PTR(a->csa_norm, "hybrid_attn_decode: csa_norm");
   }
   if (a->hca_q) {
     CHECK(a->hca_N > 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: hca_N=%d", a->hca_N);
     s = check_mqa(cfg, a->hca_q, a->hca_kv, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, a->hca_win,
                   a->hca_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->hca_out, "hybrid_attn_decode: hca");
     if (s != HCA_OK) return s;
+    if (a->hca_norm) CHECK_PTR(a->hca_norm, "hybrid_attn_decode: hca_norm");
     if (a->hca_block_cand) {
       CHECK_PTR(a->hca_block_logits, "hybrid_attn_decode: hca_block_logits");
       CHECK_PTR(a->hca_pos_bias, "hybrid_attn_decode: hca_pos_bias");
@@ -642,17 +728,49 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
   // newest complete HCA block of every request -> its cache row.  All requests
   // share one position here (q_pos is on the device), so the row is hca_N - 1:
   // the caller passes caches sized to the complete blocks.
+  char* wsb = reinterpret_cast<char*>(ws);
+  const int c = cfg->c, H = cfg->n_heads, nw = cfg->n_win;
   auto run_hca_compress = [&]() -> int {
-    CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), cfg->c,
-                             reinterpret_cast<const bf16*>(a->hca_block_logits), cfg->c, a->hca_pos_bias, cfg->c,
-                             a->B, a->hca_block_stride, cfg->m_hca, cfg->c, cfg->m_hca, false,
-                             reinterpret_cast<bf16*>(a->hca_kv) + (long long)(a->hca_N - 1) * cfg->c, cfg->c,
-                             a->hca_kv_stride, hst),
+    bf16* row = reinterpret_cast<bf16*>(a->hca_kv) + (long long)(a->hca_N - 1) * c;
+    if (!a->hca_norm) {
+      CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), c,
+                               reinterpret_cast<const bf16*>(a->hca_block_logits), c, a->hca_pos_bias, c, a->B,
+                               a->hca_block_stride, cfg->m_hca, c, cfg->m_hca, false, row, c, a->hca_kv_stride, hst),
+               "decode: hca compress");
+      return HCA_OK;
+    }
+    // f32 entries, then normalised and rotated at the entry's position into the cache row
+    float* ef = reinterpret_cast<float*>(wsb + sched.hca_ef);
+    CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), c,
+                             reinterpret_cast<const bf16*>(a->hca_block_logits), c, a->hca_pos_bias, c, a->B,
+                             a->hca_block_stride, cfg->m_hca, c, cfg->m_hca, false, nullptr, c, c, hst, ef),
              "decode: hca compress");
+    CUDA_TRY(launch_norm_rope(norm_rows(cfg, ef, true, c, c, a->B, 1, nullptr, a->hca_N * cfg->m_hca - 1, 0,
+                                        a->hca_norm + c, row, c, a->hca_kv_stride),
+                              hst),
+             "decode: hca entry normalisation");
+    return HCA_OK;
+  };
+  // normalised queries and window blocks of a layer (window row w = token max(0, t-n_win+1) + w)
+  auto normalise_layer = [&](const hca_bf16* q, const hca_bf16* win, long long win_stride, const float* norm,
+                             size_t qn, size_t wn, cudaStream_t sm) -> int {
+    CUDA_TRY(launch_norm_rope(norm_rows(cfg, q, false, c, (long long)H * c, a->B, H, a->q_pos, 0, 0, norm, wsb + qn,
+                                        c, (long long)H * c),
+                              sm),
+             "decode: query normalisation");
+    CUDA_TRY(launch_norm_rope(norm_rows(cfg, win, false, c, win_stride, a->B, nw, a->q_pos, -(nw - 1), 1, norm + c,
+                                        wsb + wn, c, (long long)nw * c),
+                              sm),
+             "decode: window normalisation");
     return HCA_OK;
   };
   auto run_hca_attention = [&]() -> int {
     MqaProblem p = decode_hca_problem(cfg, a);
+    if (a->hca_norm) {
+      int r = normalise_layer(a->hca_q, a->hca_win, a->hca_win_stride, a->hca_norm, sched.hca_qn, sched.hca_wn, hst);
+      if (r != HCA_OK) return r;
+      use_normalised(p, cfg, wsb + sched.hca_qn, wsb + sched.hca_wn, true);
+    }
     CUDA_TRY(launch_mqa(p, sched.hca_pl, hws, hst), "decode: hca attention");
     return HCA_OK;
   };
@@ -668,12 +786,19 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
     if ((s = mark()) != HCA_OK) return s;
   }
   if (a->csa_q) {
+    // (the normalisation runs before the indexer, outside the programmatic-launch chain
+    // top-k -> attention, whose attention reads its queries before it waits)
+    if (a->csa_norm) {
+      s = normalise_layer(a->csa_q, a->csa_win, a->csa_win_stride, a->csa_norm, sched.csa_qn, sched.csa_wn, st);
+      if (s != HCA_OK) return s;
+    }
     s = run_indexer_topk(reinterpret_cast<const bf16*>(a->csa_q_idx), a->csa_w_idx,
                          reinterpret_cast<const bf16*>(a->csa_k_idx), a->csa_k_stride, a->csa_N, a->q_pos, a->B,
                          HCA_MODE_DECODE, cfg, a->csa_topk_idx, ws, st, ev, n_ev, ev_i,
                          sched.overlap ? sched.sms - sched.r_hca : 0);
     if (s != HCA_OK) return s;
     MqaProblem p = decode_csa_problem(cfg, a);
+    if (a->csa_norm) use_normalised(p, cfg, wsb + sched.csa_qn, wsb + sched.csa_wn, true);
     CUDA_TRY(launch_mqa(p, sched.csa_pl, ws, st, true), "decode: csa attention");
     if ((s = mark()) != HCA_OK) return s;
   }
@@ -690,7 +815,13 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
 }
 
 // ---- prefill -----------------------------------------------------------------
-static size_t prefill_ws(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
+// Workspace: indexer / attention scratch, then (with Q/KV normalisation) the
+// normalised queries [T, H, c] and window rows [T, c] (bf16) and the f32
+// entries [N, c] before theirs; the two layers reuse these in turn.
+struct PrefillWs {
+  size_t qn = 0, wn = 0, ef = 0, total = 0;
+};
+static PrefillWs prefill_ws_layout(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
   const int T = a->T;
   const int Nc = T / cfg->m;
   size_t need = plan_indexer(T, Nc, cfg->topk).bytes;
@@ -702,7 +833,19 @@ static size_t prefill_ws(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
                              HCA_MODE_PREFILL, nullptr, nullptr);
     need = std::max(need, plan_mqa(ph).ws_bytes);
   }
-  return round256(need);
+  PrefillWs w;
+  w.total = round256(need);
+  if (a->csa_norm || (a->hca_kv && a->hca_norm)) {
+    w.qn = w.total;
+    w.wn = w.qn + round256((size_t)T * cfg->n_heads * cfg->c * 2);
+    w.ef = w.wn + round256((size_t)T * cfg->c * 2);
+    const int Nh = a->hca_kv ? T / cfg->m_hca : 0;
+    w.total = w.ef + round256((size_t)std::max(std::max(Nc, Nh), 1) * cfg->c * 4);
+  }
+  return w;
+}
+static size_t prefill_ws(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
+  return prefill_ws_layout(cfg, a).total;
 }
 
 size_t hybrid_attn_prefill_workspace(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
@@ -741,7 +884,9 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
     CHECK_PTR(a->bias_hca, "hybrid_attn_prefill: bias_hca");
     CHECK_PTR(a->hca_q, "hybrid_attn_prefill: hca_q");
     CHECK_PTR(a->hca_out, "hybrid_attn_prefill: hca_out");
+    if (a->hca_norm) CHECK_PTR(a->hca_norm, "hybrid_attn_prefill: hca_norm");
   }
+  if (a->csa_norm) CHECK_PTR(a->csa_norm, "hybrid_attn_prefill: csa_norm");
   const size_t need = prefill_ws(cfg, a);
   CHECK(ws_bytes >= need, HCA_ERR_WORKSPACE, "hybrid_attn_prefill: workspace %zu < %zu", ws_bytes, need);
   CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
@@ -758,16 +903,49 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
     if (ev && ev_i < n_ev) return cuda_status(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
     return HCA_OK;
   };
-  const int c = cfg->c, dI = cfg->d_idx;
+  const int c = cfg->c, dI = cfg->d_idx, H = cfg->n_heads;
+  const PrefillWs wl = prefill_ws_layout(cfg, a);
+  char* wsb = reinterpret_cast<char*>(ws);
+  float* ef = reinterpret_cast<float*>(wsb + wl.ef);
+  // entries of one layer: f32 from the compressor, normalised and rotated at
+  // (i+1)*rate - 1 into the cache (with normalisation), else bf16 directly
+  auto compress_entries = [&](const float* bias, int rate, bool overlap, hca_bf16* kv, const float* norm,
+                              const char* what) -> int {
+    if (!norm) {
+      CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->cand), c, reinterpret_cast<const bf16*>(a->logits), c,
+                               bias, c, 1, 0, T, c, rate, overlap, reinterpret_cast<bf16*>(kv), c, 0, st),
+               what);
+      return HCA_OK;
+    }
+    CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->cand), c, reinterpret_cast<const bf16*>(a->logits), c,
+                             bias, c, 1, 0, T, c, rate, overlap, nullptr, c, 0, st, ef),
+             what);
+    CUDA_TRY(launch_norm_rope(norm_rows(cfg, ef, true, c, 0, 1, T / rate, nullptr, rate - 1, rate, norm + c, kv, c, 0),
+                              st),
+             "prefill: entry normalisation");
+    return HCA_OK;
+  };
+  // normalised queries [T, H, c] and window rows [T, c] (row r = token r) of a layer
+  auto normalise_layer = [&](const hca_bf16* q, const float* norm) -> int {
+    CUDA_TRY(launch_norm_rope(norm_rows(cfg, q, false, c, (long long)H * c, T, H, a->q_pos, 0, 0, norm, wsb + wl.qn, c,
+                                        (long long)H * c),
+                              st),
+             "prefill: query normalisation");
+    CUDA_TRY(launch_norm_rope(norm_rows(cfg, a->cand, false, c, 0, 1, T, nullptr, 0, 1, norm + c, wsb + wl.wn, c, 0),
+                              st),
+             "prefill: window normalisation");
+    return HCA_OK;
+  };
   if ((s = mark()) != HCA_OK) return s;
   // CSA compression of KV entries and of indexer keys (logits/bias: first d_I channels)
-  CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->cand), c, reinterpret_cast<const bf16*>(a->logits), c,
-                           a->bias_csa, c, 1, 0, T, c, cfg->m, true, reinterpret_cast<bf16*>(a->csa_kv), c, 0, st),
-           "prefill: csa compress");
+  if ((s = compress_entries(a->bias_csa, cfg->m, true, a->csa_kv, a->csa_norm, "prefill: csa compress")) != HCA_OK)
+    return s;
   CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->kidx_cand), dI, reinterpret_cast<const bf16*>(a->logits),
                            c, a->bias_csa, c, 1, 0, T, dI, cfg->m, true, reinterpret_cast<bf16*>(a->csa_k_idx), dI, 0,
                            st),
            "prefill: indexer-key compress");
+  // (before the indexer: outside the programmatic-launch chain top-k -> attention)
+  if (a->csa_norm && (s = normalise_layer(a->q, a->csa_norm)) != HCA_OK) return s;
   if ((s = mark()) != HCA_OK) return s;
   s = run_indexer_topk(reinterpret_cast<const bf16*>(a->q_idx), a->w_idx, reinterpret_cast<const bf16*>(a->csa_k_idx),
                        0, Nc, a->q_pos, T, HCA_MODE_PREFILL, cfg, a->topk_idx, ws, st, ev, n_ev, ev_i);
@@ -775,17 +953,22 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
   {
     MqaProblem p = make_mqa(cfg, a->q, a->csa_kv, 0, Nc, a->topk_idx, cfg->topk, cfg->m, a->cand, T, a->q_pos, T,
                             HCA_MODE_PREFILL, a->csa_out, a->csa_sink);
+    if (a->csa_norm) use_normalised(p, cfg, wsb + wl.qn, wsb + wl.wn, false);
     CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st, true), "prefill: csa attention");
     if ((s = mark()) != HCA_OK) return s;
   }
   if (a->hca_kv) {
     const int Nh = T / cfg->m_hca;
-    CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->cand), c, reinterpret_cast<const bf16*>(a->logits), c,
-                             a->bias_hca, c, 1, 0, T, c, cfg->m_hca, false, reinterpret_cast<bf16*>(a->hca_kv), c, 0,
-                             st),
-             "prefill: hca compress");
+    if ((s = compress_entries(a->bias_hca, cfg->m_hca, false, a->hca_kv, a->hca_norm, "prefill: hca compress")) !=
+        HCA_OK)
+      return s;
     MqaProblem p = make_mqa(cfg, a->hca_q, a->hca_kv, 0, Nh, nullptr, 0, cfg->m_hca, a->cand, T, a->q_pos, T,
                             HCA_MODE_PREFILL, a->hca_out, a->hca_sink);
+    if (a->hca_norm) {
+      // (the CSA layer's normalised rows are consumed: this stream ran its attention)
+      if ((s = normalise_layer(a->hca_q, a->hca_norm)) != HCA_OK) return s;
+      use_normalised(p, cfg, wsb + wl.qn, wsb + wl.wn, false);
+    }
     CUDA_TRY(launch_mqa(p, plan_mqa(p), ws, st), "prefill: hca attention");
     if ((s = mark()) != HCA_OK) return s;
   }

@@ -60,4 +60,19 @@ __device__ __forceinline__ int n_visible(int t, int rate, int N) {
   return v < N ? v : N;
 }
 
+// Rotary angle of pair j (of d rotated channels) at position pos is
+// pos * base^(-2j/d).  Positions reach 10^6, so the angle is formed and its
+// cosine and sine taken in f64 (an f32 frequency alone would be off by
+// ~0.06 rad there).
+__device__ __forceinline__ void rope_cos_sin_f64(long long pos, int j, int d, float base, double& cs, double& sn) {
+  const double theta = pow((double)base, -2.0 * j / d);
+  sincos((double)pos * theta, &sn, &cs);
+}
+__device__ __forceinline__ void rope_cos_sin(long long pos, int j, int d, float base, float& cs, float& sn) {
+  double cd, sd;
+  rope_cos_sin_f64(pos, j, d, base, cd, sd);
+  cs = (float)cd;
+  sn = (float)sd;
+}
+
 }  // namespace hca

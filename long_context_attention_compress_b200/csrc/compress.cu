@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(256) compress_kernel(
     const bf16* __restrict__ cand, int ld_cand, const bf16* __restrict__ logits, int ld_logits,
     const float* __restrict__ bias, int ld_bias, int T, int c, int rate, int overlap,
     int n_entries, long long seq_in, bf16* __restrict__ out, int ld_out, long long seq_out,
-    int tg_log2, int toks_per_group) {
+    int tg_log2, int toks_per_group, float* __restrict__ out_f32) {
   const int TG = 1 << tg_log2;
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const int grp = (int)(gtid & (TG - 1));
@@ -53,7 +53,8 @@ __global__ void __launch_bounds__(256) compress_kernel(
   const long long b = blockIdx.y;
   cand += b * seq_in;
   logits += b * seq_in;
-  out += b * seq_out;
+  if (out_f32) out_f32 += b * seq_out;
+  else out += b * seq_out;
 
   SoftState st;
 #pragma unroll
@@ -110,6 +111,12 @@ __global__ void __launch_bounds__(256) compress_kernel(
     float o[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) o[k] = st.acc[k] / st.l[k];
+    if (out_f32) {  // handed on, unrounded, to the Q/KV normalisation
+      float4* d = reinterpret_cast<float4*>(out_f32 + (long long)i * ld_out + j0);
+      d[0] = make_float4(o[0], o[1], o[2], o[3]);
+      d[1] = make_float4(o[4], o[5], o[6], o[7]);
+      return;
+    }
     uint4 w;
     w.x = pack_bf16x2(o[0], o[1]);
     w.y = pack_bf16x2(o[2], o[3]);
@@ -122,7 +129,7 @@ __global__ void __launch_bounds__(256) compress_kernel(
 cudaError_t launch_compress(const bf16* cand, int ld_cand, const bf16* logits, int ld_logits,
                             const float* bias, int ld_bias, int B, long long seq_in, int T, int c,
                             int rate, bool overlap, bf16* out, int ld_out, long long seq_out,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, float* out_f32) {
   const int n_entries = T / rate;
   if (n_entries == 0 || B == 0) return cudaSuccess;
   const int window = overlap ? 2 * rate : rate;
@@ -137,7 +144,7 @@ cudaError_t launch_compress(const bf16* cand, int ld_cand, const bf16* logits, i
   dim3 g((unsigned)grid, (unsigned)B);
   compress_kernel<<<g, block, 0, stream>>>(cand, ld_cand, logits, ld_logits, bias, ld_bias, T, c,
                                            rate, overlap ? 1 : 0, n_entries, seq_in, out, ld_out,
-                                           seq_out, tg_log2, per);
+                                           seq_out, tg_log2, per, out_f32);
   ++g_launch_counter;
   return cudaGetLastError();
 }

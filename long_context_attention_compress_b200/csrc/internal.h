@@ -15,7 +15,26 @@ extern thread_local int g_launch_counter;
 cudaError_t launch_compress(const bf16* cand, int ld_cand, const bf16* logits, int ld_logits,
                             const float* bias, int ld_bias, int B, long long seq_in, int T, int c,
                             int rate, bool overlap, bf16* out, int ld_out, long long seq_out,
-                            cudaStream_t stream);
+                            cudaStream_t stream, float* out_f32 = nullptr);
+// (out_f32 != nullptr: the entries are written there in f32, same strides, and out is unused)
+
+// ---- norm_rope.cu -------------------------------------------------------------
+// Q/KV RMSNorm + partial RoPE of rows (see rms_norm_rope in hca.h for the row
+// addressing and positions).
+struct NormRope {
+  const void* x;
+  bool x_f32;
+  long long ld_x, seq_x;
+  int n_seq, rows_per_seq;
+  const int32_t* pos;
+  int pos_add, pos_step;
+  const float* gamma;
+  int c, rope_dims;
+  float eps, rope_base;
+  bf16* y;
+  long long ld_y, seq_y;
+};
+cudaError_t launch_norm_rope(const NormRope& p, cudaStream_t stream);
 
 // ---- topk.cu ----------------------------------------------------------------
 // Largest candidate-count a single select row may have (smem-resident).
@@ -131,6 +150,8 @@ struct MqaProblem {
   float scale;
   bf16* out;                // [Tq, H, c]
   const float* sink;        // [H] sink logits (natural units, like scale * q . k) or nullptr
+  int rope_dims;            // > 0: the output's last rope_dims channels turn back by -q_pos
+  float rope_base;
 };
 // Rows of one split; the workspace layout is decided by plan_mqa().
 struct MqaPlan {
@@ -148,6 +169,7 @@ MqaPlan plan_mqa_cuda_cores(const MqaProblem& p);
 size_t mqa_ws_upper_bound(const MqaProblem& p);  // any idx / stride / mode, rows up to max(N, n_idx)
 cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& plan, void* ws, cudaStream_t stream, bool pdl = false);
 cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out, const float* sink,
+                               const int32_t* q_pos, int rope_dims, float rope_base,
                                cudaStream_t stream,
                                bool pdl = false);
 

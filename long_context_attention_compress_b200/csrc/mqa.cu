@@ -180,11 +180,23 @@ __global__ void __launch_bounds__(kMqaThreads) mqa_split_kernel(MqaProblem p, in
       __syncthreads();
     }
     bf16* op = p.out + (long long)q * H * C;
+    const int rope0 = C - p.rope_dims;
 #pragma unroll
     for (int j = 0; j < DPT; ++j) {
       const int oi = tid + kMqaThreads * j;
       const float l = s_l[oi / C];
-      op[oi] = __float2bfloat16_rn(l > 0.f ? o[j] / l : 0.f);
+      float v = l > 0.f ? o[j] / l : 0.f;
+      if (p.rope_dims > 0) {
+        // partial-RoPE output rotation by -t: channel d pairs with d ^ 1, held by lane ^ 1
+        const float pr = __shfl_xor_sync(0xffffffffu, v, 1);
+        const int d = oi % C;
+        if (d >= rope0) {
+          float cs, sn;
+          rope_cos_sin(p.q_pos[q], (d - rope0) >> 1, p.rope_dims, p.rope_base, cs, sn);
+          v = fmaf(v, cs, pr * ((d & 1) ? -sn : sn));
+        }
+      }
+      op[oi] = __float2bfloat16_rn(v);
     }
   } else {
     float* wo = ws_o + ((long long)q * splits + sp) * H * C;
@@ -205,7 +217,9 @@ constexpr int kCombMaxSplits = 1024;  // planners never exceed this
 __global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restrict__ ws_o,
                                                           const float2* __restrict__ ws_ml, int splits,
                                                           int H, int C, bf16* __restrict__ out,
-                                                          const float* __restrict__ sink) {
+                                                          const float* __restrict__ sink,
+                                                          const int32_t* __restrict__ q_pos, int rope_dims,
+                                                          float rope_base) {
   __shared__ float s_w[kCombHeads][kCombMaxSplits];
   tc::griddep_wait();  // the partial states come from the attention kernel
   const int q = blockIdx.x, h0 = blockIdx.y * kCombHeads;
@@ -268,6 +282,16 @@ __global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restric
       acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
       acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
     }
+    if (rope_dims > 0 && d4 * 4 >= C - rope_dims) {
+      // partial-RoPE output rotation by -t of the pairs (x, y) and (z, w):
+      // a' = a cos + b sin, b' = b cos - a sin
+      const int j = (d4 * 4 - (C - rope_dims)) >> 1;
+      float c0, s0, c1, s1;
+      rope_cos_sin(q_pos[q], j, rope_dims, rope_base, c0, s0);
+      rope_cos_sin(q_pos[q], j + 1, rope_dims, rope_base, c1, s1);
+      acc = make_float4(fmaf(acc.x, c0, acc.y * s0), fmaf(acc.y, c0, -acc.x * s0),
+                        fmaf(acc.z, c1, acc.w * s1), fmaf(acc.w, c1, -acc.z * s1));
+    }
     uint2 pk;
     pk.x = pack_bf16x2(acc.x, acc.y);
     pk.y = pack_bf16x2(acc.z, acc.w);
@@ -281,9 +305,10 @@ static size_t mqa_smem() {
 }
 
 cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out,
-                               const float* sink, cudaStream_t stream, bool pdl) {
+                               const float* sink, const int32_t* q_pos, int rope_dims, float rope_base,
+                               cudaStream_t stream, bool pdl) {
   cudaError_t e = launch_pdl(pdl, mqa_combine_kernel, dim3(Tq, (H + kCombHeads - 1) / kCombHeads), dim3(256), 0,
-                             stream, ws_o, ws_ml, splits, H, C, out, sink);
+                             stream, ws_o, ws_ml, splits, H, C, out, sink, q_pos, rope_dims, rope_base);
   if (e != cudaSuccess) return e;
   ++g_launch_counter;
   return cudaGetLastError();
@@ -350,7 +375,8 @@ static cudaError_t launch_mqa_t(const MqaProblem& p, const MqaPlan& pl, void* ws
   e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;
   mqa_combine_kernel<<<dim3(p.Tq, (H + kCombHeads - 1) / kCombHeads), 256, 0, stream>>>(ws_o, ws_ml, pl.splits, H, C,
-                                                                                      p.out, p.sink);
+                                                                                      p.out, p.sink, p.q_pos,
+                                                                                      p.rope_dims, p.rope_base);
   ++g_launch_counter;
   return cudaGetLastError();
 }

@@ -179,6 +179,8 @@ struct MqaTcParams {
   float2* ws_ml;
   const float* sink;          // [H] sink logits (natural units) or nullptr; unsplit queries add it here,
                               // split ones in the combine
+  int rope_dims;              // > 0: unsplit queries turn their output's last rope_dims channels back by
+  float rope_base;            // -t here, split ones in the combine
 };
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
@@ -516,6 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       const int dim_lane = quarter * 32 + lane;
       if (p.splits == 1) {
         bf16* op = p.out + (long long)q * kH * kC + (long long)(32 * hsel) * kC;
+        const int rope0 = kC - p.rope_dims;
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
           uint32_t v[32];
@@ -524,10 +527,20 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
             tc::tmem_ld_wait();
           }
           const int d = mb * 128 + dim_lane;
+          // partial-RoPE output rotation by -t: channel d pairs with d ^ 1, the
+          // neighbouring TMEM lane (lane ^ 1 of this warp); whole warps take the branch
+          const bool rot = p.rope_dims > 0 && mb * 128 + quarter * 32 + 31 >= rope0;
+          float rc = 1.f, rsx = 0.f;
+          if (rot && d >= rope0) {
+            float sn;
+            rope_cos_sin(t_pos, (d - rope0) >> 1, p.rope_dims, p.rope_base, rc, sn);
+            rsx = (d & 1) ? -sn : sn;
+          }
 #pragma unroll
           for (int h = 0; h < 32; ++h) {
             const float l = __uint_as_float(lv[h]);
-            const float o = (nt > 0 && l > 0.f) ? __uint_as_float(v[h]) / l : 0.f;
+            float o = (nt > 0 && l > 0.f) ? __uint_as_float(v[h]) / l : 0.f;
+            if (rot) o = fmaf(o, rc, __shfl_xor_sync(0xffffffffu, o, 1) * rsx);
             op[h * kC + d] = __float2bfloat16_rn(o);
           }
         }
@@ -651,6 +664,8 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   a.rows_per_split = pl.rows_per_split;
   a.out = p.out;
   a.sink = p.sink;
+  a.rope_dims = p.rope_dims;
+  a.rope_base = p.rope_base;
   a.ws_o = pl.splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
   a.ws_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) + (size_t)p.Tq * pl.splits * kH * kC)
                           : nullptr;
@@ -662,7 +677,8 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   ++g_launch_counter;
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;
-  return launch_mqa_combine(a.ws_o, a.ws_ml, p.Tq, pl.splits, kH, kC, p.out, p.sink, stream, pdl);
+  return launch_mqa_combine(a.ws_o, a.ws_ml, p.Tq, pl.splits, kH, kC, p.out, p.sink, p.q_pos, p.rope_dims,
+                            p.rope_base, stream, pdl);
 }
 
 unsigned int read_and_clear_mqa_tc_error() {

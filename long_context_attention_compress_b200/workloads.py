@@ -35,7 +35,9 @@ import torch
 class LayerShape:
     """Hyper-parameters of one attention layer (c: KV/head dim, m: CSA rate,
     m_hca: HCA rate, topk: CSA selection size, n_idx_heads x d_idx: indexer
-    heads, n_heads: query heads sharing one KV, n_win: sliding window)."""
+    heads, n_heads: query heads sharing one KV, n_win: sliding window;
+    rope_dims / rope_base / norm_eps: the rotary part, its frequency base and
+    the RMSNorm epsilon of the optional Q/KV normalisation)."""
     c: int
     m: int
     m_hca: int
@@ -44,13 +46,16 @@ class LayerShape:
     d_idx: int
     n_heads: int
     n_win: int
+    rope_dims: int = 64
+    rope_base: float = 10000.0
+    norm_eps: float = 1e-6
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.c)
 
 
-TINY = LayerShape(c=64, m=4, m_hca=32, topk=64, n_idx_heads=4, d_idx=32, n_heads=4, n_win=32)
+TINY = LayerShape(c=64, m=4, m_hca=32, topk=64, n_idx_heads=4, d_idx=32, n_heads=4, n_win=32, rope_dims=16)
 PRO = LayerShape(c=512, m=4, m_hca=128, topk=1024, n_idx_heads=64, d_idx=128, n_heads=64, n_win=128)
 
 
@@ -101,6 +106,13 @@ def prefill_inputs(shape: LayerShape, T: int, seed: int = 0, device: str = "cpu"
         d["bias_hca"] = _normal(g, (shape.m_hca, shape.c), std=0.1, device=device, dtype=torch.float32)
     d["q_pos"] = torch.arange(T, dtype=torch.int32, device=device)
     return d
+
+
+def norm_weights(shape: LayerShape, seed: int = 0, device: str = "cpu") -> torch.Tensor:
+    """Synthetic Q/KV normalisation weights of one layer: [2, c] float32 (row 0
+    for the queries, row 1 for the KV rows), U(0.5, 1.5)."""
+    g = _gen(seed + 424_243, device)
+    return 0.5 + _uniform(g, (2, shape.c), device=device)
 
 
 def csa_decode_inputs(shape: LayerShape, B: int, ctx: int, seed: int = 0, cache_std: float = 1.0,

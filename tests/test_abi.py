@@ -82,8 +82,42 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert st == -1
     st = lib._csa_compress(FAKE, 500, FAKE, 512, FAKE, 512, 64, 512, 4, FAKE, 512, None)
     assert st == -1  # row stride too small
-    st = lib._mqa(FAKE, FAKE, 0, 100, None, 0, 0, FAKE, 0, FAKE, 4, 0, ctypes.byref(cfg), None, FAKE, None, 0, None)
+    st = lib._mqa(FAKE, FAKE, 0, 100, None, 0, 0, FAKE, 0, FAKE, 4, 0, ctypes.byref(cfg), None, 0, FAKE, None, 0,
+                  None)
     assert st == -1  # rate 0
+
+
+def test_norm_rope_arguments_checked(lib):
+    """rms_norm_rope rejects bad rows, strides and rotary settings on the host
+    (nothing is launched: no GPU needed)."""
+    from long_context_attention_compress_b200 import workloads as wl
+    cfg = _cfg(lib)
+    args = dict(x=FAKE, f32=0, ld=512, seq=0, n_seq=1, rps=4, pos=None, add=0, step=1, gamma=FAKE, y=FAKE,
+                ld_y=512, seq_y=0)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib._norm_rope(a["x"], a["f32"], a["ld"], a["seq"], a["n_seq"], a["rps"], a["pos"], a["add"],
+                              a["step"], a["gamma"], ctypes.byref(a.get("cfg", cfg)), a["y"], a["ld_y"],
+                              a["seq_y"], None)
+
+    assert call(n_seq=0) == 0 and call(rps=0) == 0          # nothing to do
+    assert call(x=None) == -1 and "x" in lib.last_error()
+    assert call(gamma=None) == -1 and "gamma" in lib.last_error()
+    assert call(x=FAKE + 4) == -1 and "aligned" in lib.last_error()
+    assert call(ld=500) == -1                                # row shorter than c
+    assert call(ld=516) == -1                                # not a 16-byte row stride for bf16
+    assert call(f32=1, y=FAKE) == -1 and "in place" in lib.last_error()
+    assert call(n_seq=-1) == -1
+    bad = lib.make_cfg(wl.PRO)
+    bad.rope_dims = 12
+    assert call(cfg=bad) == -2                               # not a multiple of 8
+    bad.rope_dims = 64
+    bad.rope_base = 0.0
+    assert call(cfg=bad) == -1
+    bad.rope_base = 10000.0
+    bad.norm_eps = -1.0
+    assert call(cfg=bad) == -1
 
 
 def test_workspace_too_small(lib):
