@@ -39,4 +39,13 @@ from .hca import (  # noqa: F401
     norm_rope_rows,
     attend_norm_rope,
     cache_entries,
+    E2M1_GRID,
+    MX_BLOCK,
+    e2m1_value,
+    mxfp4_quantize,
+    mxfp4_dequantize,
+    mxfp4_pack,
+    mxfp4_unpack,
+    indexer_scores_fp4,
+    topk_recall,
 )

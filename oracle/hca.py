@@ -52,6 +52,13 @@ notes):
     compressor's input too) and normalised when attended.  Normalised queries
     and window rows enter the attention as bf16 values, like the entries.
     The indexer is not core attention and is left as it is.
+  * FP4 indexer variant: the FP4 format is MXFP4 (E2M1 elements, one
+    power-of-two E8M0 scale per 32 consecutive elements along d_I, shared
+    exponent floor(log2 amax) - 2, nearest-even rounding saturating at +-6):
+    the pages give no format, but say FP4 values dequantise losslessly into
+    FP8 because FP8's exponent absorbs the scale -- true for power-of-two
+    scales.  Codes are packed two per byte, the even element in the low
+    nibble.  Index scores are rounded to BF16.
 """
 
 from __future__ import annotations
@@ -66,6 +73,8 @@ __all__ = [
     "hca_layer_prefill", "csa_layer_decode", "hca_layer_decode",
     "rms_norm", "rope_theta", "rope", "entry_position", "QKNorm",
     "norm_rope_rows", "attend_norm_rope", "cache_entries",
+    "E2M1_GRID", "MX_BLOCK", "e2m1_value", "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_pack",
+    "mxfp4_unpack", "indexer_scores_fp4", "topk_recall",
 ]
 
 
@@ -344,6 +353,100 @@ def cache_entries(E_exact: np.ndarray, rate: int, nrm: "QKNorm" = None, first: i
         return round_bf16(E_exact)
     pos = entry_position(np.arange(first, first + E_exact.shape[0]), rate)
     return round_bf16(norm_rope_rows(E_exact, pos, nrm.kv_gamma, nrm))
+
+
+# ----------------------------------------------------------------------------
+# (6) FP4 indexer variant  ([Tricks] "FP4 / FP8 Quantization-Aware Training":
+#     the indexer's QK activations are cached, loaded and multiplied in FP4,
+#     the index scores are kept in BF16; FP4 values dequantise losslessly into
+#     FP8 because FP8's wider exponent absorbs the fine-grained scale)
+# ----------------------------------------------------------------------------
+# E2M1 magnitudes by 3-bit code (sign in bit 3): 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+MX_BLOCK = 32        # elements sharing one scale
+E2M1_EMAX = 2        # exponent of E2M1's largest normal value (6 = 1.5 * 2^2)
+
+
+def _e2m1_code(y: np.ndarray) -> np.ndarray:
+    """Nearest E2M1 code of each value (ties to the even code), saturating at +-6."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.minimum(np.abs(y), 6.0)
+    # candidates: the grid points below and above |y|
+    hi = np.searchsorted(E2M1_GRID, a, side="left").clip(0, 7)
+    lo = (hi - 1).clip(0, 7)
+    d_lo = a - E2M1_GRID[lo]
+    d_hi = E2M1_GRID[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    mag = np.where(pick_hi, hi, lo)
+    neg = (y < 0) & (mag != 0)
+    return (mag + 8 * neg).astype(np.uint8)
+
+
+def e2m1_value(code) -> np.ndarray:
+    """Value of E2M1 codes (bit 3 = sign, bits 0-2 index E2M1_GRID)."""
+    code = np.asarray(code, dtype=np.int64)
+    v = E2M1_GRID[code & 7]
+    return np.where(code & 8, -v, v)
+
+
+def mxfp4_quantize(x: np.ndarray):
+    """MXFP4 quantisation along the last axis (length a multiple of 32).
+
+    Each block of 32 elements gets one power-of-two scale 2^X with
+    X = floor(log2(max |x|)) - 2, clamped to [-127, 127] (X = -127 for an
+    all-zero block), stored as the E8M0 byte X + 127; each element becomes
+    the E2M1 code nearest to x / 2^X (ties to even, saturating at +-6).
+    Returns (codes uint8 [..., d], scales uint8 [..., d/32])."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    assert d % MX_BLOCK == 0
+    xb = x.reshape(x.shape[:-1] + (d // MX_BLOCK, MX_BLOCK))
+    amax = np.max(np.abs(xb), axis=-1)
+    with np.errstate(divide="ignore"):
+        X = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - E2M1_EMAX, -127.0)
+    X = np.clip(X, -127, 127)
+    codes = _e2m1_code(xb / np.exp2(X)[..., None])
+    return codes.reshape(x.shape).astype(np.uint8), (X + 127).astype(np.uint8)
+
+
+def mxfp4_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Values of MXFP4 data: e2m1_value(code) * 2^(scale - 127), block by block."""
+    codes = np.asarray(codes)
+    d = codes.shape[-1]
+    v = e2m1_value(codes).reshape(codes.shape[:-1] + (d // MX_BLOCK, MX_BLOCK))
+    return (v * np.exp2(np.asarray(scales, dtype=np.float64) - 127.0)[..., None]).reshape(codes.shape)
+
+
+def mxfp4_pack(codes: np.ndarray) -> np.ndarray:
+    """Two codes per byte along the last axis: element 2i in the low nibble,
+    element 2i+1 in the high nibble (the cache format)."""
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def mxfp4_unpack(packed: np.ndarray) -> np.ndarray:
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = p & 15
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def indexer_scores_fp4(q_idx: np.ndarray, w_idx: np.ndarray, k_idx: np.ndarray) -> np.ndarray:
+    """Index scores of the FP4 variant: the queries and keys enter as their
+    MXFP4 values (quantised along d_I), the score is formed as in
+    indexer_scores and kept in BF16 (rounded to nearest even)."""
+    qd = mxfp4_dequantize(*mxfp4_quantize(q_idx))
+    kd = mxfp4_dequantize(*mxfp4_quantize(k_idx))
+    return round_bf16(indexer_scores(qd, w_idx, kd))
+
+
+def topk_recall(sel: np.ndarray, ref: np.ndarray) -> float:
+    """Fraction of the reference selection that `sel` also selects."""
+    ref = np.asarray(ref)
+    if ref.size == 0:
+        return 1.0
+    return float(np.intersect1d(np.asarray(sel), ref).size) / float(ref.size)
 
 
 # ----------------------------------------------------------------------------
