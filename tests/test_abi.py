@@ -32,7 +32,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for want in ["csa_compress", "hca_compress", "csa_indexer_topk", "sparse_mqa_attend", "hybrid_attn_decode",
+    for want in ["csa_compress", "hca_compress", "csa_indexer_topk", "sparse_mqa_attend", "rms_norm_rope",
+                 "hybrid_attn_decode",
                  "hybrid_attn_prefill", "hca_workspace_size", "hca_last_error", "hybrid_attn_decode_workspace",
                  "hybrid_attn_prefill_workspace", "hca_version"]:
         assert want in names, want
@@ -149,6 +150,39 @@ def test_decode_workspace_query(lib):
     assert 0 < need < lib.SIZE_MAX and need % 256 == 0
     a.csa_N = 1 << 26  # too many chunks to merge
     assert lib.hybrid_attn_decode_workspace(cfg, a) == lib.SIZE_MAX
+
+
+def _r256(x):
+    return (x + 255) // 256 * 256
+
+
+def test_normalisation_workspace_regions(lib):
+    """With Q/KV normalisation weights the layer calls reserve, past their other
+    scratch, the normalised queries and window rows (bf16) of each normalised
+    layer and the f32 entries ahead of the normaliser (host-side sizing, no GPU)."""
+    cfg = _cfg(lib)
+    H, c, nw = cfg.n_heads, cfg.c, cfg.n_win
+    a = lib.DecodeArgs()
+    a.B, a.csa_q, a.csa_N, a.hca_q, a.hca_N = 8, FAKE, 65536, FAKE, 8192
+    base = lib.hybrid_attn_decode_workspace(cfg, a)
+    a.csa_norm = FAKE
+    one = lib.hybrid_attn_decode_workspace(cfg, a)
+    assert one - base == _r256(8 * H * c * 2) + _r256(8 * nw * c * 2)
+    a.hca_norm = FAKE
+    two = lib.hybrid_attn_decode_workspace(cfg, a)
+    assert two - one == _r256(8 * H * c * 2) + _r256(8 * nw * c * 2) + _r256(8 * c * 4)
+    p = lib.PrefillArgs()
+    T = 65536
+    p.T = T
+    base = lib.hybrid_attn_prefill_workspace(cfg, p)
+    p.csa_norm = FAKE
+    with_norm = lib.hybrid_attn_prefill_workspace(cfg, p)
+    assert with_norm - base == _r256(T * H * c * 2) + _r256(T * c * 2) + _r256((T // cfg.m) * c * 4)
+    # the HCA layer's normalisation alone reserves the same regions (the layers share them)
+    p.csa_norm = None
+    p.hca_kv, p.hca_norm = FAKE, FAKE
+    base_h = lib.hybrid_attn_prefill_workspace(cfg, lib.PrefillArgs(T=T, hca_kv=FAKE))
+    assert lib.hybrid_attn_prefill_workspace(cfg, p) - base_h == with_norm - base
 
 
 def test_fault_injection(lib, monkeypatch):
