@@ -48,4 +48,9 @@ from .hca import (  # noqa: F401
     mxfp4_unpack,
     indexer_scores_fp4,
     topk_recall,
+    classical_block_tokens,
+    paged_rows,
+    ring_window,
+    csa_layer_decode_paged,
+    hca_attend_decode_paged,
 )

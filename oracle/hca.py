@@ -59,6 +59,12 @@ notes):
     FP8 because FP8's exponent absorbs the scale -- true for power-of-two
     scales.  Codes are packed two per byte, the even element in the low
     nibble.  Index scores are rounded to BF16.
+  * Paged cache: a classical block holds the entries of lcm(m, m') raw
+    tokens -- lcm/m CSA entries (and their indexer keys) and lcm/m' HCA
+    entries -- reached through a per-request block table (logical block j
+    covers tokens [j L, (j+1) L)); entry i sits in logical block i // (L/rate),
+    slot i % (L/rate).  The state cache keeps the window as a ring of n_win raw
+    rows, token tau at slot tau % n_win.
 """
 
 from __future__ import annotations
@@ -75,6 +81,8 @@ __all__ = [
     "norm_rope_rows", "attend_norm_rope", "cache_entries",
     "E2M1_GRID", "MX_BLOCK", "e2m1_value", "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_pack",
     "mxfp4_unpack", "indexer_scores_fp4", "topk_recall",
+    "classical_block_tokens", "paged_rows", "ring_window", "csa_layer_decode_paged",
+    "hca_attend_decode_paged",
 ]
 
 
@@ -447,6 +455,59 @@ def topk_recall(sel: np.ndarray, ref: np.ndarray) -> float:
     if ref.size == 0:
         return 1.0
     return float(np.intersect1d(np.asarray(sel), ref).size) / float(ref.size)
+
+
+# ----------------------------------------------------------------------------
+# (7) paged heterogeneous cache  ([Jiedu] cache layout: a fixed per-request
+#     state cache for the sliding window and the uncompressed tail, and a
+#     block-allocated classical cache for the compressed entries; [Tricks]
+#     "Heterogeneous KV Cache Layout": each classical block covers lcm(m, m')
+#     raw tokens)
+# ----------------------------------------------------------------------------
+def classical_block_tokens(m: int, m_hca: int) -> int:
+    """Raw tokens a classical cache block covers: lcm(m, m')."""
+    return int(np.lcm(m, m_hca))
+
+
+def paged_rows(pool: np.ndarray, block_table, idx, rows_per_block: int) -> np.ndarray:
+    """Rows of a paged cache: logical row i lives in physical block
+    block_table[i // rows_per_block], slot i % rows_per_block.
+    pool [P, rows_per_block, width]; idx: logical row indices."""
+    idx = np.asarray(idx, dtype=np.int64)
+    bt = np.asarray(block_table, dtype=np.int64)
+    return np.asarray(pool, dtype=np.float64)[bt[idx // rows_per_block], idx % rows_per_block]
+
+
+def ring_window(ring: np.ndarray, t: int, n_win: int) -> np.ndarray:
+    """Window rows of a query at t from a ring buffer of n_win rows in which
+    token tau sits at slot tau % n_win: tokens max(0, t-n_win+1) .. t, oldest first."""
+    toks = window_rows(t, n_win)
+    return np.asarray(ring, dtype=np.float64)[toks % n_win]
+
+
+def csa_layer_decode_paged(kv_pool, k_pool, block_table, N, ring, q, q_idx, w_idx, t, *, m, m_hca, topk, n_win,
+                           scale, sink=None, norm=None):
+    """csa_layer_decode with the cache in its paged form: N entries reached
+    through the request's block table (lcm(m, m')/m entry rows per block, the
+    keys in a pool of the same blocks) and the window read from the request's
+    ring buffer."""
+    rpb = classical_block_tokens(m, m_hca) // m
+    E = paged_rows(kv_pool, block_table, np.arange(N), rpb)
+    K = paged_rows(k_pool, block_table, np.arange(N), rpb)
+    return csa_layer_decode(E, K, ring_window(ring, t, n_win), q, q_idx, w_idx, t, m=m, topk=topk, n_win=n_win,
+                            scale=scale, sink=sink, norm=norm)
+
+
+def hca_attend_decode_paged(kv_pool, block_table, N, ring, q, t, *, m, m_hca, n_win, scale, sink=None, norm=None):
+    """Dense HCA attention of one decode query with the entries reached through
+    the block table (lcm(m, m')/m' rows per block) and the window from the ring."""
+    rpb = classical_block_tokens(m, m_hca) // m_hca
+    nv = n_visible(t, m_hca, N)
+    E = paged_rows(kv_pool, block_table, np.arange(nv), rpb)
+    win = ring_window(ring, t, n_win)
+    if norm is None:
+        return mqa_attend(q, np.concatenate([E, win], axis=0), scale, sink)
+    return attend_norm_rope(q, t, win, window_rows(t, n_win), scale, norm, sink, rows_ready=E)
 
 
 # ----------------------------------------------------------------------------
