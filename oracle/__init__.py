@@ -53,4 +53,7 @@ from .hca import (  # noqa: F401
     ring_window,
     csa_layer_decode_paged,
     hca_attend_decode_paged,
+    round_e4m3,
+    fp8_kv_quantize,
+    fp8_kv_dequantize,
 )

@@ -59,6 +59,10 @@ notes):
     FP8 because FP8's exponent absorbs the scale -- true for power-of-two
     scales.  Codes are packed two per byte, the even element in the low
     nibble.  Index scores are rounded to BF16.
+  * FP8 KV channels: the channels outside the rotary part are stored as
+    E4M3 (nearest even, saturating at +-448) with one f32 scale per 64
+    channels of a row, scale = group amax / 448; the rotary channels stay
+    BF16.  The pages name the split (FP8 / BF16) but no scale convention.
   * Paged cache: a classical block holds the entries of lcm(m, m') raw
     tokens -- lcm/m CSA entries (and their indexer keys) and lcm/m' HCA
     entries -- reached through a per-request block table (logical block j
@@ -82,7 +86,7 @@ __all__ = [
     "E2M1_GRID", "MX_BLOCK", "e2m1_value", "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_pack",
     "mxfp4_unpack", "indexer_scores_fp4", "topk_recall",
     "classical_block_tokens", "paged_rows", "ring_window", "csa_layer_decode_paged",
-    "hca_attend_decode_paged",
+    "hca_attend_decode_paged", "round_e4m3", "fp8_kv_quantize", "fp8_kv_dequantize",
 ]
 
 
@@ -455,6 +459,56 @@ def topk_recall(sel: np.ndarray, ref: np.ndarray) -> float:
     if ref.size == 0:
         return 1.0
     return float(np.intersect1d(np.asarray(sel), ref).size) / float(ref.size)
+
+
+# ----------------------------------------------------------------------------
+# (6b) FP8 storage of the non-rotated KV channels  ([Tricks] "Partial RoPE 和
+#      Attention Sink": the RoPE channels stay BF16 in the KV cache, the other
+#      KV channels are stored in FP8)
+# ----------------------------------------------------------------------------
+E4M3_MAX = 448.0
+FP8_GROUP = 64       # channels sharing one scale
+
+
+def round_e4m3(y) -> np.ndarray:
+    """Nearest FP8 E4M3 value (ties to even), saturating at +-448.  E4M3 keeps 3
+    mantissa bits; normal exponents -6..8, subnormals in steps of 2^-9."""
+    y = np.asarray(y, dtype=np.float64)
+    a = np.minimum(np.abs(y), E4M3_MAX)
+    with np.errstate(divide="ignore"):
+        e = np.where(a > 0, np.floor(np.log2(np.where(a > 0, a, 1.0))), -6.0)
+    e = np.maximum(e, -6.0)                     # below 2^-6: the subnormal spacing 2^-9
+    step = np.exp2(e - 3.0)
+    q = a / step
+    fl = np.floor(q)
+    frac = q - fl
+    up = (frac > 0.5) | ((frac == 0.5) & (fl % 2 == 1))
+    r = (fl + up) * step
+    return np.where(y < 0, -r, r)
+
+
+def fp8_kv_quantize(rows: np.ndarray, rope_dims: int):
+    """Cache form of KV rows [.., c]: the first c - rope_dims channels in E4M3
+    with one f32 scale per FP8_GROUP channels (scale = group amax / 448, 1 for
+    an all-zero group), the last rope_dims channels in BF16.
+    Returns (fp8 values / scale [.., c-r], scales [.., (c-r)/64], rope part bf16 [.., r])."""
+    rows = np.asarray(rows, dtype=np.float64)
+    c = rows.shape[-1]
+    n = c - rope_dims
+    assert n % FP8_GROUP == 0
+    body = rows[..., :n].reshape(rows.shape[:-1] + (n // FP8_GROUP, FP8_GROUP))
+    amax = np.max(np.abs(body), axis=-1)
+    scale = np.where(amax > 0, amax / E4M3_MAX, 1.0).astype(np.float32).astype(np.float64)
+    codes = round_e4m3(body / scale[..., None])
+    return codes.reshape(rows.shape[:-1] + (n,)), scale, round_bf16(rows[..., n:])
+
+
+def fp8_kv_dequantize(codes: np.ndarray, scales: np.ndarray, rope_part: np.ndarray) -> np.ndarray:
+    """Row values of the FP8 cache form: codes * scale per group, then the BF16 rope part."""
+    codes = np.asarray(codes, dtype=np.float64)
+    n = codes.shape[-1]
+    body = codes.reshape(codes.shape[:-1] + (n // FP8_GROUP, FP8_GROUP)) * np.asarray(scales)[..., None]
+    return np.concatenate([body.reshape(codes.shape), np.asarray(rope_part, dtype=np.float64)], axis=-1)
 
 
 # ----------------------------------------------------------------------------
