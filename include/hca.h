@@ -208,6 +208,43 @@ int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hc
                              const hca_layer_cfg* cfg, int32_t* topk_idx, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * FP4 indexer variant ([Tricks] "FP4 / FP8 Quantization-Aware Training": the
+ * indexer's QK path is cached, loaded and multiplied in FP4; index scores are
+ * kept in BF16; FP4 values dequantise losslessly because the wider format's
+ * exponent absorbs the fine-grained scale).  The FP4 format is MXFP4: E2M1
+ * elements (0, 0.5, 1, 1.5, 2, 3, 4, 6 and negatives; code bit 3 = sign), one
+ * power-of-two scale 2^X per 32 consecutive elements of a row, X =
+ * floor(log2 max|x|) - 2 clamped to [-127, 127] (-127 for an all-zero block),
+ * stored as the byte X + 127; element codes = nearest E2M1 value of x / 2^X
+ * (ties to the even code, saturating at +-6), two per byte, the even element
+ * in the low nibble.
+ *
+ * mxfp4_quantize -- MXFP4 form of `rows` rows of d elements (d a multiple of
+ *   32): x bf16 (x_is_f32 = 0) or f32, row stride ld_x elements; codes [rows]
+ *   [d/2] bytes at row stride ld_codes (a multiple of 16), scales [rows][d/32]
+ *   bytes at row stride ld_scales.  Bit-exact to the definition above.
+ *
+ * csa_indexer_topk_fp4 -- decode indexer + top-k (one query per request, as
+ *   csa_indexer_topk in HCA_MODE_DECODE) with FP4 keys and queries and BF16
+ *   scores: I(t,s) = bf16(sum_j w[t,j] ReLU(q4[t,j,:] . k4[s,:])), q4 and k4
+ *   the MXFP4 values of q_I and K_I.  Takes the 64 x 128 indexer only.
+ *   q_idx [B, 64, 128] bf16 (rounded to its MXFP4 values inside the call);
+ *   w_idx [B, 64] f32; request r's keys: codes at k_codes + r*k_seq_stride*64
+ *   ([N][64] bytes), scales at k_scales + r*k_seq_stride*4 ([N][4] bytes,
+ *   readable up to the next multiple of 4 keys); with B > 1, k_seq_stride >=
+ *   that multiple of 4 and itself a multiple of 4.  topk_idx [B, topk] as in
+ *   csa_indexer_topk.  ws: csa_indexer_topk_fp4_workspace(cfg, B, N) bytes.
+ *   Device-side waits that give up are reported by hca_check_device.
+ * ------------------------------------------------------------------------- */
+int mxfp4_quantize(const void* x, int x_is_f32, long long ld_x, int rows, int d, uint8_t* codes,
+                   long long ld_codes, uint8_t* scales, long long ld_scales, void* stream);
+int csa_indexer_topk_fp4(const hca_bf16* q_idx, const float* w_idx, const uint8_t* k_codes,
+                         const uint8_t* k_scales, long long k_seq_stride, int N, const int32_t* q_pos,
+                         int B, const hca_layer_cfg* cfg, int32_t* topk_idx, void* ws, size_t ws_bytes,
+                         void* stream);
+size_t csa_indexer_topk_fp4_workspace(const hca_layer_cfg* cfg, int B, int N);
+
+/* ---------------------------------------------------------------------------
  * sparse_mqa_attend -- core shared-KV multi-query attention over compressed
  * entries plus the sliding window, one softmax ([QbitAI] CSA step three, the
  * KV-entry-as-key-and-value remark and the sliding-window paragraph;

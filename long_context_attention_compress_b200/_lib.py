@@ -82,6 +82,12 @@ _indexer = _sig("csa_indexer_topk", c_int, [c_void_p, c_void_p, c_void_p, c_ll, 
 _mqa = _sig("sparse_mqa_attend", c_int, [c_void_p, c_void_p, c_ll, c_int, c_void_p, c_int, c_int, c_void_p, c_ll,
                                          c_void_p, c_int, c_int, ctypes.POINTER(LayerCfg), c_void_p, c_int, c_void_p,
                                          c_void_p, c_size, c_void_p])
+_mxfp4_quantize = _sig("mxfp4_quantize", c_int, [c_void_p, c_int, c_ll, c_int, c_int, c_void_p, c_ll, c_void_p, c_ll,
+                                                 c_void_p])
+_indexer_fp4 = _sig("csa_indexer_topk_fp4", c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_ll, c_int, c_void_p,
+                                                    c_int, ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_size,
+                                                    c_void_p])
+_indexer_fp4_ws = _sig("csa_indexer_topk_fp4_workspace", c_size, [ctypes.POINTER(LayerCfg), c_int, c_int])
 _norm_rope = _sig("rms_norm_rope", c_int, [c_void_p, c_int, c_ll, c_ll, c_int, c_int, c_void_p, c_int, c_int,
                                           c_void_p, ctypes.POINTER(LayerCfg), c_void_p, c_ll, c_ll, c_void_p])
 _decode = _sig("hybrid_attn_decode", c_int, [ctypes.POINTER(LayerCfg), ctypes.POINTER(DecodeArgs), c_void_p, c_size,
@@ -202,6 +208,40 @@ def csa_indexer_topk(q_idx, w_idx, k_idx, q_pos, cfg: LayerCfg, mode=HCA_MODE_PR
     _check(_indexer(_ptr(q_idx, BF16, "q_idx"), _ptr(w_idx, F32, "w_idx"), _ptr(k_idx, BF16, "k_idx"), kstride, N,
                     _ptr(q_pos, I32, "q_pos"), Tq, mode, ctypes.byref(cfg), _ptr(out, I32, "out"),
                     None if ws is None else ws.data_ptr(), nb, _stream(stream)))
+    return out
+
+
+def mxfp4_quantize(x, codes=None, scales=None, stream=None):
+    """MXFP4 form of the rows of x [rows, d] (bf16 or float32; d a multiple of 32):
+    returns (codes uint8 [rows, d/2], scales uint8 [rows, d/32])."""
+    rows, d = x.shape
+    if x.dtype not in (BF16, F32):
+        raise TypeError(f"x: dtype {x.dtype}")
+    if codes is None:
+        codes = torch.empty((rows, d // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((rows, d // 32), dtype=torch.uint8, device=x.device)
+    _check(_mxfp4_quantize(_ptr(x, None, "x"), 1 if x.dtype == F32 else 0, x.stride(0), rows, d,
+                           _ptr(codes, torch.uint8, "codes"), codes.stride(0), _ptr(scales, torch.uint8, "scales"),
+                           scales.stride(0), _stream(stream)))
+    return codes, scales
+
+
+def csa_indexer_topk_fp4(q_idx, w_idx, k_codes, k_scales, q_pos, cfg: LayerCfg, out=None, ws=None, stream=None):
+    """Decode indexer + top-k over MXFP4 keys (k_codes [B, N_alloc, 64] uint8, k_scales
+    [B, N_alloc, 4] uint8, N = q's visible range up to N_alloc) with BF16 scores."""
+    B = q_idx.shape[0]
+    N = k_codes.shape[1]
+    if out is None:
+        out = torch.empty((B, cfg.topk), dtype=I32, device=q_idx.device)
+    nb = int(_indexer_fp4_ws(ctypes.byref(cfg), B, N))
+    if nb == SIZE_MAX:
+        raise HcaError(-2, "csa_indexer_topk_fp4: unsupported configuration")
+    ws, nb = _workspace(nb, ws, q_idx.device)
+    _check(_indexer_fp4(_ptr(q_idx, BF16, "q_idx"), _ptr(w_idx, F32, "w_idx"), _ptr(k_codes, torch.uint8, "k_codes"),
+                        _ptr(k_scales, torch.uint8, "k_scales"), k_codes.stride(0) // 64, N,
+                        _ptr(q_pos, I32, "q_pos"), B, ctypes.byref(cfg), _ptr(out, I32, "out"),
+                        None if ws is None else ws.data_ptr(), nb, _stream(stream)))
     return out
 
 

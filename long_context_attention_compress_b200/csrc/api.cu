@@ -312,9 +312,10 @@ int hca_check_device(void) {
   const unsigned int w1 = read_and_clear_indexer_tc_error();
   const unsigned int w2 = read_and_clear_mqa_tc_error();
   const unsigned int w3 = read_and_clear_select_error();
-  if (w1 == 0xffffffffu || w2 == 0xffffffffu || w3 == 0xffffffffu)
+  const unsigned int w4 = read_and_clear_indexer_fp4_error();
+  if (w1 == 0xffffffffu || w2 == 0xffffffffu || w3 == 0xffffffffu || w4 == 0xffffffffu)
     return fail(HCA_ERR_CUDA, "hca_check_device: cannot read the device error word");
-  const unsigned int w = w1 | (w2 << 1);
+  const unsigned int w = w1 | (w2 << 1) | (w4 << 2);
   if (w) return fail(HCA_ERR_DEVICE_CHECK, "hca_check_device: a kernel gave up waiting (error word 0x%x)", w);
   if (w3) return fail(HCA_ERR_DEVICE_CHECK, "hca_check_device: a top-k histogram disagreed with its scores");
   return HCA_OK;
@@ -973,6 +974,111 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
     if ((s = mark()) != HCA_OK) return s;
   }
   g_last_launches = g_launch_counter;
+  return HCA_OK;
+}
+
+// ---- FP4 indexer variant -----------------------------------------------------------
+int mxfp4_quantize(const void* x, int x_is_f32, long long ld_x, int rows, int d, uint8_t* codes, long long ld_codes,
+                   uint8_t* scales, long long ld_scales, void* stream) {
+  g_err.clear();
+  CHECK(rows >= 0 && d > 0 && d % 32 == 0, HCA_ERR_INVALID_ARG, "mxfp4_quantize: rows=%d d=%d (d a multiple of 32)",
+        rows, d);
+  CHECK(ld_x >= d && ld_codes >= d / 2 && ld_scales >= d / 32, HCA_ERR_INVALID_ARG, "mxfp4_quantize: row strides");
+  CHECK(ld_codes % 16 == 0, HCA_ERR_INVALID_ARG, "mxfp4_quantize: ld_codes %lld not a multiple of 16", ld_codes);
+  if (rows == 0) return HCA_OK;
+  CHECK(x != nullptr && codes != nullptr && scales != nullptr, HCA_ERR_INVALID_ARG, "mxfp4_quantize: null pointer");
+  CHECK(aligned16(codes), HCA_ERR_INVALID_ARG, "mxfp4_quantize: codes not 16-byte aligned");
+  CHECK(((reinterpret_cast<uintptr_t>(x)) & (x_is_f32 ? 3u : 1u)) == 0, HCA_ERR_INVALID_ARG,
+        "mxfp4_quantize: x misaligned");
+  if (injected("mxfp4_quantize")) return fail(HCA_ERR_INJECTED, "mxfp4_quantize: injected");
+  CUDA_TRY(launch_mxfp4_quantize(x, x_is_f32 != 0, ld_x, rows, d, codes, ld_codes, scales, ld_scales,
+                                 as_stream(stream)),
+           "mxfp4_quantize");
+  return HCA_OK;
+}
+
+static size_t fp4_indexer_ws(const hca_layer_cfg* cfg, int B, int N) {
+  const IndexerPlan p = plan_indexer(B, N, cfg->topk);
+  return round256(p.bytes) + round256((size_t)B * cfg->n_idx_heads * cfg->d_idx * 2);
+}
+
+size_t csa_indexer_topk_fp4_workspace(const hca_layer_cfg* cfg, int B, int N) {
+  if (check_cfg(cfg) != HCA_OK || B < 0 || N < 0) return (size_t)-1;
+  if (indexer_ok(N, cfg->topk, HCA_MODE_DECODE) != HCA_OK) return (size_t)-1;
+  return fp4_indexer_ws(cfg, B, N);
+}
+
+int csa_indexer_topk_fp4(const hca_bf16* q_idx, const float* w_idx, const uint8_t* k_codes, const uint8_t* k_scales,
+                         long long k_seq_stride, int N, const int32_t* q_pos, int B, const hca_layer_cfg* cfg,
+                         int32_t* topk_idx, void* ws, size_t ws_bytes, void* stream) {
+  g_err.clear();
+  int s = check_cfg(cfg);
+  if (s != HCA_OK) return s;
+  CHECK(indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx), HCA_ERR_UNSUPPORTED,
+        "csa_indexer_topk_fp4: the FP4 indexer takes 64 heads x 128 (got %d x %d)", cfg->n_idx_heads, cfg->d_idx);
+  CHECK(B >= 0 && B <= 65535 && N > 0, HCA_ERR_INVALID_ARG, "csa_indexer_topk_fp4: B=%d N=%d", B, N);
+  s = indexer_ok(N, cfg->topk, HCA_MODE_DECODE);
+  if (s != HCA_OK) return s;
+  const long long n4 = ((long long)N + 3) / 4 * 4;
+  CHECK(B <= 1 || (k_seq_stride >= n4 && k_seq_stride % 4 == 0), HCA_ERR_INVALID_ARG,
+        "csa_indexer_topk_fp4: k_seq_stride %lld (need >= %lld keys, a multiple of 4)", k_seq_stride, n4);
+  const size_t need = fp4_indexer_ws(cfg, B, N);
+  CHECK(ws_bytes >= need, HCA_ERR_WORKSPACE, "csa_indexer_topk_fp4: workspace %zu < %zu", ws_bytes, need);
+  if (B == 0) return HCA_OK;
+  CHECK_PTR(q_idx, "csa_indexer_topk_fp4: q_idx");
+  CHECK_PTR(w_idx, "csa_indexer_topk_fp4: w_idx");
+  CHECK_PTR(k_codes, "csa_indexer_topk_fp4: k_codes");
+  CHECK_PTR(k_scales, "csa_indexer_topk_fp4: k_scales");
+  CHECK_PTR(topk_idx, "csa_indexer_topk_fp4: topk_idx");
+  CHECK(q_pos != nullptr, HCA_ERR_INVALID_ARG, "csa_indexer_topk_fp4: q_pos null");
+  CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
+        "csa_indexer_topk_fp4: ws null or not 256-byte aligned");
+  if (injected("csa_indexer_topk_fp4")) return fail(HCA_ERR_INJECTED, "csa_indexer_topk_fp4: injected");
+
+  cudaStream_t st = as_stream(stream);
+  const IndexerPlan p = plan_indexer(B, N, cfg->topk);
+  char* wsb = reinterpret_cast<char*>(ws);
+  float* scores = reinterpret_cast<float*>(ws);
+  bf16* q4 = reinterpret_cast<bf16*>(wsb + round256(p.bytes));
+  // the query's MXFP4 values (bf16), then the scores over the FP4 keys
+  CUDA_TRY(launch_mxfp4_roundtrip(reinterpret_cast<const bf16*>(q_idx), B * cfg->n_idx_heads, cfg->d_idx, q4, st),
+           "csa_indexer_topk_fp4: query rounding");
+  const bool hist = p.hist_ctas > 0;
+  if (hist)
+    CUDA_TRY(cudaMemsetAsync(wsb + p.hist_off, 0, (size_t)B * (2 * kHistBins + 1) * sizeof(int), st),
+             "histogram reset");
+  CUDA_TRY(launch_indexer_decode_fp4(q4, w_idx, k_codes, k_scales, k_seq_stride, N, q_pos, B, cfg->m, scores, p.ld,
+                                     device_sm_count(), st, hist ? reinterpret_cast<int*>(wsb + p.hist_off) : nullptr),
+           "csa_indexer_topk_fp4: scores");
+  if (hist) {
+    HistSelect a;
+    a.scores = scores;
+    a.ld = p.ld;
+    a.q_pos = q_pos;
+    a.rate = cfg->m;
+    a.N = N;
+    a.k = cfg->topk;
+    a.hist = reinterpret_cast<int*>(wsb + p.hist_off);
+    a.B = B;
+    a.done = reinterpret_cast<int*>(wsb + p.done_off);
+    a.cnt = reinterpret_cast<int2*>(wsb + p.cnt_off);
+    a.above = reinterpret_cast<int32_t*>(wsb + p.above_off);
+    a.eq = reinterpret_cast<uint64_t*>(wsb + p.eq_off);
+    a.C = p.hist_ctas;
+    a.slice = kHistSlice;
+    a.out = topk_idx;
+    CUDA_TRY(launch_select_hist(a, B, st), "csa_indexer_topk_fp4: select (histogram threshold)");
+    return HCA_OK;
+  }
+  SelectRows rows;
+  rows.chunks = p.chunks;
+  rows.chunk = p.chunk;
+  rows.n_rows = B * p.chunks;
+  rows.rate = cfg->m;
+  rows.N = N;
+  rows.q_pos = q_pos;
+  rows.ld_scores = p.ld;
+  CUDA_TRY(launch_select_rows(scores, rows, cfg->topk, topk_idx, st), "csa_indexer_topk_fp4: select");
   return HCA_OK;
 }
 

@@ -18,6 +18,18 @@ cudaError_t launch_compress(const bf16* cand, int ld_cand, const bf16* logits, i
                             cudaStream_t stream, float* out_f32 = nullptr);
 // (out_f32 != nullptr: the entries are written there in f32, same strides, and out is unused)
 
+// ---- indexer_fp4.cu (FP4 indexer variant) ----------------------------------------
+cudaError_t launch_mxfp4_quantize(const void* x, bool x_f32, long long ld_x, int rows, int d, uint8_t* codes,
+                                  long long ld_codes, uint8_t* scales, long long ld_scales, cudaStream_t stream);
+cudaError_t launch_mxfp4_roundtrip(const bf16* x, int rows, int d, bf16* y, cudaStream_t stream);
+// Decode indexer over MXFP4 keys (codes [N][64 B], scales [ceil4(N)][4 B] per request, requests
+// k_seq_stride keys apart) with a bf16 query already rounded to its MXFP4 values; BF16 scores.
+cudaError_t launch_indexer_decode_fp4(const bf16* q4, const float* w_idx, const uint8_t* k_codes,
+                                      const uint8_t* k_scales, long long k_seq_stride, int N, const int32_t* q_pos,
+                                      int B, int rate, float* scores, long long ld_scores, int num_sms,
+                                      cudaStream_t stream, int* hist);
+unsigned int read_and_clear_indexer_fp4_error();
+
 // ---- norm_rope.cu -------------------------------------------------------------
 // Q/KV RMSNorm + partial RoPE of rows (see rms_norm_rope in hca.h for the row
 // addressing and positions).

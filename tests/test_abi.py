@@ -152,6 +152,41 @@ def test_decode_workspace_query(lib):
     assert lib.hybrid_attn_decode_workspace(cfg, a) == lib.SIZE_MAX
 
 
+def test_fp4_entry_points_check_arguments(lib):
+    """mxfp4_quantize / csa_indexer_topk_fp4 reject bad shapes, strides and
+    pointers on the host (nothing is launched: no GPU needed)."""
+    from long_context_attention_compress_b200 import workloads as wl
+    cfg = _cfg(lib)
+    q = lambda **kw: lib._mxfp4_quantize(kw.get("x", FAKE), 0, kw.get("ld", 128), kw.get("rows", 4),  # noqa: E731
+                                         kw.get("d", 128), kw.get("codes", FAKE), kw.get("ldc", 64),
+                                         kw.get("scales", FAKE), kw.get("lds", 4), None)
+    assert q(rows=0) == 0
+    assert q(d=100) == -1 and "multiple of 32" in lib.last_error()
+    assert q(ld=64) == -1 and q(ldc=32) == -1 and q(lds=2) == -1
+    assert q(ldc=72) == -1 and "16" in lib.last_error()
+    assert q(x=None) == -1 and q(codes=None) == -1 and q(scales=None) == -1
+    assert q(codes=FAKE + 8) == -1 and "aligned" in lib.last_error()
+    N, B = 262144, 8
+    ws_need = lib._indexer_fp4_ws(ctypes.byref(cfg), B, N)
+    assert 0 < ws_need < lib.SIZE_MAX and ws_need % 256 == 0
+
+    def call(**kw):
+        a = dict(q=FAKE, w=FAKE, codes=FAKE, scales=FAKE, stride=N, N=N, pos=FAKE, B=B, out=FAKE, ws=FAKE,
+                 nb=ws_need, cfg=cfg)
+        a.update(kw)
+        return lib._indexer_fp4(a["q"], a["w"], a["codes"], a["scales"], a["stride"], a["N"], a["pos"], a["B"],
+                                ctypes.byref(a["cfg"]), a["out"], a["ws"], a["nb"], None)
+
+    assert call(nb=ws_need - 1) == -3
+    assert call(stride=N - 4) == -1 and "k_seq_stride" in lib.last_error()
+    assert call(stride=N + 2) == -1
+    assert call(codes=None) == -1 and call(scales=FAKE + 4) == -1 and call(pos=None) == -1
+    assert call(N=0) == -1
+    assert call(B=0) == 0                                    # nothing to do
+    small = lib.make_cfg(wl.TINY)
+    assert call(cfg=small) == -2 and "64 heads x 128" in lib.last_error()
+
+
 def _r256(x):
     return (x + 255) // 256 * 256
 
