@@ -4,8 +4,11 @@ Each case replaces one oracle function with a plausible wrong version -- a
 rotation in the wrong sense or over the wrong channels, a forgotten output
 rotation, a dropped weight or epsilon, an entry placed at its block's start,
 ties rounded away from even, a shared exponent rounded up, ReLU after the head
-sum, a dropped positional bias, a missing logit scale, a transposed page
-address -- and checks that at least one of the named pins then fails.  The
+sum, a dropped positional bias or swapped bias rows, a missing logit scale, a
+transposed page address, visibility off by one, a window without the query's
+own token, top-k ties to the higher index, a combine without its max
+rescaling or with the sink counted per part -- and checks that at least one
+of the named pins then fails.  The
 mistakes live only in this test, patched into the oracle module for its
 duration.
 """
@@ -106,7 +109,56 @@ def _paged_rows_transposed(pool, block_table, idx, rows_per_block):
     return np.asarray(pool, dtype=np.float64)[bt[idx % rows_per_block], idx // rows_per_block]
 
 
+_nvis, _wrows, _topk, _comb, _win = H.n_visible, H.window_rows, H.topk_select, H.combine_partials, H._csa_window
+
+
+def _n_visible_off_by_one(t, rate, n_entries):
+    return int(min(n_entries, t // rate))
+
+
+def _window_without_t(t, n_win):
+    return np.arange(max(0, t - n_win), t)
+
+
+def _topk_ties_to_higher_index(scores, k):
+    scores = np.asarray(scores, dtype=np.float64)
+    n = scores.shape[0]
+    return np.lexsort((-np.arange(n), -scores))[:min(k, n)].astype(np.int64)
+
+
+def _combine_without_rescale(parts, sink=None):
+    num = sum(p[2] for p in parts)
+    den = sum(p[1] for p in parts)
+    return num / den[:, None]
+
+
+def _combine_sink_per_part(parts, sink=None):
+    if sink is None:
+        return _comb(parts)
+    ms = np.stack([p[0] for p in parts])
+    M = np.max(ms, axis=0)
+    z = np.asarray(sink, dtype=np.float64)
+    num = sum(np.exp(p[0] - M)[:, None] * p[2] for p in parts)
+    den = sum(np.exp(p[0] - M) * p[1] + np.exp(z - M) for p in parts)
+    return num / den[:, None]
+
+
+def _csa_window_bias_swapped(i, m, T):
+    lo, hi, b0 = _win(i, m, T)
+    return lo, hi, (m - b0) if i > 0 else b0
+
+
 CASES = {
+    "visibility off by one": ({"n_visible": _n_visible_off_by_one},
+                              [T0.test_golden_visibility_and_window, T0.test_visibility_brute_force]),
+    "window misses the query's token": ({"window_rows": _window_without_t}, [T0.test_golden_visibility_and_window]),
+    "top-k ties to the higher index": ({"topk_select": _topk_ties_to_higher_index}, [T0.test_golden_topk_ties]),
+    "combine without max rescaling": ({"combine_partials": _combine_without_rescale},
+                                      [lambda: T0.test_split_combine_equals_unsplit([13, 29])]),
+    "sink counted once per part": ({"combine_partials": _combine_sink_per_part},
+                                   [lambda: T0.test_sink_split_combine_equals_unsplit([13, 29])]),
+    "CSA bias rows swapped": ({"_csa_window": _csa_window_bias_swapped},
+                              [T0.test_golden_csa_overlap, T0.test_csa_previous_block_bias_rows]),
     "rope turns the wrong way": ({"rope": _rope_wrong_sense}, [TN.test_rope_hand_worked]),
     "rope on the first channels": ({"rope": _rope_first_channels},
                                    [TN.test_rope_hand_worked, TN.test_rope_is_a_rotation_group]),
