@@ -187,6 +187,26 @@ def test_fp4_entry_points_check_arguments(lib):
     assert call(cfg=small) == -2 and "64 heads x 128" in lib.last_error()
 
 
+def test_empty_inputs_are_noops(lib):
+    """Zero rows, requests or tokens: every entry point returns HCA_OK without
+    touching the device (on this GPU-less host a launch or copy would fail)."""
+    cfg = _cfg(lib)
+    assert lib._csa_compress(FAKE, 512, FAKE, 512, FAKE, 512, 0, 512, 4, FAKE, 512, None) == 0
+    assert lib._csa_compress(FAKE, 512, FAKE, 512, FAKE, 512, 3, 512, 4, FAKE, 512, None) == 0  # < one block
+    assert lib._hca_compress(FAKE, 512, FAKE, 512, FAKE, 512, 0, 0, 128, 512, 128, FAKE, 512, 0, None) == 0
+    assert lib._hca_compress(FAKE, 512, FAKE, 512, FAKE, 512, 4, 65536, 0, 512, 128, FAKE, 512, 512, None) == 0
+    assert lib._indexer(FAKE, FAKE, FAKE, 0, 4096, FAKE, 0, 1, ctypes.byref(cfg), FAKE, None, 0, None) == 0
+    assert lib._mqa(FAKE, FAKE, 0, 100, None, 0, 128, FAKE, 0, FAKE, 0, 1, ctypes.byref(cfg), None, 0, FAKE, None,
+                    0, None) == 0
+    a = lib.DecodeArgs()
+    a.B, a.csa_q = 0, FAKE
+    assert lib._decode(ctypes.byref(cfg), ctypes.byref(a), None, 0, None) == 0
+    p = lib.PrefillArgs()
+    p.T = 0
+    assert lib._prefill(ctypes.byref(cfg), ctypes.byref(p), None, 0, None) == 0
+    assert lib._mxfp4_quantize(FAKE, 0, 128, 0, 128, FAKE, 64, FAKE, 4, None) == 0
+
+
 def _r256(x):
     return (x + 255) // 256 * 256
 
