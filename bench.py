@@ -128,6 +128,15 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.rows)}
 
 
+def clock_rejected(c) -> bool:
+    """A timed region whose clocks saw a hardware or thermal slowdown, or an SM clock
+    well below its maximum with no reason reported (a leftover clock lock)."""
+    if set(c.get("reasons", [])) & {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}:
+        return True
+    sm, smax = c.get("sm_mhz"), c.get("sm_max_mhz")
+    return bool(sm and smax and sm < 0.8 * smax and not c.get("reasons"))
+
+
 # ----------------------------------------------------------------------------
 # workloads
 # ----------------------------------------------------------------------------
@@ -536,10 +545,19 @@ def run_ours(a):
             a.steps = int(t.item())
     # phase breakdown pass (events between kernels, one sync per step)
     _, phase_ms = timed_steps(bench, min(a.steps, 50), flush, rank, ws, device, record=True)
-    # headline: K steps without intermediate host syncs
-    with ClockSampler(local) as clk:
-        total_ms, _ = timed_steps(bench, a.steps, flush, rank, ws, device, record=False)
-    total_ms = reduce_max(total_ms, ws, device)
+    # headline: K steps without intermediate host syncs; a run whose clock record
+    # shows a hardware/thermal slowdown (or clocks stuck low with no reason) is
+    # taken once more, on every rank alike
+    def headline():
+        with ClockSampler(local) as clk:
+            t, _ = timed_steps(bench, a.steps, flush, rank, ws, device, record=False)
+        return reduce_max(t, ws, device), clk.summary()
+
+    total_ms, clocks = headline()
+    if reduce_max(1.0 if clock_rejected(clocks) else 0.0, ws, device) > 0.0:
+        first = clocks["reasons"] or ["sm clock %s of %s MHz" % (clocks["sm_mhz"], clocks["sm_max_mhz"])]
+        total_ms, clocks = headline()
+        clocks = dict(clocks, remeasured_after=first)
     ms = total_ms / a.steps
     value = bench.units * ws / (ms / 1e3)
 
@@ -592,7 +610,7 @@ def run_ours(a):
            "gpu_launches": launches * a.steps,
            "phase_ms": {k: round(v, 4) for k, v in phase_ms.items()},
            "roofline": roof,
-           "clocks": clk.summary()}
+           "clocks": clocks}
     if a.qk_norm and isinstance(bench, PrefillBench):
         out["qk_norm_prologue"] = norm_prologue_roofline(bench, flush, pk)
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
