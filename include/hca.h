@@ -191,8 +191,12 @@ int csa_indexer_topk(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* 
  *   - Limit: calls whose scratch need (the same bytes
  *     hca_workspace_size(HCA_OP_INDEXER_TOPK, cfg, Tq, N, mode) reports)
  *     exceeds HCA_NOALLOC_SCRATCH_BYTES return HCA_ERR_WORKSPACE and launch
- *     nothing.  For the 64 x 128 indexer and top-1024 that is, e.g., up to
- *     8 requests x 262,144 entries or 32 x 32,768.
+ *     nothing.  For the 64 x 128 indexer and top-1024 in decode mode: a
+ *     request of up to 49,152 entries needs its f32 score row (4 B per
+ *     entry), so 32 requests x 32,768 entries fit (4 MiB); a longer request
+ *     also needs the histogram select's regions (about 12 B per entry in
+ *     all), so 5 requests x 262,144 entries fit (about 15.5 MiB) and 6 do
+ *     not.
  *   - The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before any
  *     stream capture.  It allocates nothing.
