@@ -36,6 +36,9 @@ from long_context_attention_compress_b200 import workloads as wl  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
 MIB = 1 << 20
+DEFAULT_WORKLOAD = "hybrid_decode_b8_1m"
+# the headline region is repeated until it has run this long (>= ~10 clock samples at 50 ms)
+HEADLINE_MIN_S = 0.75
 
 
 # ----------------------------------------------------------------------------
@@ -96,6 +99,7 @@ class ClockSampler:
                                           "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             # the timed region starts only once the sampler is producing samples
+            # (that first sample is kept with the others)
             self.first = self.proc.stdout.readline()
         except (FileNotFoundError, OSError):
             self.proc = None
@@ -111,10 +115,7 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        for line in out.splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.rows.append(parts)
+        self.rows = parse_clock_rows(self.first + out)
         return False
 
     def summary(self):
@@ -126,6 +127,16 @@ class ClockSampler:
         reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
                 "reasons": reasons, "samples": len(self.rows)}
+
+
+def parse_clock_rows(text: str):
+    """nvidia-smi CSV rows (index, sm MHz, max MHz, power, reasons...) as lists of fields."""
+    rows = []
+    for line in text.splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) >= 9:
+            rows.append(parts)
+    return rows
 
 
 def clock_rejected(c) -> bool:
@@ -176,11 +187,12 @@ def source_hash(files):
 class DecodeBench:
     """Hybrid / CSA / HCA decode.  Per step: one hybrid_attn_decode call."""
 
-    def __init__(self, name, spec, seed, device, qk_norm=False):
+    def __init__(self, name, spec, seed, device, qk_norm=False, indexer="bf16"):
         import long_context_attention_compress_b200 as hca
         self.hca = hca
         self.name = name
         self.spec = spec
+        self.indexer = indexer
         s = self.shape = spec["shape"]
         B, ctx = spec["B"], spec["ctx"]
         # Q/KV normalisation + partial RoPE: synthetic weights per layer
@@ -215,6 +227,16 @@ class DecodeBench:
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
         self.norm_kw = {k: v for k, v in self.norm_kw.items()
                         if (k == "csa_norm" and self.csa is not None) or (k == "hca_norm" and self.hcad is not None)}
+        if indexer == "fp4":
+            # the cache form of the indexer keys: MXFP4 codes + scales (64 + 4 B per key)
+            K = self.csa.pop("K_I")
+            N = K.shape[1]
+            codes = torch.empty((B, N, s.d_idx // 2), dtype=torch.uint8, device=dev)
+            scales = torch.empty((B, N, s.d_idx // 32), dtype=torch.uint8, device=dev)
+            for b in range(B):
+                hca.mxfp4_quantize(K[b], codes=codes[b], scales=scales[b])
+            del K
+            self.norm_kw["csa_k4"] = (codes, scales)
         self.args, self._keep = hca.make_decode_args(B, self.q_pos, csa=self.csa, hca=self.hcad,
                                                      csa_topk_idx=self.idx, csa_out=self.csa_out,
                                                      hca_out=self.hca_out, events=self.events, **self.norm_kw)
@@ -239,7 +261,8 @@ class DecodeBench:
             out["hca_compress"] = B * (2 * s.m_hca * s.c * 2 + s.c * 2)
         if self.csa is not None:
             N = self.csa["E"].shape[1]
-            out["indexer_scores"] = B * (N * s.d_idx * 2 + s.n_idx_heads * (s.d_idx * 2 + 4))
+            key_bytes = s.d_idx // 2 + s.d_idx // 32 if self.indexer == "fp4" else s.d_idx * 2
+            out["indexer_scores"] = B * (N * key_bytes + s.n_idx_heads * (s.d_idx * 2 + 4))
             out["topk_select"] = B * s.topk * 4
             out["csa_attention"] = B * ((min(s.topk, N) + s.n_win) * s.c * 2 + 2 * s.n_heads * s.c * 2 + s.topk * 4)
         if self.hcad is not None:
@@ -250,7 +273,9 @@ class DecodeBench:
     def config(self):
         s = self.shape
         c = {"workload": self.name, "batch": self.B, "context": self.ctx, "c": s.c, "heads": s.n_heads,
-             "topk": s.topk, "indexer": f"{s.n_idx_heads}x{s.d_idx}", "n_win": s.n_win}
+             "topk": s.topk, "indexer": f"{s.n_idx_heads}x{s.d_idx}" + (" MXFP4 keys, BF16 scores"
+                                                                         if self.indexer == "fp4" else ""),
+             "n_win": s.n_win}
         if self.csa is not None:
             c["csa_entries"] = int(self.csa["E"].shape[1])
         if self.hcad is not None:
@@ -307,9 +332,15 @@ class DecodeBench:
             if self.csa is not None:
                 d = wl.csa_decode_inputs(s, 1, self.ctx, seed=900 + b, cache_std=spec["cache_std"])
                 f = lambda x: x[0].float().numpy().astype(np.float64)  # noqa: E731
-                oracle.csa_layer_decode(f(d["E"]), f(d["K_I"]), f(d["win"]), f(d["q"]), f(d["q_idx"]),
-                                        d["w_idx"][0].double().numpy(), t, m=s.m, topk=s.topk, n_win=s.n_win,
-                                        scale=s.scale)
+                if getattr(self, "indexer", "bf16") == "fp4":
+                    nv = oracle.n_visible(t, s.m, d["E"].shape[1])
+                    sc = oracle.indexer_scores_fp4(f(d["q_idx"]), d["w_idx"][0].double().numpy(), f(d["K_I"])[:nv])
+                    sel = oracle.topk_select(sc, s.topk)
+                    oracle.mqa_attend(f(d["q"]), np.concatenate([f(d["E"])[sel], f(d["win"])]), s.scale)
+                else:
+                    oracle.csa_layer_decode(f(d["E"]), f(d["K_I"]), f(d["win"]), f(d["q"]), f(d["q_idx"]),
+                                            d["w_idx"][0].double().numpy(), t, m=s.m, topk=s.topk, n_win=s.n_win,
+                                            scale=s.scale)
             if self.hcad is not None:
                 wb = "block_cand" in self.hcad
                 d = wl.hca_decode_inputs(s, 1, self.ctx, seed=900 + b, cache_std=spec["cache_std"], with_block=wb)
@@ -399,25 +430,38 @@ class PrefillBench:
         T = self.T
         d = wl.prefill_inputs(s, T, seed=0, with_hca=False)
         f = lambda x: x.float().numpy().astype(np.float64)  # noqa: E731
+
+        class Rows:  # float64 rows of a bf16 tensor, converted one query at a time
+            def __init__(self, t):
+                self.t = t
+
+            def __getitem__(self, i):
+                return self.t[i].float().numpy().astype(np.float64)
         qs = np.linspace(T // 2, T - 1, n_q).astype(int).tolist()
         t0 = time.perf_counter()
         oracle.csa_layer_prefill(f(d["cand"]), f(d["logits"]), f(d["kidx_cand"]), f(d["bias_csa"]),
-                                 d["q_idx"], d["w_idx"].double().numpy(), d["q"], m=s.m, topk=s.topk,
+                                 Rows(d["q_idx"]), d["w_idx"].double().numpy(), Rows(d["q"]), m=s.m, topk=s.topk,
                                  d_idx=s.d_idx, n_win=s.n_win, scale=s.scale, queries=qs)
         return time.perf_counter() - t0
 
 
-def make_bench(name, seed, device, tokens=None, qk_norm=False):
+def make_bench(name, seed, device, tokens=None, qk_norm=False, indexer="bf16"):
     spec = wl.WORKLOADS[name]
     if qk_norm:
         name = f"{name}+qk_norm"  # the layer with Q/KV RMSNorm + partial RoPE (not the headline workload)
     if spec["kind"] == "prefill":
+        if indexer != "bf16":
+            raise SystemExit("--indexer fp4 is a decode variant")
         if tokens:
             # a shorter sequence of the same shape (profiling captures): not the headline workload
             spec = dict(spec, T=int(tokens))
             name = f"{name}_T{int(tokens)}"
         return PrefillBench(name, spec, seed, device, qk_norm)
-    return DecodeBench(name, spec, seed, device, qk_norm)
+    if indexer != "bf16":
+        if spec["kind"] == "hca_decode":
+            raise SystemExit("--indexer fp4 needs a CSA layer")
+        name = f"{name}+fp4_indexer"  # the FP4 indexer variant (not the headline workload)
+    return DecodeBench(name, spec, seed, device, qk_norm, indexer=indexer)
 
 
 def norm_prologue_roofline(bench, flush, pk, reps=20):
@@ -519,113 +563,208 @@ def e2e_pipelined(bench, K, device):
     return start.elapsed_time(end) / K
 
 
-def run_ours(a):
-    rank, local, ws = init_dist("nccl")
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    bench = make_bench(a.workload, shard_seed(a.seed, rank), device, tokens=a.tokens, qk_norm=a.qk_norm)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    for _ in range(a.warmup):
+def headline_region(bench, K, flush, rank, ws, device, local):
+    """The headline timing: the K-step region (no host syncs inside), repeated
+    until it has covered at least HEADLINE_MIN_S of wall time so that the clock
+    sampler holds at least ~10 samples under load; the median repeat is the
+    number.  A run whose clock record shows a hardware/thermal slowdown (or SM
+    clocks stuck low with no reason) is taken once more, on every rank alike."""
+    def once():
+        totals = []
+        with ClockSampler(local) as clk:
+            t0 = time.perf_counter()
+            while True:
+                t, _ = timed_steps(bench, K, flush, rank, ws, device, record=False)
+                totals.append(t)
+                # every rank repeats the same number of times
+                more = 1.0 if time.perf_counter() - t0 < HEADLINE_MIN_S else 0.0
+                if reduce_max(more, ws, device) == 0.0:
+                    break
+        med = float(np.median(totals))
+        return reduce_max(med, ws, device), dict(clk.summary(), region_repeats=len(totals))
+
+    total_ms, clocks = once()
+    if reduce_max(1.0 if clock_rejected(clocks) else 0.0, ws, device) > 0.0:
+        first = clocks["reasons"] or ["sm clock %s of %s MHz" % (clocks["sm_mhz"], clocks["sm_max_mhz"])]
+        total_ms, clocks = once()
+        clocks = dict(clocks, remeasured_after=first)
+    return total_ms, clocks
+
+
+def roofline_of(bench, phase_ms, pk, sustained):
+    """Roofline of the dominant phase: algorithmic bytes (or FLOPs) per launch over
+    its event time, against the measured peak (and the datasheet's)."""
+    dom = max(phase_ms, key=phase_ms.get) if phase_ms else None
+    if dom is None:
+        return None
+    flops = bench.flops() if hasattr(bench, "flops") else {}
+    bytes_ = bench.phase_bytes()
+    dur_s = phase_ms[dom] / 1e3
+    tt = traffic_table().get(dom)
+    traffic = None
+    if tt and tt.get("source_hash") == source_hash(tt.get("files", [])) and tt.get("workload") == bench.name:
+        traffic = tt["dram_bytes_per_launch"]
+    if dom in flops:
+        ach = flops[dom] / dur_s / 1e12
+        peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+        return {"bound": "tensor", "kernel": dom, "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": pk["source"],
+                "peak_kind": "sustained" if sustained else "burst",
+                "datasheet_peak": DATASHEET["bf16_tflops"], "frac_datasheet": round(ach / DATASHEET["bf16_tflops"], 4)}
+    if dom in bytes_:
+        ach = bytes_[dom] / dur_s / 1e9
+        return {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / pk["hbm_gbs"], 4), "traffic": traffic, "peak_source": pk["source"],
+                "datasheet_peak": DATASHEET["hbm_gbs"], "frac_datasheet": round(ach / DATASHEET["hbm_gbs"], 4)}
+    return {"bound": "alu", "kernel": dom, "achieved": None, "peak": None, "unit": None, "frac": None,
+            "traffic": traffic, "note": "selection kernel; no algorithmic HBM bytes"}
+
+
+def whole_step_roofline(bench, ms, pk):
+    """The whole step against the roofline its bound names: all algorithmic FLOPs
+    (prefill) or bytes (decode) of the step over the step's time."""
+    flops = bench.flops() if hasattr(bench, "flops") else {}
+    if flops:
+        ach = sum(flops.values()) / (ms / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": round(ach, 2), "unit": "TFLOP/s",
+                "frac_burst": round(ach / pk["bf16_tflops"], 4),
+                "frac_sustained": round(ach / pk["bf16_tflops_sustained"], 4),
+                "frac_datasheet": round(ach / DATASHEET["bf16_tflops"], 4)}
+    b = sum(bench.phase_bytes().values())
+    ach = b / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "bytes": int(b), "achieved": round(ach, 1), "unit": "GB/s",
+            "frac": round(ach / pk["hbm_gbs"], 4), "frac_datasheet": round(ach / DATASHEET["hbm_gbs"], 4)}
+
+
+def measure(bench, a, steps, warmup, flush, rank, ws, device, local, cpu_sample):
+    """Everything one workload reports: headline value, phases, rooflines, e2e,
+    launches, clocks and (rank 0, one GPU) the CPU oracle baseline."""
+    for _ in range(warmup):
         bench.step()
     torch.cuda.synchronize()
     launches = bench.launches_per_step()
-    if a.steps is None:
-        # default K: a timed region of about 2 s (long enough for the clock sampler)
+    if steps is None:
+        # default K: a timed region of about 2 s
         t0 = time.perf_counter()
         for _ in range(3):
             flush.zero_()
             bench.step(record=False)
         torch.cuda.synchronize()
         per = (time.perf_counter() - t0) / 3
-        a.steps = int(min(20000, max(20, math.ceil(2.0 / max(per, 1e-6)))))
-        if ws > 1:
-            import torch.distributed as dist
-            t = torch.tensor([a.steps], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            a.steps = int(t.item())
+        steps = int(min(20000, max(20, math.ceil(2.0 / max(per, 1e-6)))))
+        steps = int(reduce_max(float(steps), ws, device))
     # phase breakdown pass (events between kernels, one sync per step)
-    _, phase_ms = timed_steps(bench, min(a.steps, 50), flush, rank, ws, device, record=True)
-    # headline: K steps without intermediate host syncs; a run whose clock record
-    # shows a hardware/thermal slowdown (or clocks stuck low with no reason) is
-    # taken once more, on every rank alike
-    def headline():
-        with ClockSampler(local) as clk:
-            t, _ = timed_steps(bench, a.steps, flush, rank, ws, device, record=False)
-        return reduce_max(t, ws, device), clk.summary()
-
-    total_ms, clocks = headline()
-    if reduce_max(1.0 if clock_rejected(clocks) else 0.0, ws, device) > 0.0:
-        first = clocks["reasons"] or ["sm clock %s of %s MHz" % (clocks["sm_mhz"], clocks["sm_max_mhz"])]
-        total_ms, clocks = headline()
-        clocks = dict(clocks, remeasured_after=first)
-    ms = total_ms / a.steps
+    _, phase_ms = timed_steps(bench, min(steps, 50), flush, rank, ws, device, record=True)
+    total_ms, clocks = headline_region(bench, steps, flush, rank, ws, device, local)
+    ms = total_ms / steps
     value = bench.units * ws / (ms / 1e3)
 
     # end to end through the C ABI with host buffers
     bench.e2e_setup()
-    e2e_ms = e2e_pipelined(bench, 2, device)  # warm-up
-    e2e_ms = reduce_max(e2e_pipelined(bench, a.steps, device), ws, device)
+    e2e_pipelined(bench, 2, device)  # warm-up
+    e2e_ms = reduce_max(e2e_pipelined(bench, steps, device), ws, device)
     e2e_value = bench.units * ws / (e2e_ms / 1e3)
 
-    # roofline of the dominant kernel
     pk = peaks()
-    dom = max(phase_ms, key=phase_ms.get) if phase_ms else None
-    roof = None
-    if dom is not None:
-        flops = bench.flops() if hasattr(bench, "flops") else {}
-        bytes_ = bench.phase_bytes()
-        dur_s = phase_ms[dom] / 1e3
-        tt = traffic_table().get(dom)
-        traffic = None
-        if tt and tt.get("source_hash") == source_hash(tt.get("files", [])) and tt.get("workload") == bench.name:
-            traffic = tt["dram_bytes_per_launch"]
-        if dom in flops:
-            ach = flops[dom] / dur_s / 1e12
-            peak = pk["bf16_tflops_sustained"] if a.workload.endswith("prefill_64k") else pk["bf16_tflops"]
-            roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
-                    "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": pk["source"],
-                    "datasheet_peak": DATASHEET["bf16_tflops"],
-                    "frac_datasheet": round(ach / DATASHEET["bf16_tflops"], 4)}
-        elif dom in bytes_:
-            ach = bytes_[dom] / dur_s / 1e9
-            roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(ach / pk["hbm_gbs"], 4), "traffic": traffic, "peak_source": pk["source"],
-                    "datasheet_peak": DATASHEET["hbm_gbs"], "frac_datasheet": round(ach / DATASHEET["hbm_gbs"], 4)}
-        else:
-            roof = {"bound": "alu", "kernel": dom, "achieved": None, "peak": None, "unit": None, "frac": None,
-                    "traffic": traffic, "note": "selection kernel; no algorithmic HBM bytes"}
-
-    out = {"metric": bench.metric, "value": round(value, 2), "unit": bench.unit, "n_gpus": ws, "steps": a.steps,
-           "warmup": a.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1)/U(0,1) tensors of the workload's "
-           "shapes; caches drawn on the device)",
+    prefill = isinstance(bench, PrefillBench)
+    out = {"metric": bench.metric, "value": round(value, 2), "unit": bench.unit, "n_gpus": ws, "steps": steps,
+           "warmup": warmup, "ms_per_step": round(ms, 4),
            "config": dict(bench.config(), parallelism=f"replicas x{ws} (requests sharded, no collective)",
                           l2="flushed before every timed step (256 MiB write, outside the step's events)"),
            "e2e": {"value": round(e2e_value, 2), "unit": bench.unit, "h2d_bytes_per_step": bench.h2d,
                    "d2h_bytes_per_step": bench.d2h, "ms_per_step": round(e2e_ms, 4),
-                   "note": "every step copies its inputs (queries, indexer queries and weights, windows, new block) "
-                           "from pinned host memory and its outputs back, on copy streams that overlap the "
-                           "neighbouring steps' compute (two device buffer sets; no L2 flush: a step streams more "
-                           "than the L2 holds); KV caches resident on the device"},
-           "gpu_launches": launches * a.steps,
+                   "note": "every step copies its inputs from pinned host memory and its outputs back, on copy "
+                           "streams that overlap the neighbouring steps' compute (two device buffer sets; no L2 "
+                           "flush: a step streams more than the L2 holds); KV caches resident on the device"},
+           "gpu_launches": launches * steps,
            "phase_ms": {k: round(v, 4) for k, v in phase_ms.items()},
-           "roofline": roof,
+           # a prefill step is long: its attention runs at the sustained (power-capped) rate
+           "roofline": roofline_of(bench, phase_ms, pk, sustained=prefill),
+           "step_roofline": whole_step_roofline(bench, ms, pk),
            "clocks": clocks}
-    if a.qk_norm and isinstance(bench, PrefillBench):
+    if a.qk_norm and prefill:
         out["qk_norm_prologue"] = norm_prologue_roofline(bench, flush, pk)
     if rank == 0 and ws == 1 and not a.no_cpu_baseline:
         import oracle  # noqa: F401  (timed baseline only)
         cores = len(os.sched_getaffinity(0))
-        n = a.cpu_sample
-        secs = bench.oracle_sample(n)
-        out["cpu_baseline"] = {"value": round(n / secs, 4), "unit": bench.unit, "cores": cores, "kind": "oracle",
-                               "sample": f"{n} {'queries' if bench.unit == 'tokens/s' else 'requests'} of the same "
-                                         f"workload recipe through the float64 NumPy oracle ({secs:.1f} s)"}
+        secs = bench.oracle_sample(cpu_sample)
+        out["cpu_baseline"] = {"value": round(cpu_sample / secs, 4), "unit": bench.unit, "cores": cores,
+                               "kind": "oracle",
+                               "sample": f"{cpu_sample} {'queries' if bench.unit == 'tokens/s' else 'requests'} of "
+                                         f"the same workload recipe through the float64 NumPy oracle ({secs:.1f} s)"}
+    return out
+
+
+def run_ours(a):
+    rank, local, ws = init_dist("nccl")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    bench = make_bench(a.workload, shard_seed(a.seed, rank), device, tokens=a.tokens, qk_norm=a.qk_norm,
+                       indexer=a.indexer)
+    m = measure(bench, a, a.steps, a.warmup, flush, rank, ws, device, local, a.cpu_sample)
+    out = {"metric": bench.metric, "value": m.pop("value"), "unit": m.pop("unit"), "n_gpus": ws,
+           "steps": m.pop("steps"), "warmup": a.warmup, "ms_per_step": m.pop("ms_per_step"),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded N(0,1)/U(0,1) tensors of the workload's shapes; caches drawn on the device)"}
+    m.pop("metric")
+    m.pop("n_gpus")
+    m.pop("warmup")
+    out.update(m)
+    # The metric has two halves: decode queries/s (the headline) and prefill tokens/s.
+    # The default run measures the 64K CSA prefill as well, in the same line.
+    if a.workload == DEFAULT_WORKLOAD and not a.no_prefill and a.tokens is None and a.indexer == "bf16":
+        del bench
+        torch.cuda.empty_cache()
+        pb = make_bench("csa_prefill_64k", shard_seed(a.seed, rank), device, qk_norm=a.qk_norm)
+        # the prefill step is ~200x longer than a decode step: fewer steps cover as long a region
+        psteps = a.prefill_steps if a.prefill_steps else max(3, min(20, a.steps or 20))
+        pm = measure(pb, a, psteps, max(3, min(a.warmup, 5)), flush, rank, ws, device, local,
+                     max(4, a.cpu_sample))
+        pm["workload"] = "csa_prefill_64k"
+        out["prefill"] = pm
     if rank == 0:
         print(json.dumps(out), flush=True)
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def spawn_ranks(n: int) -> int:
+    """Re-run this command under torch.distributed.run with n ranks on this node
+    (rendezvous on 127.0.0.1); returns the launcher's exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def check_launch():
+    """Start the process group (gloo without a GPU), agree on the world size with one
+    collective, and print it from rank 0."""
+    import datetime
+    import torch.distributed as dist
+    rank, local, ws = dist_env()
+    if ws > 1:
+        dist.init_process_group(backend="nccl" if torch.cuda.is_available() else "gloo",
+                                timeout=datetime.timedelta(seconds=60))
+        dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+        if dev.type == "cuda":
+            torch.cuda.set_device(local)
+        t = torch.ones(1, device=dev)
+        dist.all_reduce(t)
+        agreed = int(t.item())
+        dist.destroy_process_group()
+    else:
+        agreed = 1
+    if rank == 0:
+        print(json.dumps({"check_launch": True, "world_size": ws, "ranks_agreed": agreed}), flush=True)
 
 
 def run_reference(a):
@@ -683,7 +822,21 @@ def main():
                     help="the layer with Q/KV RMSNorm + partial RoPE (synthetic weights)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="prefill workloads: a shorter sequence of the same shape (for profiler captures)")
+    ap.add_argument("--indexer", default="bf16", choices=["bf16", "fp4"],
+                    help="fp4: the decode indexer over MXFP4 keys with BF16 scores (a variant, not the headline)")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="default workload only: skip the 64K prefill measured in the same line")
+    ap.add_argument("--prefill-steps", type=int, default=None,
+                    help="timed steps of the 64K prefill in the default run (default: min(20, --steps))")
+    ap.add_argument("--check-launch", action="store_true",
+                    help="start the ranks and report the world size only (tests of the launcher, no GPU work)")
     a = ap.parse_args()
+    if a.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start the ranks here when not already under torchrun
+        sys.exit(spawn_ranks(a.gpus))
+    if a.check_launch:
+        check_launch()
+        return
     if a.warmup < 3:
         print("warning: fewer than 3 warm-up steps; the number is not a valid measurement", file=sys.stderr)
     if a.impl == "reference":

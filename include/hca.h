@@ -28,6 +28,13 @@
  *   - Fault injection for tests: if the environment variable
  *     HCA_INJECT_FAULT names an entry point (or is "all"), that entry point
  *     returns HCA_ERR_INJECTED after argument checking, launching nothing.
+ *   - Bounded device waits: every wait of a kernel on its own pipeline gives
+ *     up after a poll budget, records an error, lets its own copies and MMAs
+ *     drain, frees its tensor memory and returns; hca_check_device() then
+ *     reports HCA_ERR_DEVICE_CHECK.  For tests of that path only,
+ *     HCA_TEST_STALL=indexer makes the decode indexer's key producer issue
+ *     nothing, with a budget of a few thousand polls, so that its waits run
+ *     out (the call's top-k output is then meaningless).
  *   - Supported shapes: c in {64, 512}, d_idx in {32, 128}; n_heads,
  *     n_idx_heads <= 64; topk <= 2048; n_win <= 256.  Other shapes return
  *     HCA_ERR_UNSUPPORTED.
@@ -335,6 +342,15 @@ typedef struct {
   const float* hca_sink;      /* [H] sink logits of the HCA layer, or NULL */
   const float* csa_norm;      /* [2, c] Q/KV normalisation weights of the CSA layer, or NULL */
   const float* hca_norm;      /* [2, c] of the HCA layer, or NULL */
+  /* FP4 indexer variant (see csa_indexer_topk_fp4), or NULL: the CSA layer's indexer
+   * reads MXFP4 keys instead of csa_k_idx (which is then not read): request b's codes
+   * at csa_k_codes + b*csa_k4_stride*64 ([csa_N][64] bytes) and scales at
+   * csa_k_scales + b*csa_k4_stride*4 ([csa_N][4] bytes, readable up to the next
+   * multiple of 4 keys); csa_k4_stride in keys, a multiple of 4 (B > 1). 64 x 128
+   * indexer only; the index scores are BF16. */
+  const uint8_t* csa_k_codes;
+  const uint8_t* csa_k_scales;
+  long long csa_k4_stride;
 } hca_decode_args;
 
 int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* args, void* ws,

@@ -54,7 +54,8 @@ class DecodeArgs(ctypes.Structure):
                 ("hca_block_cand", c_void_p), ("hca_block_logits", c_void_p), ("hca_block_stride", c_ll),
                 ("hca_pos_bias", c_void_p), ("hca_win", c_void_p), ("hca_win_stride", c_ll), ("hca_out", c_void_p),
                 ("events", c_void_p), ("n_events", c_int), ("csa_sink", c_void_p), ("hca_sink", c_void_p),
-                ("csa_norm", c_void_p), ("hca_norm", c_void_p)]
+                ("csa_norm", c_void_p), ("hca_norm", c_void_p),
+                ("csa_k_codes", c_void_p), ("csa_k_scales", c_void_p), ("csa_k4_stride", c_ll)]
 
 
 class PrefillArgs(ctypes.Structure):
@@ -303,12 +304,19 @@ def _events_array(events):
 
 
 def make_decode_args(B, q_pos, csa=None, hca=None, csa_topk_idx=None, csa_out=None, hca_out=None, events=None,
-                     csa_sink=None, hca_sink=None, csa_norm=None, hca_norm=None):
+                     csa_sink=None, hca_sink=None, csa_norm=None, hca_norm=None, csa_k4=None):
     """Build DecodeArgs from dicts of tensors (see workloads.csa_decode_inputs /
     hca_decode_inputs); csa_sink / hca_sink: optional [H] float32 sink logits;
-    csa_norm / hca_norm: optional [2, c] float32 Q/KV normalisation weights.
+    csa_norm / hca_norm: optional [2, c] float32 Q/KV normalisation weights;
+    csa_k4: optional (codes uint8 [B, N_alloc, 64], scales uint8 [B, N_alloc, 4]),
+    the MXFP4 indexer keys of the FP4 indexer variant (see mxfp4_quantize).
     Returns (args, keepalive)."""
     a = DecodeArgs()
+    if csa_k4 is not None:
+        codes, scales = csa_k4
+        a.csa_k_codes = _ptr(codes, torch.uint8, "csa_k4 codes")
+        a.csa_k_scales = _ptr(scales, torch.uint8, "csa_k4 scales")
+        a.csa_k4_stride = codes.stride(0) // 64
     a.csa_sink = _ptr(csa_sink, F32, "csa_sink")
     a.hca_sink = _ptr(hca_sink, F32, "hca_sink")
     a.csa_norm = _ptr(csa_norm, F32, "csa_norm")
@@ -316,16 +324,16 @@ def make_decode_args(B, q_pos, csa=None, hca=None, csa_topk_idx=None, csa_out=No
     a.B = B
     a.q_pos = _ptr(q_pos, I32, "q_pos")
     # every tensor the struct points at stays alive with the returned keepalive
-    keep = [q_pos, csa_sink, hca_sink, csa_norm, hca_norm, csa, hca, csa_topk_idx, csa_out, hca_out]
+    keep = [q_pos, csa_sink, hca_sink, csa_norm, hca_norm, csa, hca, csa_topk_idx, csa_out, hca_out, csa_k4]
     if csa is not None:
         a.csa_q = _ptr(csa["q"], BF16, "csa.q")
         a.csa_q_idx = _ptr(csa["q_idx"], BF16, "csa.q_idx")
         a.csa_w_idx = _ptr(csa["w_idx"], F32, "csa.w_idx")
         a.csa_kv = _ptr(csa["E"], BF16, "csa.E")
-        a.csa_k_idx = _ptr(csa["K_I"], BF16, "csa.K_I")
+        a.csa_k_idx = _ptr(csa.get("K_I"), BF16, "csa.K_I")  # (not read by the FP4 variant)
         a.csa_N = csa["E"].shape[1]
         a.csa_kv_stride = csa["E"].stride(0)
-        a.csa_k_stride = csa["K_I"].stride(0)
+        a.csa_k_stride = csa["K_I"].stride(0) if csa.get("K_I") is not None else 0
         a.csa_win = _ptr(csa["win"], BF16, "csa.win")
         a.csa_win_stride = csa["win"].stride(0)
         a.csa_topk_idx = _ptr(csa_topk_idx, I32, "csa_topk_idx")

@@ -57,6 +57,14 @@ bool injected(const char* name) {
   return strcmp(v, "all") == 0 || strcmp(v, name) == 0;
 }
 
+// Tests of the bounded device waits: HCA_TEST_STALL=indexer makes the decode
+// indexer's key producer issue nothing, with a tiny poll budget, so that every
+// consumer wait runs out; the kernel records the error and returns.
+bool test_stall_indexer() {
+  const char* v = getenv("HCA_TEST_STALL");
+  return v && strcmp(v, "indexer") == 0;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 #define CHECK_PTR(p, name)                                                          \
@@ -182,22 +190,44 @@ int indexer_ok(int N, int k, int mode) {
   return HCA_OK;
 }
 
+// Keys of the FP4 indexer variant (decode only): MXFP4 codes [N][64 B] and scales
+// [N][4 B] per request, `stride` keys apart; q4 = workspace for the queries'
+// MXFP4 values in bf16 [Tq, 64, 128].
+struct Fp4Keys {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  long long stride;
+  bf16* q4;
+};
+
 int run_indexer_topk(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride, int N,
                      const int32_t* q_pos, int Tq, int mode, const hca_layer_cfg* cfg, int32_t* topk_idx,
-                     void* ws, cudaStream_t st, void* const* ev, int n_ev, int& ev_i, int grid_sms = 0) {
+                     void* ws, cudaStream_t st, void* const* ev, int n_ev, int& ev_i, int grid_sms = 0,
+                     const Fp4Keys* fp4 = nullptr) {
   const IndexerPlan p = plan_indexer(Tq, N, cfg->topk);
   float* scores = reinterpret_cast<float*>(ws);
   // decode with more entries than one select CTA holds: the indexer also builds
   // each request's score-key histogram, and one threshold select follows
-  const bool hist = mode == HCA_MODE_DECODE && p.hist_ctas > 0 && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx);
+  const bool hist = mode == HCA_MODE_DECODE && p.hist_ctas > 0 &&
+                    (fp4 != nullptr || indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx));
   char* wsb = reinterpret_cast<char*>(ws);
+  if (fp4) {
+    // the queries' MXFP4 values (bf16), then the scores over the FP4 keys
+    CUDA_TRY(launch_mxfp4_roundtrip(q_idx, Tq * cfg->n_idx_heads, cfg->d_idx, fp4->q4, st), "fp4 query rounding");
+  }
   if (hist)
     CUDA_TRY(cudaMemsetAsync(wsb + p.hist_off, 0, (size_t)Tq * (2 * kHistBins + 1) * sizeof(int), st),
              "histogram reset");
-  if (mode == HCA_MODE_DECODE && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx)) {
+  if (fp4) {
+    CUDA_TRY(launch_indexer_decode_fp4(fp4->q4, w_idx, fp4->codes, fp4->scales, fp4->stride, N, q_pos, Tq, cfg->m,
+                                       scores, p.ld, grid_sms > 0 ? grid_sms : device_sm_count(), st,
+                                       hist ? reinterpret_cast<int*>(wsb + p.hist_off) : nullptr),
+             "indexer scores (fp4)");
+  } else if (mode == HCA_MODE_DECODE && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx)) {
     CUDA_TRY(launch_indexer_decode_tc(q_idx, w_idx, k_idx, k_seq_stride, N, q_pos, Tq, cfg->m, scores, p.ld,
                                       grid_sms > 0 ? grid_sms : device_sm_count(), st,
-                                      hist ? reinterpret_cast<int*>(wsb + p.hist_off) : nullptr),
+                                      hist ? reinterpret_cast<int*>(wsb + p.hist_off) : nullptr,
+                                      test_stall_indexer()),
              "indexer scores (tcgen05)");
   } else if (mode == HCA_MODE_PREFILL && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx)) {
     CUDA_TRY(launch_indexer_prefill_tc(q_idx, w_idx, k_idx, N, q_pos, Tq, cfg->m, scores, p.ld,
@@ -557,6 +587,8 @@ struct DecodeSched {
   // Q/KV normalisation: normalised queries [B, H, c] and window blocks [B, n_win, c]
   // (bf16) of each normalised layer, and the HCA entries in f32 [B, c] before theirs
   size_t csa_qn = 0, csa_wn = 0, hca_qn = 0, hca_wn = 0, hca_ef = 0;
+  // FP4 indexer: the queries' MXFP4 values in bf16 [B, H_I, d_I]
+  size_t q4 = 0;
 };
 
 static MqaProblem decode_csa_problem(const hca_layer_cfg* cfg, const hca_decode_args* a) {
@@ -624,6 +656,10 @@ static DecodeSched decode_schedule(const hca_layer_cfg* cfg, const hca_decode_ar
     d.hca_ef = d.hca_wn + wbytes;
     d.total = d.hca_ef + round256((size_t)a->B * cfg->c * 4);
   }
+  if (csa && a->csa_k_codes) {
+    d.q4 = d.total;
+    d.total = d.q4 + round256((size_t)a->B * cfg->n_idx_heads * cfg->d_idx * 2);
+  }
   return d;
 }
 
@@ -678,9 +714,19 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
     CHECK(a->csa_N > 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: csa_N=%d", a->csa_N);
     CHECK_PTR(a->csa_q_idx, "hybrid_attn_decode: csa_q_idx");
     CHECK_PTR(a->csa_w_idx, "hybrid_attn_decode: csa_w_idx");
-    CHECK_PTR(a->csa_k_idx, "hybrid_attn_decode: csa_k_idx");
+    if (a->csa_k_codes) {
+      CHECK(indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx), HCA_ERR_UNSUPPORTED,
+            "hybrid_attn_decode: the FP4 indexer takes 64 heads x 128 (got %d x %d)", cfg->n_idx_heads, cfg->d_idx);
+      CHECK_PTR(a->csa_k_codes, "hybrid_attn_decode: csa_k_codes");
+      CHECK_PTR(a->csa_k_scales, "hybrid_attn_decode: csa_k_scales");
+      const long long n4 = ((long long)a->csa_N + 3) / 4 * 4;
+      CHECK(a->B <= 1 || (a->csa_k4_stride >= n4 && a->csa_k4_stride % 4 == 0), HCA_ERR_INVALID_ARG,
+            "hybrid_attn_decode: csa_k4_stride %lld (need >= %lld keys, a multiple of 4)", a->csa_k4_stride, n4);
+    } else {
+      CHECK_PTR(a->csa_k_idx, "hybrid_attn_decode: csa_k_idx");
+      CHECK(a->csa_k_stride % 8 == 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: csa_k_stride");
+    }
     CHECK_PTR(a->csa_topk_idx, "hybrid_attn_decode: csa_topk_idx");
-    CHECK(a->csa_k_stride % 8 == 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: csa_k_stride");
     s = check_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_N, a->csa_topk_idx, cfg->topk, cfg->m,
                   a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out, "hybrid_attn_decode: csa");
     if (s != HCA_OK) return s;
@@ -793,10 +839,13 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
       s = normalise_layer(a->csa_q, a->csa_win, a->csa_win_stride, a->csa_norm, sched.csa_qn, sched.csa_wn, st);
       if (s != HCA_OK) return s;
     }
+    Fp4Keys k4{a->csa_k_codes, a->csa_k_scales,
+               a->B > 1 ? a->csa_k4_stride : ((long long)a->csa_N + 3) / 4 * 4,
+               reinterpret_cast<bf16*>(wsb + sched.q4)};
     s = run_indexer_topk(reinterpret_cast<const bf16*>(a->csa_q_idx), a->csa_w_idx,
                          reinterpret_cast<const bf16*>(a->csa_k_idx), a->csa_k_stride, a->csa_N, a->q_pos, a->B,
                          HCA_MODE_DECODE, cfg, a->csa_topk_idx, ws, st, ev, n_ev, ev_i,
-                         sched.overlap ? sched.sms - sched.r_hca : 0);
+                         sched.overlap ? sched.sms - sched.r_hca : 0, a->csa_k_codes ? &k4 : nullptr);
     if (s != HCA_OK) return s;
     MqaProblem p = decode_csa_problem(cfg, a);
     if (a->csa_norm) use_normalised(p, cfg, wsb + sched.csa_qn, wsb + sched.csa_wn, true);
@@ -1035,51 +1084,12 @@ int csa_indexer_topk_fp4(const hca_bf16* q_idx, const float* w_idx, const uint8_
         "csa_indexer_topk_fp4: ws null or not 256-byte aligned");
   if (injected("csa_indexer_topk_fp4")) return fail(HCA_ERR_INJECTED, "csa_indexer_topk_fp4: injected");
 
-  cudaStream_t st = as_stream(stream);
   const IndexerPlan p = plan_indexer(B, N, cfg->topk);
-  char* wsb = reinterpret_cast<char*>(ws);
-  float* scores = reinterpret_cast<float*>(ws);
-  bf16* q4 = reinterpret_cast<bf16*>(wsb + round256(p.bytes));
-  // the query's MXFP4 values (bf16), then the scores over the FP4 keys
-  CUDA_TRY(launch_mxfp4_roundtrip(reinterpret_cast<const bf16*>(q_idx), B * cfg->n_idx_heads, cfg->d_idx, q4, st),
-           "csa_indexer_topk_fp4: query rounding");
-  const bool hist = p.hist_ctas > 0;
-  if (hist)
-    CUDA_TRY(cudaMemsetAsync(wsb + p.hist_off, 0, (size_t)B * (2 * kHistBins + 1) * sizeof(int), st),
-             "histogram reset");
-  CUDA_TRY(launch_indexer_decode_fp4(q4, w_idx, k_codes, k_scales, k_seq_stride, N, q_pos, B, cfg->m, scores, p.ld,
-                                     device_sm_count(), st, hist ? reinterpret_cast<int*>(wsb + p.hist_off) : nullptr),
-           "csa_indexer_topk_fp4: scores");
-  if (hist) {
-    HistSelect a;
-    a.scores = scores;
-    a.ld = p.ld;
-    a.q_pos = q_pos;
-    a.rate = cfg->m;
-    a.N = N;
-    a.k = cfg->topk;
-    a.hist = reinterpret_cast<int*>(wsb + p.hist_off);
-    a.B = B;
-    a.done = reinterpret_cast<int*>(wsb + p.done_off);
-    a.cnt = reinterpret_cast<int2*>(wsb + p.cnt_off);
-    a.above = reinterpret_cast<int32_t*>(wsb + p.above_off);
-    a.eq = reinterpret_cast<uint64_t*>(wsb + p.eq_off);
-    a.C = p.hist_ctas;
-    a.slice = kHistSlice;
-    a.out = topk_idx;
-    CUDA_TRY(launch_select_hist(a, B, st), "csa_indexer_topk_fp4: select (histogram threshold)");
-    return HCA_OK;
-  }
-  SelectRows rows;
-  rows.chunks = p.chunks;
-  rows.chunk = p.chunk;
-  rows.n_rows = B * p.chunks;
-  rows.rate = cfg->m;
-  rows.N = N;
-  rows.q_pos = q_pos;
-  rows.ld_scores = p.ld;
-  CUDA_TRY(launch_select_rows(scores, rows, cfg->topk, topk_idx, st), "csa_indexer_topk_fp4: select");
-  return HCA_OK;
+  Fp4Keys k4{k_codes, k_scales, B > 1 ? k_seq_stride : (long long)(N + 3) / 4 * 4,
+             reinterpret_cast<bf16*>(reinterpret_cast<char*>(ws) + round256(p.bytes))};
+  int ev_i = 0;
+  return run_indexer_topk(reinterpret_cast<const bf16*>(q_idx), w_idx, nullptr, 0, N, q_pos, B, HCA_MODE_DECODE,
+                          cfg, topk_idx, ws, as_stream(stream), nullptr, 0, ev_i, 0, &k4);
 }
 
 }  // extern "C"

@@ -60,7 +60,10 @@ __device__ unsigned int g_indexer_tc_error = 0;
 __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
     const float* __restrict__ w_idx, const int32_t* __restrict__ q_pos, int B, int N, int rate,
-    int tiles_per_req, float* __restrict__ scores, long long ld_scores, int* __restrict__ hist_g) {
+    int tiles_per_req, float* __restrict__ scores, long long ld_scores, int* __restrict__ hist_g,
+    uint32_t spin, int stall) {
+  // spin: poll budget of every wait (tc::kSpinLimit in normal use).  stall != 0 (tests of
+  // the bounded waits only): the producer issues nothing, so every consumer wait runs out.
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* k_smem = base;                              // [stages][2][128][128 B]
@@ -96,13 +99,13 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
       tc::tma_prefetch_desc(&tm_k);
       tc::tma_prefetch_desc(&tm_q);
       int it = 0, rq = 0, cur_r = -1;
-      for (long long g = g0; g < g1; ++g) {
+      for (long long g = stall ? g1 : g0; g < g1; ++g) {
         const int r = (int)(g / tiles_per_req);
         const int row0 = (int)(g % tiles_per_req) * kTile;
         if (row0 >= n_visible(q_pos[r], rate, N)) continue;
         if (r != cur_r) {
           const int qb = rq & 1;
-          if (!tc::mbar_wait(&bars->qempty[qb], ((rq >> 1) & 1) ^ 1, abort)) break;
+          if (!tc::mbar_wait(&bars->qempty[qb], ((rq >> 1) & 1) ^ 1, abort, spin)) break;
           tc::mbar_arrive_expect_tx(&bars->qfull[qb], kQBytes);
           tc::tma_load_2d(q_smem + qb * kQBytes, &tm_q, &bars->qfull[qb], 0, r * kHeads);
           tc::tma_load_2d(q_smem + qb * kQBytes + kQChunkBytes, &tm_q, &bars->qfull[qb], 64, r * kHeads);
@@ -110,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
           ++rq;
         }
         const int s = it % kStages;
-        if (!tc::mbar_wait(&bars->empty[s], ((it / kStages) & 1) ^ 1, abort)) break;
+        if (!tc::mbar_wait(&bars->empty[s], ((it / kStages) & 1) ^ 1, abort, spin)) break;
         tc::mbar_arrive_expect_tx(&bars->full[s], kTileBytes);
         tc::tma_load_3d(k_smem + s * kTileBytes, &tm_k, &bars->full[s], 0, row0, r);
         tc::tma_load_3d(k_smem + s * kTileBytes + kChunkBytes, &tm_k, &bars->full[s], 64, row0, r);
@@ -135,15 +138,15 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
         if (r != cur_r) {
           if (cur_r >= 0) tc::mma_commit(&bars->qempty[qb]);  // previous q buffer free once its MMAs finish
           qb = rq & 1;
-          if (!tc::mbar_wait(&bars->qfull[qb], (rq >> 1) & 1, abort)) break;
+          if (!tc::mbar_wait(&bars->qfull[qb], (rq >> 1) & 1, abort, spin)) break;
           tc::fence_after_sync();
           cur_r = r;
           ++rq;
         }
         const int s = it % kStages;
         const int a = it % kAcc;
-        if (!tc::mbar_wait(&bars->full[s], (it / kStages) & 1, abort)) break;
-        if (!tc::mbar_wait(&bars->tempty[a], ((it / kAcc) & 1) ^ 1, abort)) break;
+        if (!tc::mbar_wait(&bars->full[s], (it / kStages) & 1, abort, spin)) break;
+        if (!tc::mbar_wait(&bars->tempty[a], ((it / kAcc) & 1) ^ 1, abort, spin)) break;
         tc::fence_after_sync();
 #pragma unroll
         for (int k = 0; k < kDim / 16; ++k) {
@@ -197,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
       }
       const int a = it % kAcc;
       ++it;
-      if (!failed) failed = !tc::mbar_wait(&bars->tfull[a], ((it - 1) / kAcc) & 1, abort);
+      if (!failed) failed = !tc::mbar_wait(&bars->tfull[a], ((it - 1) / kAcc) & 1, abort, spin);
       if (failed) continue;
       tc::fence_after_sync();
       uint32_t v[kHeads];
@@ -466,7 +469,8 @@ bool indexer_tc_supported(int H_I, int d_I) { return H_I == kHeads && d_I == kDi
 
 cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride,
                                      int N, const int32_t* q_pos, int B, int rate, float* scores, long long ld_scores,
-                                     int num_sms, cudaStream_t stream, int* hist) {
+                                     int num_sms, cudaStream_t stream, int* hist, bool stall) {
+  constexpr uint32_t kStallSpin = 4096;  // a stalled test launch gives up after ~4k polls
   if (B == 0 || N == 0) return cudaSuccess;
   CUtensorMap tm_k, tm_q;
   const uint64_t kd[3] = {(uint64_t)kDim, (uint64_t)N, (uint64_t)B};
@@ -484,7 +488,9 @@ cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, cons
                            (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   indexer_decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_k, tm_q, w_idx, q_pos, B, N, rate,
-                                                                   tiles_per_req, scores, ld_scores, hist);
+                                                                   tiles_per_req, scores, ld_scores, hist,
+                                                                   stall ? kStallSpin : tc::kSpinLimit,
+                                                                   stall ? 1 : 0);
   ++g_launch_counter;
   return cudaGetLastError();
 }

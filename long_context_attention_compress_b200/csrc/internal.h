@@ -133,7 +133,9 @@ bool indexer_tc_supported(int H_I, int d_I);
 cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride,
                                      int N, const int32_t* q_pos, int B, int rate, float* scores, long long ld_scores,
                                      int num_sms, cudaStream_t stream,
-                                     int* hist = nullptr);
+                                     int* hist = nullptr, bool stall = false);
+// (stall: tests of the bounded waits only -- the key producer issues nothing and every
+// wait gives up after a few thousand polls; the kernel records an error and returns)
 // Prefill: queries of one sequence against its keys [N, d_I]; scores[q*ld + s] for visible s.
 cudaError_t launch_indexer_prefill_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, int N,
                                       const int32_t* q_pos, int Tq, int rate, float* scores, long long ld_scores,

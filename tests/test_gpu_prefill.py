@@ -70,6 +70,14 @@ def test_prefill_pro_shape_ragged(hca=None):
     _check(s, d, csa_kv, csa_k, topk, out, qs, check_all_entries=True)
 
 
+def cfg4_subsample(T=65536):
+    """The 1,024-query subsample of the 64K prefill: every 64th position, shifted by
+    i mod 4 so that all four queries of a 4-query indexer group occur (t = 64 i + i mod 4),
+    plus the edges of causality and of the window and the last query."""
+    qs = [64 * i + (i % 4) for i in range(T // 64)]
+    return sorted(set(qs + [0, 1, 2, 3, 4, 127, 128, 4095, 4096, 4097, T - 1]))
+
+
 def test_prefill_64k_sampled():
     import long_context_attention_compress_b200 as hca
     s = wl.PRO
@@ -77,7 +85,8 @@ def test_prefill_64k_sampled():
     d = wl.prefill_inputs(s, T=T, seed=0, with_hca=False)
     csa_kv, csa_k, topk, out = _prefill(hca, s, d)
     rng = np.random.default_rng(0)
-    qs = sorted(set([0, 1, 2, 3, 4, 127, 128, 4095, 4096, 4097, 65535] + rng.integers(0, T, 24).tolist()))
+    qs = cfg4_subsample(T)
+    assert len(qs) >= 1024 and {t % 4 for t in qs} == {0, 1, 2, 3}
     # entries compared on a sample (the float64 compressor over 16,384 entries is checked in full elsewhere)
     _check(s, d, csa_kv, csa_k, topk, out, qs, check_all_entries=False)
     f = lambda x: x.float().numpy().astype(np.float64)  # noqa: E731
@@ -86,3 +95,30 @@ def test_prefill_64k_sampled():
         ref = oracle.csa_compress(f(d["cand"][lo:(i + 1) * s.m]), f(d["logits"][lo:(i + 1) * s.m]),
                                   f(d["bias_csa"]), s.m)[-1]
         assert_bf16_close(to64(csa_kv[i]), ref, f"entry {i}")
+
+
+def test_prefill_indexer_long_rows():
+    """Prefill-mode indexer + top-k on queries whose visible rows cross 49,152
+    entries (the most one on-chip select pass of 32-bit keys holds), up to
+    65,536 entries, plus short rows in the same call."""
+    import long_context_attention_compress_b200 as hca
+    s = wl.PRO
+    N = 65536
+    g = torch.Generator().manual_seed(77)
+    K = torch.randn((N, s.d_idx), generator=g).bfloat16()
+    pos = [0, 3, 4 * 1024 - 1, 4 * 1024, 4 * 49152 - 2, 4 * 49152 - 1, 4 * 49152 + 3, 4 * 50000 + 1,
+           4 * 60000 + 2, 4 * 65535, 4 * 65536 - 2, 4 * 65536 - 1]
+    Tq = len(pos)
+    q_idx = torch.randn((Tq, s.n_idx_heads, s.d_idx), generator=g).bfloat16()
+    w_idx = torch.rand((Tq, s.n_idx_heads), generator=g)
+    q_pos = torch.tensor(pos, dtype=torch.int32)
+    cfg = hca.make_cfg(s)
+    ti = hca.csa_indexer_topk(q_idx.cuda(), w_idx.cuda(), K.cuda(), q_pos.cuda(), cfg, mode=hca.HCA_MODE_PREFILL)
+    torch.cuda.synchronize()
+    assert hca.lib.hca_check_device() == 0, hca.last_error()
+    ti = ti.cpu().numpy()
+    K64 = to64(K)
+    for i, t in enumerate(pos):
+        nv = oracle.n_visible(t, s.m, N)
+        sc = oracle.indexer_scores(to64(q_idx[i]), w_idx[i].double().numpy(), K64[:nv])
+        check_topk_row(ti[i], oracle.topk_select(sc, s.topk), sc, s.topk, nv)

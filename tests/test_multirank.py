@@ -63,3 +63,20 @@ def test_single_rank_needs_no_process_group(monkeypatch):
     r, local, w = bench.init_dist("gloo")
     assert (r, local, w) == (0, 0, 1)
     assert bench.reduce_max(3.5, w, "cpu") == 3.5
+
+
+@pytest.mark.timeout(180)
+def test_gpus_flag_starts_that_many_ranks():
+    """`bench.py --gpus 2` outside torchrun starts two ranks itself (here gloo ranks
+    on the CPU, via --check-launch, which runs one collective and no GPU work)."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "LOCAL_RANK", "WORLD_SIZE", "MASTER_ADDR",
+                                                             "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--check-launch"],
+                       capture_output=True, text=True, timeout=170, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["world_size"] == 2 and d["ranks_agreed"] == 2
