@@ -187,12 +187,13 @@ def source_hash(files):
 class DecodeBench:
     """Hybrid / CSA / HCA decode.  Per step: one hybrid_attn_decode call."""
 
-    def __init__(self, name, spec, seed, device, qk_norm=False, indexer="bf16"):
+    def __init__(self, name, spec, seed, device, qk_norm=False, indexer="bf16", paged=False, kv_fp8=False):
         import long_context_attention_compress_b200 as hca
         self.hca = hca
         self.name = name
         self.spec = spec
         self.indexer = indexer
+        self.kv_fp8 = kv_fp8
         s = self.shape = spec["shape"]
         B, ctx = spec["B"], spec["ctx"]
         # Q/KV normalisation + partial RoPE: synthetic weights per layer
@@ -237,14 +238,66 @@ class DecodeBench:
                 hca.mxfp4_quantize(K[b], codes=codes[b], scales=scales[b])
             del K
             self.norm_kw["csa_k4"] = (codes, scales)
+        self.n_entries = {"csa": self.csa["E"].shape[1] if self.csa is not None else 0,
+                          "hca": self.hcad["E_h"].shape[1] if self.hcad is not None else 0}
+        self.paged = None
+        if paged:
+            self._make_paged(seed, dev)
+        if kv_fp8:
+            # FP8 cache form of both layers' entries (E4M3 + f32 group scales, bf16 rotary part)
+            for key, d, arg in (("E", self.csa, "csa_kv8"), ("E_h", self.hcad, "hca_kv8")):
+                if d is not None:
+                    self.norm_kw[arg] = hca.kv_fp8_quantize(d.pop(key), self.cfg)
+            torch.cuda.empty_cache()
         self.args, self._keep = hca.make_decode_args(B, self.q_pos, csa=self.csa, hca=self.hcad,
                                                      csa_topk_idx=self.idx, csa_out=self.csa_out,
                                                      hca_out=self.hca_out, events=self.events, **self.norm_kw)
+        self._apply_paged(self.args)
         self.ws = torch.empty(max(1, hca.hybrid_attn_decode_workspace(self.cfg, self.args)), dtype=torch.uint8,
                               device=dev)
         self.units = B
         self.metric = "hybrid CSA+HCA decode queries/s at 1M ctx"
         self.unit = "queries/s"
+
+    def _make_paged(self, seed, dev):
+        """The caches in paged form: blocks of lcm(m, m') = 128 raw tokens (32 CSA entries
+        and keys, 1 HCA entry per block) in pools, reached through a shuffled block table."""
+        s, B = self.shape, self.B
+        L = s.m * s.m_hca // math.gcd(s.m, s.m_hca)
+        rc, rh = L // s.m, L // s.m_hca
+        N = self.csa["E"].shape[1] if self.csa is not None else 0
+        Nh = self.hcad["E_h"].shape[1] if self.hcad is not None else 0
+        nblk = max((N + rc - 1) // rc, (Nh + rh - 1) // rh)
+        P = B * nblk
+        g = torch.Generator(device="cpu").manual_seed(seed + 99)
+        perm = torch.randperm(P, generator=g).to(torch.int32)
+        bt = perm.view(B, nblk).to(dev)
+        # physical block perm[b * nblk + j] holds request b's logical block j
+        inv = torch.empty_like(perm)
+        inv[perm.long()] = torch.arange(P, dtype=torch.int32)
+        inv = inv.long().to(dev)
+
+        def pool(flat, rpb):  # [B, n, w] -> [P, rpb, w] in shuffled block order
+            Bn, n, w = flat.shape
+            fb = flat.new_zeros((Bn, nblk * rpb, w))
+            fb[:, :n] = flat
+            return fb.view(Bn * nblk, rpb, w)[inv].contiguous()
+        if self.csa is not None:
+            self.csa["E"] = pool(self.csa["E"], rc)
+            if "K_I" in self.csa:
+                self.csa["K_I"] = pool(self.csa["K_I"], rc)
+        if self.hcad is not None:
+            self.hcad["E_h"] = pool(self.hcad["E_h"], rh)
+        torch.cuda.empty_cache()
+        self.paged = {"bt": bt, "nblk": nblk, "P": P, "N": N, "Nh": Nh}
+
+    def _apply_paged(self, args):
+        if self.paged is None:
+            return
+        pg = self.paged
+        args.csa_N, args.hca_N = pg["N"], pg["Nh"]
+        args.block_table, args.bt_stride, args.n_pool_blocks = pg["bt"].data_ptr(), pg["nblk"], pg["P"]
+        args.csa_kv_stride = args.csa_k_stride = args.hca_kv_stride = 0
 
     def step(self, record=True):
         self.args.n_events = len(self.events) if record else 0
@@ -260,14 +313,16 @@ class DecodeBench:
         if "hca_compress" in self.phases:
             out["hca_compress"] = B * (2 * s.m_hca * s.c * 2 + s.c * 2)
         if self.csa is not None:
-            N = self.csa["E"].shape[1]
+            N = self.n_entries["csa"]
             key_bytes = s.d_idx // 2 + s.d_idx // 32 if self.indexer == "fp4" else s.d_idx * 2
             out["indexer_scores"] = B * (N * key_bytes + s.n_idx_heads * (s.d_idx * 2 + 4))
             out["topk_select"] = B * s.topk * 4
-            out["csa_attention"] = B * ((min(s.topk, N) + s.n_win) * s.c * 2 + 2 * s.n_heads * s.c * 2 + s.topk * 4)
+            row = (s.c - s.rope_dims) + 4 * (s.c - s.rope_dims) // 64 + 2 * s.rope_dims if self.kv_fp8 else s.c * 2
+            out["csa_attention"] = B * (min(s.topk, N) * row + s.n_win * s.c * 2 + 2 * s.n_heads * s.c * 2 + s.topk * 4)
         if self.hcad is not None:
-            Nh = self.hcad["E_h"].shape[1]
-            out["hca_attention"] = B * ((Nh + s.n_win) * s.c * 2 + 2 * s.n_heads * s.c * 2)
+            Nh = self.n_entries["hca"]
+            row = (s.c - s.rope_dims) + 4 * (s.c - s.rope_dims) // 64 + 2 * s.rope_dims if self.kv_fp8 else s.c * 2
+            out["hca_attention"] = B * (Nh * row + s.n_win * s.c * 2 + 2 * s.n_heads * s.c * 2)
         return out
 
     def config(self):
@@ -277,9 +332,14 @@ class DecodeBench:
                                                                          if self.indexer == "fp4" else ""),
              "n_win": s.n_win}
         if self.csa is not None:
-            c["csa_entries"] = int(self.csa["E"].shape[1])
+            c["csa_entries"] = int(self.n_entries["csa"])
         if self.hcad is not None:
-            c["hca_entries"] = int(self.hcad["E_h"].shape[1])
+            c["hca_entries"] = int(self.n_entries["hca"])
+        if self.kv_fp8:
+            c["kv_cache"] = "FP8 E4M3 (448 channels, f32 scale per 64) + bf16 rotary 64 channels"
+        if self.paged:
+            c["cache"] = (f"paged: blocks of 128 raw tokens (32 CSA entries + keys, 1 HCA entry), "
+                          f"{self.paged['P']} blocks, shuffled block table")
         return c
 
     # --- end to end: per-step inputs from pinned host memory, outputs back ---
@@ -312,6 +372,7 @@ class DecodeBench:
             d_out = [t for t in outs if t is not None]
             args, keep = self.hca.make_decode_args(self.B, self.q_pos, csa=csa, hca=hcad, csa_topk_idx=outs[0],
                                                    csa_out=outs[1], hca_out=outs[2], **self.norm_kw)
+            self._apply_paged(args)
             h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d_out]
             self.sets.append({"args": args, "keep": (keep, csa, hcad, outs), "d_in": d_in, "d_out": d_out,
                               "h_out": h_out})
@@ -445,7 +506,7 @@ class PrefillBench:
         return time.perf_counter() - t0
 
 
-def make_bench(name, seed, device, tokens=None, qk_norm=False, indexer="bf16"):
+def make_bench(name, seed, device, tokens=None, qk_norm=False, indexer="bf16", paged=False, kv_fp8=False):
     spec = wl.WORKLOADS[name]
     if qk_norm:
         name = f"{name}+qk_norm"  # the layer with Q/KV RMSNorm + partial RoPE (not the headline workload)
@@ -461,7 +522,13 @@ def make_bench(name, seed, device, tokens=None, qk_norm=False, indexer="bf16"):
         if spec["kind"] == "hca_decode":
             raise SystemExit("--indexer fp4 needs a CSA layer")
         name = f"{name}+fp4_indexer"  # the FP4 indexer variant (not the headline workload)
-    return DecodeBench(name, spec, seed, device, qk_norm, indexer=indexer)
+    if paged:
+        if indexer != "bf16" or kv_fp8:
+            raise SystemExit("--paged takes the bf16 indexer and bf16 caches")
+        name = f"{name}+paged"  # the paged-cache variant (not the headline workload)
+    if kv_fp8:
+        name = f"{name}+kv_fp8"  # the FP8 KV-cache variant (not the headline workload)
+    return DecodeBench(name, spec, seed, device, qk_norm, indexer=indexer, paged=paged, kv_fp8=kv_fp8)
 
 
 def norm_prologue_roofline(bench, flush, pk, reps=20):
@@ -701,7 +768,7 @@ def run_ours(a):
     device = torch.device("cuda", local)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     bench = make_bench(a.workload, shard_seed(a.seed, rank), device, tokens=a.tokens, qk_norm=a.qk_norm,
-                       indexer=a.indexer)
+                       indexer=a.indexer, paged=a.paged, kv_fp8=a.kv_fp8)
     m = measure(bench, a, a.steps, a.warmup, flush, rank, ws, device, local, a.cpu_sample)
     out = {"metric": bench.metric, "value": m.pop("value"), "unit": m.pop("unit"), "n_gpus": ws,
            "steps": m.pop("steps"), "warmup": a.warmup, "ms_per_step": m.pop("ms_per_step"),
@@ -713,7 +780,8 @@ def run_ours(a):
     out.update(m)
     # The metric has two halves: decode queries/s (the headline) and prefill tokens/s.
     # The default run measures the 64K CSA prefill as well, in the same line.
-    if a.workload == DEFAULT_WORKLOAD and not a.no_prefill and a.tokens is None and a.indexer == "bf16":
+    if (a.workload == DEFAULT_WORKLOAD and not a.no_prefill and a.tokens is None and a.indexer == "bf16"
+            and not a.paged and not a.kv_fp8):
         del bench
         torch.cuda.empty_cache()
         pb = make_bench("csa_prefill_64k", shard_seed(a.seed, rank), device, qk_norm=a.qk_norm)
@@ -824,6 +892,10 @@ def main():
                     help="prefill workloads: a shorter sequence of the same shape (for profiler captures)")
     ap.add_argument("--indexer", default="bf16", choices=["bf16", "fp4"],
                     help="fp4: the decode indexer over MXFP4 keys with BF16 scores (a variant, not the headline)")
+    ap.add_argument("--kv-fp8", action="store_true",
+                    help="decode workloads: the KV caches in FP8 form (E4M3 + bf16 rotary channels)")
+    ap.add_argument("--paged", action="store_true",
+                    help="decode workloads: the caches in paged form (blocks of 128 raw tokens, shuffled block table)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="default workload only: skip the 64K prefill measured in the same line")
     ap.add_argument("--prefill-steps", type=int, default=None,

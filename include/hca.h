@@ -256,6 +256,36 @@ int csa_indexer_topk_fp4(const hca_bf16* q_idx, const float* w_idx, const uint8_
 size_t csa_indexer_topk_fp4_workspace(const hca_layer_cfg* cfg, int B, int N);
 
 /* ---------------------------------------------------------------------------
+ * FP8 storage of the KV channels outside the rotary part ([Tricks] "Partial
+ * RoPE 和 Attention Sink": the rotary channels of the KV cache stay BF16, the
+ * other channels are stored in FP8).  Cache form of a row of c channels, with
+ * n = c - cfg->rope_dims (a multiple of 64) and rope_dims a multiple of 8:
+ *   codes  [n] E4M3 bytes (sign bit 7, exponent bits 3-6 with bias 7 and field 0
+ *          subnormal, mantissa bits 0-2): the E4M3 value nearest to x / scale of
+ *          the channel's group (ties to the even mantissa, saturating at +-448;
+ *          a negative value that rounds to zero keeps its sign);
+ *   scales [n / 64] f32: scale of a group of 64 channels = f32(max |x| / 448),
+ *          1 for an all-zero group;
+ *   rope   [rope_dims] bf16: the last rope_dims channels, rounded to bf16.
+ * A row's value is code * scale on the first n channels, then the rope part.
+ *
+ * kv_fp8_quantize -- the cache form of `rows` rows x [c] (x bf16, or f32 with
+ *   x_is_f32 = 1; row stride ld_x elements); codes row stride ld_codes bytes (a
+ *   multiple of 16), scales ld_scales floats, rope ld_rope bf16 (a multiple of 8).
+ *   Every code is decided on the f64 quotient of the f32 values x and scale.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  uint8_t* codes;      /* [rows][ld_codes] */
+  float* scales;       /* [rows][ld_scales] */
+  hca_bf16* rope;      /* [rows][ld_rope] */
+  long long ld_codes, ld_scales, ld_rope;
+  long long seq_rows;  /* rows between requests (decode) */
+} hca_kv_fp8;
+int kv_fp8_quantize(const void* x, int x_is_f32, long long ld_x, long long rows, const hca_layer_cfg* cfg,
+                    uint8_t* codes, long long ld_codes, float* scales, long long ld_scales, hca_bf16* rope,
+                    long long ld_rope, void* stream);
+
+/* ---------------------------------------------------------------------------
  * sparse_mqa_attend -- core shared-KV multi-query attention over compressed
  * entries plus the sliding window, one softmax ([QbitAI] CSA step three, the
  * KV-entry-as-key-and-value remark and the sliding-window paragraph;
@@ -351,6 +381,33 @@ typedef struct {
   const uint8_t* csa_k_codes;
   const uint8_t* csa_k_scales;
   long long csa_k4_stride;
+  /* Paged caches ([Tricks] "Heterogeneous KV Cache Layout": the compressed
+   * ("classical") cache is allocated in blocks that each cover L = lcm(m, m')
+   * raw tokens, i.e. L/m CSA entries with their indexer keys and L/m' HCA
+   * entries; [Jiedu] 核心创新一: the window sits in a separate state cache), or
+   * NULL: flat caches as above.  With block_table, request b's logical block j
+   * is physical block block_table[b*bt_stride + j] (int32, device) of every
+   * pool: csa_kv is a pool [n_pool_blocks][L/m][c], csa_k_idx
+   * [n_pool_blocks][L/m][d_I], hca_kv [n_pool_blocks][L/m'][c]; entry i of a
+   * request is row i % (L/m) of its block i / (L/m) (likewise for HCA); the
+   * request strides csa_kv_stride, csa_k_stride and hca_kv_stride are not read.
+   * The newest HCA entry (hca_block_cand) is written to its pool row.  Each
+   * window block [n_win, c] is a ring: token tau at row tau mod n_win (this
+   * only matters with Q/KV normalisation; rows >= q_pos+1 are not read).
+   * Needs c = 512, 64 heads, the 64 x 128 indexer with bf16 keys, L/m a
+   * multiple of 8 dividing 128, and bt_stride >= the blocks each layer's
+   * entries span. */
+  const int32_t* block_table;
+  long long bt_stride;
+  int n_pool_blocks;
+  /* FP8 caches (see kv_fp8_quantize; host pointers to descriptors), or NULL: the
+   * layer's entries are read from their FP8 form (csa_kv / hca_kv are not read):
+   * request b's entry i is row b*seq_rows + i.  The rows an attention reads are
+   * first widened to bf16 (code * scale, rounded once) in the workspace: the CSA
+   * layer's selected rows, the HCA layer's visible rows.  With hca_block_cand the
+   * newest HCA entry is written in FP8 form to row hca_N-1.  Not with paged caches. */
+  const hca_kv_fp8* csa_kv8;
+  const hca_kv_fp8* hca_kv8;
 } hca_decode_args;
 
 int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* args, void* ws,

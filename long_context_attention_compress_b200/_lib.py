@@ -55,7 +55,14 @@ class DecodeArgs(ctypes.Structure):
                 ("hca_pos_bias", c_void_p), ("hca_win", c_void_p), ("hca_win_stride", c_ll), ("hca_out", c_void_p),
                 ("events", c_void_p), ("n_events", c_int), ("csa_sink", c_void_p), ("hca_sink", c_void_p),
                 ("csa_norm", c_void_p), ("hca_norm", c_void_p),
-                ("csa_k_codes", c_void_p), ("csa_k_scales", c_void_p), ("csa_k4_stride", c_ll)]
+                ("csa_k_codes", c_void_p), ("csa_k_scales", c_void_p), ("csa_k4_stride", c_ll),
+                ("block_table", c_void_p), ("bt_stride", c_ll), ("n_pool_blocks", c_int),
+                ("csa_kv8", c_void_p), ("hca_kv8", c_void_p)]
+
+
+class KvFp8(ctypes.Structure):
+    _fields_ = [("codes", c_void_p), ("scales", c_void_p), ("rope", c_void_p), ("ld_codes", c_ll),
+                ("ld_scales", c_ll), ("ld_rope", c_ll), ("seq_rows", c_ll)]
 
 
 class PrefillArgs(ctypes.Structure):
@@ -88,6 +95,8 @@ _mxfp4_quantize = _sig("mxfp4_quantize", c_int, [c_void_p, c_int, c_ll, c_int, c
 _indexer_fp4 = _sig("csa_indexer_topk_fp4", c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_ll, c_int, c_void_p,
                                                     c_int, ctypes.POINTER(LayerCfg), c_void_p, c_void_p, c_size,
                                                     c_void_p])
+_kv_fp8_quantize = _sig("kv_fp8_quantize", c_int, [c_void_p, c_int, c_ll, c_ll, ctypes.POINTER(LayerCfg), c_void_p,
+                                                   c_ll, c_void_p, c_ll, c_void_p, c_ll, c_void_p])
 _indexer_fp4_ws = _sig("csa_indexer_topk_fp4_workspace", c_size, [ctypes.POINTER(LayerCfg), c_int, c_int])
 _norm_rope = _sig("rms_norm_rope", c_int, [c_void_p, c_int, c_ll, c_ll, c_int, c_int, c_void_p, c_int, c_int,
                                           c_void_p, ctypes.POINTER(LayerCfg), c_void_p, c_ll, c_ll, c_void_p])
@@ -228,6 +237,36 @@ def mxfp4_quantize(x, codes=None, scales=None, stream=None):
     return codes, scales
 
 
+def kv_fp8_quantize(x, cfg: LayerCfg, out=None, stream=None):
+    """FP8 cache form of KV rows x [..., c] (bf16 or float32): returns (codes uint8
+    [..., c - rope_dims], scales float32 [..., (c - rope_dims) / 64], rope bf16
+    [..., rope_dims]); `out` may give that triple to write into."""
+    c = x.shape[-1]
+    rows = x.numel() // c
+    n, r = c - cfg.rope_dims, cfg.rope_dims
+    lead = x.shape[:-1]
+    if out is None:
+        out = (torch.empty(lead + (n,), dtype=torch.uint8, device=x.device),
+               torch.empty(lead + (n // 64,), dtype=F32, device=x.device),
+               torch.empty(lead + (r,), dtype=BF16, device=x.device))
+    codes, scales, rope = out
+    if x.dtype not in (BF16, F32):
+        raise TypeError(f"x: dtype {x.dtype}")
+    _check(_kv_fp8_quantize(_ptr(x, None, "x"), 1 if x.dtype == F32 else 0, c, rows, ctypes.byref(cfg),
+                            _ptr(codes, torch.uint8, "codes"), n, _ptr(scales, F32, "scales"), n // 64,
+                            _ptr(rope, BF16, "rope"), r, _stream(stream)))
+    return codes, scales, rope
+
+
+def make_kv_fp8(codes, scales, rope):
+    """KvFp8 descriptor of an FP8 cache (codes [B, N, n], scales [B, N, n/64], rope [B, N, r])."""
+    d = KvFp8()
+    d.codes, d.scales, d.rope = _ptr(codes, torch.uint8, "codes"), _ptr(scales, F32, "scales"), _ptr(rope, BF16, "rope")
+    d.ld_codes, d.ld_scales, d.ld_rope = codes.shape[-1], scales.shape[-1], rope.shape[-1]
+    d.seq_rows = codes.shape[-2] if codes.dim() == 3 else 0
+    return d
+
+
 def csa_indexer_topk_fp4(q_idx, w_idx, k_codes, k_scales, q_pos, cfg: LayerCfg, out=None, ws=None, stream=None):
     """Decode indexer + top-k over MXFP4 keys (k_codes [B, N_alloc, 64] uint8, k_scales
     [B, N_alloc, 4] uint8, N = q's visible range up to N_alloc) with BF16 scores."""
@@ -304,7 +343,8 @@ def _events_array(events):
 
 
 def make_decode_args(B, q_pos, csa=None, hca=None, csa_topk_idx=None, csa_out=None, hca_out=None, events=None,
-                     csa_sink=None, hca_sink=None, csa_norm=None, hca_norm=None, csa_k4=None):
+                     csa_sink=None, hca_sink=None, csa_norm=None, hca_norm=None, csa_k4=None, csa_kv8=None,
+                     hca_kv8=None):
     """Build DecodeArgs from dicts of tensors (see workloads.csa_decode_inputs /
     hca_decode_inputs); csa_sink / hca_sink: optional [H] float32 sink logits;
     csa_norm / hca_norm: optional [2, c] float32 Q/KV normalisation weights;
@@ -312,6 +352,13 @@ def make_decode_args(B, q_pos, csa=None, hca=None, csa_topk_idx=None, csa_out=No
     the MXFP4 indexer keys of the FP4 indexer variant (see mxfp4_quantize).
     Returns (args, keepalive)."""
     a = DecodeArgs()
+    # FP8 caches: (codes, scales, rope) triples from kv_fp8_quantize
+    d8 = []
+    for name, t in (("csa_kv8", csa_kv8), ("hca_kv8", hca_kv8)):
+        if t is not None:
+            desc = make_kv_fp8(*t)
+            setattr(a, name, ctypes.cast(ctypes.pointer(desc), c_void_p))
+            d8.append(desc)
     if csa_k4 is not None:
         codes, scales = csa_k4
         a.csa_k_codes = _ptr(codes, torch.uint8, "csa_k4 codes")
@@ -324,15 +371,17 @@ def make_decode_args(B, q_pos, csa=None, hca=None, csa_topk_idx=None, csa_out=No
     a.B = B
     a.q_pos = _ptr(q_pos, I32, "q_pos")
     # every tensor the struct points at stays alive with the returned keepalive
-    keep = [q_pos, csa_sink, hca_sink, csa_norm, hca_norm, csa, hca, csa_topk_idx, csa_out, hca_out, csa_k4]
+    keep = [q_pos, csa_sink, hca_sink, csa_norm, hca_norm, csa, hca, csa_topk_idx, csa_out, hca_out, csa_k4, csa_kv8,
+            hca_kv8, d8]
     if csa is not None:
         a.csa_q = _ptr(csa["q"], BF16, "csa.q")
         a.csa_q_idx = _ptr(csa["q_idx"], BF16, "csa.q_idx")
         a.csa_w_idx = _ptr(csa["w_idx"], F32, "csa.w_idx")
-        a.csa_kv = _ptr(csa["E"], BF16, "csa.E")
+        E = csa.get("E")  # (not read with an FP8 cache)
+        a.csa_kv = _ptr(E, BF16, "csa.E")
         a.csa_k_idx = _ptr(csa.get("K_I"), BF16, "csa.K_I")  # (not read by the FP4 variant)
-        a.csa_N = csa["E"].shape[1]
-        a.csa_kv_stride = csa["E"].stride(0)
+        a.csa_N = E.shape[1] if E is not None else csa_kv8[0].shape[1]
+        a.csa_kv_stride = E.stride(0) if E is not None else 0
         a.csa_k_stride = csa["K_I"].stride(0) if csa.get("K_I") is not None else 0
         a.csa_win = _ptr(csa["win"], BF16, "csa.win")
         a.csa_win_stride = csa["win"].stride(0)
@@ -340,9 +389,10 @@ def make_decode_args(B, q_pos, csa=None, hca=None, csa_topk_idx=None, csa_out=No
         a.csa_out = _ptr(csa_out, BF16, "csa_out")
     if hca is not None:
         a.hca_q = _ptr(hca["q"], BF16, "hca.q")
-        a.hca_kv = _ptr(hca["E_h"], BF16, "hca.E_h")
-        a.hca_N = hca["E_h"].shape[1]
-        a.hca_kv_stride = hca["E_h"].stride(0)
+        Eh = hca.get("E_h")  # (not read with an FP8 cache)
+        a.hca_kv = _ptr(Eh, BF16, "hca.E_h")
+        a.hca_N = Eh.shape[1] if Eh is not None else hca_kv8[0].shape[1]
+        a.hca_kv_stride = Eh.stride(0) if Eh is not None else 0
         if hca.get("block_cand") is not None:
             a.hca_block_cand = _ptr(hca["block_cand"], BF16, "hca.block_cand")
             a.hca_block_logits = _ptr(hca["block_logits"], BF16, "hca.block_logits")

@@ -146,9 +146,16 @@ struct IndexerPlan {
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Prefill on the tensor cores takes its top-k on chip (no workspace at all).
+bool fused_prefill(const hca_layer_cfg* cfg, int mode) {
+  return mode == HCA_MODE_PREFILL && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx) &&
+         indexer_prefill_topk_fused(cfg->topk);
+}
+
 // Workspace: the f32 score rows, then either select layout (they share the space;
-// only one is used per call).
-IndexerPlan plan_indexer(int Tq, int N, int k) {
+// only one is used per call); nothing for the fused prefill.
+IndexerPlan plan_indexer(const hca_layer_cfg* cfg, int Tq, int N, int mode) {
+  const int k = cfg->topk;
   IndexerPlan p;
   p.ld = ((long long)N + 3) / 4 * 4;
   if (N <= kSelectRowMaxN) {
@@ -174,12 +181,14 @@ IndexerPlan plan_indexer(int Tq, int N, int k) {
     const size_t hist_end = p.eq_off + (size_t)Tq * C * kHistSlice * sizeof(uint64_t);
     end = end > hist_end ? end : hist_end;
   }
-  p.bytes = end;
+  p.bytes = fused_prefill(cfg, mode) ? 0 : end;
   return p;
 }
 
-int indexer_ok(int N, int k, int mode) {
-  const IndexerPlan p = plan_indexer(1, N, k);
+int indexer_ok(const hca_layer_cfg* cfg, int N, int mode) {
+  const int k = cfg->topk;
+  const IndexerPlan p = plan_indexer(cfg, 1, N, mode);
+  if (fused_prefill(cfg, mode)) return HCA_OK;  // any number of entries
   if (mode == HCA_MODE_DECODE) {
     CHECK(p.hist_ctas <= kHistMaxCtas, HCA_ERR_UNSUPPORTED, "indexer: N=%d exceeds %d entries per request", N,
           kHistMaxCtas * kHistSlice);
@@ -203,8 +212,8 @@ struct Fp4Keys {
 int run_indexer_topk(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride, int N,
                      const int32_t* q_pos, int Tq, int mode, const hca_layer_cfg* cfg, int32_t* topk_idx,
                      void* ws, cudaStream_t st, void* const* ev, int n_ev, int& ev_i, int grid_sms = 0,
-                     const Fp4Keys* fp4 = nullptr) {
-  const IndexerPlan p = plan_indexer(Tq, N, cfg->topk);
+                     const Fp4Keys* fp4 = nullptr, const PagedKeys* paged = nullptr) {
+  const IndexerPlan p = plan_indexer(cfg, Tq, N, mode);
   float* scores = reinterpret_cast<float*>(ws);
   // decode with more entries than one select CTA holds: the indexer also builds
   // each request's score-key histogram, and one threshold select follows
@@ -227,8 +236,16 @@ int run_indexer_topk(const bf16* q_idx, const float* w_idx, const bf16* k_idx, l
     CUDA_TRY(launch_indexer_decode_tc(q_idx, w_idx, k_idx, k_seq_stride, N, q_pos, Tq, cfg->m, scores, p.ld,
                                       grid_sms > 0 ? grid_sms : device_sm_count(), st,
                                       hist ? reinterpret_cast<int*>(wsb + p.hist_off) : nullptr,
-                                      test_stall_indexer()),
+                                      test_stall_indexer(), paged),
              "indexer scores (tcgen05)");
+  } else if (fused_prefill(cfg, mode)) {
+    // scores and top-k in one kernel: nothing goes through memory but the indices
+    CUDA_TRY(launch_indexer_prefill_tc(q_idx, w_idx, k_idx, N, q_pos, Tq, cfg->m, nullptr, 0,
+                                       grid_sms > 0 ? grid_sms : device_sm_count(), st, cfg->topk, topk_idx),
+             "indexer + top-k (tcgen05, prefill)");
+    if (ev && ev_i < n_ev) CUDA_TRY(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
+    if (ev && ev_i < n_ev) CUDA_TRY(cudaEventRecord((cudaEvent_t)ev[ev_i++], st), "event");
+    return HCA_OK;
   } else if (mode == HCA_MODE_PREFILL && indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx)) {
     CUDA_TRY(launch_indexer_prefill_tc(q_idx, w_idx, k_idx, N, q_pos, Tq, cfg->m, scores, p.ld,
                                        grid_sms > 0 ? grid_sms : device_sm_count(), st),
@@ -399,8 +416,8 @@ size_t hca_workspace_size(int op, const hca_layer_cfg* cfg, int Tq, int N, int m
   if (check_cfg(cfg) != HCA_OK || Tq < 0 || N < 0) return (size_t)-1;
   switch (op) {
     case HCA_OP_INDEXER_TOPK:
-      if (indexer_ok(N, cfg->topk, mode) != HCA_OK) return (size_t)-1;
-      return plan_indexer(Tq, N, cfg->topk).bytes;
+      if (indexer_ok(cfg, N, mode) != HCA_OK) return (size_t)-1;
+      return plan_indexer(cfg, Tq, N, mode).bytes;
     case HCA_OP_SPARSE_MQA:
       return mqa_ws_bound(cfg, Tq, N, cfg->topk);
     default:
@@ -417,7 +434,7 @@ int csa_indexer_topk(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* 
   CHECK(Tq >= 0 && N >= 0, HCA_ERR_INVALID_ARG, "csa_indexer_topk: Tq=%d N=%d", Tq, N);
   CHECK(mode == HCA_MODE_PREFILL || mode == HCA_MODE_DECODE, HCA_ERR_INVALID_ARG, "csa_indexer_topk: mode=%d", mode);
   CHECK(mode == HCA_MODE_PREFILL || k_seq_stride % 8 == 0, HCA_ERR_INVALID_ARG, "csa_indexer_topk: k_seq_stride");
-  s = indexer_ok(N, cfg->topk, mode);
+  s = indexer_ok(cfg, N, mode);
   if (s != HCA_OK) return s;
   if (Tq == 0) return injected("csa_indexer_topk") ? fail(HCA_ERR_INJECTED, "injected") : HCA_OK;
   CHECK_PTR(q_idx, "csa_indexer_topk: q_idx");
@@ -425,7 +442,7 @@ int csa_indexer_topk(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* 
   CHECK_PTR(q_pos, "csa_indexer_topk: q_pos");
   CHECK_PTR(topk_idx, "csa_indexer_topk: topk_idx");
   if (N > 0) CHECK_PTR(k_idx, "csa_indexer_topk: k_idx");
-  const size_t need = plan_indexer(Tq, N, cfg->topk).bytes;
+  const size_t need = plan_indexer(cfg, Tq, N, mode).bytes;
   CHECK(ws_bytes >= need, HCA_ERR_WORKSPACE, "csa_indexer_topk: workspace %zu < %zu", ws_bytes, need);
   if (need) CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
                   "csa_indexer_topk: ws null or not 256-byte aligned");
@@ -476,9 +493,9 @@ int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hc
         "csa_indexer_topk_noalloc: mode=%d", mode);
   CHECK(mode == HCA_MODE_PREFILL || k_seq_stride % 8 == 0, HCA_ERR_INVALID_ARG,
         "csa_indexer_topk_noalloc: k_seq_stride");
-  s = indexer_ok(N, cfg->topk, mode);
+  s = indexer_ok(cfg, N, mode);
   if (s != HCA_OK) return s;
-  const size_t need = plan_indexer(Tq, N, cfg->topk).bytes;
+  const size_t need = plan_indexer(cfg, Tq, N, mode).bytes;
   CHECK(need <= (size_t)HCA_NOALLOC_SCRATCH_BYTES, HCA_ERR_WORKSPACE,
         "csa_indexer_topk_noalloc: Tq=%d x N=%d needs %zu bytes of scratch, more than the built-in %zu; "
         "use csa_indexer_topk with a workspace",
@@ -573,6 +590,62 @@ int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_st
   return HCA_OK;
 }
 
+// ---- FP8 storage of the non-rotary KV channels ----------------------------------
+static int check_fp8_layout(const hca_layer_cfg* cfg, long long ld_codes, long long ld_scales, long long ld_rope,
+                            const char* who) {
+  const int n = cfg->c - cfg->rope_dims;
+  CHECK(n > 0 && n % 64 == 0 && cfg->rope_dims % 8 == 0, HCA_ERR_UNSUPPORTED,
+        "%s: c - rope_dims = %d must be a positive multiple of 64 (rope_dims a multiple of 8)", who, n);
+  CHECK(ld_codes >= n && ld_codes % 16 == 0 && ld_scales >= n / 64 && ld_rope >= cfg->rope_dims && ld_rope % 8 == 0,
+        HCA_ERR_INVALID_ARG, "%s: row strides (codes %lld, scales %lld, rope %lld)", who, ld_codes, ld_scales, ld_rope);
+  return HCA_OK;
+}
+
+static KvFp8 kv_fp8_of(const hca_kv_fp8* d) {
+  KvFp8 k;
+  k.codes = d->codes;
+  k.scales = d->scales;
+  k.rope = reinterpret_cast<const bf16*>(d->rope);
+  k.ld_codes = d->ld_codes;
+  k.ld_scales = d->ld_scales;
+  k.ld_rope = d->ld_rope;
+  k.seq_rows = d->seq_rows;
+  return k;
+}
+
+extern "C" int kv_fp8_quantize(const void* x, int x_is_f32, long long ld_x, long long rows, const hca_layer_cfg* cfg,
+                               uint8_t* codes, long long ld_codes, float* scales, long long ld_scales, hca_bf16* rope,
+                               long long ld_rope, void* stream) {
+  g_err.clear();
+  int s = check_cfg(cfg);
+  if (s != HCA_OK) return s;
+  CHECK(rows >= 0, HCA_ERR_INVALID_ARG, "kv_fp8_quantize: rows=%lld", rows);
+  if ((s = check_fp8_layout(cfg, ld_codes, ld_scales, ld_rope, "kv_fp8_quantize")) != HCA_OK) return s;
+  CHECK(ld_x >= cfg->c && ld_x % (x_is_f32 ? 4 : 8) == 0, HCA_ERR_INVALID_ARG, "kv_fp8_quantize: ld_x %lld", ld_x);
+  if (rows == 0) return HCA_OK;
+  CHECK_PTR(x, "kv_fp8_quantize: x");
+  CHECK_PTR(codes, "kv_fp8_quantize: codes");
+  CHECK(scales != nullptr && (reinterpret_cast<uintptr_t>(scales) & 3u) == 0, HCA_ERR_INVALID_ARG,
+        "kv_fp8_quantize: scales null or misaligned");
+  if (cfg->rope_dims) CHECK_PTR(rope, "kv_fp8_quantize: rope");
+  if (injected("kv_fp8_quantize")) return fail(HCA_ERR_INJECTED, "kv_fp8_quantize: injected");
+  CUDA_TRY(launch_kv_fp8_quantize(x, x_is_f32 != 0, ld_x, rows, cfg->c, cfg->rope_dims, codes, ld_codes, scales,
+                                  ld_scales, reinterpret_cast<bf16*>(rope), ld_rope, as_stream(stream)),
+           "kv_fp8_quantize");
+  return HCA_OK;
+}
+
+static int check_kv8(const hca_layer_cfg* cfg, const hca_kv_fp8* d, const char* who) {
+  int s = check_fp8_layout(cfg, d->ld_codes, d->ld_scales, d->ld_rope, who);
+  if (s != HCA_OK) return s;
+  CHECK_PTR(d->codes, who);
+  CHECK(d->scales != nullptr && (reinterpret_cast<uintptr_t>(d->scales) & 3u) == 0, HCA_ERR_INVALID_ARG,
+        "%s: scales null or misaligned", who);
+  if (cfg->rope_dims) CHECK_PTR(d->rope, who);
+  CHECK(d->seq_rows >= 0, HCA_ERR_INVALID_ARG, "%s: seq_rows", who);
+  return HCA_OK;
+}
+
 // ---- decode ------------------------------------------------------------------
 // When both layers are present, the HCA layer (its block compression and dense
 // attention) runs on a side stream, concurrently with the CSA indexer, on a
@@ -589,16 +662,47 @@ struct DecodeSched {
   size_t csa_qn = 0, csa_wn = 0, hca_qn = 0, hca_wn = 0, hca_ef = 0;
   // FP4 indexer: the queries' MXFP4 values in bf16 [B, H_I, d_I]
   size_t q4 = 0;
+  // paged caches: the newest HCA entries [B, c] bf16 before they go to their pool rows
+  size_t hca_new = 0;
+  // FP8 caches: the CSA layer's selected rows widened to bf16 [B, k, c] and their
+  // slot indices [B, k]; the HCA layer's visible rows [B, hca_N, c]; the newest HCA
+  // entries [B, c] (f32, or bf16 after normalisation) before their FP8 form
+  size_t csa8_rows = 0, csa8_idx = 0, hca8_rows = 0, hca8_new = 0;
 };
 
+// Geometry of the paged (classical) cache: blocks of lcm(m, m') raw tokens.
+struct PagedGeom {
+  int rpb_csa = 0, rpb_hca = 0;
+};
+static PagedGeom paged_geom(const hca_layer_cfg* cfg) {
+  int a = cfg->m, b = cfg->m_hca;
+  while (b) { const int t = a % b; a = b; b = t; }
+  const long long L = (long long)cfg->m / a * cfg->m_hca;
+  PagedGeom g;
+  g.rpb_csa = (int)(L / cfg->m);
+  g.rpb_hca = (int)(L / cfg->m_hca);
+  return g;
+}
+static void make_paged(MqaProblem& p, const hca_decode_args* a, int rpb) {
+  p.bt = a->block_table;
+  p.bt_stride = a->bt_stride;
+  p.rpb = rpb;
+  p.pool_rows = (long long)a->n_pool_blocks * rpb;
+  p.kv_seq_stride = 0;
+}
+
 static MqaProblem decode_csa_problem(const hca_layer_cfg* cfg, const hca_decode_args* a) {
-  return make_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_N,
-                  a->csa_topk_idx ? a->csa_topk_idx : reinterpret_cast<const int32_t*>(1), cfg->topk, cfg->m,
-                  a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out, a->csa_sink);
+  MqaProblem p = make_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_N,
+                          a->csa_topk_idx ? a->csa_topk_idx : reinterpret_cast<const int32_t*>(1), cfg->topk, cfg->m,
+                          a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out, a->csa_sink);
+  if (a->block_table) make_paged(p, a, paged_geom(cfg).rpb_csa);
+  return p;
 }
 static MqaProblem decode_hca_problem(const hca_layer_cfg* cfg, const hca_decode_args* a) {
-  return make_mqa(cfg, a->hca_q, a->hca_kv, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, a->hca_win,
-                  a->hca_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->hca_out, a->hca_sink);
+  MqaProblem p = make_mqa(cfg, a->hca_q, a->hca_kv, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, a->hca_win,
+                          a->hca_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->hca_out, a->hca_sink);
+  if (a->block_table) make_paged(p, a, paged_geom(cfg).rpb_hca);
+  return p;
 }
 
 static DecodeSched decode_schedule(const hca_layer_cfg* cfg, const hca_decode_args* a) {
@@ -634,7 +738,7 @@ static DecodeSched decode_schedule(const hca_layer_cfg* cfg, const hca_decode_ar
   }
   if (csa) {
     d.csa_pl = plan_mqa(pc);
-    d.main_bytes = std::max(plan_indexer(a->B, a->csa_N, cfg->topk).bytes, d.csa_pl.ws_bytes);
+    d.main_bytes = std::max(plan_indexer(cfg, a->B, a->csa_N, HCA_MODE_DECODE).bytes, d.csa_pl.ws_bytes);
   }
   if (d.overlap) {
     d.hca_off = round256(d.main_bytes);
@@ -659,6 +763,20 @@ static DecodeSched decode_schedule(const hca_layer_cfg* cfg, const hca_decode_ar
   if (csa && a->csa_k_codes) {
     d.q4 = d.total;
     d.total = d.q4 + round256((size_t)a->B * cfg->n_idx_heads * cfg->d_idx * 2);
+  }
+  if (hcl && a->block_table && a->hca_block_cand) {
+    d.hca_new = d.total;
+    d.total = d.hca_new + round256((size_t)a->B * cfg->c * 2);
+  }
+  if (csa && a->csa_kv8) {
+    d.csa8_rows = d.total;
+    d.csa8_idx = d.csa8_rows + round256((size_t)a->B * cfg->topk * cfg->c * 2);
+    d.total = d.csa8_idx + round256((size_t)a->B * cfg->topk * 4);
+  }
+  if (hcl && a->hca_kv8) {
+    d.hca8_rows = d.total;
+    d.hca8_new = d.hca8_rows + round256((size_t)a->B * a->hca_N * cfg->c * 2);
+    d.total = d.hca8_new + round256((size_t)a->B * cfg->c * 4);
   }
   return d;
 }
@@ -694,7 +812,7 @@ static int side_stream(SideStream** out) {
 
 size_t hybrid_attn_decode_workspace(const hca_layer_cfg* cfg, const hca_decode_args* a) {
   if (check_cfg(cfg) != HCA_OK || !a || a->B < 0) return (size_t)-1;
-  if (a->csa_q && indexer_ok(a->csa_N, cfg->topk, HCA_MODE_DECODE) != HCA_OK) return (size_t)-1;
+  if (a->csa_q && indexer_ok(cfg, a->csa_N, HCA_MODE_DECODE) != HCA_OK) return (size_t)-1;
   return decode_ws(cfg, a);
 }
 
@@ -708,8 +826,32 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
   CHECK(a->n_events >= 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: n_events");
   if (a->B == 0) return HCA_OK;
   CHECK_PTR(a->q_pos, "hybrid_attn_decode: q_pos");
+  const PagedGeom pg = paged_geom(cfg);
+  if (a->block_table) {
+    CHECK_PTR(a->block_table, "hybrid_attn_decode: block_table");
+    CHECK(cfg->c == 512 && cfg->n_heads == 64, HCA_ERR_UNSUPPORTED,
+          "hybrid_attn_decode: paged caches need c = 512 and 64 heads");
+    CHECK(a->n_pool_blocks > 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: n_pool_blocks=%d", a->n_pool_blocks);
+    if (a->csa_q) {
+      CHECK(indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx) && !a->csa_k_codes, HCA_ERR_UNSUPPORTED,
+            "hybrid_attn_decode: paged caches need the 64 x 128 indexer with bf16 keys");
+      CHECK(pg.rpb_csa % 8 == 0 && 128 % pg.rpb_csa == 0, HCA_ERR_UNSUPPORTED,
+            "hybrid_attn_decode: paged CSA blocks of %d entries (need a multiple of 8 dividing 128)", pg.rpb_csa);
+      CHECK(a->bt_stride >= ((long long)a->csa_N + pg.rpb_csa - 1) / pg.rpb_csa, HCA_ERR_INVALID_ARG,
+            "hybrid_attn_decode: bt_stride %lld < the %d CSA blocks", a->bt_stride,
+            (a->csa_N + pg.rpb_csa - 1) / pg.rpb_csa);
+    }
+    if (a->hca_q)
+      CHECK(a->bt_stride >= ((long long)a->hca_N + pg.rpb_hca - 1) / pg.rpb_hca, HCA_ERR_INVALID_ARG,
+            "hybrid_attn_decode: bt_stride %lld < the %d HCA blocks", a->bt_stride,
+            (a->hca_N + pg.rpb_hca - 1) / pg.rpb_hca);
+  }
+  if (a->csa_kv8 || a->hca_kv8)
+    CHECK(!a->block_table, HCA_ERR_UNSUPPORTED, "hybrid_attn_decode: FP8 caches are not paged");
+  if (a->csa_q && a->csa_kv8 && (s = check_kv8(cfg, a->csa_kv8, "hybrid_attn_decode: csa_kv8")) != HCA_OK) return s;
+  if (a->hca_q && a->hca_kv8 && (s = check_kv8(cfg, a->hca_kv8, "hybrid_attn_decode: hca_kv8")) != HCA_OK) return s;
   if (a->csa_q) {
-    s = indexer_ok(a->csa_N, cfg->topk, HCA_MODE_DECODE);
+    s = indexer_ok(cfg, a->csa_N, HCA_MODE_DECODE);
     if (s != HCA_OK) return s;
     CHECK(a->csa_N > 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: csa_N=%d", a->csa_N);
     CHECK_PTR(a->csa_q_idx, "hybrid_attn_decode: csa_q_idx");
@@ -727,14 +869,16 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
       CHECK(a->csa_k_stride % 8 == 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: csa_k_stride");
     }
     CHECK_PTR(a->csa_topk_idx, "hybrid_attn_decode: csa_topk_idx");
-    s = check_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_N, a->csa_topk_idx, cfg->topk, cfg->m,
+    s = check_mqa(cfg, a->csa_q, a->csa_kv, a->csa_kv_stride, a->csa_kv8 ? 0 : a->csa_N, a->csa_topk_idx, cfg->topk,
+                  cfg->m,
                   a->csa_win, a->csa_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->csa_out, "hybrid_attn_decode: csa");
     if (s != HCA_OK) return s;
     if (a->csa_norm) CHECK_PTR(a->csa_norm, "hybrid_attn_decode: csa_norm");
   }
   if (a->hca_q) {
     CHECK(a->hca_N > 0, HCA_ERR_INVALID_ARG, "hybrid_attn_decode: hca_N=%d", a->hca_N);
-    s = check_mqa(cfg, a->hca_q, a->hca_kv, a->hca_kv_stride, a->hca_N, nullptr, 0, cfg->m_hca, a->hca_win,
+    s = check_mqa(cfg, a->hca_q, a->hca_kv, a->hca_kv_stride, a->hca_kv8 ? 0 : a->hca_N, nullptr, 0, cfg->m_hca,
+                  a->hca_win,
                   a->hca_win_stride, a->q_pos, a->B, HCA_MODE_DECODE, a->hca_out, "hybrid_attn_decode: hca");
     if (s != HCA_OK) return s;
     if (a->hca_norm) CHECK_PTR(a->hca_norm, "hybrid_attn_decode: hca_norm");
@@ -778,24 +922,59 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
   char* wsb = reinterpret_cast<char*>(ws);
   const int c = cfg->c, H = cfg->n_heads, nw = cfg->n_win;
   auto run_hca_compress = [&]() -> int {
-    bf16* row = reinterpret_cast<bf16*>(a->hca_kv) + (long long)(a->hca_N - 1) * c;
+    if (a->hca_kv8) {
+      // FP8 cache: the f32 entries (normalised to bf16 when asked), then their FP8 form in
+      // row hca_N-1 of every request
+      const hca_kv_fp8* d = a->hca_kv8;
+      float* ef = reinterpret_cast<float*>(wsb + (a->hca_norm ? sched.hca_ef : sched.hca8_new));
+      CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), c,
+                               reinterpret_cast<const bf16*>(a->hca_block_logits), c, a->hca_pos_bias, c, a->B,
+                               a->hca_block_stride, cfg->m_hca, c, cfg->m_hca, false, nullptr, c, c, hst, ef),
+               "decode: hca compress");
+      const void* src = ef;
+      if (a->hca_norm) {
+        CUDA_TRY(launch_norm_rope(norm_rows(cfg, ef, true, c, c, a->B, 1, nullptr, a->hca_N * cfg->m_hca - 1, 0,
+                                            a->hca_norm + c, wsb + sched.hca8_new, c, c),
+                                  hst),
+                 "decode: hca entry normalisation");
+        src = wsb + sched.hca8_new;
+      }
+      const long long r0 = a->hca_N - 1;
+      CUDA_TRY(launch_kv_fp8_quantize(src, a->hca_norm == nullptr, c, a->B, c, cfg->rope_dims,
+                                      d->codes + r0 * d->ld_codes, d->seq_rows * d->ld_codes,
+                                      d->scales + r0 * d->ld_scales, d->seq_rows * d->ld_scales,
+                                      reinterpret_cast<bf16*>(d->rope) + r0 * d->ld_rope, d->seq_rows * d->ld_rope,
+                                      hst),
+               "decode: hca entry to its FP8 form");
+      return HCA_OK;
+    }
+    // flat: straight into row hca_N-1 of every request's cache; paged: into [B, c] in the
+    // workspace, then each row to its pool row
+    const bool pgd = a->block_table != nullptr;
+    bf16* row = pgd ? reinterpret_cast<bf16*>(wsb + sched.hca_new)
+                    : reinterpret_cast<bf16*>(a->hca_kv) + (long long)(a->hca_N - 1) * c;
+    const long long row_stride = pgd ? (long long)c : a->hca_kv_stride;
     if (!a->hca_norm) {
       CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), c,
                                reinterpret_cast<const bf16*>(a->hca_block_logits), c, a->hca_pos_bias, c, a->B,
-                               a->hca_block_stride, cfg->m_hca, c, cfg->m_hca, false, row, c, a->hca_kv_stride, hst),
+                               a->hca_block_stride, cfg->m_hca, c, cfg->m_hca, false, row, c, row_stride, hst),
                "decode: hca compress");
-      return HCA_OK;
+    } else {
+      // f32 entries, then normalised and rotated at the entry's position into the cache row
+      float* ef = reinterpret_cast<float*>(wsb + sched.hca_ef);
+      CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), c,
+                               reinterpret_cast<const bf16*>(a->hca_block_logits), c, a->hca_pos_bias, c, a->B,
+                               a->hca_block_stride, cfg->m_hca, c, cfg->m_hca, false, nullptr, c, c, hst, ef),
+               "decode: hca compress");
+      CUDA_TRY(launch_norm_rope(norm_rows(cfg, ef, true, c, c, a->B, 1, nullptr, a->hca_N * cfg->m_hca - 1, 0,
+                                          a->hca_norm + c, row, c, row_stride),
+                                hst),
+               "decode: hca entry normalisation");
     }
-    // f32 entries, then normalised and rotated at the entry's position into the cache row
-    float* ef = reinterpret_cast<float*>(wsb + sched.hca_ef);
-    CUDA_TRY(launch_compress(reinterpret_cast<const bf16*>(a->hca_block_cand), c,
-                             reinterpret_cast<const bf16*>(a->hca_block_logits), c, a->hca_pos_bias, c, a->B,
-                             a->hca_block_stride, cfg->m_hca, c, cfg->m_hca, false, nullptr, c, c, hst, ef),
-             "decode: hca compress");
-    CUDA_TRY(launch_norm_rope(norm_rows(cfg, ef, true, c, c, a->B, 1, nullptr, a->hca_N * cfg->m_hca - 1, 0,
-                                        a->hca_norm + c, row, c, a->hca_kv_stride),
-                              hst),
-             "decode: hca entry normalisation");
+    if (pgd)
+      CUDA_TRY(launch_scatter_rows(row, a->B, c, a->block_table, a->bt_stride, a->hca_N - 1, pg.rpb_hca,
+                                   reinterpret_cast<bf16*>(a->hca_kv), hst),
+               "decode: hca entry to its pool row");
     return HCA_OK;
   };
   // normalised queries and window blocks of a layer (window row w = token max(0, t-n_win+1) + w)
@@ -805,14 +984,23 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
                                         c, (long long)H * c),
                               sm),
              "decode: query normalisation");
-    CUDA_TRY(launch_norm_rope(norm_rows(cfg, win, false, c, win_stride, a->B, nw, a->q_pos, -(nw - 1), 1, norm + c,
-                                        wsb + wn, c, (long long)nw * c),
-                              sm),
-             "decode: window normalisation");
+    NormRope wr = norm_rows(cfg, win, false, c, win_stride, a->B, nw, a->q_pos, -(nw - 1), 1, norm + c, wsb + wn, c,
+                            (long long)nw * c);
+    wr.ring = a->block_table ? 1 : 0;  // paged: the window block is a ring of the last n_win tokens
+    CUDA_TRY(launch_norm_rope(wr, sm), "decode: window normalisation");
     return HCA_OK;
   };
   auto run_hca_attention = [&]() -> int {
     MqaProblem p = decode_hca_problem(cfg, a);
+    if (a->hca_kv8) {
+      // the visible rows widened to bf16, read by the attention as its cache
+      bf16* rows = reinterpret_cast<bf16*>(wsb + sched.hca8_rows);
+      CUDA_TRY(launch_kv_fp8_gather(kv_fp8_of(a->hca_kv8), c, cfg->rope_dims, a->B, a->hca_N, nullptr, a->hca_N, rows,
+                                    nullptr, hst),
+               "decode: hca FP8 rows");
+      p.kv = rows;
+      p.kv_seq_stride = (long long)a->hca_N * c;
+    }
     if (a->hca_norm) {
       int r = normalise_layer(a->hca_q, a->hca_win, a->hca_win_stride, a->hca_norm, sched.hca_qn, sched.hca_wn, hst);
       if (r != HCA_OK) return r;
@@ -842,13 +1030,28 @@ int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void*
     Fp4Keys k4{a->csa_k_codes, a->csa_k_scales,
                a->B > 1 ? a->csa_k4_stride : ((long long)a->csa_N + 3) / 4 * 4,
                reinterpret_cast<bf16*>(wsb + sched.q4)};
+    const PagedKeys pk{a->block_table, a->bt_stride, pg.rpb_csa, (long long)a->n_pool_blocks};
     s = run_indexer_topk(reinterpret_cast<const bf16*>(a->csa_q_idx), a->csa_w_idx,
                          reinterpret_cast<const bf16*>(a->csa_k_idx), a->csa_k_stride, a->csa_N, a->q_pos, a->B,
                          HCA_MODE_DECODE, cfg, a->csa_topk_idx, ws, st, ev, n_ev, ev_i,
-                         sched.overlap ? sched.sms - sched.r_hca : 0, a->csa_k_codes ? &k4 : nullptr);
+                         sched.overlap ? sched.sms - sched.r_hca : 0, a->csa_k_codes ? &k4 : nullptr,
+                         a->block_table ? &pk : nullptr);
     if (s != HCA_OK) return s;
     MqaProblem p = decode_csa_problem(cfg, a);
     if (a->csa_norm) use_normalised(p, cfg, wsb + sched.csa_qn, wsb + sched.csa_wn, true);
+    if (a->csa_kv8) {
+      // the selected rows widened to bf16 in slot order; the attention reads them as a
+      // cache of k rows through the slot indices (empty slots stay -1)
+      bf16* rows = reinterpret_cast<bf16*>(wsb + sched.csa8_rows);
+      int32_t* slots = reinterpret_cast<int32_t*>(wsb + sched.csa8_idx);
+      CUDA_TRY(launch_kv_fp8_gather(kv_fp8_of(a->csa_kv8), c, cfg->rope_dims, a->B, cfg->topk, a->csa_topk_idx,
+                                    a->csa_N, rows, slots, st),
+               "decode: csa FP8 rows");
+      p.kv = rows;
+      p.kv_seq_stride = (long long)cfg->topk * c;
+      p.N = cfg->topk;
+      p.idx = slots;
+    }
     CUDA_TRY(launch_mqa(p, sched.csa_pl, ws, st, true), "decode: csa attention");
     if ((s = mark()) != HCA_OK) return s;
   }
@@ -874,7 +1077,7 @@ struct PrefillWs {
 static PrefillWs prefill_ws_layout(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
   const int T = a->T;
   const int Nc = T / cfg->m;
-  size_t need = plan_indexer(T, Nc, cfg->topk).bytes;
+  size_t need = plan_indexer(cfg, T, Nc, HCA_MODE_PREFILL).bytes;
   MqaProblem p = make_mqa(cfg, nullptr, nullptr, 0, Nc, reinterpret_cast<const int32_t*>(1), cfg->topk, cfg->m,
                           nullptr, T, nullptr, T, HCA_MODE_PREFILL, nullptr, nullptr);
   need = std::max(need, plan_mqa(p).ws_bytes);
@@ -900,7 +1103,7 @@ static size_t prefill_ws(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
 
 size_t hybrid_attn_prefill_workspace(const hca_layer_cfg* cfg, const hca_prefill_args* a) {
   if (check_cfg(cfg) != HCA_OK || !a || a->T < 0) return (size_t)-1;
-  if (indexer_ok(a->T / cfg->m, cfg->topk, HCA_MODE_PREFILL) != HCA_OK) return (size_t)-1;
+  if (indexer_ok(cfg, a->T / cfg->m, HCA_MODE_PREFILL) != HCA_OK) return (size_t)-1;
   return prefill_ws(cfg, a);
 }
 
@@ -914,7 +1117,7 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
   const int T = a->T;
   if (T == 0) return HCA_OK;
   const int Nc = T / cfg->m;
-  s = indexer_ok(Nc, cfg->topk, HCA_MODE_PREFILL);
+  s = indexer_ok(cfg, Nc, HCA_MODE_PREFILL);
   if (s != HCA_OK) return s;
   CHECK_PTR(a->q_pos, "hybrid_attn_prefill: q_pos");
   CHECK_PTR(a->cand, "hybrid_attn_prefill: cand");
@@ -939,8 +1142,8 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
   if (a->csa_norm) CHECK_PTR(a->csa_norm, "hybrid_attn_prefill: csa_norm");
   const size_t need = prefill_ws(cfg, a);
   CHECK(ws_bytes >= need, HCA_ERR_WORKSPACE, "hybrid_attn_prefill: workspace %zu < %zu", ws_bytes, need);
-  CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
-        "hybrid_attn_prefill: ws null or not 256-byte aligned");
+  if (need) CHECK(ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0, HCA_ERR_INVALID_ARG,
+                  "hybrid_attn_prefill: ws null or not 256-byte aligned");
   if (injected("hybrid_attn_prefill")) return fail(HCA_ERR_INJECTED, "hybrid_attn_prefill: injected");
 
   cudaStream_t st = as_stream(stream);
@@ -1047,13 +1250,13 @@ int mxfp4_quantize(const void* x, int x_is_f32, long long ld_x, int rows, int d,
 }
 
 static size_t fp4_indexer_ws(const hca_layer_cfg* cfg, int B, int N) {
-  const IndexerPlan p = plan_indexer(B, N, cfg->topk);
+  const IndexerPlan p = plan_indexer(cfg, B, N, HCA_MODE_DECODE);
   return round256(p.bytes) + round256((size_t)B * cfg->n_idx_heads * cfg->d_idx * 2);
 }
 
 size_t csa_indexer_topk_fp4_workspace(const hca_layer_cfg* cfg, int B, int N) {
   if (check_cfg(cfg) != HCA_OK || B < 0 || N < 0) return (size_t)-1;
-  if (indexer_ok(N, cfg->topk, HCA_MODE_DECODE) != HCA_OK) return (size_t)-1;
+  if (indexer_ok(cfg, N, HCA_MODE_DECODE) != HCA_OK) return (size_t)-1;
   return fp4_indexer_ws(cfg, B, N);
 }
 
@@ -1066,7 +1269,7 @@ int csa_indexer_topk_fp4(const hca_bf16* q_idx, const float* w_idx, const uint8_
   CHECK(indexer_tc_supported(cfg->n_idx_heads, cfg->d_idx), HCA_ERR_UNSUPPORTED,
         "csa_indexer_topk_fp4: the FP4 indexer takes 64 heads x 128 (got %d x %d)", cfg->n_idx_heads, cfg->d_idx);
   CHECK(B >= 0 && B <= 65535 && N > 0, HCA_ERR_INVALID_ARG, "csa_indexer_topk_fp4: B=%d N=%d", B, N);
-  s = indexer_ok(N, cfg->topk, HCA_MODE_DECODE);
+  s = indexer_ok(cfg, N, HCA_MODE_DECODE);
   if (s != HCA_OK) return s;
   const long long n4 = ((long long)N + 3) / 4 * 4;
   CHECK(B <= 1 || (k_seq_stride >= n4 && k_seq_stride % 4 == 0), HCA_ERR_INVALID_ARG,
@@ -1084,7 +1287,7 @@ int csa_indexer_topk_fp4(const hca_bf16* q_idx, const float* w_idx, const uint8_
         "csa_indexer_topk_fp4: ws null or not 256-byte aligned");
   if (injected("csa_indexer_topk_fp4")) return fail(HCA_ERR_INJECTED, "csa_indexer_topk_fp4: injected");
 
-  const IndexerPlan p = plan_indexer(B, N, cfg->topk);
+  const IndexerPlan p = plan_indexer(cfg, B, N, HCA_MODE_DECODE);
   Fp4Keys k4{k_codes, k_scales, B > 1 ? k_seq_stride : (long long)(N + 3) / 4 * 4,
              reinterpret_cast<bf16*>(reinterpret_cast<char*>(ws) + round256(p.bytes))};
   int ev_i = 0;

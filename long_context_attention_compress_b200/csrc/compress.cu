@@ -149,4 +149,23 @@ cudaError_t launch_compress(const bf16* cand, int ld_cand, const bf16* logits, i
   return cudaGetLastError();
 }
 
+// Row b of src [B][c] (bf16) into its paged pool row:
+// pool + (bt[b*bt_stride + entry / rpb] * rpb + entry % rpb) * c.
+__global__ void __launch_bounds__(64) scatter_rows_kernel(const bf16* __restrict__ src, int c,
+                                                          const int32_t* __restrict__ bt, long long bt_stride,
+                                                          int entry, int rpb, bf16* __restrict__ pool) {
+  const long long b = blockIdx.x;
+  const long long row = (long long)bt[b * bt_stride + entry / rpb] * rpb + entry % rpb;
+  for (int j = threadIdx.x * 8; j < c; j += blockDim.x * 8)
+    *reinterpret_cast<uint4*>(pool + row * c + j) = *reinterpret_cast<const uint4*>(src + b * c + j);
+}
+
+cudaError_t launch_scatter_rows(const bf16* src, int B, int c, const int32_t* bt, long long bt_stride, int entry,
+                                int rpb, bf16* pool, cudaStream_t stream) {
+  if (B == 0) return cudaSuccess;
+  scatter_rows_kernel<<<B, 64, 0, stream>>>(src, c, bt, bt_stride, entry, rpb, pool);
+  ++g_launch_counter;
+  return cudaGetLastError();
+}
+
 }  // namespace hca

@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
     int B, int N, int rate, int tiles_per_req, float* __restrict__ scores, long long ld_scores,
     int* __restrict__ hist_g) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* base = tc::smem_align1024(smem_raw);
   unsigned char* k_smem = base;                                   // [kFBuf][2][128][128 B] bf16, swizzled
   unsigned char* q_smem = k_smem + kFBuf * kFTileBytes;           // [2][2][64][128 B]
   unsigned char* st_smem = q_smem + 2 * kFQBytes;                 // [kFStages][codes 8 KiB | scales 512 B]

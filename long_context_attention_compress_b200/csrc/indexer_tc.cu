@@ -61,11 +61,13 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
     const float* __restrict__ w_idx, const int32_t* __restrict__ q_pos, int B, int N, int rate,
     int tiles_per_req, float* __restrict__ scores, long long ld_scores, int* __restrict__ hist_g,
-    uint32_t spin, int stall) {
+    uint32_t spin, int stall, const int32_t* __restrict__ bt, long long bt_stride, int rpb) {
+  // bt != nullptr: paged keys -- request r's logical block j (rpb keys) is physical block
+  // bt[r*bt_stride + j] of a pool that tm_k maps as [blocks * rpb rows, 128 dims].
   // spin: poll budget of every wait (tc::kSpinLimit in normal use).  stall != 0 (tests of
   // the bounded waits only): the producer issues nothing, so every consumer wait runs out.
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* base = tc::smem_align1024(smem_raw);
   unsigned char* k_smem = base;                              // [stages][2][128][128 B]
   unsigned char* q_smem = base + kStages * kTileBytes;        // [2][2][64][128 B]
   Bars* bars = reinterpret_cast<Bars*>(q_smem + 2 * kQBytes);
@@ -113,10 +115,35 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
           ++rq;
         }
         const int s = it % kStages;
+        // paged: the tile's blocks that hold visible keys (their ids are loaded before the
+        // wait for a free stage, so the loads' latency hides behind it)
+        int pb[kTile / 8];
+        int nb = 0;
+        if (bt) {
+          const int nvis = n_visible(q_pos[r], rate, N);
+          nb = min(kTile / rpb, (nvis - row0 + rpb - 1) / rpb);
+          const int32_t* btr = bt + (long long)r * bt_stride + row0 / rpb;
+#pragma unroll
+          for (int i = 0; i < kTile / 8; ++i) pb[i] = i < nb ? __ldg(btr + i) : 0;
+        }
         if (!tc::mbar_wait(&bars->empty[s], ((it / kStages) & 1) ^ 1, abort, spin)) break;
-        tc::mbar_arrive_expect_tx(&bars->full[s], kTileBytes);
-        tc::tma_load_3d(k_smem + s * kTileBytes, &tm_k, &bars->full[s], 0, row0, r);
-        tc::tma_load_3d(k_smem + s * kTileBytes + kChunkBytes, &tm_k, &bars->full[s], 64, row0, r);
+        if (bt) {
+          // one box of rpb rows per block and 64-dim chunk (rows past the visible blocks
+          // keep stale data: their scores are never used)
+          tc::mbar_arrive_expect_tx(&bars->full[s], (uint32_t)(nb * rpb * kDim * 2));
+#pragma unroll
+          for (int i = 0; i < kTile / 8; ++i) {
+            if (i < nb) {
+              const int prow = pb[i] * rpb;
+              tc::tma_load_2d(k_smem + s * kTileBytes + i * rpb * 128, &tm_k, &bars->full[s], 0, prow);
+              tc::tma_load_2d(k_smem + s * kTileBytes + kChunkBytes + i * rpb * 128, &tm_k, &bars->full[s], 64, prow);
+            }
+          }
+        } else {
+          tc::mbar_arrive_expect_tx(&bars->full[s], kTileBytes);
+          tc::tma_load_3d(k_smem + s * kTileBytes, &tm_k, &bars->full[s], 0, row0, r);
+          tc::tma_load_3d(k_smem + s * kTileBytes + kChunkBytes, &tm_k, &bars->full[s], 64, row0, r);
+        }
         ++it;
       }
       // make sure no copy of ours is still landing in shared memory
@@ -237,23 +264,51 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
   if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// ---- prefill: groups of 4 queries (N = 4 x 64 heads = 256) ---------------------
+// ---- prefill: groups of 4 queries (N = 4 x 64 heads = 256), top-k on chip -----------
 // One sequence: query t sees entries s < n_visible(q_pos[t]).  A CTA owns
 // groups of four consecutive queries (their q_I rows form the 256-row B
-// operand, 64 KiB) and streams the key tiles visible to the group's last
-// query through a 4-stage ring; two 256-column TMEM accumulators let the
-// epilogue of one tile overlap the MMAs of the next.  Groups are dealt to the
-// persistent grid largest first, interleaved, which balances the causal
-// triangle.  Epilogue: per query, ReLU of 64 head dot products weighted by the
-// f32 head weights (staged in shared memory per group).
+// operand, 64 KiB) and streams the key tiles visible to the group's queries
+// through a 3-stage ring; two 256-column TMEM accumulators let the epilogue of
+// one tile overlap the MMAs of the next.  Groups are dealt to the persistent
+// grid largest first, interleaved, which balances the causal triangle.
+// Epilogue: per query, ReLU of 64 head dot products weighted by the f32 head
+// weights (staged in shared memory per group).
+//
+// Top-k fused into the epilogue (the per-query selection of the QbitAI
+// write-up, CSA step two; "DeepSeek V4 Architecture Tricks", CSA section,
+// top-k 1024): the scores never leave the SM.  Each query of the group keeps,
+// in shared memory, a list of candidates -- 64-bit composites (order-
+// preserving score key, inverted entry index; distinct, and larger = preferred,
+// so ties go to the lower index) in entry order -- and a threshold, the
+// smallest composite of its last cut.  Per tile, the two warps of each TMEM
+// lane quarter append the entries that beat the threshold, at offsets agreed
+// per lane quarter so that the list stays in entry order.  When the next tile
+// could overflow the list, an exact MSB-first radix select cuts it back to its
+// k largest, in order, and raises the threshold to the smallest one kept (no
+// later entry below it can be among the k largest).  After the group's last
+// tile a final cut leaves exactly the k largest, written out in entry order.
+// A query that sees at most k entries takes all of them without scoring.
+// Without the fused top-k (k above kPCand - kTile) the epilogue writes the f32
+// scores instead, for a separate select.
 namespace {
-constexpr int kPStages = 4;
+constexpr int kPStages = 3;
 constexpr int kPQ = 4;                       // queries per group
 constexpr int kPN = kPQ * kHeads;            // 256 = MMA N
 constexpr uint32_t kPQBytes = kPN * kDim * 2;        // 64 KiB
 constexpr uint32_t kPQChunkBytes = kPN * 128;        // 32 KiB
 constexpr int kPAcc = 2;
 constexpr int kPThreads = 320;  // producer, MMA, 8 epilogue warps (two per TMEM lane quarter)
+constexpr int kPCand = 1536;    // candidate slots per query
+constexpr int kPPer = kPCand / 128;  // candidates per thread of a half in a cut
+
+// Scratch of one half of the epilogue (the 128 threads serving two queries).
+struct __align__(16) PHalf {
+  unsigned long long wmin[4], wmax[4];
+  int hist[256];
+  int wsum[4];
+  int wcnt[2][4][2];  // [tile parity][TMEM lane quarter][query of the half]: appends per warp
+  int bucket, greater;
+};
 struct __align__(16) PBars {
   float w[kPN];  // first: read with 16-byte vector loads
   int nvis[kPQ];
@@ -262,32 +317,177 @@ struct __align__(16) PBars {
   uint64_t qfull, qempty, drain;
   uint32_t tmem_base;
   int abort;
+  PHalf half[2];
 };
 static_assert(offsetof(PBars, w) % 16 == 0 && offsetof(PBars, full) % 8 == 0, "PBars alignment");
-static_assert((kPStages * kTileBytes + kPQBytes) % 16 == 0, "PBars starts 16-byte aligned");
-constexpr size_t kPSmemBytes = 1024 + kPStages * kTileBytes + kPQBytes + sizeof(PBars);
+static_assert((kPStages * kTileBytes + kPQBytes) % 1024 == 0, "candidate lists start 1024-byte aligned");
+constexpr size_t kPCandBytes = (size_t)kPQ * kPCand * sizeof(uint64_t);  // 48 KiB
+constexpr size_t kPSmemBytes = 1024 + kPStages * kTileBytes + kPQBytes + kPCandBytes + sizeof(PBars);
+static_assert(kPSmemBytes <= 232448, "shared memory budget");
+
+// Exclusive prefix of v over the 128 threads of a half (hl = 0..127, in order);
+// *total receives the sum.  Every thread of the half calls it.
+__device__ __forceinline__ int half_scan(int v, int hl, PHalf* hs, uint32_t bar, int* total) {
+  const int lane = hl & 31, w = hl >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) hs->wsum[w] = x;
+  tc::named_bar(bar, 128);
+  int before = 0, tot = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int s = hs->wsum[i];
+    before += i < w ? s : 0;
+    tot += s;
+  }
+  tc::named_bar(bar, 128);  // wsum is free again
+  *total = tot;
+  return before + x - v;
+}
+
+// Cut the candidate list buf[0..n) (distinct composites, k < n <= kPCand) to its k
+// largest, keeping their order; returns the smallest composite kept.  All 128
+// threads of the half call it with the same n and k.  Thread hl holds the
+// contiguous run [hl*per, hl*per + per) in registers, so the ordered rewrite is
+// a scan of the per-thread counts; every write stays inside [0, n).
+__device__ __forceinline__ uint64_t cut_to_topk(uint64_t* buf, int n, int k, PHalf* hs, uint32_t bar, int hl) {
+  const int lane = hl & 31, w = hl >> 5;
+  tc::named_bar(bar, 128);  // every warp's appends are in place
+  const int per = (n + 127) / 128;
+  const int i0 = hl * per;
+  uint64_t v[kPPer];
+  unsigned long long mn = ~0ull, mx = 0ull;
+#pragma unroll
+  for (int u = 0; u < kPPer; ++u) {
+    const int i = i0 + u;
+    const bool ok = u < per && i < n;
+    v[u] = ok ? buf[i] : 0ull;
+    if (ok) {
+      mn = v[u] < mn ? v[u] : mn;
+      mx = v[u] > mx ? v[u] : mx;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const unsigned long long a = __shfl_xor_sync(0xffffffffu, mn, o);
+    const unsigned long long b = __shfl_xor_sync(0xffffffffu, mx, o);
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
+  }
+  if (lane == 0) {
+    hs->wmin[w] = mn;
+    hs->wmax[w] = mx;
+  }
+  tc::named_bar(bar, 128);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    mn = hs->wmin[i] < mn ? hs->wmin[i] : mn;
+    mx = hs->wmax[i] > mx ? hs->wmax[i] : mx;
+  }
+  // MSB-first radix select of the k-th largest, 8-bit digits, from the highest bit
+  // where the candidates differ (distinct and n > k >= 1, so mn < mx)
+  int hi = mn == mx ? -1 : 63 - __clzll((long long)(mn ^ mx));
+  uint64_t prefix = hi >= 63 ? 0ull : (mn >> (hi + 1)) << (hi + 1);
+  int lo = hi + 1;
+  int remaining = k;
+  while (hi >= 0) {
+    lo = hi >= 7 ? hi - 7 : 0;
+    const uint32_t dmask = (1u << (hi - lo + 1)) - 1u;
+    hs->hist[hl] = 0;
+    hs->hist[hl + 128] = 0;
+    tc::named_bar(bar, 128);
+#pragma unroll
+    for (int u = 0; u < kPPer; ++u) {
+      const int i = i0 + u;
+      if (u < per && i < n && (hi >= 63 || (v[u] >> (hi + 1)) == (prefix >> (hi + 1))))
+        atomicAdd(&hs->hist[(int)((v[u] >> lo) & dmask)], 1);
+    }
+    tc::named_bar(bar, 128);
+    // thread hl owns bins 255 - 2hl and 254 - 2hl: a prefix over the threads is a
+    // suffix over the bins
+    const int b0 = 255 - 2 * hl, b1 = b0 - 1;
+    const int h0 = hs->hist[b0], h1 = hs->hist[b1];
+    int tot;
+    const int ex = half_scan(h0 + h1, hl, hs, bar, &tot);  // candidates in bins above b0
+    if (ex < remaining && ex + h0 >= remaining) {
+      hs->bucket = b0;
+      hs->greater = ex;
+    } else if (ex + h0 < remaining && ex + h0 + h1 >= remaining) {
+      hs->bucket = b1;
+      hs->greater = ex + h0;
+    }
+    tc::named_bar(bar, 128);
+    const int b = hs->bucket;
+    remaining -= hs->greater;
+    prefix |= (uint64_t)b << lo;
+    const int cnt = hs->hist[b];
+    tc::named_bar(bar, 128);  // bucket and histogram read by all before they are rewritten
+    hi = lo - 1;
+    if (cnt == remaining) break;
+  }
+  // kept: the composites whose decided bits are at least the prefix's (exactly k of them)
+  const int shift = lo;
+  const uint64_t P = prefix >> shift;
+  int nk = 0;
+  unsigned long long kmin = ~0ull;
+#pragma unroll
+  for (int u = 0; u < kPPer; ++u) {
+    const int i = i0 + u;
+    if (u < per && i < n && (v[u] >> shift) >= P) {
+      ++nk;
+      kmin = v[u] < kmin ? v[u] : kmin;
+    }
+  }
+  int tot;
+  int off = half_scan(nk, hl, hs, bar, &tot);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
+    kmin = a < kmin ? a : kmin;
+  }
+  if (lane == 0) hs->wmin[w] = kmin;
+#pragma unroll
+  for (int u = 0; u < kPPer; ++u) {
+    const int i = i0 + u;
+    if (u < per && i < n && (v[u] >> shift) >= P) buf[off++] = v[u];
+  }
+  tc::named_bar(bar, 128);  // the cut list and the warp minima are in place
+#pragma unroll
+  for (int i = 0; i < 4; ++i) kmin = hs->wmin[i] < kmin ? hs->wmin[i] : kmin;
+  return kmin;
+}
 }  // namespace
+
+bool indexer_prefill_topk_fused(int k) { return k >= 1 && k <= kPCand - kTile; }
 
 __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
     const float* __restrict__ w_idx, const int32_t* __restrict__ q_pos, int Tq, int N, int rate,
-    float* __restrict__ scores, long long ld_scores) {
+    float* __restrict__ scores, long long ld_scores, int k, int32_t* __restrict__ topk_idx) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* base = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* base = tc::smem_align1024(smem_raw);
   unsigned char* k_smem = base;                           // [stages][2][128][128 B]
   unsigned char* q_smem = base + kPStages * kTileBytes;   // [2][256][128 B]
-  PBars* bars = reinterpret_cast<PBars*>(q_smem + kPQBytes);
+  uint64_t* cand_smem = reinterpret_cast<uint64_t*>(q_smem + kPQBytes);  // [4][kPCand]
+  PBars* bars = reinterpret_cast<PBars*>(q_smem + kPQBytes + kPCandBytes);
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_groups = (Tq + kPQ - 1) / kPQ;
+  const bool fused = topk_idx != nullptr;
   // tiles of group g: entries visible to its queries (q_pos is non-decreasing within a group
-  // in the layer call; the maximum over the group is used in general)
+  // in the layer call; the maximum over the group is used in general).  With the fused
+  // top-k a group whose queries all see at most k entries needs no scores at all.
   auto group_tiles = [&](int g) -> int {
     int nv = 0;
     for (int j = 0; j < kPQ; ++j) {
       const int q = g * kPQ + j;
       if (q < Tq) nv = max(nv, n_visible(q_pos[q], rate, N));
     }
+    if (fused && nv <= k) return 0;
     return (nv + kTile - 1) / kTile;
   };
 
@@ -351,10 +551,10 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
           tc::fence_after_sync();
           const uint64_t ad0 = tc::sdesc_sw128(k_base + s * kTileBytes, 16, 1024);
 #pragma unroll
-          for (int k = 0; k < kDim / 16; ++k) {
-            const uint32_t aoff = ((k >> 2) * kChunkBytes + (k & 3) * 32) >> 4;
-            const uint32_t boff = ((k >> 2) * kPQChunkBytes + (k & 3) * 32) >> 4;
-            tc::mma_bf16(tmem + a * kPN, ad0 + aoff, qd0 + boff, idesc, k > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kDim / 16; ++kk) {
+            const uint32_t aoff = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
+            const uint32_t boff = ((kk >> 2) * kPQChunkBytes + (kk & 3) * 32) >> 4;
+            tc::mma_bf16(tmem + a * kPN, ad0 + aoff, qd0 + boff, idesc, kk > 0 ? 1u : 0u);
           }
           tc::mma_commit(&bars->empty[s]);
           tc::mma_commit(&bars->tfull[a]);
@@ -367,16 +567,23 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
     __syncwarp();
   } else {
     // epilogue: warps 2..9, one TMEM lane (= entry) per thread; the two warps of a
-    // lane quarter score two of the group's four queries each
+    // lane quarter score two of the group's four queries each.  Warps 2-5 (half 0)
+    // serve queries 0 and 1, warps 6-9 (half 1) queries 2 and 3.
     const int lq = warp & 3;
     const int row_in_tile = lq * 32 + lane;
     const int et = threadIdx.x - 64;  // 0..255
-    const int j0 = 2 * ((warp - 2) >> 2);
-    int it = 0;
+    const int half = (warp - 2) >> 2;
+    const int j0 = 2 * half;
+    const int hl = et - 128 * half;  // 0..127 within the half
+    const uint32_t hbar = 2 + half;
+    PHalf* hs = &bars->half[half];
+    uint64_t* cbuf[2] = {cand_smem + (size_t)j0 * kPCand, cand_smem + (size_t)(j0 + 1) * kPCand};
+    const unsigned lt = (1u << lane) - 1u;
+    int it = 0, par = 0;
     bool failed = false;
     for (int g = n_groups - 1 - (int)blockIdx.x; g >= 0; g -= (int)gridDim.x) {
       const int nt = group_tiles(g);
-      if (nt == 0) continue;
+      if (nt == 0 && !fused) continue;
       // stage this group's weights and visible counts (the previous group's readers are done)
       tc::named_bar(1, 256);
       for (int e = et; e < kPN; e += 256) {
@@ -388,41 +595,105 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
         bars->nvis[et] = q < Tq ? n_visible(q_pos[q], rate, N) : 0;
       }
       tc::named_bar(1, 256);
+      // fused top-k state of this half's two queries (uniform over the half)
+      bool sel[2];
+      int cnt[2] = {0, 0};
+      uint64_t thr[2] = {0ull, 0ull};  // every real composite is > 0
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) sel[jj] = fused && g * kPQ + j0 + jj < Tq && bars->nvis[j0 + jj] > k;
       for (int t = 0; t < nt; ++t, ++it) {
         const int a = it % kPAcc;
         if (!failed) failed = !tc::warp_wait(&bars->tfull[a], (it / kPAcc) & 1, abort);
-        if (failed) continue;
-        tc::fence_after_sync();
         const int e = t * kTile + row_in_tile;
-        float sc[2];
+        float sc[2] = {0.f, 0.f};
+        if (!failed) {
+          tc::fence_after_sync();
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int j = j0 + jj;
-          uint32_t v[kHeads];
-          const uint32_t taddr = tmem + ((uint32_t)(lq * 32) << 16) + a * kPN + j * kHeads;
-          tc::tmem_ld32(taddr, v);
-          tc::tmem_ld32(taddr + 32, v + 32);
-          tc::tmem_ld_wait();
-          const float* w = bars->w + j * kHeads;
-          float s0 = 0.f, s1 = 0.f;
+          for (int jj = 0; jj < 2; ++jj) {
+            const int j = j0 + jj;
+            uint32_t v[kHeads];
+            const uint32_t taddr = tmem + ((uint32_t)(lq * 32) << 16) + a * kPN + j * kHeads;
+            tc::tmem_ld32(taddr, v);
+            tc::tmem_ld32(taddr + 32, v + 32);
+            tc::tmem_ld_wait();
+            const float* w = bars->w + j * kHeads;
+            float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-          for (int h = 0; h < kHeads; h += 4) {
-            const float4 wv = *reinterpret_cast<const float4*>(w + h);
-            s0 = fmaf(wv.x, fmaxf(__uint_as_float(v[h]), 0.f), s0);
-            s1 = fmaf(wv.y, fmaxf(__uint_as_float(v[h + 1]), 0.f), s1);
-            s0 = fmaf(wv.z, fmaxf(__uint_as_float(v[h + 2]), 0.f), s0);
-            s1 = fmaf(wv.w, fmaxf(__uint_as_float(v[h + 3]), 0.f), s1);
+            for (int h = 0; h < kHeads; h += 4) {
+              const float4 wv = *reinterpret_cast<const float4*>(w + h);
+              s0 = fmaf(wv.x, fmaxf(__uint_as_float(v[h]), 0.f), s0);
+              s1 = fmaf(wv.y, fmaxf(__uint_as_float(v[h + 1]), 0.f), s1);
+              s0 = fmaf(wv.z, fmaxf(__uint_as_float(v[h + 2]), 0.f), s0);
+              s1 = fmaf(wv.w, fmaxf(__uint_as_float(v[h + 3]), 0.f), s1);
+            }
+            sc[jj] = s0 + s1;
           }
-          sc[jj] = s0 + s1;
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&bars->tempty[a]);
         }
-        tc::fence_before_sync();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars->tempty[a]);
+        if (!fused) {
+          if (failed) continue;
+#pragma unroll
+          for (int jj = 0; jj < 2; ++jj) {
+            const int q = g * kPQ + j0 + jj;
+            if (q < Tq && e < bars->nvis[j0 + jj]) scores[(long long)q * ld_scores + e] = sc[jj];
+          }
+          continue;
+        }
+        // fused: candidates that beat the threshold, appended in entry order
+        uint64_t c[2];
+        unsigned bal[2];
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
-          const int q = g * kPQ + j0 + jj;
-          if (q < Tq && e < bars->nvis[j0 + jj]) scores[(long long)q * ld_scores + e] = sc[jj];
+          c[jj] = make_cand(sc[jj], e);
+          const bool take = !failed && sel[jj] && e < bars->nvis[j0 + jj] && c[jj] > thr[jj];
+          bal[jj] = __ballot_sync(0xffffffffu, take);
+          if (lane == 0) hs->wcnt[par][lq][jj] = __popc(bal[jj]);
         }
+        // one barrier per tile: the warps' counts are in, and every thread agrees on failure
+        if (tc::named_bar_or(hbar, 128, failed || *abort)) { failed = true; break; }
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          int off = cnt[jj], tot = 0;
+#pragma unroll
+          for (int l = 0; l < 4; ++l) {
+            const int n_l = hs->wcnt[par][l][jj];
+            off += l < lq ? n_l : 0;
+            tot += n_l;
+          }
+          if ((bal[jj] >> lane) & 1u) cbuf[jj][off + __popc(bal[jj] & lt)] = c[jj];
+          cnt[jj] += tot;
+        }
+        par ^= 1;
+        // room for one more tile of appends in each list, else cut it to its k largest
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          if (cnt[jj] > kPCand - kTile) {
+            thr[jj] = cut_to_topk(cbuf[jj], cnt[jj], k, hs, hbar, hl);
+            cnt[jj] = k;
+          }
+        }
+      }
+      if (!fused) continue;
+      if (failed) continue;  // (uniform over the half: agreed at the per-tile barrier)
+      tc::named_bar(hbar, 128);  // the last tile's appends are in place
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int q = g * kPQ + j0 + jj;
+        if (q >= Tq) continue;
+        int32_t* out = topk_idx + (long long)q * k;
+        if (!sel[jj]) {
+          // at most k visible entries: all of them, then empty slots
+          const int nv = bars->nvis[j0 + jj];
+          for (int i = hl; i < k; i += 128) out[i] = i < nv ? i : -1;
+          continue;
+        }
+        if (cnt[jj] > k) {
+          thr[jj] = cut_to_topk(cbuf[jj], cnt[jj], k, hs, hbar, hl);
+          cnt[jj] = k;
+        }
+        for (int i = hl; i < k; i += 128) out[i] = cand_index(cbuf[jj][i]);
       }
     }
   }
@@ -469,13 +740,22 @@ bool indexer_tc_supported(int H_I, int d_I) { return H_I == kHeads && d_I == kDi
 
 cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride,
                                      int N, const int32_t* q_pos, int B, int rate, float* scores, long long ld_scores,
-                                     int num_sms, cudaStream_t stream, int* hist, bool stall) {
+                                     int num_sms, cudaStream_t stream, int* hist, bool stall, const PagedKeys* paged) {
   constexpr uint32_t kStallSpin = 4096;  // a stalled test launch gives up after ~4k polls
   if (B == 0 || N == 0) return cudaSuccess;
   CUtensorMap tm_k, tm_q;
-  const uint64_t kd[3] = {(uint64_t)kDim, (uint64_t)N, (uint64_t)B};
-  const uint64_t ks[2] = {(uint64_t)kDim * 2, (uint64_t)(B > 1 ? k_seq_stride : (long long)N * kDim) * 2};
-  cudaError_t e = make_tmap_bf16(&tm_k, k_idx, 3, kd, ks, kTile);
+  cudaError_t e;
+  if (paged) {
+    if (paged->rpb < 8 || paged->rpb > kTile || kTile % paged->rpb != 0 || paged->rpb % 8 != 0)
+      return cudaErrorInvalidValue;
+    const uint64_t kd[2] = {(uint64_t)kDim, (uint64_t)paged->n_blocks * paged->rpb};
+    const uint64_t ks[1] = {(uint64_t)kDim * 2};
+    e = make_tmap_bf16(&tm_k, k_idx, 2, kd, ks, (uint32_t)paged->rpb);
+  } else {
+    const uint64_t kd[3] = {(uint64_t)kDim, (uint64_t)N, (uint64_t)B};
+    const uint64_t ks[2] = {(uint64_t)kDim * 2, (uint64_t)(B > 1 ? k_seq_stride : (long long)N * kDim) * 2};
+    e = make_tmap_bf16(&tm_k, k_idx, 3, kd, ks, kTile);
+  }
   if (e != cudaSuccess) return e;
   const uint64_t qd[2] = {(uint64_t)kDim, (uint64_t)B * kHeads};
   const uint64_t qs[1] = {(uint64_t)kDim * 2};
@@ -490,15 +770,24 @@ cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, cons
   indexer_decode_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_k, tm_q, w_idx, q_pos, B, N, rate,
                                                                    tiles_per_req, scores, ld_scores, hist,
                                                                    stall ? kStallSpin : tc::kSpinLimit,
-                                                                   stall ? 1 : 0);
+                                                                   stall ? 1 : 0, paged ? paged->bt : nullptr,
+                                                                   paged ? paged->bt_stride : 0,
+                                                                   paged ? paged->rpb : 0);
   ++g_launch_counter;
   return cudaGetLastError();
 }
 
 cudaError_t launch_indexer_prefill_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, int N,
                                       const int32_t* q_pos, int Tq, int rate, float* scores, long long ld_scores,
-                                      int num_sms, cudaStream_t stream) {
-  if (Tq == 0 || N == 0) return cudaSuccess;
+                                      int num_sms, cudaStream_t stream, int k, int32_t* topk_idx) {
+  if (Tq == 0) return cudaSuccess;
+  if (N == 0) {
+    // nothing is visible to any query: every slot of the fused top-k is empty (-1)
+    if (!topk_idx) return cudaSuccess;
+    ++g_launch_counter;
+    return cudaMemsetAsync(topk_idx, 0xff, (size_t)Tq * k * sizeof(int32_t), stream);
+  }
+  if (topk_idx && !indexer_prefill_topk_fused(k)) return cudaErrorInvalidValue;
   CUtensorMap tm_k, tm_q;
   const uint64_t kd[3] = {(uint64_t)kDim, (uint64_t)N, 1};
   const uint64_t ks[2] = {(uint64_t)kDim * 2, (uint64_t)N * kDim * 2};
@@ -514,7 +803,7 @@ cudaError_t launch_indexer_prefill_tc(const bf16* q_idx, const float* w_idx, con
                            (int)kPSmemBytes);
   if (e != cudaSuccess) return e;
   indexer_prefill_tc_kernel<<<grid, kPThreads, kPSmemBytes, stream>>>(tm_k, tm_q, w_idx, q_pos, Tq, N, rate, scores,
-                                                                      ld_scores);
+                                                                      ld_scores, k, topk_idx);
   ++g_launch_counter;
   return cudaGetLastError();
 }

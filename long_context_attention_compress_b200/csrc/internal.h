@@ -17,6 +17,9 @@ cudaError_t launch_compress(const bf16* cand, int ld_cand, const bf16* logits, i
                             int rate, bool overlap, bf16* out, int ld_out, long long seq_out,
                             cudaStream_t stream, float* out_f32 = nullptr);
 // (out_f32 != nullptr: the entries are written there in f32, same strides, and out is unused)
+// Row b of src [B][c] into a paged pool [blocks * rpb][c]: row bt[b*bt_stride + entry/rpb]*rpb + entry%rpb.
+cudaError_t launch_scatter_rows(const bf16* src, int B, int c, const int32_t* bt, long long bt_stride, int entry,
+                                int rpb, bf16* pool, cudaStream_t stream);
 
 // ---- indexer_fp4.cu (FP4 indexer variant) ----------------------------------------
 cudaError_t launch_mxfp4_quantize(const void* x, bool x_f32, long long ld_x, int rows, int d, uint8_t* codes,
@@ -29,6 +32,24 @@ cudaError_t launch_indexer_decode_fp4(const bf16* q4, const float* w_idx, const 
                                       int B, int rate, float* scores, long long ld_scores, int num_sms,
                                       cudaStream_t stream, int* hist);
 unsigned int read_and_clear_indexer_fp4_error();
+
+// ---- kv_fp8.cu (FP8 storage of the non-rotary KV channels) -------------------------
+// Cache form of KV rows: codes [rows][ld_codes] E4M3 bytes (the first c - rope_dims
+// channels), scales [rows][ld_scales] f32 (one per 64 channels), rope [rows][ld_rope]
+// bf16 (the last rope_dims channels); sequences seq_rows rows apart.
+struct KvFp8 {
+  const uint8_t* codes;
+  const float* scales;
+  const bf16* rope;
+  long long ld_codes, ld_scales, ld_rope, seq_rows;
+};
+cudaError_t launch_kv_fp8_quantize(const void* x, bool x_f32, long long ld_x, long long rows, int c, int rope_dims,
+                                   uint8_t* codes, long long ld_codes, float* scales, long long ld_scales, bf16* rope,
+                                   long long ld_rope, cudaStream_t stream);
+// bf16 rows [B][n_out][c] from an FP8 cache: row j of sequence b <- source row idx[b][j]
+// (or j without idx); invalid or negative -> zeros (and idx_out -1, else j).
+cudaError_t launch_kv_fp8_gather(const KvFp8& kv, int c, int rope_dims, int B, int n_out, const int32_t* idx,
+                                 int n_src, bf16* out, int32_t* idx_out, cudaStream_t stream);
 
 // ---- norm_rope.cu -------------------------------------------------------------
 // Q/KV RMSNorm + partial RoPE of rows (see rms_norm_rope in hca.h for the row
@@ -45,6 +66,10 @@ struct NormRope {
   float eps, rope_base;
   bf16* y;
   long long ld_y, seq_y;
+  // ring != 0: the rows of a sequence are a ring buffer of rows_per_seq tokens ending
+  // at pos[s]: row r holds the one token of [pos[s] - rows_per_seq + 1, pos[s]] that is
+  // congruent to r mod rows_per_seq (pos_add and pos_step are not read)
+  int ring = 0;
 };
 cudaError_t launch_norm_rope(const NormRope& p, cudaStream_t stream);
 
@@ -129,17 +154,29 @@ cudaError_t launch_indexer_scores(const bf16* q_idx, const float* w_idx, const b
 
 // ---- indexer_tc.cu (tcgen05) -------------------------------------------------------
 bool indexer_tc_supported(int H_I, int d_I);
+// Paged indexer keys: request r's logical block j (rpb keys) is physical block
+// bt[r*bt_stride + j] of a pool of n_blocks blocks, [n_blocks * rpb, d_I] bf16.
+struct PagedKeys {
+  const int32_t* bt;
+  long long bt_stride;
+  int rpb;
+  long long n_blocks;
+};
 // Decode: query r scores request r's keys (k_idx + r*k_seq_stride), scores[r*ld + s].
 cudaError_t launch_indexer_decode_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, long long k_seq_stride,
                                      int N, const int32_t* q_pos, int B, int rate, float* scores, long long ld_scores,
                                      int num_sms, cudaStream_t stream,
-                                     int* hist = nullptr, bool stall = false);
+                                     int* hist = nullptr, bool stall = false, const PagedKeys* paged = nullptr);
 // (stall: tests of the bounded waits only -- the key producer issues nothing and every
 // wait gives up after a few thousand polls; the kernel records an error and returns)
-// Prefill: queries of one sequence against its keys [N, d_I]; scores[q*ld + s] for visible s.
+// Prefill: queries of one sequence against its keys [N, d_I].  With topk_idx (k <= the
+// fused limit, indexer_prefill_topk_fused) the top-k is taken on chip and written to
+// topk_idx [Tq, k] in entry order (-1 padded), scores unused; without it, scores[q*ld + s]
+// for visible s.
+bool indexer_prefill_topk_fused(int k);
 cudaError_t launch_indexer_prefill_tc(const bf16* q_idx, const float* w_idx, const bf16* k_idx, int N,
                                       const int32_t* q_pos, int Tq, int rate, float* scores, long long ld_scores,
-                                      int num_sms, cudaStream_t stream);
+                                      int num_sms, cudaStream_t stream, int k = 0, int32_t* topk_idx = nullptr);
 unsigned int read_and_clear_indexer_tc_error();
 
 // SM count of the current device (cached per device).
@@ -166,6 +203,12 @@ struct MqaProblem {
   const float* sink;        // [H] sink logits (natural units, like scale * q . k) or nullptr
   int rope_dims;            // > 0: the output's last rope_dims channels turn back by -q_pos
   float rope_base;
+  // paged entries (decode, tensor-core kernel only): request r's entry e is row
+  // bt[r*bt_stride + e / rpb] * rpb + e % rpb of a pool of pool_rows rows at kv
+  const int32_t* bt = nullptr;
+  long long bt_stride = 0;
+  int rpb = 0;
+  long long pool_rows = 0;
 };
 // Rows of one split; the workspace layout is decided by plan_mqa().
 struct MqaPlan {

@@ -384,6 +384,7 @@ static cudaError_t launch_mqa_t(const MqaProblem& p, const MqaPlan& pl, void* ws
 cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream, bool pdl) {
   if (p.Tq == 0) return cudaSuccess;
   if (mqa_tc_supported(p)) return launch_mqa_decode_tc(p, pl, ws, stream, pdl);
+  if (p.bt) return cudaErrorInvalidValue;  // paged entries: tensor-core kernel only
   if (p.H == 64 && p.c == 512) return launch_mqa_t<64, 512>(p, pl, ws, stream);
   if (p.H == 4 && p.c == 64) return launch_mqa_t<4, 64>(p, pl, ws, stream);
   return cudaErrorInvalidValue;

@@ -181,6 +181,9 @@ struct MqaTcParams {
                               // split ones in the combine
   int rope_dims;              // > 0: unsplit queries turn their output's last rope_dims channels back by
   float rope_base;            // -t here, split ones in the combine
+  const int32_t* bt;          // paged entries (see MqaProblem), or nullptr
+  long long bt_stride;
+  int rpb;
 };
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
@@ -188,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_kvg, const __grid_constant__ CUtensorMap tm_win, MqaTcParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base =
-      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+      tc::smem_align1024(smem_raw);
   Bars* bars = reinterpret_cast<Bars*>(base + kOffBars);
   volatile int* abort = &bars->abort;
   volatile int* need_flag = bars->need;
@@ -312,6 +315,9 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
 
     // Rows of tile j this issuer gathers (map rows; invalid slots read the request's row 0,
     // masked by the softmax).
+    // With paged entries every entry row is gathered: selected rows (idx) or the
+    // dense rows t.row0 + r, translated through the request's block table.
+    const int32_t* bt_q = p.bt ? p.bt + (long long)q * p.bt_stride : nullptr;
     auto gather_rows = [&](int j, int (&y)[4 * kGroupsPerIssuer]) {
       const Tile t = tiles.get(j);
 #pragma unroll
@@ -319,9 +325,10 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
 #pragma unroll
         for (int r4 = 0; r4 < 4; ++r4) {
           const int r = 4 * (g0 + gg * kCompute * kIssueLanes) + r4;
-          int e = (t.seg == 0 && idx_q != nullptr && r < t.nrows) ? idx_q[t.row0 + r] : 0;
+          int e = 0;
+          if (t.seg == 0 && r < t.nrows) e = idx_q != nullptr ? idx_q[t.row0 + r] : t.row0 + r;
           if (e < 0 || e >= p.N) e = 0;
-          y[4 * gg + r4] = (int)(kv_row_base + e);
+          y[4 * gg + r4] = bt_q ? bt_q[e / p.rpb] * p.rpb + e % p.rpb : (int)(kv_row_base + e);
         }
       }
     };
@@ -329,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     // tile has released it.  Returns false on a failed wait (warp-uniform).
     auto issue_tile = [&](int j, const int (&y)[4 * kGroupsPerIssuer]) -> bool {
       const Tile t = tiles.get(j);
-      const bool gathered = t.seg == 0 && idx_q != nullptr;
+      const bool gathered = t.seg == 0 && (idx_q != nullptr || bt_q != nullptr);
       for (int b = 0; b < kBlocks; ++b) {
         if (!tc::warp_wait(&bars->kvempty[b], (j & 1) ^ 1, abort)) return false;
         if (st == 0) tc::mbar_arrive_expect_tx(&bars->kvfull[b], kBlockBytes);
@@ -585,7 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
 // ---- host side ------------------------------------------------------------------
 bool mqa_tc_supported(const MqaProblem& p) {
   if (p.H != kH || p.c != kC || p.n_win > 256) return false;
-  if (p.mode == HCA_MODE_PREFILL) return p.win_rows > 0;
+  if (p.mode == HCA_MODE_PREFILL) return p.win_rows > 0 && p.bt == nullptr;
+  if (p.bt) return p.mode == HCA_MODE_DECODE && p.rpb >= 1 && p.pool_rows >= 1 && p.win_seq_stride % kC == 0;
   return p.mode == HCA_MODE_DECODE && p.kv_seq_stride % kC == 0 && p.win_seq_stride % kC == 0;
 }
 
@@ -626,15 +634,17 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   cudaError_t e = make_tmap_bf16(&tm_q, p.q, 2, qd, rstride, 64);
   if (e != cudaSuccess) return e;
   const bool prefill = p.mode == HCA_MODE_PREFILL;
-  const long long kv_rs = prefill ? 0 : p.kv_seq_stride / kC;
-  const uint64_t n_kv = (uint64_t)(p.N > 0 ? p.N : 1);
+  const long long kv_rs = (prefill || p.bt) ? 0 : p.kv_seq_stride / kC;
+  // (paged: the maps cover the whole pool; only the gather map is used)
+  const uint64_t n_kv = p.bt ? (uint64_t)p.pool_rows : (uint64_t)(p.N > 0 ? p.N : 1);
   // With no entries the entry maps are never used (no entry tiles): point them at
   // the window rows, which exist, instead of a cache that may have no rows.
   const void* kv_base = p.N > 0 ? (const void*)p.kv : (const void*)p.win;
   // dense tiles: (dims, rows of one request, request), so a tile never reads
   // another request's rows or the unused capacity behind a request's entries
-  const uint64_t kvd3[3] = {(uint64_t)kC, n_kv, prefill ? 1ull : (uint64_t)p.Tq};
-  const long long kv_req_elems = (prefill || p.Tq == 1 || p.N <= 0) ? (long long)n_kv * kC : p.kv_seq_stride;
+  const uint64_t kvd3[3] = {(uint64_t)kC, n_kv, (prefill || p.bt) ? 1ull : (uint64_t)p.Tq};
+  const long long kv_req_elems =
+      (prefill || p.bt || p.Tq == 1 || p.N <= 0) ? (long long)n_kv * kC : p.kv_seq_stride;
   const uint64_t kvs3[2] = {(uint64_t)kC * 2, (uint64_t)kv_req_elems * 2};
   e = make_tmap_bf16(&tm_kv, kv_base, 3, kvd3, kvs3, kRows);
   if (e != cudaSuccess) return e;
@@ -666,6 +676,9 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   a.sink = p.sink;
   a.rope_dims = p.rope_dims;
   a.rope_base = p.rope_base;
+  a.bt = p.bt;
+  a.bt_stride = p.bt_stride;
+  a.rpb = p.rpb > 0 ? p.rpb : 1;
   a.ws_o = pl.splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
   a.ws_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) + (size_t)p.Tq * pl.splits * kH * kC)
                           : nullptr;

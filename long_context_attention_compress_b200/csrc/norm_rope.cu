@@ -104,7 +104,16 @@ __global__ void __launch_bounds__(kNrThreads) norm_rope_kernel(NormRope p, long 
   int slot = 0;
   for (long long R = r0; R < r1; ++R) {
     issue(R + C::kStages - 1, slot == 0 ? C::kStages - 1 : slot - 1);
-    const long long pos = (long long)max((p.pos ? p.pos[sq] : 0) + p.pos_add, 0) + rr * p.pos_step;
+    long long pos;
+    if (p.ring) {
+      // ring block of rows_per_seq rows ending at t: row rr holds the token in
+      // [t - rows_per_seq + 1, t] that is congruent to rr
+      const long long t = p.pos ? p.pos[sq] : 0;
+      const long long n = p.rows_per_seq;
+      pos = t - (((t - rr) % n) + n) % n;
+    } else {
+      pos = (long long)max((p.pos ? p.pos[sq] : 0) + p.pos_add, 0) + rr * p.pos_step;
+    }
     if (pos != last_pos && n_pairs > 0) {  // warp-uniform
       last_pos = pos;
       __syncwarp();

@@ -20,6 +20,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte aligned byte of a dynamic shared-memory block, derived from
+// the block's own pointer by an offset.  (Rounding the address as an integer would
+// lose the pointer's shared address space, and every load, store and atomic
+// through it would become a slower generic one.)
+__device__ __forceinline__ unsigned char* smem_align1024(unsigned char* p) {
+  return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
+}
+
 // ---- mbarrier ------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
