@@ -241,8 +241,8 @@ int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hc
  *   the MXFP4 values of q_I and K_I.  Takes the 64 x 128 indexer only.
  *   q_idx [B, 64, 128] bf16 (rounded to its MXFP4 values inside the call);
  *   w_idx [B, 64] f32; request r's keys: codes at k_codes + r*k_seq_stride*64
- *   ([N][64] bytes), scales at k_scales + r*k_seq_stride*4 ([N][4] bytes,
- *   readable up to the next multiple of 4 keys); with B > 1, k_seq_stride >=
+ *   ([N][64] bytes), scales at k_scales + r*k_seq_stride*4 ([N][4] bytes), both
+ *   readable up to the next multiple of 4 keys; with B > 1, k_seq_stride >=
  *   that multiple of 4 and itself a multiple of 4.  topk_idx [B, topk] as in
  *   csa_indexer_topk.  ws: csa_indexer_topk_fp4_workspace(cfg, B, N) bytes.
  *   Device-side waits that give up are reported by hca_check_device.
@@ -375,8 +375,8 @@ typedef struct {
   /* FP4 indexer variant (see csa_indexer_topk_fp4), or NULL: the CSA layer's indexer
    * reads MXFP4 keys instead of csa_k_idx (which is then not read): request b's codes
    * at csa_k_codes + b*csa_k4_stride*64 ([csa_N][64] bytes) and scales at
-   * csa_k_scales + b*csa_k4_stride*4 ([csa_N][4] bytes, readable up to the next
-   * multiple of 4 keys); csa_k4_stride in keys, a multiple of 4 (B > 1). 64 x 128
+   * csa_k_scales + b*csa_k4_stride*4 ([csa_N][4] bytes), both readable up to the
+   * next multiple of 4 keys; csa_k4_stride in keys, a multiple of 4 (B > 1). 64 x 128
    * indexer only; the index scores are BF16. */
   const uint8_t* csa_k_codes;
   const uint8_t* csa_k_scales;

@@ -22,8 +22,9 @@
 //               (FP4-rounded, bf16) query on request change
 //   warp 1      MMA issuer
 //   warps 2..5  epilogue: ReLU, head weights, BF16 rounding, score-key histogram
-//   warps 6..9  converters: one key row per thread, codes x scale -> bf16 into
-//               the 128B-swizzled K-major tile ring (3 deep) the MMA reads
+//   warps 6..13 converters: half a key row per thread, codes x scale -> bf16 (byte
+//               permutes and one bf16x2 multiply per pair) into the 128B-swizzled
+//               K-major tile ring (3 deep) the MMA reads
 // Every wait is bounded; a CTA that gives up records an error, lets its own
 // copies and MMAs drain, frees its TMEM and returns.
 //
@@ -57,7 +58,8 @@ constexpr uint32_t kFTileBytes = kFTile * kFDim * 2;       // 32 KiB
 constexpr uint32_t kFChunkBytes = kFTile * 128;            // 16 KiB (64 dims)
 constexpr uint32_t kFQBytes = kFHeads * kFDim * 2;         // 16 KiB
 constexpr uint32_t kFQChunkBytes = kFHeads * 128;          // 8 KiB
-constexpr int kFThreads = 320;
+constexpr int kFConvWarps = 8;                             // converter warps (two per scheduler)
+constexpr int kFThreads = 192 + 32 * kFConvWarps;          // producer, MMA, 4 epilogue warps, converters
 constexpr int kFConv0 = 192;                               // first converter thread
 
 struct __align__(8) FBars {
@@ -79,6 +81,43 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
   const uint32_t e = (c >> 1) & 3u, m = c & 1u;
   const uint32_t mag = e ? (((126u + e) << 23) | (m << 22)) : (m ? 0x3F000000u : 0u);
   return __uint_as_float(mag | ((c & 8u) << 28));
+}
+
+// Eight E2M1 codes (word nibbles 0..7, element order) times 2^X -> eight bf16, packed in
+// pairs (o[k] = element 2k | element 2k+1 << 16).  The magnitudes come from byte
+// tables by byte permutes (bf16 bits of 0, 0.5, 1, 1.5, 2, 3, 4, 6: high bytes
+// 00 3F 3F 3F 40 40 40 40, low bytes 00 00 80 C0 00 40 80 C0), the signs are moved
+// to bit 15 / 31, and 2^X is applied by one bf16x2 multiply, exact while every
+// nonzero product stays a normal bf16 (|X| <= 125: 0.5 * 2^X .. 6 * 2^X); beyond
+// that the values are formed in f32 (as exact) and rounded once.
+__device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, int X, uint32_t* o) {
+  constexpr uint32_t kHiLo = 0x3F3F3F00u, kHiHi = 0x40404040u, kLoLo = 0xC0800000u, kLoHi = 0xC0804000u;
+  if (X >= -125 && X <= 125) {
+    const uint32_t m = w & 0x77777777u, sg = w & 0x88888888u;
+    const uint32_t h0 = __byte_perm(kHiLo, kHiHi, m & 0xffffu), l0 = __byte_perm(kLoLo, kLoHi, m & 0xffffu);
+    const uint32_t h1 = __byte_perm(kHiLo, kHiHi, m >> 16), l1 = __byte_perm(kLoLo, kLoHi, m >> 16);
+    uint32_t p[4];
+    p[0] = __byte_perm(l0, h0, 0x5140u) | ((sg << 12) & 0x8000u) | ((sg << 24) & 0x80000000u);
+    p[1] = __byte_perm(l0, h0, 0x7362u) | ((sg << 4) & 0x8000u) | ((sg << 16) & 0x80000000u);
+    p[2] = __byte_perm(l1, h1, 0x5140u) | ((sg >> 4) & 0x8000u) | ((sg << 8) & 0x80000000u);
+    p[3] = __byte_perm(l1, h1, 0x7362u) | ((sg >> 12) & 0x8000u) | (sg & 0x80000000u);
+    const uint32_t sb = (uint32_t)(127 + X) << 7;  // bf16 bits of 2^X
+    const uint32_t sbits = sb | (sb << 16);
+    __nv_bfloat162 sc;
+    memcpy(&sc, &sbits, 4);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      __nv_bfloat162 v;
+      memcpy(&v, &p[k], 4);
+      v = __hmul2(v, sc);
+      memcpy(&o[k], &v, 4);
+    }
+    return;
+  }
+  const float scf = ldexpf(1.f, X);
+#pragma unroll
+  for (int j = 0; j < 8; j += 2)
+    o[j >> 1] = pack_bf16x2(e2m1_value((w >> (4 * j)) & 15u) * scf, e2m1_value((w >> (4 * j + 4)) & 15u) * scf);
 }
 
 // Nearest E2M1 code of a (already scaled) value, ties to the even code, saturating.
@@ -179,8 +218,14 @@ __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
   const long long g1 = total * (blockIdx.x + 1) / gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kFStages; ++s) { tc::mbar_init(&bars->sfull[s], 1); tc::mbar_init(&bars->sempty[s], 4); }
-    for (int b = 0; b < kFBuf; ++b) { tc::mbar_init(&bars->cfull[b], 4); tc::mbar_init(&bars->bempty[b], 1); }
+    for (int s = 0; s < kFStages; ++s) {
+      tc::mbar_init(&bars->sfull[s], 1);
+      tc::mbar_init(&bars->sempty[s], kFConvWarps);
+    }
+    for (int b = 0; b < kFBuf; ++b) {
+      tc::mbar_init(&bars->cfull[b], kFConvWarps);
+      tc::mbar_init(&bars->bempty[b], 1);
+    }
     for (int a = 0; a < kFAcc; ++a) { tc::mbar_init(&bars->tfull[a], 1); tc::mbar_init(&bars->tempty[a], 4); }
     for (int b = 0; b < 2; ++b) { tc::mbar_init(&bars->qfull[b], 1); tc::mbar_init(&bars->qempty[b], 1); }
     tc::mbar_init(&bars->drain, 1);
@@ -219,7 +264,7 @@ __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
         if (!tc::mbar_wait(&bars->sempty[s], ((it / kFStages) & 1) ^ 1, abort)) break;
         tc::mbar_arrive_expect_tx(&bars->sfull[s], kFCodeBytes + kFScaleBytes);
         unsigned char* slot = st_smem + s * kFStageStride;
-        tc::tma_load_3d(slot, &tm_codes, &bars->sfull[s], 0, row0, r);                  // [128][64 B]
+        tc::tma_load_3d(slot, &tm_codes, &bars->sfull[s], 0, row0 / 2, r);              // [64][128 B]
         tc::tma_load_3d(slot + kFCodeBytes, &tm_scales, &bars->sfull[s], 0, row0 / 4, r);  // [32][16 B]
         ++it;
       }
@@ -330,10 +375,11 @@ __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
     if (hist_g && cur_r >= 0) flush(cur_r);
   } else {
     // ------------------------------ converters ------------------------------
-    // thread ci widens key row ci of each tile: 128 codes x its 4 block scales -> bf16,
-    // written in the K-major 128B-swizzled layout (unit u of a 64-dim chunk at
-    // row * 128 + ((u ^ (row & 7)) * 16)).
+    // thread ci widens half a key row of each tile: row ci % 128, 64-dim chunk ci / 128
+    // (its 32 code bytes and 2 block scales) -> bf16, written in the K-major
+    // 128B-swizzled layout (16-byte unit u of the chunk at row * 128 + ((u ^ (row & 7)) * 16)).
     const int ci = threadIdx.x - kFConv0;
+    const int crw = ci & (kFTile - 1), chh = ci >> 7;
     int it = 0;
     for (long long g = g0; g < g1; ++g) {
       const int r = (int)(g / tiles_per_req);
@@ -343,28 +389,20 @@ __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
       if (!tc::warp_wait(&bars->sfull[s], (it / kFStages) & 1, abort)) break;
       if (!tc::warp_wait(&bars->bempty[b], ((it / kFBuf) & 1) ^ 1, abort)) break;
       const unsigned char* slot = st_smem + s * kFStageStride;
-      const uint4* crow = reinterpret_cast<const uint4*>(slot + ci * 64);
-      const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(slot + kFCodeBytes + ci * 4);
-      unsigned char* trow = k_smem + b * kFTileBytes + ci * 128;
+      const uint4* crow = reinterpret_cast<const uint4*>(slot + crw * 64 + chh * 32);
+      const uint32_t sc2 = *reinterpret_cast<const uint32_t*>(slot + kFCodeBytes + crw * 4) >> (16 * chh);
+      unsigned char* trow = k_smem + b * kFTileBytes + chh * kFChunkBytes + crw * 128;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {  // 32-dim block q: codes crow[q], scale byte q
+      for (int q = 0; q < 2; ++q) {  // 32-dim block q of the chunk: codes crow[q], scale byte q
         const uint4 cw = crow[q];
-        const float scf = ldexpf(1.f, (int)((sc4 >> (8 * q)) & 0xffu) - 127);  // 2^X, exact
+        const int X = (int)((sc2 >> (8 * q)) & 0xffu) - 127;
         const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {  // 8 dims: unit 4q + h
-          const uint32_t word = words[h];
+        for (int h = 0; h < 4; ++h) {  // 8 dims: unit 4q + h of the chunk
           uint32_t o[4];
-#pragma unroll
-          for (int j = 0; j < 8; j += 2) {
-            // (a power-of-two product of a two-significant-bit value: exact in f32 and in bf16)
-            o[j >> 1] = pack_bf16x2(e2m1_value((word >> (4 * j)) & 15u) * scf,
-                                    e2m1_value((word >> (4 * j + 4)) & 15u) * scf);
-          }
-          const int u = 4 * q + h;             // 16-byte unit along the row (0..15)
-          const int chunk = u >> 3, uu = u & 7;  // 64-dim chunk and unit within it
-          *reinterpret_cast<uint4*>(trow + chunk * kFChunkBytes + ((uu ^ (ci & 7)) << 4)) =
-              make_uint4(o[0], o[1], o[2], o[3]);
+          e2m1x8_to_bf16(words[h], X, o);
+          const int uu = 4 * q + h;
+          *reinterpret_cast<uint4*>(trow + ((uu ^ (crw & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }
       tc::fence_proxy_async_smem();  // the tensor cores read the tile through the async proxy
@@ -442,9 +480,11 @@ cudaError_t launch_indexer_decode_fp4(const bf16* q4, const float* w_idx, const 
   if (B == 0 || N == 0) return cudaSuccess;
   CUtensorMap tm_codes, tm_scales, tm_q;
   const long long per_req = B > 1 ? k_seq_stride : (long long)(N + 3) / 4 * 4;  // keys between requests
-  const uint64_t cd[3] = {64, (uint64_t)N, (uint64_t)B};
-  const uint64_t cs[2] = {64, (uint64_t)per_req * 64};
-  cudaError_t e = make_tmap_u8(&tm_codes, k_codes, cd, cs, 64, kFTile);
+  // codes as 128-byte rows of two keys (contiguous, so the staged bytes are the same as
+  // key rows of 64 B): half the row requests of 64-byte rows
+  const uint64_t cd[3] = {128, (uint64_t)(N + 3) / 4 * 2, (uint64_t)B};
+  const uint64_t cs[2] = {128, (uint64_t)per_req * 64};
+  cudaError_t e = make_tmap_u8(&tm_codes, k_codes, cd, cs, 128, kFTile / 2);
   if (e != cudaSuccess) return e;
   const uint64_t sd[3] = {16, (uint64_t)(N + 3) / 4, (uint64_t)B};
   const uint64_t ss[2] = {16, (uint64_t)per_req * 4};

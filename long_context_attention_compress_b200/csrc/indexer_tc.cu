@@ -298,7 +298,7 @@ constexpr uint32_t kPQBytes = kPN * kDim * 2;        // 64 KiB
 constexpr uint32_t kPQChunkBytes = kPN * 128;        // 32 KiB
 constexpr int kPAcc = 2;
 constexpr int kPThreads = 320;  // producer, MMA, 8 epilogue warps (two per TMEM lane quarter)
-constexpr int kPCand = 1536;    // candidate slots per query
+constexpr int kPCand = 1792;    // candidate slots per query
 constexpr int kPPer = kPCand / 128;  // candidates per thread of a half in a cut
 
 // Scratch of one half of the epilogue (the 128 threads serving two queries).
@@ -459,6 +459,96 @@ __device__ __forceinline__ uint64_t cut_to_topk(uint64_t* buf, int n, int k, PHa
 #pragma unroll
   for (int i = 0; i < 4; ++i) kmin = hs->wmin[i] < kmin ? hs->wmin[i] : kmin;
   return kmin;
+}
+// Cut the candidate list buf[0..n) (distinct composites, k < n <= kPCand) to the
+// candidates at or above the bucket of its k-th largest, in one histogram pass over
+// the 8 highest bits where the list differs; keeps their order and returns how many
+// were kept (at least k) through *kept, and as the new threshold the largest
+// composite below every kept one.  No later entry at or under it can be among the k
+// largest: the kept ones are at least k and all larger.  Falls back to the exact cut
+// when the bucket would leave less than two tiles of room.
+__device__ __forceinline__ uint64_t cut_coarse(uint64_t* buf, int n, int k, PHalf* hs, uint32_t bar, int hl,
+                                               int* kept) {
+  const int lane = hl & 31, w = hl >> 5;
+  tc::named_bar(bar, 128);  // every warp's appends are in place
+  const int per = (n + 127) / 128;
+  const int i0 = hl * per;
+  uint64_t v[kPPer];
+  unsigned long long mn = ~0ull, mx = 0ull;
+#pragma unroll
+  for (int u = 0; u < kPPer; ++u) {
+    const int i = i0 + u;
+    const bool ok = u < per && i < n;
+    v[u] = ok ? buf[i] : 0ull;
+    if (ok) {
+      mn = v[u] < mn ? v[u] : mn;
+      mx = v[u] > mx ? v[u] : mx;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const unsigned long long a = __shfl_xor_sync(0xffffffffu, mn, o);
+    const unsigned long long b = __shfl_xor_sync(0xffffffffu, mx, o);
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
+  }
+  if (lane == 0) {
+    hs->wmin[w] = mn;
+    hs->wmax[w] = mx;
+  }
+  tc::named_bar(bar, 128);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    mn = hs->wmin[i] < mn ? hs->wmin[i] : mn;
+    mx = hs->wmax[i] > mx ? hs->wmax[i] : mx;
+  }
+  const int hi = 63 - __clzll((long long)(mn ^ mx));  // mn < mx: distinct and n > k >= 1
+  const int lo = hi >= 7 ? hi - 7 : 0;
+  const uint32_t dmask = (1u << (hi - lo + 1)) - 1u;
+  hs->hist[hl] = 0;
+  hs->hist[hl + 128] = 0;
+  tc::named_bar(bar, 128);
+#pragma unroll
+  for (int u = 0; u < kPPer; ++u) {
+    const int i = i0 + u;
+    if (u < per && i < n) atomicAdd(&hs->hist[(int)((v[u] >> lo) & dmask)], 1);
+  }
+  tc::named_bar(bar, 128);
+  const int b0 = 255 - 2 * hl, b1 = b0 - 1;
+  const int h0 = hs->hist[b0], h1 = hs->hist[b1];
+  int tot;
+  const int ex = half_scan(h0 + h1, hl, hs, bar, &tot);  // candidates in bins above b0
+  if (ex < k && ex + h0 >= k) {
+    hs->bucket = b0;
+    hs->greater = ex + h0;  // kept: everything in bin b0 and above
+  } else if (ex + h0 < k && ex + h0 + h1 >= k) {
+    hs->bucket = b1;
+    hs->greater = ex + h0 + h1;
+  }
+  tc::named_bar(bar, 128);
+  const int nkeep = hs->greater;
+  const uint64_t P = ((mn >> lo) & ~(uint64_t)dmask) | (uint64_t)hs->bucket;  // bucket's value of v >> lo
+  tc::named_bar(bar, 128);  // bucket read by all before it is rewritten
+  if (nkeep > kPCand - 2 * kTile) {  // a fat bucket: the exact cut
+    // (buf is unchanged; cut_to_topk reloads it)
+    *kept = k;
+    return cut_to_topk(buf, n, k, hs, bar, hl);
+  }
+  int nk = 0;
+#pragma unroll
+  for (int u = 0; u < kPPer; ++u) {
+    const int i = i0 + u;
+    nk += (u < per && i < n && (v[u] >> lo) >= P) ? 1 : 0;
+  }
+  int off = half_scan(nk, hl, hs, bar, &tot);
+#pragma unroll
+  for (int u = 0; u < kPPer; ++u) {
+    const int i = i0 + u;
+    if (u < per && i < n && (v[u] >> lo) >= P) buf[off++] = v[u];
+  }
+  tc::named_bar(bar, 128);  // the cut list is in place
+  *kept = tot;
+  return (P << lo) - 1;  // every kept composite is >= P << lo > 0
 }
 }  // namespace
 
@@ -666,12 +756,14 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
           cnt[jj] += tot;
         }
         par ^= 1;
-        // room for one more tile of appends in each list, else cut it to its k largest
+        // room for one more tile of appends in each list, else cut it back (coarsely: the
+        // exact k largest are taken once, after the group's last tile)
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
           if (cnt[jj] > kPCand - kTile) {
-            thr[jj] = cut_to_topk(cbuf[jj], cnt[jj], k, hs, hbar, hl);
-            cnt[jj] = k;
+            int kept;
+            thr[jj] = cut_coarse(cbuf[jj], cnt[jj], k, hs, hbar, hl, &kept);
+            cnt[jj] = kept;
           }
         }
       }
