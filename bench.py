@@ -788,7 +788,7 @@ def run_ours(a):
         # the prefill step is ~200x longer than a decode step: fewer steps cover as long a region
         psteps = a.prefill_steps if a.prefill_steps else max(3, min(20, a.steps or 20))
         pm = measure(pb, a, psteps, max(3, min(a.warmup, 5)), flush, rank, ws, device, local,
-                     max(4, a.cpu_sample))
+                     4 * a.cpu_sample)
         pm["workload"] = "csa_prefill_64k"
         out["prefill"] = pm
     if rank == 0:
@@ -884,7 +884,8 @@ def main():
                                                                           if k != "tiny_prefill_1k"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--cpu-sample", type=int, default=4, help="requests (decode) / queries (prefill) for the oracle")
+    ap.add_argument("--cpu-sample", type=int, default=10,
+                    help="requests (decode; the 64K prefill in the same line takes 4x as many queries) for the oracle")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--qk-norm", action="store_true",
                     help="the layer with Q/KV RMSNorm + partial RoPE (synthetic weights)")
