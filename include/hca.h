@@ -35,6 +35,16 @@
  *     HCA_TEST_STALL=indexer makes the decode indexer's key producer issue
  *     nothing, with a budget of a few thousand polls, so that its waits run
  *     out (the call's top-k output is then meaningless).
+ *   - Index check: with HCA_DEBUG=1 in the environment at call time, the
+ *     attention kernels of sparse_mqa_attend, hybrid_attn_decode and
+ *     hybrid_attn_prefill record every selected entry outside [-1, N), every
+ *     entry e that its query at position t cannot see yet ((e+1)*rate - 1 > t)
+ *     and every block-table entry outside the pool; hca_check_device() then
+ *     reports HCA_ERR_DEVICE_CHECK naming the kinds found.  Out-of-range
+ *     entries are skipped (as empty slots) with or without the check; the
+ *     check changes no result.
+ *   - Every entry point that launches work opens an NVTX range named after
+ *     itself for the duration of the host call (no cost without a tool).
  *   - Supported shapes: c in {64, 512}, d_idx in {32, 128}; n_heads,
  *     n_idx_heads <= 64; topk <= 2048; n_win <= 256.  Other shapes return
  *     HCA_ERR_UNSUPPORTED.

@@ -10,6 +10,8 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -64,6 +66,23 @@ bool test_stall_indexer() {
   const char* v = getenv("HCA_TEST_STALL");
   return v && strcmp(v, "indexer") == 0;
 }
+
+// HCA_DEBUG=1: the attention kernels record selected entries that are out of
+// range or not causally visible, and block-table entries outside the pool
+// (reported by hca_check_device; the results are as without the check).
+bool debug_checks() {
+  const char* v = getenv("HCA_DEBUG");
+  return v && strcmp(v, "1") == 0;
+}
+
+// One NVTX range per entry point call (named after it), for timeline tools.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define HCA_RANGE(name) NvtxRange nvtx_range_(name)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -322,6 +341,7 @@ MqaProblem make_mqa(const hca_layer_cfg* cfg, const hca_bf16* q, const hca_bf16*
   p.sink = sink;
   p.rope_dims = 0;
   p.rope_base = cfg->rope_base;
+  p.check = debug_checks() ? 1 : 0;
   return p;
 }
 
@@ -362,14 +382,23 @@ int hca_check_device(void) {
   const unsigned int w4 = read_and_clear_indexer_fp4_error();
   if (w1 == 0xffffffffu || w2 == 0xffffffffu || w3 == 0xffffffffu || w4 == 0xffffffffu)
     return fail(HCA_ERR_CUDA, "hca_check_device: cannot read the device error word");
-  const unsigned int w = w1 | (w2 << 1) | (w4 << 2);
+  const unsigned int w5 = read_and_clear_mqa_index_error();
+  if (w5 == 0xffffffffu) return fail(HCA_ERR_CUDA, "hca_check_device: cannot read the device error word");
+  const unsigned int w = w1 | ((w2 & 1u) << 1) | (w4 << 2);
+  const unsigned int idx_bad = (w2 >> 1) | w5;
   if (w) return fail(HCA_ERR_DEVICE_CHECK, "hca_check_device: a kernel gave up waiting (error word 0x%x)", w);
   if (w3) return fail(HCA_ERR_DEVICE_CHECK, "hca_check_device: a top-k histogram disagreed with its scores");
+  if (idx_bad)
+    return fail(HCA_ERR_DEVICE_CHECK, "hca_check_device: the attention was given %s%s%s",
+                (idx_bad & kIdxRange) ? "entries out of range; " : "",
+                (idx_bad & kIdxCausal) ? "entries not yet visible to their query; " : "",
+                (idx_bad & kIdxBlock) ? "block-table entries outside the pool; " : "");
   return HCA_OK;
 }
 
 int csa_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int ld_logits, const float* pos_bias,
                  int ld_bias, int T, int c, int m, hca_bf16* out, int ld_out, void* stream) {
+  HCA_RANGE("csa_compress");
   g_err.clear();
   CHECK(T >= 0 && c > 0 && m >= 1 && m <= 16, HCA_ERR_INVALID_ARG, "csa_compress: T=%d c=%d m=%d", T, c, m);
   CHECK(c % 8 == 0, HCA_ERR_UNSUPPORTED, "csa_compress: c=%d not a multiple of 8", c);
@@ -392,6 +421,7 @@ int csa_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int 
 int hca_compress(const hca_bf16* cand, int ld_cand, const hca_bf16* logits, int ld_logits, const float* pos_bias,
                  int ld_bias, int B, long long seq_stride_in, int T, int c, int m_hca, hca_bf16* out, int ld_out,
                  long long seq_stride_out, void* stream) {
+  HCA_RANGE("hca_compress");
   g_err.clear();
   CHECK(B >= 0 && B <= 65535 && T >= 0 && c > 0 && m_hca >= 1 && m_hca <= 1024, HCA_ERR_INVALID_ARG,
         "hca_compress: B=%d T=%d c=%d m'=%d", B, T, c, m_hca);
@@ -428,6 +458,7 @@ size_t hca_workspace_size(int op, const hca_layer_cfg* cfg, int Tq, int N, int m
 int csa_indexer_topk(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* k_idx, long long k_seq_stride, int N,
                      const int32_t* q_pos, int Tq, int mode, const hca_layer_cfg* cfg, int32_t* topk_idx, void* ws,
                      size_t ws_bytes, void* stream) {
+  HCA_RANGE("csa_indexer_topk");
   g_err.clear();
   int s = check_cfg(cfg);
   if (s != HCA_OK) return s;
@@ -485,6 +516,7 @@ int noalloc_scratch(void** out) {
 int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hca_bf16* k_idx,
                              long long k_seq_stride, int N, const int32_t* q_pos, int Tq, int mode,
                              const hca_layer_cfg* cfg, int32_t* topk_idx, void* stream) {
+  HCA_RANGE("csa_indexer_topk_noalloc");
   g_err.clear();
   int s = check_cfg(cfg);
   if (s != HCA_OK) return s;
@@ -522,6 +554,7 @@ int csa_indexer_topk_noalloc(const hca_bf16* q_idx, const float* w_idx, const hc
 int rms_norm_rope(const void* x, int x_is_f32, long long ld_x, long long seq_stride_x, int n_seq, int rows_per_seq,
                   const int32_t* pos, int pos_add, int pos_step, const float* gamma, const hca_layer_cfg* cfg,
                   hca_bf16* y, long long ld_y, long long seq_stride_y, void* stream) {
+  HCA_RANGE("rms_norm_rope");
   g_err.clear();
   int s = check_cfg(cfg);
   if (s != HCA_OK) return s;
@@ -571,6 +604,7 @@ int sparse_mqa_attend(const hca_bf16* q, const hca_bf16* kv, long long kv_seq_st
                       int n_idx, int rate, const hca_bf16* win, long long win_seq_stride, const int32_t* q_pos, int Tq,
                       int mode, const hca_layer_cfg* cfg, const float* sink, int rotate_out, hca_bf16* out,
                       void* ws, size_t ws_bytes, void* stream) {
+  HCA_RANGE("sparse_mqa_attend");
   g_err.clear();
   int s = check_cfg(cfg);
   if (s != HCA_OK) return s;
@@ -616,6 +650,7 @@ static KvFp8 kv_fp8_of(const hca_kv_fp8* d) {
 extern "C" int kv_fp8_quantize(const void* x, int x_is_f32, long long ld_x, long long rows, const hca_layer_cfg* cfg,
                                uint8_t* codes, long long ld_codes, float* scales, long long ld_scales, hca_bf16* rope,
                                long long ld_rope, void* stream) {
+  HCA_RANGE("kv_fp8_quantize");
   g_err.clear();
   int s = check_cfg(cfg);
   if (s != HCA_OK) return s;
@@ -817,6 +852,7 @@ size_t hybrid_attn_decode_workspace(const hca_layer_cfg* cfg, const hca_decode_a
 }
 
 int hybrid_attn_decode(const hca_layer_cfg* cfg, const hca_decode_args* a, void* ws, size_t ws_bytes, void* stream) {
+  HCA_RANGE("hybrid_attn_decode");
   g_err.clear();
   int s = check_cfg(cfg);
   if (s != HCA_OK) return s;
@@ -1108,6 +1144,7 @@ size_t hybrid_attn_prefill_workspace(const hca_layer_cfg* cfg, const hca_prefill
 }
 
 int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, void* ws, size_t ws_bytes, void* stream) {
+  HCA_RANGE("hybrid_attn_prefill");
   g_err.clear();
   int s = check_cfg(cfg);
   if (s != HCA_OK) return s;
@@ -1232,6 +1269,7 @@ int hybrid_attn_prefill(const hca_layer_cfg* cfg, const hca_prefill_args* a, voi
 // ---- FP4 indexer variant -----------------------------------------------------------
 int mxfp4_quantize(const void* x, int x_is_f32, long long ld_x, int rows, int d, uint8_t* codes, long long ld_codes,
                    uint8_t* scales, long long ld_scales, void* stream) {
+  HCA_RANGE("mxfp4_quantize");
   g_err.clear();
   CHECK(rows >= 0 && d > 0 && d % 32 == 0, HCA_ERR_INVALID_ARG, "mxfp4_quantize: rows=%d d=%d (d a multiple of 32)",
         rows, d);
@@ -1263,6 +1301,7 @@ size_t csa_indexer_topk_fp4_workspace(const hca_layer_cfg* cfg, int B, int N) {
 int csa_indexer_topk_fp4(const hca_bf16* q_idx, const float* w_idx, const uint8_t* k_codes, const uint8_t* k_scales,
                          long long k_seq_stride, int N, const int32_t* q_pos, int B, const hca_layer_cfg* cfg,
                          int32_t* topk_idx, void* ws, size_t ws_bytes, void* stream) {
+  HCA_RANGE("csa_indexer_topk_fp4");
   g_err.clear();
   int s = check_cfg(cfg);
   if (s != HCA_OK) return s;

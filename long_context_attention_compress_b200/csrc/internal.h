@@ -209,7 +209,19 @@ struct MqaProblem {
   long long bt_stride = 0;
   int rpb = 0;
   long long pool_rows = 0;
+  // opt-in index check: record selected entries outside [-1, N), entries that the
+  // query cannot see yet (last token after q_pos) and block-table entries outside
+  // the pool; results are computed as without the check
+  int check = 0;
 };
+// Bits of the index-check record (hca_check_device reports them).
+constexpr unsigned int kIdxRange = 1u, kIdxCausal = 2u, kIdxBlock = 4u;
+// Kind of a selected entry e of a query at position t (0: acceptable).
+__host__ __device__ __forceinline__ unsigned int entry_check(int e, int t, int rate, int N) {
+  if (e < -1 || e >= N) return kIdxRange;
+  if (e >= 0 && (long long)(e + 1) * rate - 1 > t) return kIdxCausal;
+  return 0u;
+}
 // Rows of one split; the workspace layout is decided by plan_mqa().
 struct MqaPlan {
   int splits;          // splits per query (1 = no combine)
@@ -234,6 +246,7 @@ cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, i
 bool mqa_tc_supported(const MqaProblem& p);
 MqaPlan plan_mqa_tc(const MqaProblem& p, int num_sms);
 cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream, bool pdl);
-unsigned int read_and_clear_mqa_tc_error();
+unsigned int read_and_clear_mqa_tc_error();     // bit 0: a wait gave up; entry_check bits << 1
+unsigned int read_and_clear_mqa_index_error();  // entry_check bits of the CUDA-core attention
 
 }  // namespace hca

@@ -20,21 +20,26 @@
 namespace hca {
 
 constexpr int kMqaThreads = 256;
+
+// index-check record of this kernel (entry_check bits)
+__device__ unsigned int g_mqa_index_error = 0;
 constexpr int kTR = 16;  // rows per tile
 
 struct RowList {
   const bf16* kv;       // this request's entries
   const int32_t* idx;   // this query's selected entries or nullptr
   int n_first;          // length of the entry part
+  int N;                // entries of the request
+  int t;                // the query's position
   const bf16* win;      // first window row
   int n_win;            // window rows
   int c;
   __device__ __forceinline__ int length() const { return n_first + n_win; }
-  // pointer of list row u, or nullptr for an empty selected slot
+  // pointer of list row u, or nullptr for an empty (or out-of-range) selected slot
   __device__ __forceinline__ const bf16* row(int u) const {
     if (u < n_first) {
       int s = idx ? idx[u] : u;
-      return s < 0 ? nullptr : kv + (long long)s * c;
+      return (s < 0 || s >= N) ? nullptr : kv + (long long)s * c;
     }
     return win + (long long)(u - n_first) * c;
   }
@@ -46,6 +51,8 @@ __device__ __forceinline__ RowList make_rows(const MqaProblem& p, int q) {
   const long long rs = p.mode == HCA_MODE_DECODE ? q : 0;
   L.kv = p.kv + rs * p.kv_seq_stride;
   L.c = p.c;
+  L.N = p.N;
+  L.t = t;
   if (p.idx) {
     L.idx = p.idx + (long long)q * p.n_idx;
     L.n_first = p.n_idx;
@@ -109,7 +116,13 @@ __global__ void __launch_bounds__(kMqaThreads) mqa_split_kernel(MqaProblem p, in
       uint4 v = make_uint4(0, 0, 0, 0);
       if (rp) v = *reinterpret_cast<const uint4*>(rp + d);
       *reinterpret_cast<uint4*>(s_r + r * CP + d) = v;
-      if (d == 0) s_valid[r] = rp != nullptr;
+      if (d == 0) {
+        s_valid[r] = rp != nullptr;
+        if (p.check && L.idx && u < u_end && u < L.n_first) {
+          const unsigned int k = entry_check(L.idx[u], L.t, p.rate, p.N);
+          if (k) atomicOr(&g_mqa_index_error, k);
+        }
+      }
     }
     __syncthreads();
     // scores S[h][u] (base-2 scaled)
@@ -379,6 +392,13 @@ static cudaError_t launch_mqa_t(const MqaProblem& p, const MqaPlan& pl, void* ws
                                                                                       p.rope_dims, p.rope_base);
   ++g_launch_counter;
   return cudaGetLastError();
+}
+
+unsigned int read_and_clear_mqa_index_error() {
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_mqa_index_error, sizeof(v)) != cudaSuccess) return 0xffffffffu;
+  if (v) cudaMemcpyToSymbol(g_mqa_index_error, &zero, sizeof(zero));
+  return v;
 }
 
 cudaError_t launch_mqa(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream, bool pdl) {

@@ -184,6 +184,8 @@ struct MqaTcParams {
   const int32_t* bt;          // paged entries (see MqaProblem), or nullptr
   long long bt_stride;
   int rpb;
+  long long pool_blocks;      // blocks of the pool the block table points into
+  int check;                  // record entry_check failures (bits << 1 of the error word)
 };
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
@@ -385,9 +387,17 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       const Tile t = tiles.get(i);
       const uint32_t ph = i & 1;
       bool valid = row < t.nrows;
-      if (valid && t.seg == 0 && idx_q != nullptr) {
-        const int e = idx_q[t.row0 + row];
-        valid = e >= 0 && e < p.N;
+      if (valid && t.seg == 0) {
+        const int e = idx_q != nullptr ? idx_q[t.row0 + row] : t.row0 + row;
+        if (idx_q != nullptr) valid = e >= 0 && e < p.N;
+        if (p.check) {
+          unsigned int k = idx_q != nullptr ? entry_check(e, t_pos, p.rate, p.N) : 0u;
+          if (valid && p.bt) {
+            const int blk = p.bt[(long long)q * p.bt_stride + e / p.rpb];
+            if (blk < 0 || blk >= p.pool_blocks) k |= kIdxBlock;
+          }
+          if (k) atomicOr(&g_mqa_tc_error, k << 1);
+        }
       }
       if (i + 1 < nt) gather_rows(i + 1, y);  // index loads overlap the wait below
       float sv[32];
@@ -679,6 +689,8 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   a.bt = p.bt;
   a.bt_stride = p.bt_stride;
   a.rpb = p.rpb > 0 ? p.rpb : 1;
+  a.pool_blocks = p.bt ? p.pool_rows / a.rpb : 0;
+  a.check = p.check;
   a.ws_o = pl.splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
   a.ws_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) + (size_t)p.Tq * pl.splits * kH * kC)
                           : nullptr;

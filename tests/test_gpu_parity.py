@@ -2,7 +2,7 @@
 
 Sizes: the tiny shape (c=64, 4 heads) over several tiles with ragged tails,
 and the full-size decode workloads with the oracle run per request.  The
-64K-token prefill is covered in test_gpu_prefill_full.py on sampled queries.
+64K-token prefill is covered in test_gpu_prefill.py on sampled queries.
 """
 
 import numpy as np
