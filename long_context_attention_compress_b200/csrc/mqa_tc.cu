@@ -18,10 +18,13 @@
 // each) with their own full/empty barriers: PV runs block by block and
 // releases each block as soon as its MMAs finish, so the next tile's loads of
 // that block, and its QK^T over it, start while PV is still running.
-// Dense rows arrive as 2-D TMA tiles.  Selected rows arrive as tile::gather4
-// loads (four 128-byte row pieces each), issued by two lanes of each of the
-// eight compute warps: the TMA issue rate is per warp, and sixteen issuers in
-// eight warps gather about three times faster than one warp.
+// Dense rows arrive as 2-D TMA tiles.  Selected rows of column blocks 0-1
+// arrive as tile::gather4 loads (four 128-byte row pieces each), one per issuer
+// lane, eight lanes in each of the eight compute warps (the TMA issue rate is
+// per warp); those of blocks 2-3 are copied by all compute threads with 16-byte
+// cp.async (the swizzle applied by hand), which roughly halves the time the
+// TMA unit alone needs for a gathered tile.  The query's output leaves as one
+// contiguous 64 KiB bulk copy staged in the free tile buffer.
 //   warp 0     MMA issuer (and TMEM owner)
 //   warps 1-8  two per TMEM lane quarter (32 rows of S^T), each owning 32 of
 //              the 64 heads: per-head tile maxima by a warp reduce-scatter plus
@@ -32,7 +35,7 @@
 //              next tile; the final epilogue.
 // Row sums l_h are warp reduce-scatter sums of exactly the bf16 P_hi + P_lo
 // that PV multiplies (kept per warp across tiles, rescaled with O).
-// TMEM: S^T 64 columns, O^T 4 blocks x 64.
+// TMEM: S^T 64 columns, O^T 3 blocks x 128 (P_hi and P_lo products apart) + 1 x 64.
 
 #include <cudaTypedefs.h>
 
@@ -52,8 +55,18 @@ constexpr int kC = 512;
 constexpr int kH = 64;
 constexpr int kChunks = kC / 64;
 constexpr int kBlocks = 4;                           // 128-dim column blocks
-constexpr int kIssueLanes = 2;                       // gather issuers per compute warp
-constexpr int kGroupsPerIssuer = kRows / 4 / (kCompute * kIssueLanes);  // 4-row groups per issuer
+constexpr int kIssueLanes = 8;                       // gather issuers per compute warp
+// A column block of a tile is 64 gathers of four 128-byte row pieces: (4-row group,
+// 64-dim chunk) slots, dealt round-robin to the issuer lanes of all compute warps.
+constexpr int kSlots = kRows / 4 * 2;
+constexpr int kSlotsPerIssuer = kSlots / (kCompute * kIssueLanes);
+// Column blocks whose selected rows are copied by the compute threads themselves
+// (16-byte cp.async, the 128-byte swizzle applied by hand) instead of the TMA
+// unit: the TMA unit gathers about 36 bytes per clock, so a tile of 128 KiB
+// takes longer than the PV it overlaps; the two paths together halve that.
+constexpr unsigned kLsuBlocks = 0xCu;  // blocks 2 and 3
+__host__ __device__ constexpr bool lsu_block(int b) { return ((kLsuBlocks >> b) & 1u) != 0; }
+constexpr int kLsuRows = 4;            // rows per lane and block (16 rows per warp, 8 lanes per row)
 constexpr uint32_t kQBytes = kH * kC * 2;            // 64 KiB
 constexpr uint32_t kQChunk = kH * 128;               // 8 KiB
 constexpr uint32_t kKvChunk = kRows * 128;           // 16 KiB
@@ -62,8 +75,18 @@ constexpr uint32_t kBlockBytes = 2 * kKvChunk;       // 32 KiB
 constexpr uint32_t kPBytes = kRows * kH * 2;         // 16 KiB per P term
 constexpr uint32_t kOffQ = 0, kOffKv = kQBytes, kOffP = kOffKv + kKvBytes, kOffBars = kOffP + 2 * kPBytes;
 constexpr uint32_t kColS = 0, kColO = 64, kTmemCols = 512;
+// O^T column blocks.  Blocks 0-2 keep the P_hi and P_lo products apart (128
+// columns, hi then lo: one N = 128 MMA per K-step reads the V^T tile once for
+// both terms); block 3 accumulates both terms in 64 columns (two N = 64 MMAs).
+// TMEM: S^T 64 + 3 x 128 + 64 = 512 columns.
+constexpr int kWideBlocks = 3;
+__host__ __device__ constexpr bool wide_block(int b) { return b < kWideBlocks; }
+__host__ __device__ constexpr uint32_t col_o(int b) {
+  return kColO + (b < kWideBlocks ? b * 2 * kH : kWideBlocks * 2 * kH + (b - kWideBlocks) * kH);
+}
+static_assert(col_o(kBlocks - 1) + kH == kTmemCols, "TMEM columns");
 constexpr float kRescaleLog2 = 8.f;
-static_assert(kGroupsPerIssuer * kCompute * kIssueLanes * 4 == kRows, "issuers cover the tile");
+static_assert(kSlotsPerIssuer * kCompute * kIssueLanes == kSlots, "issuers cover the tile");
 
 struct __align__(16) Bars {
   // float arrays first: mref is read with 16-byte vector loads
@@ -186,6 +209,8 @@ struct MqaTcParams {
   int rpb;
   long long pool_blocks;      // blocks of the pool the block table points into
   int check;                  // record entry_check failures (bits << 1 of the error word)
+  const bf16* kvg;            // base of the gathered-row map (rows of kC elements)
+  long long kvg_rows;         // its rows (a copy never reads outside them)
 };
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
@@ -216,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
   if (threadIdx.x == 0) {
     tc::mbar_init(&bars->qfull, 1);
     for (int b = 0; b < kBlocks; ++b) {
-      tc::mbar_init(&bars->kvfull[b], 1);
+      tc::mbar_init(&bars->kvfull[b], lsu_block(b) ? kCompute : 1);
       tc::mbar_init(&bars->kvempty[b], 1);
     }
     tc::mbar_init(&bars->sfull, 1);
@@ -249,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     if (lane == 0) {
       constexpr uint32_t id_qk = tc::idesc_bf16_f32(kRows, kH, false, false);
       constexpr uint32_t id_pv = tc::idesc_bf16_f32(128, kH, true, true);
+      constexpr uint32_t id_pv2 = tc::idesc_bf16_f32(128, 2 * kH, true, true);  // B = [P_hi | P_lo]
       const uint32_t q_base = tc::smem_u32(base + kOffQ), kv_base = tc::smem_u32(base + kOffKv),
                      p_base = tc::smem_u32(base + kOffP);
       // Descriptors are built once; each K-step only adds a compile-time
@@ -287,8 +313,13 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
             const uint32_t koff = (kk * 2048) >> 4;
             const uint32_t first = kk > 0 ? 1u : acc0;
             const uint64_t ad = v_desc0 + (((2 * b) * kKvChunk) >> 4) + koff;
-            tc::mma_bf16(tmem + kColO + b * kH, ad, p_hi0 + koff, id_pv, first);
-            tc::mma_bf16(tmem + kColO + b * kH, ad, p_lo0 + koff, id_pv, 1u);
+            if (wide_block(b)) {
+              // N = 128: the P_lo columns are the next 64-column block of the operand (LBO)
+              tc::mma_bf16(tmem + col_o(b), ad, p_hi0 + koff, id_pv2, first);
+            } else {
+              tc::mma_bf16(tmem + col_o(b), ad, p_hi0 + koff, id_pv, first);
+              tc::mma_bf16(tmem + col_o(b), ad, p_lo0 + koff, id_pv, 1u);
+            }
           }
           tc::mma_commit(&bars->kvempty[b]);  // this block's columns of the tile may be reloaded
         }
@@ -307,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     const int st = cw * 32 + lane;                 // 0..255 within the compute group
     const uint32_t lanebase = (uint32_t)(quarter * 32) << 16;
     const bool issuer = lane < kIssueLanes;
-    const int g0 = cw * kIssueLanes + lane;        // first 4-row group of this issuer
+    const int g0 = cw * kIssueLanes + lane;        // first gather slot of this issuer
     // decode: request q's cache and window block; prefill: one sequence whose
     // window is the raw token rows [max(0, t - n_win + 1), t]
     const long long kv_row_base = p.prefill ? 0ll : (long long)q * p.kv_rows_stride;
@@ -315,43 +346,85 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     const int win_row0 = p.prefill ? max(0, t_pos - p.n_win + 1) : 0;
     int loaded = 0;  // tiles whose loads were issued (thread st == 0 drains them)
 
-    // Rows of tile j this issuer gathers (map rows; invalid slots read the request's row 0,
-    // masked by the softmax).
-    // With paged entries every entry row is gathered: selected rows (idx) or the
-    // dense rows t.row0 + r, translated through the request's block table.
+    // Entries of tile j this issuer gathers (issuer lanes only; 0 elsewhere).  They
+    // are loaded one tile ahead of their use so that no global-load latency lies
+    // on the path from one tile to the next.
     const int32_t* bt_q = p.bt ? p.bt + (long long)q * p.bt_stride : nullptr;
-    auto gather_rows = [&](int j, int (&y)[4 * kGroupsPerIssuer]) {
+    auto load_entries = [&](int j, int (&e)[4 * kSlotsPerIssuer]) {
       const Tile t = tiles.get(j);
 #pragma unroll
-      for (int gg = 0; gg < kGroupsPerIssuer; ++gg) {
+      for (int gg = 0; gg < kSlotsPerIssuer; ++gg) {
 #pragma unroll
         for (int r4 = 0; r4 < 4; ++r4) {
-          const int r = 4 * (g0 + gg * kCompute * kIssueLanes) + r4;
-          int e = 0;
-          if (t.seg == 0 && r < t.nrows) e = idx_q != nullptr ? idx_q[t.row0 + r] : t.row0 + r;
-          if (e < 0 || e >= p.N) e = 0;
-          y[4 * gg + r4] = bt_q ? bt_q[e / p.rpb] * p.rpb + e % p.rpb : (int)(kv_row_base + e);
+          const int r = 4 * ((g0 + gg * kCompute * kIssueLanes) >> 1) + r4;
+          int v = 0;
+          if (issuer && t.seg == 0 && r < t.nrows) v = idx_q != nullptr ? idx_q[t.row0 + r] : t.row0 + r;
+          e[4 * gg + r4] = v;
         }
       }
     };
+    // Map rows of those entries (invalid slots read the request's row 0, masked by
+    // the softmax).  With paged entries every entry row is gathered: selected rows
+    // (idx) or the dense rows, translated through the request's block table.
+    auto rows_of = [&](const auto& e, auto& y) {
+#pragma unroll
+      for (int k = 0; k < (int)(sizeof(e) / sizeof(e[0])); ++k) {
+        int v = e[k];
+        if (v < 0 || v >= p.N) v = 0;
+        y[k] = bt_q ? bt_q[v / p.rpb] * p.rpb + v % p.rpb : (int)(kv_row_base + v);
+      }
+    };
+    // Entries of the rows this lane copies in the cp.async blocks: rows
+    // 16 cw + 4 k + lane / 8 (k < 4), 16-byte unit lane % 8 of each 128-byte piece.
+    auto load_lsu_entries = [&](int j, int (&e)[kLsuRows]) {
+      const Tile t = tiles.get(j);
+#pragma unroll
+      for (int k = 0; k < kLsuRows; ++k) {
+        const int r = 16 * cw + 4 * k + (lane >> 3);
+        int v = 0;
+        if (t.seg == 0 && r < t.nrows) v = idx_q != nullptr ? idx_q[t.row0 + r] : t.row0 + r;
+        e[k] = v;
+      }
+    };
+    // The entry of this thread's row of tile j (its validity), also loaded a tile ahead.
+    auto row_entry = [&](int j) -> int {
+      const Tile t = tiles.get(j);
+      if (row >= t.nrows || t.seg != 0) return 0;
+      return idx_q != nullptr ? idx_q[t.row0 + row] : t.row0 + row;
+    };
     // Issue the loads of tile j, block by block, each once PV of the previous
     // tile has released it.  Returns false on a failed wait (warp-uniform).
-    auto issue_tile = [&](int j, const int (&y)[4 * kGroupsPerIssuer]) -> bool {
+    auto issue_tile = [&](int j, const int (&y)[4 * kSlotsPerIssuer], const int (&ly)[kLsuRows]) -> bool {
       const Tile t = tiles.get(j);
       const bool gathered = t.seg == 0 && (idx_q != nullptr || bt_q != nullptr);
       for (int b = 0; b < kBlocks; ++b) {
         if (!tc::warp_wait(&bars->kvempty[b], (j & 1) ^ 1, abort)) return false;
-        if (st == 0) tc::mbar_arrive_expect_tx(&bars->kvfull[b], kBlockBytes);
         unsigned char* dst = base + kOffKv + 2 * b * kKvChunk;
+        if (gathered && lsu_block(b)) {
+          // eight 16-byte copies per lane: (row group k, chunk c), swizzled as TMA would
+          const int u = lane & 7;
+#pragma unroll
+          for (int k = 0; k < kLsuRows; ++k) {
+            const int r = 16 * cw + 4 * k + (lane >> 3);
+            const long long mr = (ly[k] >= 0 && ly[k] < p.kvg_rows) ? ly[k] : 0;
+            const bf16* src = p.kvg + mr * kC + 2 * b * 64 + u * 8;
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+              tc::cp_async16(tc::smem_u32(dst + c * kKvChunk + r * 128 + ((u ^ (r & 7)) << 4)), src + c * 64, 16);
+          }
+          tc::cp_async_commit();
+          continue;
+        }
+        if (st == 0) tc::mbar_arrive_expect_tx(&bars->kvfull[b], kBlockBytes);
+        else if (lsu_block(b) && lane == 0) tc::mbar_arrive(&bars->kvfull[b]);  // the other warps' arrivals
         if (gathered) {
           if (issuer) {
 #pragma unroll
-            for (int gg = 0; gg < kGroupsPerIssuer; ++gg) {
-              const int g = g0 + gg * kCompute * kIssueLanes;
-#pragma unroll
-              for (int c = 0; c < 2; ++c)
-                tc::tma_gather4(dst + c * kKvChunk + g * 512, &tm_kvg, &bars->kvfull[b], (2 * b + c) * 64,
-                                y[4 * gg], y[4 * gg + 1], y[4 * gg + 2], y[4 * gg + 3]);
+            for (int gg = 0; gg < kSlotsPerIssuer; ++gg) {
+              const int slot = g0 + gg * kCompute * kIssueLanes;
+              const int g = slot >> 1, c = slot & 1;
+              tc::tma_gather4(dst + c * kKvChunk + g * 512, &tm_kvg, &bars->kvfull[b], (2 * b + c) * 64,
+                              y[4 * gg], y[4 * gg + 1], y[4 * gg + 2], y[4 * gg + 3]);
             }
           }
         } else if (st == 0) {
@@ -367,6 +440,19 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
         }
         __syncwarp();
       }
+      if (gathered) {
+        // The copies of each cp.async block complete in order; make them visible to
+        // the tensor core (async proxy) and arrive once per warp.
+        static_assert(kLsuBlocks == 0xCu, "completion order below");
+        tc::cp_async_wait<1>();
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars->kvfull[2]);
+        tc::cp_async_wait<0>();
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars->kvfull[3]);
+      }
       return true;
     };
 
@@ -377,18 +463,39 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     // P[row, 32 hsel + l] (exactly the bf16 P_hi + P_lo that PV multiplies), over
     // all tiles so far, relative to the running maxima.
     float lw = 0.f;
-    int y[4 * kGroupsPerIssuer];
+    int y[4 * kSlotsPerIssuer];   // map rows of the next tile to issue
+    int en[4 * kSlotsPerIssuer];  // entries of the tile after it (loads in flight)
+    int ly[kLsuRows], le[kLsuRows];  // the same for this lane's cp.async rows
+    int ev = 0;                    // entry of this thread's row in the current tile
     if (nt > 0) {
-      gather_rows(0, y);
-      failed = !issue_tile(0, y);
+      load_entries(0, en);
+      load_lsu_entries(0, le);
+      ev = row_entry(0);
+      rows_of(en, y);
+      rows_of(le, ly);
+      failed = !issue_tile(0, y, ly);
       if (!failed) loaded = 1;
+      if (nt > 1) {
+        load_entries(1, en);
+        load_lsu_entries(1, le);
+      }
     }
     for (int i = 0; i < nt; ++i) {
       const Tile t = tiles.get(i);
       const uint32_t ph = i & 1;
       bool valid = row < t.nrows;
+      const int e_row = ev;
+      if (i + 1 < nt) {
+        ev = row_entry(i + 1);
+        rows_of(en, y);  // entries loaded during the previous tile
+        rows_of(le, ly);
+        if (i + 2 < nt) {
+          load_entries(i + 2, en);
+          load_lsu_entries(i + 2, le);
+        }
+      }
       if (valid && t.seg == 0) {
-        const int e = idx_q != nullptr ? idx_q[t.row0 + row] : t.row0 + row;
+        const int e = e_row;
         if (idx_q != nullptr) valid = e >= 0 && e < p.N;
         if (p.check) {
           unsigned int k = idx_q != nullptr ? entry_check(e, t_pos, p.rate, p.N) : 0u;
@@ -399,7 +506,6 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
           if (k) atomicOr(&g_mqa_tc_error, k << 1);
         }
       }
-      if (i + 1 < nt) gather_rows(i + 1, y);  // index loads overlap the wait below
       float sv[32];
       bool need = false;  // a score above its head's running maximum + 2^8 (or the first valid one)
       if (!failed) failed = !tc::warp_wait(&bars->sfull, ph, abort);
@@ -462,8 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
           // O^T holds the sums up to tile i-1: scale column h by alpha[h]
           tc::fence_after_sync();
 #pragma unroll 1
-          for (int blk = 0; blk < 4; ++blk) {
-            const uint32_t ta = tmem + lanebase + kColO + blk * kH + 32 * hsel;
+          for (int part = 0; part < kBlocks + kWideBlocks; ++part) {
+            const int blk = part < kBlocks ? part : part - kBlocks;  // then the lo halves of the wide blocks
+            const uint32_t ta = tmem + lanebase + col_o(blk) + (part < kBlocks ? 0u : (uint32_t)kH) + 32 * hsel;
             uint32_t v[32];
             tc::tmem_ld32(ta, v);
             tc::tmem_ld_wait();
@@ -508,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       lw += warp_sum32(sv, lane);
       // next tile's rows, block by block as PV(i) releases them
       if (!failed && i + 1 < nt) {
-        if (issue_tile(i + 1, y)) loaded = i + 2;
+        if (issue_tile(i + 1, y, ly)) loaded = i + 2;
         else failed = true;
       }
     }
@@ -519,6 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     bars->red[quarter][32 * hsel + lane] = lw;
     bool ok = !tc::named_bar_or(1, 32 * kCompute, failed || *abort);
     if (ok && nt > 0) ok = tc::warp_wait(&bars->odone, (nt - 1) & 1, abort);
+    // every compute warp takes the same branch below (the unsplit path has a barrier)
+    ok = !tc::named_bar_or(1, 32 * kCompute, !ok);
     if (ok) {
       tc::fence_after_sync();
       uint32_t lv[32];
@@ -534,14 +643,33 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       }
       const int dim_lane = quarter * 32 + lane;
       if (p.splits == 1) {
-        bf16* op = p.out + (long long)q * kH * kC + (long long)(32 * hsel) * kC;
+        // The output leaves as one contiguous 64 KiB block (the query's [head][dim]
+        // rows are adjacent): bf16 values are staged in the tile buffer, which the
+        // last PV has released and no load refills, then sent by bulk copies.
+        bf16* stage = reinterpret_cast<bf16*>(base + kOffKv) + (32 * hsel) * kC;
         const int rope0 = kC - p.rope_dims;
+        float inv[32];
+#pragma unroll
+        for (int h = 0; h < 32; ++h) {
+          const float l = __uint_as_float(lv[h]);
+          inv[h] = (nt > 0 && l > 0.f) ? __frcp_rn(l) : 0.f;
+        }
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
           uint32_t v[32];
           if (nt > 0) {
-            tc::tmem_ld32(tmem + lanebase + kColO + mb * kH + 32 * hsel, v);
+            tc::tmem_ld32(tmem + lanebase + col_o(mb) + 32 * hsel, v);
+            if (wide_block(mb)) {
+              uint32_t w[32];
+              tc::tmem_ld32(tmem + lanebase + col_o(mb) + kH + 32 * hsel, w);
+              tc::tmem_ld_wait();
+#pragma unroll
+              for (int h = 0; h < 32; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) + __uint_as_float(w[h]));
+            }
             tc::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int h = 0; h < 32; ++h) v[h] = 0u;
           }
           const int d = mb * 128 + dim_lane;
           // partial-RoPE output rotation by -t: channel d pairs with d ^ 1, the
@@ -555,11 +683,20 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
           }
 #pragma unroll
           for (int h = 0; h < 32; ++h) {
-            const float l = __uint_as_float(lv[h]);
-            float o = (nt > 0 && l > 0.f) ? __uint_as_float(v[h]) / l : 0.f;
+            float o = inv[h] != 0.f ? __uint_as_float(v[h]) * inv[h] : 0.f;
             if (rot) o = fmaf(o, rc, __shfl_xor_sync(0xffffffffu, o, 1) * rsx);
-            op[h * kC + d] = __float2bfloat16_rn(o);
+            stage[h * kC + d] = __float2bfloat16_rn(o);
           }
+        }
+        tc::fence_proxy_async_smem();
+        tc::named_bar(1, 32 * kCompute);
+        if (st == 0) {
+          char* dst = reinterpret_cast<char*>(p.out + (long long)q * kH * kC);
+          const uint32_t src = tc::smem_u32(base + kOffKv);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tc::bulk_store(dst + c * (kQBytes / 4), src + c * (kQBytes / 4), kQBytes / 4);
+          tc::bulk_commit();
+          tc::bulk_wait_read_all();
         }
       } else {
         float* wo = p.ws_o + ((long long)q * p.splits + sp) * kH * kC + (long long)(32 * hsel) * kC;
@@ -567,7 +704,14 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
         for (int mb = 0; mb < 4; ++mb) {
           uint32_t v[32];
           if (nt > 0) {
-            tc::tmem_ld32(tmem + lanebase + kColO + mb * kH + 32 * hsel, v);
+            tc::tmem_ld32(tmem + lanebase + col_o(mb) + 32 * hsel, v);
+            if (wide_block(mb)) {
+              uint32_t w[32];
+              tc::tmem_ld32(tmem + lanebase + col_o(mb) + kH + 32 * hsel, w);
+              tc::tmem_ld_wait();
+#pragma unroll
+              for (int h = 0; h < 32; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) + __uint_as_float(w[h]));
+            }
             tc::tmem_ld_wait();
           }
           const int d = mb * 128 + dim_lane;
@@ -585,6 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       }
     }
     // drain: every block load issued has landed before the CTA may exit
+    tc::cp_async_wait<0>();
     if (st == 0 && loaded > 0) {
       const int j = loaded - 1;
       for (int b = 0; b < kBlocks; ++b)
@@ -691,6 +836,8 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   a.rpb = p.rpb > 0 ? p.rpb : 1;
   a.pool_blocks = p.bt ? p.pool_rows / a.rpb : 0;
   a.check = p.check;
+  a.kvg = reinterpret_cast<const bf16*>(kv_base);
+  a.kvg_rows = (long long)kvd[1];
   a.ws_o = pl.splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
   a.ws_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) + (size_t)p.Tq * pl.splits * kH * kC)
                           : nullptr;
