@@ -18,13 +18,13 @@
 // each) with their own full/empty barriers: PV runs block by block and
 // releases each block as soon as its MMAs finish, so the next tile's loads of
 // that block, and its QK^T over it, start while PV is still running.
-// Dense rows arrive as 2-D TMA tiles.  Selected rows of column blocks 0-1
-// arrive as tile::gather4 loads (four 128-byte row pieces each), one per issuer
-// lane, eight lanes in each of the eight compute warps (the TMA issue rate is
-// per warp); those of blocks 2-3 are copied by all compute threads with 16-byte
-// cp.async (the swizzle applied by hand), which roughly halves the time the
-// TMA unit alone needs for a gathered tile.  The query's output leaves as one
-// contiguous 64 KiB bulk copy staged in the free tile buffer.
+// Dense rows arrive as 3-D TMA tiles.  Selected (gathered) rows are copied by
+// the compute threads with 16-byte cp.async, the 128-byte swizzle applied by
+// hand: the TMA unit gathers only about 36 bytes per clock (tile::gather4 of
+// 128-byte row pieces), less than the tile rate PV sustains, while the
+// threads' copies keep up; each column block is signalled as soon as its
+// copies have landed.  The query's output leaves as one contiguous 64 KiB bulk
+// copy staged in the free tile buffer.
 //   warp 0     MMA issuer (and TMEM owner)
 //   warps 1-8  two per TMEM lane quarter (32 rows of S^T), each owning 32 of
 //              the 64 heads: per-head tile maxima by a warp reduce-scatter plus
@@ -55,18 +55,9 @@ constexpr int kC = 512;
 constexpr int kH = 64;
 constexpr int kChunks = kC / 64;
 constexpr int kBlocks = 4;                           // 128-dim column blocks
-constexpr int kIssueLanes = 8;                       // gather issuers per compute warp
-// A column block of a tile is 64 gathers of four 128-byte row pieces: (4-row group,
-// 64-dim chunk) slots, dealt round-robin to the issuer lanes of all compute warps.
-constexpr int kSlots = kRows / 4 * 2;
-constexpr int kSlotsPerIssuer = kSlots / (kCompute * kIssueLanes);
-// Column blocks whose selected rows are copied by the compute threads themselves
-// (16-byte cp.async, the 128-byte swizzle applied by hand) instead of the TMA
-// unit: the TMA unit gathers about 36 bytes per clock, so a tile of 128 KiB
-// takes longer than the PV it overlaps; the two paths together halve that.
-constexpr unsigned kLsuBlocks = 0xCu;  // blocks 2 and 3
-__host__ __device__ constexpr bool lsu_block(int b) { return ((kLsuBlocks >> b) & 1u) != 0; }
-constexpr int kLsuRows = 4;            // rows per lane and block (16 rows per warp, 8 lanes per row)
+// Gathered rows: warp w copies tile rows [16 w, 16 w + 16) of every column block,
+// lane l the 16-byte unit l % 8 of rows 16 w + 4 k + l / 8 (k < 4), both chunks.
+constexpr int kCopyRows = 4;
 constexpr uint32_t kQBytes = kH * kC * 2;            // 64 KiB
 constexpr uint32_t kQChunk = kH * 128;               // 8 KiB
 constexpr uint32_t kKvChunk = kRows * 128;           // 16 KiB
@@ -86,7 +77,7 @@ __host__ __device__ constexpr uint32_t col_o(int b) {
 }
 static_assert(col_o(kBlocks - 1) + kH == kTmemCols, "TMEM columns");
 constexpr float kRescaleLog2 = 8.f;
-static_assert(kSlotsPerIssuer * kCompute * kIssueLanes == kSlots, "issuers cover the tile");
+static_assert(kCompute * 16 == kRows && kCopyRows * 4 == 16, "copies cover the tile");
 
 struct __align__(16) Bars {
   // float arrays first: mref is read with 16-byte vector loads
@@ -215,7 +206,7 @@ struct MqaTcParams {
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-    const __grid_constant__ CUtensorMap tm_kvg, const __grid_constant__ CUtensorMap tm_win, MqaTcParams p) {
+    const __grid_constant__ CUtensorMap tm_win, MqaTcParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base =
       tc::smem_align1024(smem_raw);
@@ -241,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
   if (threadIdx.x == 0) {
     tc::mbar_init(&bars->qfull, 1);
     for (int b = 0; b < kBlocks; ++b) {
-      tc::mbar_init(&bars->kvfull[b], lsu_block(b) ? kCompute : 1);
+      tc::mbar_init(&bars->kvfull[b], kCompute);  // one arrival per compute warp
       tc::mbar_init(&bars->kvempty[b], 1);
     }
     tc::mbar_init(&bars->sfull, 1);
@@ -337,8 +328,6 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     const int row = quarter * 32 + lane;           // S^T row (tile row) / O^T lane
     const int st = cw * 32 + lane;                 // 0..255 within the compute group
     const uint32_t lanebase = (uint32_t)(quarter * 32) << 16;
-    const bool issuer = lane < kIssueLanes;
-    const int g0 = cw * kIssueLanes + lane;        // first gather slot of this issuer
     // decode: request q's cache and window block; prefill: one sequence whose
     // window is the raw token rows [max(0, t - n_win + 1), t]
     const long long kv_row_base = p.prefill ? 0ll : (long long)q * p.kv_rows_stride;
@@ -346,25 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     const int win_row0 = p.prefill ? max(0, t_pos - p.n_win + 1) : 0;
     int loaded = 0;  // tiles whose loads were issued (thread st == 0 drains them)
 
-    // Entries of tile j this issuer gathers (issuer lanes only; 0 elsewhere).  They
-    // are loaded one tile ahead of their use so that no global-load latency lies
-    // on the path from one tile to the next.
     const int32_t* bt_q = p.bt ? p.bt + (long long)q * p.bt_stride : nullptr;
-    auto load_entries = [&](int j, int (&e)[4 * kSlotsPerIssuer]) {
-      const Tile t = tiles.get(j);
-#pragma unroll
-      for (int gg = 0; gg < kSlotsPerIssuer; ++gg) {
-#pragma unroll
-        for (int r4 = 0; r4 < 4; ++r4) {
-          const int r = 4 * ((g0 + gg * kCompute * kIssueLanes) >> 1) + r4;
-          int v = 0;
-          if (issuer && t.seg == 0 && r < t.nrows) v = idx_q != nullptr ? idx_q[t.row0 + r] : t.row0 + r;
-          e[4 * gg + r4] = v;
-        }
-      }
-    };
-    // Map rows of those entries (invalid slots read the request's row 0, masked by
-    // the softmax).  With paged entries every entry row is gathered: selected rows
+    // Map rows of entries (invalid slots read the request's row 0, masked by the
+    // softmax).  With paged entries every entry row is gathered: selected rows
     // (idx) or the dense rows, translated through the request's block table.
     auto rows_of = [&](const auto& e, auto& y) {
 #pragma unroll
@@ -374,12 +347,13 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
         y[k] = bt_q ? bt_q[v / p.rpb] * p.rpb + v % p.rpb : (int)(kv_row_base + v);
       }
     };
-    // Entries of the rows this lane copies in the cp.async blocks: rows
-    // 16 cw + 4 k + lane / 8 (k < 4), 16-byte unit lane % 8 of each 128-byte piece.
-    auto load_lsu_entries = [&](int j, int (&e)[kLsuRows]) {
+    // Entries of the rows this lane copies in tile j (rows 16 cw + 4 k + lane / 8),
+    // loaded one tile ahead of their use so that no global-load latency lies on
+    // the path from one tile to the next.
+    auto load_copy_entries = [&](int j, int (&e)[kCopyRows]) {
       const Tile t = tiles.get(j);
 #pragma unroll
-      for (int k = 0; k < kLsuRows; ++k) {
+      for (int k = 0; k < kCopyRows; ++k) {
         const int r = 16 * cw + 4 * k + (lane >> 3);
         int v = 0;
         if (t.seg == 0 && r < t.nrows) v = idx_q != nullptr ? idx_q[t.row0 + r] : t.row0 + r;
@@ -394,17 +368,17 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     };
     // Issue the loads of tile j, block by block, each once PV of the previous
     // tile has released it.  Returns false on a failed wait (warp-uniform).
-    auto issue_tile = [&](int j, const int (&y)[4 * kSlotsPerIssuer], const int (&ly)[kLsuRows]) -> bool {
+    auto issue_tile = [&](int j, const int (&ly)[kCopyRows]) -> bool {
       const Tile t = tiles.get(j);
       const bool gathered = t.seg == 0 && (idx_q != nullptr || bt_q != nullptr);
+      const int u = lane & 7;
       for (int b = 0; b < kBlocks; ++b) {
         if (!tc::warp_wait(&bars->kvempty[b], (j & 1) ^ 1, abort)) return false;
         unsigned char* dst = base + kOffKv + 2 * b * kKvChunk;
-        if (gathered && lsu_block(b)) {
+        if (gathered) {
           // eight 16-byte copies per lane: (row group k, chunk c), swizzled as TMA would
-          const int u = lane & 7;
 #pragma unroll
-          for (int k = 0; k < kLsuRows; ++k) {
+          for (int k = 0; k < kCopyRows; ++k) {
             const int r = 16 * cw + 4 * k + (lane >> 3);
             const long long mr = (ly[k] >= 0 && ly[k] < p.kvg_rows) ? ly[k] : 0;
             const bf16* src = p.kvg + mr * kC + 2 * b * 64 + u * 8;
@@ -413,45 +387,36 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
               tc::cp_async16(tc::smem_u32(dst + c * kKvChunk + r * 128 + ((u ^ (r & 7)) << 4)), src + c * 64, 16);
           }
           tc::cp_async_commit();
-          continue;
-        }
-        if (st == 0) tc::mbar_arrive_expect_tx(&bars->kvfull[b], kBlockBytes);
-        else if (lsu_block(b) && lane == 0) tc::mbar_arrive(&bars->kvfull[b]);  // the other warps' arrivals
-        if (gathered) {
-          if (issuer) {
-#pragma unroll
-            for (int gg = 0; gg < kSlotsPerIssuer; ++gg) {
-              const int slot = g0 + gg * kCompute * kIssueLanes;
-              const int g = slot >> 1, c = slot & 1;
-              tc::tma_gather4(dst + c * kKvChunk + g * 512, &tm_kvg, &bars->kvfull[b], (2 * b + c) * 64,
-                              y[4 * gg], y[4 * gg + 1], y[4 * gg + 2], y[4 * gg + 3]);
-            }
+          if (b > 0) {
+            // block b-1 has landed: visible to the tensor core (async proxy), one arrival per warp
+            tc::cp_async_wait<1>();
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->kvfull[b - 1]);
           }
-        } else if (st == 0) {
+        } else {
           // 3-D maps (dims, rows, request): rows past the request's own extent read as zeros
+          if (st == 0) {
+            tc::mbar_arrive_expect_tx(&bars->kvfull[b], kBlockBytes);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            if (t.seg == 0)
-              tc::tma_load_3d(dst + c * kKvChunk, &tm_kv, &bars->kvfull[b], (2 * b + c) * 64, t.row0, req);
-            else
-              tc::tma_load_3d(dst + c * kKvChunk, &tm_win, &bars->kvfull[b], (2 * b + c) * 64,
-                              (int)(win_row0 + t.row0), req);
+            for (int c = 0; c < 2; ++c) {
+              if (t.seg == 0)
+                tc::tma_load_3d(dst + c * kKvChunk, &tm_kv, &bars->kvfull[b], (2 * b + c) * 64, t.row0, req);
+              else
+                tc::tma_load_3d(dst + c * kKvChunk, &tm_win, &bars->kvfull[b], (2 * b + c) * 64,
+                                (int)(win_row0 + t.row0), req);
+            }
+          } else if (lane == 0) {
+            tc::mbar_arrive(&bars->kvfull[b]);
           }
+          __syncwarp();
         }
-        __syncwarp();
       }
       if (gathered) {
-        // The copies of each cp.async block complete in order; make them visible to
-        // the tensor core (async proxy) and arrive once per warp.
-        static_assert(kLsuBlocks == 0xCu, "completion order below");
-        tc::cp_async_wait<1>();
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars->kvfull[2]);
         tc::cp_async_wait<0>();
         tc::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars->kvfull[3]);
+        if (lane == 0) tc::mbar_arrive(&bars->kvfull[kBlocks - 1]);
       }
       return true;
     };
@@ -463,22 +428,16 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     // P[row, 32 hsel + l] (exactly the bf16 P_hi + P_lo that PV multiplies), over
     // all tiles so far, relative to the running maxima.
     float lw = 0.f;
-    int y[4 * kSlotsPerIssuer];   // map rows of the next tile to issue
-    int en[4 * kSlotsPerIssuer];  // entries of the tile after it (loads in flight)
-    int ly[kLsuRows], le[kLsuRows];  // the same for this lane's cp.async rows
-    int ev = 0;                    // entry of this thread's row in the current tile
+    int ly[kCopyRows];  // map rows this lane copies in the next tile to load
+    int le[kCopyRows];  // entries of those rows in the tile after it (loads in flight)
+    int ev = 0;         // entry of this thread's row in the current tile
     if (nt > 0) {
-      load_entries(0, en);
-      load_lsu_entries(0, le);
+      load_copy_entries(0, le);
       ev = row_entry(0);
-      rows_of(en, y);
       rows_of(le, ly);
-      failed = !issue_tile(0, y, ly);
+      failed = !issue_tile(0, ly);
       if (!failed) loaded = 1;
-      if (nt > 1) {
-        load_entries(1, en);
-        load_lsu_entries(1, le);
-      }
+      if (nt > 1) load_copy_entries(1, le);
     }
     for (int i = 0; i < nt; ++i) {
       const Tile t = tiles.get(i);
@@ -487,12 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       const int e_row = ev;
       if (i + 1 < nt) {
         ev = row_entry(i + 1);
-        rows_of(en, y);  // entries loaded during the previous tile
-        rows_of(le, ly);
-        if (i + 2 < nt) {
-          load_entries(i + 2, en);
-          load_lsu_entries(i + 2, le);
-        }
+        rows_of(le, ly);  // entries loaded during the previous tile
+        if (i + 2 < nt) load_copy_entries(i + 2, le);
       }
       if (valid && t.seg == 0) {
         const int e = e_row;
@@ -615,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       lw += warp_sum32(sv, lane);
       // next tile's rows, block by block as PV(i) releases them
       if (!failed && i + 1 < nt) {
-        if (issue_tile(i + 1, y, ly)) loaded = i + 2;
+        if (issue_tile(i + 1, ly)) loaded = i + 2;
         else failed = true;
       }
     }
@@ -783,7 +738,7 @@ extern cudaError_t make_tmap_bf16(CUtensorMap* m, const void* ptr, int rank, con
 
 cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream, bool pdl) {
   if (p.Tq == 0) return cudaSuccess;
-  CUtensorMap tm_q, tm_kv, tm_kvg, tm_win;
+  CUtensorMap tm_q, tm_kv, tm_win;
   const uint64_t rstride[1] = {(uint64_t)kC * 2};
   const uint64_t qd[2] = {(uint64_t)kC, (uint64_t)p.Tq * kH};
   cudaError_t e = make_tmap_bf16(&tm_q, p.q, 2, qd, rstride, 64);
@@ -803,10 +758,8 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   const uint64_t kvs3[2] = {(uint64_t)kC * 2, (uint64_t)kv_req_elems * 2};
   e = make_tmap_bf16(&tm_kv, kv_base, 3, kvd3, kvs3, kRows);
   if (e != cudaSuccess) return e;
-  // gathered rows: one 2-D map over every request's rows
-  const uint64_t kvd[2] = {(uint64_t)kC, (uint64_t)((long long)(p.Tq - 1) * kv_rs) + n_kv};
-  e = make_tmap_bf16(&tm_kvg, kv_base, 2, kvd, rstride, 1);
-  if (e != cudaSuccess) return e;
+  // gathered rows: copied by the threads from one range over every request's rows
+  const long long kvg_rows = (long long)(p.Tq - 1) * kv_rs + (long long)n_kv;
   const long long win_rs = prefill ? 0 : p.win_seq_stride / kC;
   const uint64_t wd3[3] = {(uint64_t)kC, prefill ? (uint64_t)p.win_rows : (uint64_t)p.n_win,
                            prefill ? 1ull : (uint64_t)p.Tq};
@@ -837,7 +790,7 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
   a.pool_blocks = p.bt ? p.pool_rows / a.rpb : 0;
   a.check = p.check;
   a.kvg = reinterpret_cast<const bf16*>(kv_base);
-  a.kvg_rows = (long long)kvd[1];
+  a.kvg_rows = kvg_rows;
   a.ws_o = pl.splits > 1 ? reinterpret_cast<float*>(ws) : nullptr;
   a.ws_ml = pl.splits > 1 ? reinterpret_cast<float2*>(reinterpret_cast<float*>(ws) + (size_t)p.Tq * pl.splits * kH * kC)
                           : nullptr;
@@ -845,7 +798,7 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
                            (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   e = launch_pdl(pdl, mqa_decode_tc_kernel, dim3(p.Tq * pl.splits), dim3(kThreads), kSmemBytes, stream, tm_q, tm_kv,
-                 tm_kvg, tm_win, a);
+                 tm_win, a);
   ++g_launch_counter;
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;

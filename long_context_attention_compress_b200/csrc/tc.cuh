@@ -125,6 +125,14 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Wait until at most n (0..3, unrolled by the caller) committed groups are pending.
+__device__ __forceinline__ void cp_async_wait_n(int n) {
+  if (n <= 0) cp_async_wait<0>();
+  else if (n == 1) cp_async_wait<1>();
+  else if (n == 2) cp_async_wait<2>();
+  else cp_async_wait<3>();
+}
+
 // ---- bulk shared -> global copies (no tensor map) ---------------------------------
 // Both addresses 16-byte aligned, bytes a multiple of 16; tracked by the issuing
 // thread's bulk groups.
