@@ -29,8 +29,8 @@
 //   warps 1-8  two per TMEM lane quarter (32 rows of S^T), each owning 32 of
 //              the 64 heads: per-head tile maxima by a warp reduce-scatter plus
 //              a 4-way shared-memory step; P = 2^(s - m) written as two bf16
-//              terms P_hi + P_lo (MN-major B operands of PV, so P keeps ~16
-//              significant bits); lazy rescale of the TMEM accumulators (only
+//              terms P_hi + P_lo, each truncated (MN-major B operands of PV; P
+//              keeps ~15 significant bits); lazy rescale of the TMEM accumulators (only
 //              when a head's maximum grows by more than 2^8); the loads of the
 //              next tile; the final epilogue.
 // Row sums l_h are warp reduce-scatter sums of exactly the bf16 P_hi + P_lo
@@ -513,10 +513,9 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
         }
         if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
       }
-      // Wait for PV(i-1) on every tile, in order: the odone barrier completes once per
-      // tile, and a parity wait is only unambiguous while the waiter is at most one
-      // phase behind (PV(i) cannot complete before this group publishes P(i)).
-      if (i > 0 && !tc::warp_wait(&bars->odone, (i - 1) & 1, abort)) failed = true;
+      // PV(i-1) has completed here: the MMA thread issued it before QK(i), and the
+      // commit that signalled S(i) tracks every MMA issued before it.  So the O^T
+      // accumulators may be rescaled and the P buffers rewritten without a wait.
       if (full) {
         lw *= bars->alpha[32 * hsel + lane];
         if (!failed && bars->rescale && i > 0) {
@@ -555,10 +554,15 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
           const float m0 = mm[2 * j], m1 = mm[2 * j + 1];
           const float p0 = (m0 == neg_inf()) ? 0.f : fast_exp2(sv[h] - m0);
           const float p1 = (m1 == neg_inf()) ? 0.f : fast_exp2(sv[h + 1] - m1);
-          wh[j] = pack_bf16x2(p0, p1);
-          wl[j] = pack_bf16x2(p0 - bf16_lo(wh[j]), p1 - bf16_hi(wh[j]));
-          sv[h] = bf16_lo(wh[j]) + bf16_lo(wl[j]);  // the probability PV uses (exact in f32)
-          sv[h + 1] = bf16_hi(wh[j]) + bf16_hi(wl[j]);
+          // P_hi = p truncated to bf16, P_lo = the (exact) remainder truncated to bf16:
+          // relative error below 2^-14, by integer masks instead of conversions
+          const uint32_t h0 = __float_as_uint(p0) & 0xffff0000u, h1 = __float_as_uint(p1) & 0xffff0000u;
+          const uint32_t l0 = __float_as_uint(p0 - __uint_as_float(h0)) & 0xffff0000u;
+          const uint32_t l1 = __float_as_uint(p1 - __uint_as_float(h1)) & 0xffff0000u;
+          wh[j] = __byte_perm(h0, h1, 0x7632);
+          wl[j] = __byte_perm(l0, l1, 0x7632);
+          sv[h] = __uint_as_float(h0) + __uint_as_float(l0);  // the probability PV uses (exact in f32)
+          sv[h + 1] = __uint_as_float(h1) + __uint_as_float(l1);
         }
         const uint32_t sw = (uint32_t)((c ^ (row & 7)) << 4);
         *reinterpret_cast<uint4*>(phi + sw) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
