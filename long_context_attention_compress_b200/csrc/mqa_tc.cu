@@ -206,7 +206,7 @@ struct MqaTcParams {
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-    const __grid_constant__ CUtensorMap tm_win, MqaTcParams p) {
+    const __grid_constant__ CUtensorMap tm_win, const __grid_constant__ CUtensorMap tm_out, MqaTcParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* base =
       tc::smem_align1024(smem_raw);
@@ -602,17 +602,19 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       }
       const int dim_lane = quarter * 32 + lane;
       if (p.splits == 1) {
-        // The output leaves as one contiguous 64 KiB block (the query's [head][dim]
-        // rows are adjacent): bf16 values are staged in the tile buffer, which the
-        // last PV has released and no load refills, then sent by bulk copies.
-        bf16* stage = reinterpret_cast<bf16*>(base + kOffKv) + (32 * hsel) * kC;
+        // The output leaves block by block as TMA tensor stores (a map of the same
+        // shape as the queries'): each 128-dim block is staged as two 128B-swizzled
+        // [64 heads x 64 dims] boxes in the tile buffer, which the last PV has
+        // released and no load refills, and its store overlaps the next block's staging.
         const int rope0 = kC - p.rope_dims;
         float inv[32];
 #pragma unroll
         for (int h = 0; h < 32; ++h) {
           const float l = __uint_as_float(lv[h]);
-          inv[h] = (nt > 0 && l > 0.f) ? __frcp_rn(l) : 0.f;
+          inv[h] = (nt > 0 && l > 0.f) ? __fdividef(1.f, l) : 0.f;
         }
+        const int dl = dim_lane & 63;                    // dim within its 64-dim chunk
+        const uint32_t ubyte = (uint32_t)(dl * 2);       // byte within the 128-byte row
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
           uint32_t v[32];
@@ -631,6 +633,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
             for (int h = 0; h < 32; ++h) v[h] = 0u;
           }
           const int d = mb * 128 + dim_lane;
+          // chunk 2 mb + dim_lane / 64 of the output, rows = heads
+          unsigned char* box = base + kOffKv + (2 * mb + (dim_lane >> 6)) * kQChunk;
           // partial-RoPE output rotation by -t: channel d pairs with d ^ 1, the
           // neighbouring TMEM lane (lane ^ 1 of this warp); whole warps take the branch
           const bool rot = p.rope_dims > 0 && mb * 128 + quarter * 32 + 31 >= rope0;
@@ -644,19 +648,20 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
           for (int h = 0; h < 32; ++h) {
             float o = inv[h] != 0.f ? __uint_as_float(v[h]) * inv[h] : 0.f;
             if (rot) o = fmaf(o, rc, __shfl_xor_sync(0xffffffffu, o, 1) * rsx);
-            stage[h * kC + d] = __float2bfloat16_rn(o);
+            const int hh = 32 * hsel + h;
+            *reinterpret_cast<bf16*>(box + hh * 128 + ((((ubyte >> 4) ^ (hh & 7)) << 4) | (ubyte & 15))) =
+                __float2bfloat16_rn(o);
+          }
+          tc::fence_proxy_async_smem();
+          tc::named_bar(1, 32 * kCompute);
+          if (st == 0) {
+            for (int c = 0; c < 2; ++c)
+              tc::tma_store_2d(&tm_out, (2 * mb + c) * 64, q * kH,
+                               tc::smem_u32(base + kOffKv + (2 * mb + c) * kQChunk));
+            tc::bulk_commit();
           }
         }
-        tc::fence_proxy_async_smem();
-        tc::named_bar(1, 32 * kCompute);
-        if (st == 0) {
-          char* dst = reinterpret_cast<char*>(p.out + (long long)q * kH * kC);
-          const uint32_t src = tc::smem_u32(base + kOffKv);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tc::bulk_store(dst + c * (kQBytes / 4), src + c * (kQBytes / 4), kQBytes / 4);
-          tc::bulk_commit();
-          tc::bulk_wait_read_all();
-        }
+        if (st == 0) tc::bulk_wait_read_all();
       } else {
         float* wo = p.ws_o + ((long long)q * p.splits + sp) * kH * kC + (long long)(32 * hsel) * kC;
 #pragma unroll 1
@@ -742,10 +747,12 @@ extern cudaError_t make_tmap_bf16(CUtensorMap* m, const void* ptr, int rank, con
 
 cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* ws, cudaStream_t stream, bool pdl) {
   if (p.Tq == 0) return cudaSuccess;
-  CUtensorMap tm_q, tm_kv, tm_win;
+  CUtensorMap tm_q, tm_kv, tm_win, tm_out;
   const uint64_t rstride[1] = {(uint64_t)kC * 2};
   const uint64_t qd[2] = {(uint64_t)kC, (uint64_t)p.Tq * kH};
   cudaError_t e = make_tmap_bf16(&tm_q, p.q, 2, qd, rstride, 64);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_bf16(&tm_out, p.out, 2, qd, rstride, 64);  // unsplit queries store through it
   if (e != cudaSuccess) return e;
   const bool prefill = p.mode == HCA_MODE_PREFILL;
   const long long kv_rs = (prefill || p.bt) ? 0 : p.kv_seq_stride / kC;
@@ -802,7 +809,7 @@ cudaError_t launch_mqa_decode_tc(const MqaProblem& p, const MqaPlan& pl, void* w
                            (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   e = launch_pdl(pdl, mqa_decode_tc_kernel, dim3(p.Tq * pl.splits), dim3(kThreads), kSmemBytes, stream, tm_q, tm_kv,
-                 tm_win, a);
+                 tm_win, tm_out, a);
   ++g_launch_counter;
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;
