@@ -707,16 +707,22 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
             tc::tmem_ld32(taddr + 32, v + 32);
             tc::tmem_ld_wait();
             const float* w = bars->w + j * kHeads;
-            float s0 = 0.f, s1 = 0.f;
+            // eight independent chains (a fixed association, the same for every entry)
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int h = 0; h < kHeads; h += 4) {
-              const float4 wv = *reinterpret_cast<const float4*>(w + h);
-              s0 = fmaf(wv.x, fmaxf(__uint_as_float(v[h]), 0.f), s0);
-              s1 = fmaf(wv.y, fmaxf(__uint_as_float(v[h + 1]), 0.f), s1);
-              s0 = fmaf(wv.z, fmaxf(__uint_as_float(v[h + 2]), 0.f), s0);
-              s1 = fmaf(wv.w, fmaxf(__uint_as_float(v[h + 3]), 0.f), s1);
+            for (int h = 0; h < kHeads; h += 8) {
+              const float4 wa = *reinterpret_cast<const float4*>(w + h);
+              const float4 wb = *reinterpret_cast<const float4*>(w + h + 4);
+              acc[0] = fmaf(wa.x, fmaxf(__uint_as_float(v[h]), 0.f), acc[0]);
+              acc[1] = fmaf(wa.y, fmaxf(__uint_as_float(v[h + 1]), 0.f), acc[1]);
+              acc[2] = fmaf(wa.z, fmaxf(__uint_as_float(v[h + 2]), 0.f), acc[2]);
+              acc[3] = fmaf(wa.w, fmaxf(__uint_as_float(v[h + 3]), 0.f), acc[3]);
+              acc[4] = fmaf(wb.x, fmaxf(__uint_as_float(v[h + 4]), 0.f), acc[4]);
+              acc[5] = fmaf(wb.y, fmaxf(__uint_as_float(v[h + 5]), 0.f), acc[5]);
+              acc[6] = fmaf(wb.z, fmaxf(__uint_as_float(v[h + 6]), 0.f), acc[6]);
+              acc[7] = fmaf(wb.w, fmaxf(__uint_as_float(v[h + 7]), 0.f), acc[7]);
             }
-            sc[jj] = s0 + s1;
+            sc[jj] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
           }
           tc::fence_before_sync();
           __syncwarp();
