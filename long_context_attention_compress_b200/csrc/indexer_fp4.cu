@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
       }
       const int a = it % kFAcc;
       ++it;
-      if (!failed) failed = !tc::mbar_wait(&bars->tfull[a], ((it - 1) / kFAcc) & 1, abort);
+      if (!failed) failed = !tc::warp_wait(&bars->tfull[a], ((it - 1) / kFAcc) & 1, abort);
       if (failed) continue;
       tc::fence_after_sync();
       uint32_t v[kFHeads];

@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
       }
       const int a = it % kAcc;
       ++it;
-      if (!failed) failed = !tc::mbar_wait(&bars->tfull[a], ((it - 1) / kAcc) & 1, abort, spin);
+      if (!failed) failed = !tc::warp_wait(&bars->tfull[a], ((it - 1) / kAcc) & 1, abort, spin);
       if (failed) continue;
       tc::fence_after_sync();
       uint32_t v[kHeads];

@@ -173,8 +173,9 @@ __device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t count, bool p
 // every lane has observed the completed phase (each lane acquires it itself).
 // No lane runs ahead in divergent code: a lane-0 wait followed by a broadcast
 // costs about 400 cycles even on a completed phase, this about 90.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint32_t limit = kSpinLimit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
     if ((i & 255u) == 255u) {
       if (__any_sync(0xffffffffu, *abort != 0)) return false;
