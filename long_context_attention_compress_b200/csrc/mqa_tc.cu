@@ -48,16 +48,16 @@
 namespace hca {
 
 namespace {
-constexpr int kCompute = 8;                          // compute warps
+constexpr int kCompute = 16;                         // compute warps (four per TMEM lane quarter)
 constexpr int kThreads = 32 * (1 + kCompute);
 constexpr int kRows = 128;                           // rows per tile
 constexpr int kC = 512;
 constexpr int kH = 64;
 constexpr int kChunks = kC / 64;
 constexpr int kBlocks = 4;                           // 128-dim column blocks
-// Gathered rows: warp w copies tile rows [16 w, 16 w + 16) of every column block,
-// lane l the 16-byte unit l % 8 of rows 16 w + 4 k + l / 8 (k < 4), both chunks.
-constexpr int kCopyRows = 4;
+// Gathered rows: warp w copies tile rows [8 w, 8 w + 8) of every column block,
+// lane l the 16-byte unit l % 8 of rows 8 w + 4 k + l / 8 (k < 2), both chunks.
+constexpr int kCopyRows = 2;
 constexpr uint32_t kQBytes = kH * kC * 2;            // 64 KiB
 constexpr uint32_t kQChunk = kH * 128;               // 8 KiB
 constexpr uint32_t kKvChunk = kRows * 128;           // 16 KiB
@@ -77,7 +77,9 @@ __host__ __device__ constexpr uint32_t col_o(int b) {
 }
 static_assert(col_o(kBlocks - 1) + kH == kTmemCols, "TMEM columns");
 constexpr float kRescaleLog2 = 8.f;
-static_assert(kCompute * 16 == kRows && kCopyRows * 4 == 16, "copies cover the tile");
+constexpr int kHpt = kH * 4 / kCompute;  // heads per compute thread (16)
+static_assert(kCompute * 8 == kRows && kCopyRows * 4 == 8, "copies cover the tile");
+static_assert(kHpt == 16, "the reductions below are written for 16 heads per thread");
 
 struct __align__(16) Bars {
   // float arrays first: mref is read with 16-byte vector loads
@@ -136,8 +138,8 @@ struct SplitTiles {
 
 // One reduce-scatter step over lane bit O: of the NV values held, keep the
 // half selected by the bit and fold in the partner's copy of that half.
-template <int O, int NV>
-__device__ __forceinline__ void rs_max_step(float (&a)[32], int lane) {
+template <int O, int NV, int SZ>
+__device__ __forceinline__ void rs_max_step(float (&a)[SZ], int lane) {
   const bool hi = (lane & O) != 0;
 #pragma unroll
   for (int j = 0; j < NV / 2; ++j) {
@@ -146,8 +148,8 @@ __device__ __forceinline__ void rs_max_step(float (&a)[32], int lane) {
     a[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, O));
   }
 }
-template <int O, int NV>
-__device__ __forceinline__ void rs_sum_step(float (&a)[32], int lane) {
+template <int O, int NV, int SZ>
+__device__ __forceinline__ void rs_sum_step(float (&a)[SZ], int lane) {
   const bool hi = (lane & O) != 0;
 #pragma unroll
   for (int j = 0; j < NV / 2; ++j) {
@@ -156,23 +158,21 @@ __device__ __forceinline__ void rs_sum_step(float (&a)[32], int lane) {
     a[j] = keep + __shfl_xor_sync(0xffffffffu, send, O);
   }
 }
-// Afterwards lane l holds the warp-wide sum of value l (31 shuffles).
-__device__ __forceinline__ float warp_sum32(float (&a)[32], int lane) {
-  rs_sum_step<16, 32>(a, lane);
+// Afterwards lane l holds the warp-wide sum of value l % 16 (16 shuffles).
+__device__ __forceinline__ float warp_sum16(float (&a)[16], int lane) {
   rs_sum_step<8, 16>(a, lane);
   rs_sum_step<4, 8>(a, lane);
   rs_sum_step<2, 4>(a, lane);
   rs_sum_step<1, 2>(a, lane);
-  return a[0];
+  return a[0] + __shfl_xor_sync(0xffffffffu, a[0], 16);
 }
-// Afterwards lane l holds the warp-wide maximum of value l (31 shuffles).
-__device__ __forceinline__ float warp_max32(float (&a)[32], int lane) {
-  rs_max_step<16, 32>(a, lane);
+// Afterwards lane l holds the warp-wide maximum of value l % 16 (16 shuffles).
+__device__ __forceinline__ float warp_max16(float (&a)[16], int lane) {
   rs_max_step<8, 16>(a, lane);
   rs_max_step<4, 8>(a, lane);
   rs_max_step<2, 4>(a, lane);
   rs_max_step<1, 2>(a, lane);
-  return a[0];
+  return fmaxf(a[0], __shfl_xor_sync(0xffffffffu, a[0], 16));
 }
 }  // namespace
 
@@ -324,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     // --------------------- loads, softmax / correction / epilogue ---------------------
     const int cw = warp - 1;                       // compute warp 0..7
     const int quarter = warp & 3;                  // TMEM lane quarter
-    const int hsel = cw >> 2;                      // heads [32 hsel, 32 hsel + 32)
+    const int hsel = cw >> 2;                      // heads [16 hsel, 16 hsel + 16)
     const int row = quarter * 32 + lane;           // S^T row (tile row) / O^T lane
     const int st = cw * 32 + lane;                 // 0..255 within the compute group
     const uint32_t lanebase = (uint32_t)(quarter * 32) << 16;
@@ -347,14 +347,14 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
         y[k] = bt_q ? bt_q[v / p.rpb] * p.rpb + v % p.rpb : (int)(kv_row_base + v);
       }
     };
-    // Entries of the rows this lane copies in tile j (rows 16 cw + 4 k + lane / 8),
+    // Entries of the rows this lane copies in tile j (rows 8 cw + 4 k + lane / 8),
     // loaded one tile ahead of their use so that no global-load latency lies on
     // the path from one tile to the next.
     auto load_copy_entries = [&](int j, int (&e)[kCopyRows]) {
       const Tile t = tiles.get(j);
 #pragma unroll
       for (int k = 0; k < kCopyRows; ++k) {
-        const int r = 16 * cw + 4 * k + (lane >> 3);
+        const int r = 8 * cw + 4 * k + (lane >> 3);
         int v = 0;
         if (t.seg == 0 && r < t.nrows) v = idx_q != nullptr ? idx_q[t.row0 + r] : t.row0 + r;
         e[k] = v;
@@ -376,10 +376,10 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
         if (!tc::warp_wait(&bars->kvempty[b], (j & 1) ^ 1, abort)) return false;
         unsigned char* dst = base + kOffKv + 2 * b * kKvChunk;
         if (gathered) {
-          // eight 16-byte copies per lane: (row group k, chunk c), swizzled as TMA would
+          // four 16-byte copies per lane: (row group k, chunk c), swizzled as TMA would
 #pragma unroll
           for (int k = 0; k < kCopyRows; ++k) {
-            const int r = 16 * cw + 4 * k + (lane >> 3);
+            const int r = 8 * cw + 4 * k + (lane >> 3);
             const long long mr = (ly[k] >= 0 && ly[k] < p.kvg_rows) ? ly[k] : 0;
             const bf16* src = p.kvg + mr * kC + 2 * b * 64 + u * 8;
 #pragma unroll
@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     // iteration; failures are agreed through bar.red.or before anyone leaves.
     bool failed = false;
     // Row sums: lane l of this warp carries the sum over its quarter's rows of
-    // P[row, 32 hsel + l] (exactly the bf16 P_hi + P_lo that PV multiplies), over
+    // P[row, 16 hsel + l % 16] (exactly the bf16 P_hi + P_lo that PV multiplies), over
     // all tiles so far, relative to the running maxima.
     float lw = 0.f;
     int ly[kCopyRows];  // map rows this lane copies in the next tile to load
@@ -461,20 +461,20 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
           if (k) atomicOr(&g_mqa_tc_error, k << 1);
         }
       }
-      float sv[32];
+      float sv[kHpt];
       bool need = false;  // a score above its head's running maximum + 2^8 (or the first valid one)
       if (!failed) failed = !tc::warp_wait(&bars->sfull, ph, abort);
       if (!failed) {
         tc::fence_after_sync();
-        uint32_t v[32];
-        tc::tmem_ld32(tmem + lanebase + kColS + 32 * hsel, v);
+        uint32_t v[kHpt];
+        tc::tmem_ld16(tmem + lanebase + kColS + kHpt * hsel, v);
         tc::tmem_ld_wait();
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&bars->sempty);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float4 m4 = *reinterpret_cast<const float4*>(bars->mref + 32 * hsel + 4 * c);
+        for (int c = 0; c < kHpt / 4; ++c) {
+          const float4 m4 = *reinterpret_cast<const float4*>(bars->mref + kHpt * hsel + 4 * c);
           const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -494,10 +494,11 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       // every head keeps its running maximum, exactly as the full path would decide.
       const bool full = need_flag[i % 3] != 0;
       if (full) {
-        float tmp[32];
+        float tmp[kHpt];
 #pragma unroll
-        for (int h = 0; h < 32; ++h) tmp[h] = sv[h];
-        bars->red[quarter][32 * hsel + lane] = warp_max32(tmp, lane);
+        for (int h = 0; h < kHpt; ++h) tmp[h] = sv[h];
+        const float tmax = warp_max16(tmp, lane);
+        if (lane < kHpt) bars->red[quarter][kHpt * hsel + lane] = tmax;
         if (tc::named_bar_or(1, 32 * kCompute, failed || *abort)) { failed = true; break; }
         if (st < kH) {
           const int h = st;
@@ -517,20 +518,20 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       // commit that signalled S(i) tracks every MMA issued before it.  So the O^T
       // accumulators may be rescaled and the P buffers rewritten without a wait.
       if (full) {
-        lw *= bars->alpha[32 * hsel + lane];
+        lw *= bars->alpha[kHpt * hsel + (lane & (kHpt - 1))];
         if (!failed && bars->rescale && i > 0) {
           // O^T holds the sums up to tile i-1: scale column h by alpha[h]
           tc::fence_after_sync();
 #pragma unroll 1
           for (int part = 0; part < kBlocks + kWideBlocks; ++part) {
             const int blk = part < kBlocks ? part : part - kBlocks;  // then the lo halves of the wide blocks
-            const uint32_t ta = tmem + lanebase + col_o(blk) + (part < kBlocks ? 0u : (uint32_t)kH) + 32 * hsel;
-            uint32_t v[32];
-            tc::tmem_ld32(ta, v);
+            const uint32_t ta = tmem + lanebase + col_o(blk) + (part < kBlocks ? 0u : (uint32_t)kH) + kHpt * hsel;
+            uint32_t v[kHpt];
+            tc::tmem_ld16(ta, v);
             tc::tmem_ld_wait();
 #pragma unroll
-            for (int h = 0; h < 32; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * bars->alpha[32 * hsel + h]);
-            tc::tmem_st32(ta, v);
+            for (int h = 0; h < kHpt; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * bars->alpha[kHpt * hsel + h]);
+            tc::tmem_st16(ta, v);
           }
           tc::tmem_st_wait();
           tc::fence_before_sync();
@@ -542,8 +543,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       unsigned char* phi = base + kOffP + row * 128;
       unsigned char* plo = phi + kPBytes;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c = 4 * hsel + cc;  // 16-byte unit of the row: heads 8c .. 8c+7
+      for (int cc = 0; cc < kHpt / 8; ++cc) {
+        const int c = (kHpt / 8) * hsel + cc;  // 16-byte unit of the row: heads 8c .. 8c+7
         const float4 ma = *reinterpret_cast<const float4*>(bars->mref + c * 8);
         const float4 mb = *reinterpret_cast<const float4*>(bars->mref + c * 8 + 4);
         const float mm[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
@@ -571,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
       tc::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&bars->pfull);
-      lw += warp_sum32(sv, lane);
+      lw += warp_sum16(sv, lane);
       // next tile's rows, block by block as PV(i) releases them
       if (!failed && i + 1 < nt) {
         if (issue_tile(i + 1, ly)) loaded = i + 2;
@@ -582,20 +583,20 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
     // The four quarters' row-sum partials meet in shared memory.  Every compute
     // thread reaches this barrier (the loop only ends together or normally) and
     // it also settles, for all of them, whether a wait failed on the last tile.
-    bars->red[quarter][32 * hsel + lane] = lw;
+    if (lane < kHpt) bars->red[quarter][kHpt * hsel + lane] = lw;
     bool ok = !tc::named_bar_or(1, 32 * kCompute, failed || *abort);
     if (ok && nt > 0) ok = tc::warp_wait(&bars->odone, (nt - 1) & 1, abort);
     // every compute warp takes the same branch below (the unsplit path has a barrier)
     ok = !tc::named_bar_or(1, 32 * kCompute, !ok);
     if (ok) {
       tc::fence_after_sync();
-      uint32_t lv[32];
+      uint32_t lv[kHpt];
       // an unsplit query's sink logit joins its denominator here (base-2 scale, against the
       // head's running maximum); split queries leave it to the combine
       const bool sink_here = p.sink != nullptr && p.splits == 1;
 #pragma unroll
-      for (int h = 0; h < 32; ++h) {
-        const int hh = 32 * hsel + h;
+      for (int h = 0; h < kHpt; ++h) {
+        const int hh = kHpt * hsel + h;
         float l = (bars->red[0][hh] + bars->red[1][hh]) + (bars->red[2][hh] + bars->red[3][hh]);
         if (sink_here) l += fast_exp2(p.sink[hh] * kLog2e - bars->mref[hh]);
         lv[h] = __float_as_uint(l);
@@ -607,9 +608,9 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
         // [64 heads x 64 dims] boxes in the tile buffer, which the last PV has
         // released and no load refills, and its store overlaps the next block's staging.
         const int rope0 = kC - p.rope_dims;
-        float inv[32];
+        float inv[kHpt];
 #pragma unroll
-        for (int h = 0; h < 32; ++h) {
+        for (int h = 0; h < kHpt; ++h) {
           const float l = __uint_as_float(lv[h]);
           inv[h] = (nt > 0 && l > 0.f) ? __fdividef(1.f, l) : 0.f;
         }
@@ -617,20 +618,20 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
         const uint32_t ubyte = (uint32_t)(dl * 2);       // byte within the 128-byte row
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
-          uint32_t v[32];
+          uint32_t v[kHpt];
           if (nt > 0) {
-            tc::tmem_ld32(tmem + lanebase + col_o(mb) + 32 * hsel, v);
+            tc::tmem_ld16(tmem + lanebase + col_o(mb) + kHpt * hsel, v);
             if (wide_block(mb)) {
-              uint32_t w[32];
-              tc::tmem_ld32(tmem + lanebase + col_o(mb) + kH + 32 * hsel, w);
+              uint32_t w[kHpt];
+              tc::tmem_ld16(tmem + lanebase + col_o(mb) + kH + kHpt * hsel, w);
               tc::tmem_ld_wait();
 #pragma unroll
-              for (int h = 0; h < 32; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) + __uint_as_float(w[h]));
+              for (int h = 0; h < kHpt; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) + __uint_as_float(w[h]));
             }
             tc::tmem_ld_wait();
           } else {
 #pragma unroll
-            for (int h = 0; h < 32; ++h) v[h] = 0u;
+            for (int h = 0; h < kHpt; ++h) v[h] = 0u;
           }
           const int d = mb * 128 + dim_lane;
           // chunk 2 mb + dim_lane / 64 of the output, rows = heads
@@ -645,10 +646,10 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
             rsx = (d & 1) ? -sn : sn;
           }
 #pragma unroll
-          for (int h = 0; h < 32; ++h) {
+          for (int h = 0; h < kHpt; ++h) {
             float o = inv[h] != 0.f ? __uint_as_float(v[h]) * inv[h] : 0.f;
             if (rot) o = fmaf(o, rc, __shfl_xor_sync(0xffffffffu, o, 1) * rsx);
-            const int hh = 32 * hsel + h;
+            const int hh = kHpt * hsel + h;
             *reinterpret_cast<bf16*>(box + hh * 128 + ((((ubyte >> 4) ^ (hh & 7)) << 4) | (ubyte & 15))) =
                 __float2bfloat16_rn(o);
           }
@@ -663,32 +664,33 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_decode_tc_kernel(
         }
         if (st == 0) tc::bulk_wait_read_all();
       } else {
-        float* wo = p.ws_o + ((long long)q * p.splits + sp) * kH * kC + (long long)(32 * hsel) * kC;
+        float* wo = p.ws_o + ((long long)q * p.splits + sp) * kH * kC + (long long)(kHpt * hsel) * kC;
 #pragma unroll 1
         for (int mb = 0; mb < 4; ++mb) {
-          uint32_t v[32];
+          uint32_t v[kHpt];
           if (nt > 0) {
-            tc::tmem_ld32(tmem + lanebase + col_o(mb) + 32 * hsel, v);
+            tc::tmem_ld16(tmem + lanebase + col_o(mb) + kHpt * hsel, v);
             if (wide_block(mb)) {
-              uint32_t w[32];
-              tc::tmem_ld32(tmem + lanebase + col_o(mb) + kH + 32 * hsel, w);
+              uint32_t w[kHpt];
+              tc::tmem_ld16(tmem + lanebase + col_o(mb) + kH + kHpt * hsel, w);
               tc::tmem_ld_wait();
 #pragma unroll
-              for (int h = 0; h < 32; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) + __uint_as_float(w[h]));
+              for (int h = 0; h < kHpt; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) + __uint_as_float(w[h]));
             }
             tc::tmem_ld_wait();
           }
           const int d = mb * 128 + dim_lane;
 #pragma unroll
-          for (int h = 0; h < 32; ++h) wo[h * kC + d] = nt > 0 ? __uint_as_float(v[h]) : 0.f;
+          for (int h = 0; h < kHpt; ++h) wo[h * kC + d] = nt > 0 ? __uint_as_float(v[h]) : 0.f;
         }
         if (quarter == 0) {
-          // lane l of the quarter-0 warps: head 32 hsel + l (l is the same in every TMEM lane)
+          // lane l < 16 of the quarter-0 warps: head 16 hsel + l (l is the same in every TMEM lane)
           float l = 0.f;  // lv[lane] without a dynamically indexed register array
 #pragma unroll
-          for (int h = 0; h < 32; ++h) l = (h == lane && nt > 0) ? __uint_as_float(lv[h]) : l;
-          const int hh = 32 * hsel + lane;
-          p.ws_ml[((long long)q * p.splits + sp) * kH + hh] = make_float2(l > 0.f ? bars->mref[hh] : neg_inf(), l);
+          for (int h = 0; h < kHpt; ++h) l = (h == lane && nt > 0) ? __uint_as_float(lv[h]) : l;
+          const int hh = kHpt * hsel + lane;
+          if (lane < kHpt)
+            p.ws_ml[((long long)q * p.splits + sp) * kH + hh] = make_float2(l > 0.f ? bars->mref[hh] : neg_inf(), l);
         }
       }
     }
