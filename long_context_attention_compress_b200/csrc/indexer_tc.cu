@@ -297,16 +297,19 @@ constexpr int kPN = kPQ * kHeads;            // 256 = MMA N
 constexpr uint32_t kPQBytes = kPN * kDim * 2;        // 64 KiB
 constexpr uint32_t kPQChunkBytes = kPN * 128;        // 32 KiB
 constexpr int kPAcc = 2;
-constexpr int kPThreads = 320;  // producer, MMA, 8 epilogue warps (two per TMEM lane quarter)
+constexpr int kPEpi = 16;       // epilogue warps (four per TMEM lane quarter)
+constexpr int kPQT = kPQ * 4 / kPEpi;  // queries per epilogue thread (1)
+constexpr int kPParts = kPQ / kPQT;    // 128-thread parts of the epilogue, one per query
+constexpr int kPThreads = 64 + 32 * kPEpi;  // producer, MMA, epilogue
 constexpr int kPCand = 1792;    // candidate slots per query
 constexpr int kPPer = kPCand / 128;  // candidates per thread of a half in a cut
 
-// Scratch of one half of the epilogue (the 128 threads serving two queries).
+// Scratch of one part of the epilogue (the 128 threads serving kPQT queries).
 struct __align__(16) PHalf {
   unsigned long long wmin[4], wmax[4];
   int hist[256];
   int wsum[4];
-  int wcnt[2][4][2];  // [tile parity][TMEM lane quarter][query of the half]: appends per warp
+  int wcnt[2][4][kPQT];  // [tile parity][TMEM lane quarter][query of the part]: appends per warp
   int bucket, greater;
 };
 struct __align__(16) PBars {
@@ -317,7 +320,7 @@ struct __align__(16) PBars {
   uint64_t qfull, qempty, drain;
   uint32_t tmem_base;
   int abort;
-  PHalf half[2];
+  PHalf half[kPParts];
 };
 static_assert(offsetof(PBars, w) % 16 == 0 && offsetof(PBars, full) % 8 == 0, "PBars alignment");
 static_assert((kPStages * kTileBytes + kPQBytes) % 1024 == 0, "candidate lists start 1024-byte aligned");
@@ -583,7 +586,7 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPStages; ++s) { tc::mbar_init(&bars->full[s], 1); tc::mbar_init(&bars->empty[s], 1); }
-    for (int a = 0; a < kPAcc; ++a) { tc::mbar_init(&bars->tfull[a], 1); tc::mbar_init(&bars->tempty[a], 8); }
+    for (int a = 0; a < kPAcc; ++a) { tc::mbar_init(&bars->tfull[a], 1); tc::mbar_init(&bars->tempty[a], kPEpi); }
     tc::mbar_init(&bars->qfull, 1);
     tc::mbar_init(&bars->qempty, 1);
     tc::mbar_init(&bars->drain, 1);
@@ -656,18 +659,20 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
     }
     __syncwarp();
   } else {
-    // epilogue: warps 2..9, one TMEM lane (= entry) per thread; the two warps of a
-    // lane quarter score two of the group's four queries each.  Warps 2-5 (half 0)
-    // serve queries 0 and 1, warps 6-9 (half 1) queries 2 and 3.
+    // epilogue: warps 2..17, one TMEM lane (= entry) per thread; the four warps of a
+    // lane quarter score one of the group's four queries each.  Warps 2-5 (part 0)
+    // serve query 0, warps 6-9 query 1, and so on.
     const int lq = warp & 3;
     const int row_in_tile = lq * 32 + lane;
     const int et = threadIdx.x - 64;  // 0..255
-    const int half = (warp - 2) >> 2;
-    const int j0 = 2 * half;
-    const int hl = et - 128 * half;  // 0..127 within the half
+    const int half = (warp - 2) >> 2;  // the part: kPQT queries
+    const int j0 = kPQT * half;
+    const int hl = et - 128 * half;  // 0..127 within the part
     const uint32_t hbar = 2 + half;
     PHalf* hs = &bars->half[half];
-    uint64_t* cbuf[2] = {cand_smem + (size_t)j0 * kPCand, cand_smem + (size_t)(j0 + 1) * kPCand};
+    uint64_t* cbuf[kPQT];
+#pragma unroll
+    for (int jj = 0; jj < kPQT; ++jj) cbuf[jj] = cand_smem + (size_t)(j0 + jj) * kPCand;
     const unsigned lt = (1u << lane) - 1u;
     int it = 0, par = 0;
     bool failed = false;
@@ -675,8 +680,8 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
       const int nt = group_tiles(g);
       if (nt == 0 && !fused) continue;
       // stage this group's weights and visible counts (the previous group's readers are done)
-      tc::named_bar(1, 256);
-      for (int e = et; e < kPN; e += 256) {
+      tc::named_bar(1, 32 * kPEpi);
+      for (int e = et; e < kPN; e += 32 * kPEpi) {
         const int q = g * kPQ + e / kHeads;
         bars->w[e] = q < Tq ? w_idx[(long long)q * kHeads + (e % kHeads)] : 0.f;
       }
@@ -684,22 +689,26 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
         const int q = g * kPQ + et;
         bars->nvis[et] = q < Tq ? n_visible(q_pos[q], rate, N) : 0;
       }
-      tc::named_bar(1, 256);
-      // fused top-k state of this half's two queries (uniform over the half)
-      bool sel[2];
-      int cnt[2] = {0, 0};
-      uint64_t thr[2] = {0ull, 0ull};  // every real composite is > 0
+      tc::named_bar(1, 32 * kPEpi);
+      // fused top-k state of this part's queries (uniform over the part)
+      bool sel[kPQT];
+      int cnt[kPQT];
+      uint64_t thr[kPQT];  // every real composite is > 0
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) sel[jj] = fused && g * kPQ + j0 + jj < Tq && bars->nvis[j0 + jj] > k;
+      for (int jj = 0; jj < kPQT; ++jj) { cnt[jj] = 0; thr[jj] = 0ull; }
+#pragma unroll
+      for (int jj = 0; jj < kPQT; ++jj) sel[jj] = fused && g * kPQ + j0 + jj < Tq && bars->nvis[j0 + jj] > k;
       for (int t = 0; t < nt; ++t, ++it) {
         const int a = it % kPAcc;
         if (!failed) failed = !tc::warp_wait(&bars->tfull[a], (it / kPAcc) & 1, abort);
         const int e = t * kTile + row_in_tile;
-        float sc[2] = {0.f, 0.f};
+        float sc[kPQT];
+#pragma unroll
+        for (int jj = 0; jj < kPQT; ++jj) sc[jj] = 0.f;
         if (!failed) {
           tc::fence_after_sync();
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
+          for (int jj = 0; jj < kPQT; ++jj) {
             const int j = j0 + jj;
             uint32_t v[kHeads];
             const uint32_t taddr = tmem + ((uint32_t)(lq * 32) << 16) + a * kPN + j * kHeads;
@@ -731,17 +740,17 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
         if (!fused) {
           if (failed) continue;
 #pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
+          for (int jj = 0; jj < kPQT; ++jj) {
             const int q = g * kPQ + j0 + jj;
             if (q < Tq && e < bars->nvis[j0 + jj]) scores[(long long)q * ld_scores + e] = sc[jj];
           }
           continue;
         }
         // fused: candidates that beat the threshold, appended in entry order
-        uint64_t c[2];
-        unsigned bal[2];
+        uint64_t c[kPQT];
+        unsigned bal[kPQT];
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
+        for (int jj = 0; jj < kPQT; ++jj) {
           c[jj] = make_cand(sc[jj], e);
           const bool take = !failed && sel[jj] && e < bars->nvis[j0 + jj] && c[jj] > thr[jj];
           bal[jj] = __ballot_sync(0xffffffffu, take);
@@ -750,7 +759,7 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
         // one barrier per tile: the warps' counts are in, and every thread agrees on failure
         if (tc::named_bar_or(hbar, 128, failed || *abort)) { failed = true; break; }
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
+        for (int jj = 0; jj < kPQT; ++jj) {
           int off = cnt[jj], tot = 0;
 #pragma unroll
           for (int l = 0; l < 4; ++l) {
@@ -765,7 +774,7 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
         // room for one more tile of appends in each list, else cut it back (coarsely: the
         // exact k largest are taken once, after the group's last tile)
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
+        for (int jj = 0; jj < kPQT; ++jj) {
           if (cnt[jj] > kPCand - kTile) {
             int kept;
             thr[jj] = cut_coarse(cbuf[jj], cnt[jj], k, hs, hbar, hl, &kept);
@@ -777,7 +786,7 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
       if (failed) continue;  // (uniform over the half: agreed at the per-tile barrier)
       tc::named_bar(hbar, 128);  // the last tile's appends are in place
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
+      for (int jj = 0; jj < kPQT; ++jj) {
         const int q = g * kPQ + j0 + jj;
         if (q >= Tq) continue;
         int32_t* out = topk_idx + (long long)q * k;
