@@ -612,6 +612,13 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
         tc::mbar_arrive_expect_tx(&bars->qfull, kPQBytes);
         tc::tma_load_2d(q_smem, &tm_q, &bars->qfull, 0, g * kPN);
         tc::tma_load_2d(q_smem + kPQChunkBytes, &tm_q, &bars->qfull, 64, g * kPN);
+        // the next group's queries into L2 while this group streams: its load above
+        // then waits on L2, not on HBM (the q buffer holds one group)
+        {
+          int gn = g - (int)gridDim.x;
+          while (gn >= 0 && group_tiles(gn) == 0) gn -= (int)gridDim.x;
+          if (gn >= 0) tc::tma_prefetch_2d(&tm_q, 0, gn * kPN), tc::tma_prefetch_2d(&tm_q, 64, gn * kPN);
+        }
         for (int t = 0; t < nt; ++t, ++it) {
           const int s = it % kPStages;
           if (!tc::mbar_wait(&bars->empty[s], ((it / kPStages) & 1) ^ 1, abort)) { ok = false; break; }
@@ -707,6 +714,7 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
         for (int jj = 0; jj < kPQT; ++jj) sc[jj] = 0.f;
         if (!failed) {
           tc::fence_after_sync();
+          static_assert(kPQT == 1, "the accumulator is released right after its one read below");
 #pragma unroll
           for (int jj = 0; jj < kPQT; ++jj) {
             const int j = j0 + jj;
@@ -715,6 +723,10 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
             tc::tmem_ld32(taddr, v);
             tc::tmem_ld32(taddr + 32, v + 32);
             tc::tmem_ld_wait();
+            // the accumulator may take tile it + 2's MMAs while this warp sums
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->tempty[a]);
             const float* w = bars->w + j * kHeads;
             // eight independent chains (a fixed association, the same for every entry)
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -733,9 +745,6 @@ __global__ void __launch_bounds__(kPThreads, 1) indexer_prefill_tc_kernel(
             }
             sc[jj] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
           }
-          tc::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&bars->tempty[a]);
         }
         if (!fused) {
           if (failed) continue;
