@@ -752,9 +752,10 @@ static DecodeSched decode_schedule(const hca_layer_cfg* cfg, const hca_decode_ar
     // Balance the two sides' SM-time: the attention costs about kAttnTileUs per
     // 64 rows on one SM, the indexer streams about kIdxBytesPerSmUs bytes per
     // microsecond per SM (calibrated on B200 by sweeping the HCA share of the
-    // 8-request 1M-context step: 24 of 148 SMs is best there).  The HCA share is
-    // a whole number of splits per request so that it runs as a single wave.
-    constexpr double kAttnTileUs = 3.0, kIdxBytesPerSmUs = 35e3;
+    // 8-request 1M-context step: 16 of 148 SMs is best there, 0.178 against
+    // 0.188 ms with 24).  The HCA share is a whole number of splits per request
+    // so that it runs as a single wave.
+    constexpr double kAttnTileUs = 2.0, kIdxBytesPerSmUs = 35e3;
     const double hca_tiles = (double)a->B * std::ceil(((double)a->hca_N + cfg->n_win) / 64.0);
     const double hca_us = hca_tiles * kAttnTileUs;
     const double idx_us = (double)a->B * a->csa_N * cfg->d_idx * 2.0 / kIdxBytesPerSmUs;
