@@ -8,7 +8,8 @@
 // streamed once.  The (request, 128-entry tile) space is split evenly over a
 // persistent grid (one CTA per SM).  Per CTA:
 //   warp 0      TMA producer: key tiles [128 entries x 128 dims] bf16 (two
-//               64-dim 128B-swizzled boxes, 32 KiB) into a ring of stages;
+//               64-dim 128B-swizzled boxes, 32 KiB, L2 evict-first) into a
+//               ring of stages;
 //               the request's q_I [64 heads x 128] when the request changes.
 //   warp 1      MMA issuer (one thread): S^T[128 entries, 64 heads] =
 //               K_tile . q_I^T with eight M=128 N=64 K=16 tcgen05.mma into one
@@ -100,6 +101,9 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
     if (lane == 0) {
       tc::tma_prefetch_desc(&tm_k);
       tc::tma_prefetch_desc(&tm_q);
+      // the keys are read once per step: their lines go first, so that the scores and
+      // histograms stay in L2 for the select that reads them next
+      const uint64_t stream_pol = tc::l2_evict_first_policy();
       int it = 0, rq = 0, cur_r = -1;
       for (long long g = stall ? g1 : g0; g < g1; ++g) {
         const int r = (int)(g / tiles_per_req);
@@ -135,14 +139,15 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_decode_tc_kernel(
           for (int i = 0; i < kTile / 8; ++i) {
             if (i < nb) {
               const int prow = pb[i] * rpb;
-              tc::tma_load_2d(k_smem + s * kTileBytes + i * rpb * 128, &tm_k, &bars->full[s], 0, prow);
-              tc::tma_load_2d(k_smem + s * kTileBytes + kChunkBytes + i * rpb * 128, &tm_k, &bars->full[s], 64, prow);
+              tc::tma_load_2d_hint(k_smem + s * kTileBytes + i * rpb * 128, &tm_k, &bars->full[s], 0, prow, stream_pol);
+              tc::tma_load_2d_hint(k_smem + s * kTileBytes + kChunkBytes + i * rpb * 128, &tm_k, &bars->full[s], 64,
+                                   prow, stream_pol);
             }
           }
         } else {
           tc::mbar_arrive_expect_tx(&bars->full[s], kTileBytes);
-          tc::tma_load_3d(k_smem + s * kTileBytes, &tm_k, &bars->full[s], 0, row0, r);
-          tc::tma_load_3d(k_smem + s * kTileBytes + kChunkBytes, &tm_k, &bars->full[s], 64, row0, r);
+          tc::tma_load_3d_hint(k_smem + s * kTileBytes, &tm_k, &bars->full[s], 0, row0, r, stream_pol);
+          tc::tma_load_3d_hint(k_smem + s * kTileBytes + kChunkBytes, &tm_k, &bars->full[s], 64, row0, r, stream_pol);
         }
         ++it;
       }

@@ -221,11 +221,14 @@ __global__ void __launch_bounds__(kMqaThreads) mqa_split_kernel(MqaProblem p, in
 }
 
 // combine: o = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i per (query, head).
-// grid (Tq, ceil(H/4)), 256 threads: one CTA merges 4 heads; the per-split
-// weights are computed once into shared memory, then every thread owns a
-// float4 of one head's output and loads that float4 from all splits with
-// independent loads (the split loop is unrolled by 4).
-constexpr int kCombHeads = 4;
+// grid (Tq, ceil(H/2)), 256 threads: 128 threads merge one head, each owning one
+// float4 of the head's output (C <= 512).  The first kCombBatch splits' float4s
+// are loaded before the weights are formed, so that their latency overlaps the
+// reductions over the splits' (m, l); later batches follow one load round each.
+// The sum runs over the splits in order with the normalised weights, as
+// w_i / den computed at use.
+constexpr int kCombHeads = 2;
+constexpr int kCombBatch = 16;        // partial float4s in flight per thread
 constexpr int kCombMaxSplits = 1024;  // planners never exceed this
 __global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restrict__ ws_o,
                                                           const float2* __restrict__ ws_ml, int splits,
@@ -234,82 +237,77 @@ __global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restric
                                                           const int32_t* __restrict__ q_pos, int rope_dims,
                                                           float rope_base) {
   __shared__ float s_w[kCombHeads][kCombMaxSplits];
+  __shared__ float s_red[kCombHeads][2][4];
   tc::griddep_wait();  // the partial states come from the attention kernel
-  const int q = blockIdx.x, h0 = blockIdx.y * kCombHeads;
-  const int nh = min(kCombHeads, H - h0);
-  // weights: thread hh*64 + lane-group handles head hh
-  for (int hh = threadIdx.x >> 6; hh < nh; hh += 4) {
-    const int h = h0 + hh;
-    const int t = threadIdx.x & 63;
-    float M = neg_inf();
-    for (int s = t; s < splits; s += 64) M = fmaxf(M, ws_ml[((long long)q * splits + s) * H + h].x);
+  const int hh = threadIdx.x >> 7, t = threadIdx.x & 127, lane = t & 31, wq = t >> 5;
+  const int q = blockIdx.x, h = blockIdx.y * kCombHeads + hh;
+  if (h >= H) return;  // the whole 128-thread group: its named barrier counts no one else
+  const int bar = 1 + hh;
+  const bool has = t < (C >> 2);
+  const long long sstride = (long long)H * C / 4;  // float4s between splits
+  const float4* src = reinterpret_cast<const float4*>(ws_o + ((long long)q * splits * H + h) * C) + t;
+  float4 v[kCombBatch];
 #pragma unroll
-    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    __shared__ float s_red[4][2];
-    if ((t & 31) == 0) s_red[hh & 3][t >> 5] = M;
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + (hh & 3)) : "memory");
-    M = fmaxf(s_red[hh & 3][0], s_red[hh & 3][1]);
-    // a sink logit (base-2 scale like the maxima) joins the denominator once per query
-    const float z = sink ? sink[h] * kLog2e : neg_inf();
-    M = fmaxf(M, z);
-    float den = 0.f;
-    for (int s = t; s < splits; s += 64) {
-      const float2 ml = ws_ml[((long long)q * splits + s) * H + h];
-      const float w = ml.y > 0.f ? fast_exp2(ml.x - M) : 0.f;
-      s_w[hh][s] = w;
-      den += w * ml.y;
+  for (int u = 0; u < kCombBatch; ++u)
+    v[u] = (has && u < splits) ? src[u * sstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+  // weights: the maximum over the splits (and the sink logit), then the denominator
+  const float2* ml = ws_ml + (long long)q * splits * H + h;  // split s at ml[s * H]
+  float M = neg_inf();
+  for (int s = t; s < splits; s += 128) M = fmaxf(M, ml[(long long)s * H].x);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) s_red[hh][0][wq] = M;
+  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+  M = fmaxf(fmaxf(s_red[hh][0][0], s_red[hh][0][1]), fmaxf(s_red[hh][0][2], s_red[hh][0][3]));
+  // a sink logit (base-2 scale like the maxima) joins the denominator once per query
+  const float z = sink ? sink[h] * kLog2e : neg_inf();
+  M = fmaxf(M, z);
+  float den = 0.f;
+  for (int s = t; s < splits; s += 128) {
+    const float2 m_l = ml[(long long)s * H];
+    const float w = m_l.y > 0.f ? fast_exp2(m_l.x - M) : 0.f;
+    s_w[hh][s] = w;
+    den += w * m_l.y;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane == 0) s_red[hh][1][wq] = den;
+  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
+  den = (s_red[hh][1][0] + s_red[hh][1][1]) + (s_red[hh][1][2] + s_red[hh][1][3]);
+  if (sink) den += fast_exp2(z - M);
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  if (!has) return;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < splits; s0 += kCombBatch) {
+    if (s0 > 0) {
+#pragma unroll
+      for (int u = 0; u < kCombBatch; ++u)
+        if (s0 + u < splits) v[u] = src[(s0 + u) * sstride];
     }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + (hh & 3)) : "memory");
-    if ((t & 31) == 0) s_red[hh & 3][t >> 5] = den;
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + (hh & 3)) : "memory");
-    den = s_red[hh & 3][0] + s_red[hh & 3][1];
-    if (sink) den += fast_exp2(z - M);
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    for (int s = t; s < splits; s += 64) s_w[hh][s] *= inv;
-  }
-  __syncthreads();
-  const int per_head = C / 4;  // float4 per head
-  for (int e = threadIdx.x; e < nh * per_head; e += 256) {
-    const int hh = e / per_head, d4 = e % per_head;
-    const int h = h0 + hh;
-    const float4* src = reinterpret_cast<const float4*>(ws_o + ((long long)q * splits * H + h) * C) + d4;
-    const long long sstride = (long long)H * C / 4;  // float4s between splits
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int s = 0;
-    for (; s + 4 <= splits; s += 4) {
-      float4 v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = src[(s + u) * sstride];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float w = s_w[hh][s + u];
+    for (int u = 0; u < kCombBatch; ++u) {
+      if (s0 + u < splits) {
+        const float w = s_w[hh][s0 + u] * inv;
         acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
         acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
       }
     }
-    for (; s < splits; ++s) {
-      const float4 v = src[s * sstride];
-      const float w = s_w[hh][s];
-      acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
-    }
-    if (rope_dims > 0 && d4 * 4 >= C - rope_dims) {
-      // partial-RoPE output rotation by -t of the pairs (x, y) and (z, w):
-      // a' = a cos + b sin, b' = b cos - a sin
-      const int j = (d4 * 4 - (C - rope_dims)) >> 1;
-      float c0, s0, c1, s1;
-      rope_cos_sin(q_pos[q], j, rope_dims, rope_base, c0, s0);
-      rope_cos_sin(q_pos[q], j + 1, rope_dims, rope_base, c1, s1);
-      acc = make_float4(fmaf(acc.x, c0, acc.y * s0), fmaf(acc.y, c0, -acc.x * s0),
-                        fmaf(acc.z, c1, acc.w * s1), fmaf(acc.w, c1, -acc.z * s1));
-    }
-    uint2 pk;
-    pk.x = pack_bf16x2(acc.x, acc.y);
-    pk.y = pack_bf16x2(acc.z, acc.w);
-    *reinterpret_cast<uint2*>(out + ((long long)q * H + h) * C + d4 * 4) = pk;
   }
+  const int d4 = t;
+  if (rope_dims > 0 && d4 * 4 >= C - rope_dims) {
+    // partial-RoPE output rotation by -t of the pairs (x, y) and (z, w):
+    // a' = a cos + b sin, b' = b cos - a sin
+    const int j = (d4 * 4 - (C - rope_dims)) >> 1;
+    float c0, s0, c1, s1;
+    rope_cos_sin(q_pos[q], j, rope_dims, rope_base, c0, s0);
+    rope_cos_sin(q_pos[q], j + 1, rope_dims, rope_base, c1, s1);
+    acc = make_float4(fmaf(acc.x, c0, acc.y * s0), fmaf(acc.y, c0, -acc.x * s0),
+                      fmaf(acc.z, c1, acc.w * s1), fmaf(acc.w, c1, -acc.z * s1));
+  }
+  uint2 pk;
+  pk.x = pack_bf16x2(acc.x, acc.y);
+  pk.y = pack_bf16x2(acc.z, acc.w);
+  *reinterpret_cast<uint2*>(out + ((long long)q * H + h) * C + d4 * 4) = pk;
 }
 
 template <int H, int C>
@@ -320,6 +318,7 @@ static size_t mqa_smem() {
 cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, int splits, int H, int C, bf16* out,
                                const float* sink, const int32_t* q_pos, int rope_dims, float rope_base,
                                cudaStream_t stream, bool pdl) {
+  if (C % 4 != 0 || C > 4 * 128 || splits < 1 || splits > kCombMaxSplits) return cudaErrorInvalidValue;
   cudaError_t e = launch_pdl(pdl, mqa_combine_kernel, dim3(Tq, (H + kCombHeads - 1) / kCombHeads), dim3(256), 0,
                              stream, ws_o, ws_ml, splits, H, C, out, sink, q_pos, rope_dims, rope_base);
   if (e != cudaSuccess) return e;
@@ -387,11 +386,8 @@ static cudaError_t launch_mqa_t(const MqaProblem& p, const MqaPlan& pl, void* ws
   ++g_launch_counter;
   e = cudaGetLastError();
   if (e != cudaSuccess || pl.splits == 1) return e;
-  mqa_combine_kernel<<<dim3(p.Tq, (H + kCombHeads - 1) / kCombHeads), 256, 0, stream>>>(ws_o, ws_ml, pl.splits, H, C,
-                                                                                      p.out, p.sink, p.q_pos,
-                                                                                      p.rope_dims, p.rope_base);
-  ++g_launch_counter;
-  return cudaGetLastError();
+  return launch_mqa_combine(ws_o, ws_ml, p.Tq, pl.splits, H, C, p.out, p.sink, p.q_pos, p.rope_dims, p.rope_base,
+                            stream, false);
 }
 
 unsigned int read_and_clear_mqa_index_error() {

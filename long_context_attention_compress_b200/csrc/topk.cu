@@ -404,12 +404,18 @@ __global__ void __launch_bounds__(kSelThreads) select_merge_kernel(const uint64_
 // entries above T in index order, then the chosen bin-T entries in index order.
 // Threshold over a 4096-bin histogram read from global memory: the bin holding the
 // `k`-th largest entry, and the number of entries in higher bins.  All NT threads.
+// The thread's four bins, as hist_threshold_from takes them.
 template <int NT>
-__device__ void hist_threshold(const int* h, int k, int* s_bin, int* s_higher, int2* s_warp) {
+__device__ __forceinline__ int4 hist_bins(const int* h) {
+  static_assert(NT * 4 == kHistBins, "four bins per thread");
+  return __ldcg(reinterpret_cast<const int4*>(h + kHistBins - 4 * (threadIdx.x + 1)));
+}
+// (h4: this thread's bins, loaded by hist_bins)
+template <int NT>
+__device__ void hist_threshold_from(int4 h4, int k, int* s_bin, int* s_higher, int2* s_warp) {
   static_assert(NT * 4 == kHistBins, "four bins per thread");
   const int tid = threadIdx.x;
   if (tid == 0) { *s_bin = -1; *s_higher = 0; }
-  const int4 h4 = __ldcg(reinterpret_cast<const int4*>(h + kHistBins - 4 * (tid + 1)));
   const int hv[4] = {h4.w, h4.z, h4.y, h4.x};  // bins 4095 - 4t, 4094 - 4t, ...
   int ex, dummy, tot, tdummy;
   block_scan2<NT>(hv[0] + hv[1] + hv[2] + hv[3], 0, ex, dummy, tot, tdummy, s_warp);
@@ -420,6 +426,21 @@ __device__ void hist_threshold(const int* h, int k, int* s_bin, int* s_higher, i
     run += hv[u];
   }
   __syncthreads();
+}
+template <int NT>
+__device__ void hist_threshold(const int* h, int k, int* s_bin, int* s_higher, int2* s_warp) {
+  hist_threshold_from<NT>(hist_bins<NT>(h), k, s_bin, s_higher, s_warp);
+}
+
+// Largest j in [0, n) with off[j] <= i, for off[0] <= i < off[n] (a prefix sum:
+// the list of a concatenation that holds element i, skipping empty lists).
+__device__ __forceinline__ int list_of(const int* off, int stride, int n, int i) {
+  int lo = 0, hi = n;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (off[mid * stride] <= i) lo = mid; else hi = mid;
+  }
+  return lo;
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_hist_kernel(HistSelect a) {
@@ -501,8 +522,10 @@ __global__ void __launch_bounds__(kSelThreads) select_hist_kernel(HistSelect a) 
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // every CTA's counts (written by other CTAs: read from L2), exclusive offsets by warp 0
+  // every CTA's counts (written by other CTAs: read from L2), exclusive offsets by warp 0;
+  // the level-2 histogram is complete too: its bins load alongside
   if (tid < a.C) s_cnt[tid] = __ldcg(a.cnt + (long long)r * a.C + tid);
+  const int4 h2 = hist_bins<kSelThreads>(hist2);
   __syncthreads();
   if (warp == 0) {
     int ca = 0, ce = 0;
@@ -529,19 +552,42 @@ __global__ void __launch_bounds__(kSelThreads) select_hist_kernel(HistSelect a) 
     return;
   }
   const int need = k - n_above;
-  // one warp per slice list: the "above" entries go straight to the output
-  for (int j = warp; j < a.C; j += kSelThreads / 32) {
-    const int32_t* src_a = a.above + ((long long)r * a.C + j) * k;
-    for (int t = lane; t < s_cnt[j].x; t += 32) out[s_off[j].x + t] = __ldcg(src_a + t);
-  }
-  if (n_eq <= kSelectMaxN) {
-    // bin-T candidates staged in shared memory in entry order
-    for (int j = warp; j < a.C; j += kSelThreads / 32) {
-      const uint64_t* src_e = a.eq + ((long long)r * a.C + j) * a.slice;
-      for (int t = lane; t < s_cnt[j].y; t += 32) s_c[s_off[j].y + t] = __ldcg(src_e + t);
+  const bool staged = n_eq <= kSelectMaxN;
+  // The "above" entries go straight to the output and, when they fit, the bin-T
+  // candidates to shared memory, both in entry order: element i of the lists'
+  // concatenation (above lists, then bin-T lists) is found in its list by a search
+  // over the offsets, with all of a thread's loads in flight before its stores.
+  {
+    const int n_cp = n_above + (staged ? n_eq : 0);
+    const int* off_a = &s_off[0].x;
+    const int* off_e = &s_off[0].y;
+    for (int i0 = 0; i0 < n_cp; i0 += 4 * kSelThreads) {
+      uint64_t val[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kSelThreads + tid;
+        val[u] = 0ull;
+        if (i < n_above) {
+          const int j = list_of(off_a, 2, a.C, i);
+          val[u] = (uint32_t)__ldcg(a.above + ((long long)r * a.C + j) * k + (i - off_a[2 * j]));
+        } else if (i < n_cp) {
+          const int ie = i - n_above;
+          const int j = list_of(off_e, 2, a.C, ie);
+          val[u] = __ldcg(a.eq + ((long long)r * a.C + j) * a.slice + (ie - off_e[2 * j]));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kSelThreads + tid;
+        if (i < n_above) out[i] = (int32_t)(uint32_t)val[u];
+        else if (i < n_cp) s_c[i - n_above] = val[u];
+      }
     }
-    // level 2 threshold among them (the histogram's total is n_eq)
-    hist_threshold<kSelThreads>(hist2, need, &s_T2, &s_above2, s_warp);
+  }
+  if (staged) {
+    // level 2 threshold among the staged candidates (the histogram's total is n_eq;
+    // its barriers also publish the staged candidates)
+    hist_threshold_from<kSelThreads>(h2, need, &s_T2, &s_above2, s_warp);
     const int T2 = s_T2, above2 = s_above2;
     if (T2 < 0) {
       if (tid == 0) atomicOr(&g_select_error, 1u);
