@@ -221,49 +221,55 @@ __global__ void __launch_bounds__(kMqaThreads) mqa_split_kernel(MqaProblem p, in
 }
 
 // combine: o = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i per (query, head).
-// grid (Tq, ceil(H/2)), 256 threads: 128 threads merge one head, each owning one
-// float4 of the head's output (C <= 512).  The first kCombBatch splits' float4s
-// are loaded before the weights are formed, so that their latency overlaps the
-// reductions over the splits' (m, l); later batches follow one load round each.
-// The sum runs over the splits in order with the normalised weights, as
-// w_i / den computed at use.
-constexpr int kCombHeads = 2;
-constexpr int kCombBatch = 16;        // partial float4s in flight per thread
+// 256 threads per CTA, TPH per head (256 / TPH heads per CTA), each thread owning
+// the float4s t, t + TPH, ... of its head's output (C <= 512).  The first BATCH
+// splits' float4s are loaded before the weights are formed, so that their latency
+// overlaps the reductions over the splits' (m, l); later batches follow one load
+// round each.  The sum runs over the splits in order with the normalised weights
+// w_i / den formed at use.  Few queries take TPH = 128 with 16 splits in flight
+// (one wave at two CTAs per SM); many take TPH = 64 with 4, which needs fewer
+// registers, so that more CTAs share an SM.
 constexpr int kCombMaxSplits = 1024;  // planners never exceed this
+template <int TPH, int BATCH>
 __global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restrict__ ws_o,
                                                           const float2* __restrict__ ws_ml, int splits,
                                                           int H, int C, bf16* __restrict__ out,
                                                           const float* __restrict__ sink,
                                                           const int32_t* __restrict__ q_pos, int rope_dims,
                                                           float rope_base) {
-  __shared__ float s_w[kCombHeads][kCombMaxSplits];
-  __shared__ float s_red[kCombHeads][2][4];
+  constexpr int kHeads = 256 / TPH, kWarps = TPH / 32, kF = 128 / TPH;
+  __shared__ float s_w[kHeads][kCombMaxSplits];
+  __shared__ float s_red[kHeads][2][kWarps];
   tc::griddep_wait();  // the partial states come from the attention kernel
-  const int hh = threadIdx.x >> 7, t = threadIdx.x & 127, lane = t & 31, wq = t >> 5;
-  const int q = blockIdx.x, h = blockIdx.y * kCombHeads + hh;
-  if (h >= H) return;  // the whole 128-thread group: its named barrier counts no one else
+  const int hh = threadIdx.x / TPH, t = threadIdx.x % TPH, lane = t & 31, wq = t >> 5;
+  const int q = blockIdx.x, h = blockIdx.y * kHeads + hh;
+  if (h >= H) return;  // the whole TPH-thread group: its named barrier counts no one else
   const int bar = 1 + hh;
-  const bool has = t < (C >> 2);
+  const int per_head = C >> 2;
   const long long sstride = (long long)H * C / 4;  // float4s between splits
   const float4* src = reinterpret_cast<const float4*>(ws_o + ((long long)q * splits * H + h) * C) + t;
-  float4 v[kCombBatch];
+  float4 v[BATCH][kF];
 #pragma unroll
-  for (int u = 0; u < kCombBatch; ++u)
-    v[u] = (has && u < splits) ? src[u * sstride] : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int u = 0; u < BATCH; ++u)
+#pragma unroll
+    for (int f = 0; f < kF; ++f)
+      v[u][f] = (t + f * TPH < per_head && u < splits) ? src[u * sstride + f * TPH] : make_float4(0.f, 0.f, 0.f, 0.f);
   // weights: the maximum over the splits (and the sink logit), then the denominator
   const float2* ml = ws_ml + (long long)q * splits * H + h;  // split s at ml[s * H]
   float M = neg_inf();
-  for (int s = t; s < splits; s += 128) M = fmaxf(M, ml[(long long)s * H].x);
+  for (int s = t; s < splits; s += TPH) M = fmaxf(M, ml[(long long)s * H].x);
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   if (lane == 0) s_red[hh][0][wq] = M;
-  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
-  M = fmaxf(fmaxf(s_red[hh][0][0], s_red[hh][0][1]), fmaxf(s_red[hh][0][2], s_red[hh][0][3]));
+  asm volatile("bar.sync %0, %1;" ::"r"(bar), "n"(TPH) : "memory");
+  M = s_red[hh][0][0];
+#pragma unroll
+  for (int w = 1; w < kWarps; ++w) M = fmaxf(M, s_red[hh][0][w]);
   // a sink logit (base-2 scale like the maxima) joins the denominator once per query
   const float z = sink ? sink[h] * kLog2e : neg_inf();
   M = fmaxf(M, z);
   float den = 0.f;
-  for (int s = t; s < splits; s += 128) {
+  for (int s = t; s < splits; s += TPH) {
     const float2 m_l = ml[(long long)s * H];
     const float w = m_l.y > 0.f ? fast_exp2(m_l.x - M) : 0.f;
     s_w[hh][s] = w;
@@ -272,42 +278,55 @@ __global__ void __launch_bounds__(256) mqa_combine_kernel(const float* __restric
 #pragma unroll
   for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
   if (lane == 0) s_red[hh][1][wq] = den;
-  asm volatile("bar.sync %0, 128;" ::"r"(bar) : "memory");
-  den = (s_red[hh][1][0] + s_red[hh][1][1]) + (s_red[hh][1][2] + s_red[hh][1][3]);
+  asm volatile("bar.sync %0, %1;" ::"r"(bar), "n"(TPH) : "memory");
+  den = s_red[hh][1][0];
+#pragma unroll
+  for (int w = 1; w < kWarps; ++w) den += s_red[hh][1][w];
   if (sink) den += fast_exp2(z - M);
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  if (!has) return;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < splits; s0 += kCombBatch) {
+  float4 acc[kF];
+#pragma unroll
+  for (int f = 0; f < kF; ++f) acc[f] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < splits; s0 += BATCH) {
     if (s0 > 0) {
 #pragma unroll
-      for (int u = 0; u < kCombBatch; ++u)
-        if (s0 + u < splits) v[u] = src[(s0 + u) * sstride];
+      for (int u = 0; u < BATCH; ++u)
+#pragma unroll
+        for (int f = 0; f < kF; ++f)
+          if (t + f * TPH < per_head && s0 + u < splits) v[u][f] = src[(s0 + u) * sstride + f * TPH];
     }
 #pragma unroll
-    for (int u = 0; u < kCombBatch; ++u) {
+    for (int u = 0; u < BATCH; ++u) {
       if (s0 + u < splits) {
         const float w = s_w[hh][s0 + u] * inv;
-        acc.x = fmaf(w, v[u].x, acc.x); acc.y = fmaf(w, v[u].y, acc.y);
-        acc.z = fmaf(w, v[u].z, acc.z); acc.w = fmaf(w, v[u].w, acc.w);
+#pragma unroll
+        for (int f = 0; f < kF; ++f) {
+          acc[f].x = fmaf(w, v[u][f].x, acc[f].x); acc[f].y = fmaf(w, v[u][f].y, acc[f].y);
+          acc[f].z = fmaf(w, v[u][f].z, acc[f].z); acc[f].w = fmaf(w, v[u][f].w, acc[f].w);
+        }
       }
     }
   }
-  const int d4 = t;
-  if (rope_dims > 0 && d4 * 4 >= C - rope_dims) {
-    // partial-RoPE output rotation by -t of the pairs (x, y) and (z, w):
-    // a' = a cos + b sin, b' = b cos - a sin
-    const int j = (d4 * 4 - (C - rope_dims)) >> 1;
-    float c0, s0, c1, s1;
-    rope_cos_sin(q_pos[q], j, rope_dims, rope_base, c0, s0);
-    rope_cos_sin(q_pos[q], j + 1, rope_dims, rope_base, c1, s1);
-    acc = make_float4(fmaf(acc.x, c0, acc.y * s0), fmaf(acc.y, c0, -acc.x * s0),
-                      fmaf(acc.z, c1, acc.w * s1), fmaf(acc.w, c1, -acc.z * s1));
+#pragma unroll
+  for (int f = 0; f < kF; ++f) {
+    const int d4 = t + f * TPH;
+    if (d4 >= per_head) break;
+    float4 o = acc[f];
+    if (rope_dims > 0 && d4 * 4 >= C - rope_dims) {
+      // partial-RoPE output rotation by -t of the pairs (x, y) and (z, w):
+      // a' = a cos + b sin, b' = b cos - a sin
+      const int j = (d4 * 4 - (C - rope_dims)) >> 1;
+      float c0, s0, c1, s1;
+      rope_cos_sin(q_pos[q], j, rope_dims, rope_base, c0, s0);
+      rope_cos_sin(q_pos[q], j + 1, rope_dims, rope_base, c1, s1);
+      o = make_float4(fmaf(o.x, c0, o.y * s0), fmaf(o.y, c0, -o.x * s0), fmaf(o.z, c1, o.w * s1),
+                      fmaf(o.w, c1, -o.z * s1));
+    }
+    uint2 pk;
+    pk.x = pack_bf16x2(o.x, o.y);
+    pk.y = pack_bf16x2(o.z, o.w);
+    *reinterpret_cast<uint2*>(out + ((long long)q * H + h) * C + d4 * 4) = pk;
   }
-  uint2 pk;
-  pk.x = pack_bf16x2(acc.x, acc.y);
-  pk.y = pack_bf16x2(acc.z, acc.w);
-  *reinterpret_cast<uint2*>(out + ((long long)q * H + h) * C + d4 * 4) = pk;
 }
 
 template <int H, int C>
@@ -319,8 +338,13 @@ cudaError_t launch_mqa_combine(const float* ws_o, const float2* ws_ml, int Tq, i
                                const float* sink, const int32_t* q_pos, int rope_dims, float rope_base,
                                cudaStream_t stream, bool pdl) {
   if (C % 4 != 0 || C > 4 * 128 || splits < 1 || splits > kCombMaxSplits) return cudaErrorInvalidValue;
-  cudaError_t e = launch_pdl(pdl, mqa_combine_kernel, dim3(Tq, (H + kCombHeads - 1) / kCombHeads), dim3(256), 0,
-                             stream, ws_o, ws_ml, splits, H, C, out, sink, q_pos, rope_dims, rope_base);
+  cudaError_t e;
+  if ((long long)Tq * ((H + 1) / 2) <= 2ll * device_sm_count())
+    e = launch_pdl(pdl, mqa_combine_kernel<128, 16>, dim3(Tq, (H + 1) / 2), dim3(256), 0, stream, ws_o, ws_ml, splits,
+                   H, C, out, sink, q_pos, rope_dims, rope_base);
+  else
+    e = launch_pdl(pdl, mqa_combine_kernel<64, 4>, dim3(Tq, (H + 3) / 4), dim3(256), 0, stream, ws_o, ws_ml, splits,
+                   H, C, out, sink, q_pos, rope_dims, rope_base);
   if (e != cudaSuccess) return e;
   ++g_launch_counter;
   return cudaGetLastError();
