@@ -86,21 +86,25 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
 // Eight E2M1 codes (word nibbles 0..7, element order) times 2^X -> eight bf16, packed in
 // pairs (o[k] = element 2k | element 2k+1 << 16).  The magnitudes come from byte
 // tables by byte permutes (bf16 bits of 0, 0.5, 1, 1.5, 2, 3, 4, 6: high bytes
-// 00 3F 3F 3F 40 40 40 40, low bytes 00 00 80 C0 00 40 80 C0), the signs are moved
-// to bit 15 / 31, and 2^X is applied by one bf16x2 multiply, exact while every
-// nonzero product stays a normal bf16 (|X| <= 125: 0.5 * 2^X .. 6 * 2^X); beyond
-// that the values are formed in f32 (as exact) and rounded once.
+// 00 3F 3F 3F 40 40 40 40, low bytes 00 00 80 C0 00 40 80 C0; a permute reads only
+// the low 16 bits of its selector).  The signs (bit 3 of each nibble) reach bits 15
+// and 31 by one more permute per pair: byte k of (signs << 4) holds element 2k's sign
+// in its bit 7 and byte k of the signs element 2k+1's, so placing them in bytes 1
+// and 3 and masking bits 15 and 31 gives the pair's sign bits.  2^X is applied by one
+// bf16x2 multiply, exact while every nonzero product stays a normal bf16
+// (|X| <= 125: 0.5 * 2^X .. 6 * 2^X); beyond that the values are formed in f32 (as
+// exact) and rounded once.
 __device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, int X, uint32_t* o) {
   constexpr uint32_t kHiLo = 0x3F3F3F00u, kHiHi = 0x40404040u, kLoLo = 0xC0800000u, kLoHi = 0xC0804000u;
   if (X >= -125 && X <= 125) {
-    const uint32_t m = w & 0x77777777u, sg = w & 0x88888888u;
-    const uint32_t h0 = __byte_perm(kHiLo, kHiHi, m & 0xffffu), l0 = __byte_perm(kLoLo, kLoHi, m & 0xffffu);
+    const uint32_t m = w & 0x77777777u, sg = w & 0x88888888u, sg4 = sg << 4;
+    const uint32_t h0 = __byte_perm(kHiLo, kHiHi, m), l0 = __byte_perm(kLoLo, kLoHi, m);
     const uint32_t h1 = __byte_perm(kHiLo, kHiHi, m >> 16), l1 = __byte_perm(kLoLo, kLoHi, m >> 16);
     uint32_t p[4];
-    p[0] = __byte_perm(l0, h0, 0x5140u) | ((sg << 12) & 0x8000u) | ((sg << 24) & 0x80000000u);
-    p[1] = __byte_perm(l0, h0, 0x7362u) | ((sg << 4) & 0x8000u) | ((sg << 16) & 0x80000000u);
-    p[2] = __byte_perm(l1, h1, 0x5140u) | ((sg >> 4) & 0x8000u) | ((sg << 8) & 0x80000000u);
-    p[3] = __byte_perm(l1, h1, 0x7362u) | ((sg >> 12) & 0x8000u) | (sg & 0x80000000u);
+    p[0] = __byte_perm(l0, h0, 0x5140u) | (__byte_perm(sg4, sg, 0x4000u) & 0x80008000u);
+    p[1] = __byte_perm(l0, h0, 0x7362u) | (__byte_perm(sg4, sg, 0x5111u) & 0x80008000u);
+    p[2] = __byte_perm(l1, h1, 0x5140u) | (__byte_perm(sg4, sg, 0x6222u) & 0x80008000u);
+    p[3] = __byte_perm(l1, h1, 0x7362u) | (__byte_perm(sg4, sg, 0x7333u) & 0x80008000u);
     const uint32_t sb = (uint32_t)(127 + X) << 7;  // bf16 bits of 2^X
     const uint32_t sbits = sb | (sb << 16);
     __nv_bfloat162 sc;
