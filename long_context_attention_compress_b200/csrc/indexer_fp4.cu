@@ -87,10 +87,10 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
 // pairs (o[k] = element 2k | element 2k+1 << 16).  The magnitudes come from byte
 // tables by byte permutes (bf16 bits of 0, 0.5, 1, 1.5, 2, 3, 4, 6: high bytes
 // 00 3F 3F 3F 40 40 40 40, low bytes 00 00 80 C0 00 40 80 C0; a permute reads only
-// the low 16 bits of its selector).  The signs (bit 3 of each nibble) reach bits 15
-// and 31 by one more permute per pair: byte k of (signs << 4) holds element 2k's sign
-// in its bit 7 and byte k of the signs element 2k+1's, so placing them in bytes 1
-// and 3 and masking bits 15 and 31 gives the pair's sign bits.  2^X is applied by one
+// the low 16 bits of its selector).  The signs (bit 3 of each nibble) join the high
+// bytes before the pairs are formed: byte k of (signs << 4) holds element 2k's sign in
+// its bit 7 and byte k of the signs element 2k+1's, so one permute per four elements
+// lines them up with the high bytes of those elements.  2^X is applied by one
 // bf16x2 multiply, exact while every nonzero product stays a normal bf16
 // (|X| <= 125: 0.5 * 2^X .. 6 * 2^X); beyond that the values are formed in f32 (as
 // exact) and rounded once.
@@ -98,13 +98,15 @@ __device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, int X, uint32_t* o) {
   constexpr uint32_t kHiLo = 0x3F3F3F00u, kHiHi = 0x40404040u, kLoLo = 0xC0800000u, kLoHi = 0xC0804000u;
   if (X >= -125 && X <= 125) {
     const uint32_t m = w & 0x77777777u, sg = w & 0x88888888u, sg4 = sg << 4;
-    const uint32_t h0 = __byte_perm(kHiLo, kHiHi, m), l0 = __byte_perm(kLoLo, kLoHi, m);
-    const uint32_t h1 = __byte_perm(kHiLo, kHiHi, m >> 16), l1 = __byte_perm(kLoLo, kLoHi, m >> 16);
+    // high bytes of elements 0-3 and 4-7, signs included; low bytes likewise
+    const uint32_t h0 = __byte_perm(kHiLo, kHiHi, m) | (__byte_perm(sg4, sg, 0x5140u) & 0x80808080u);
+    const uint32_t h1 = __byte_perm(kHiLo, kHiHi, m >> 16) | (__byte_perm(sg4, sg, 0x7362u) & 0x80808080u);
+    const uint32_t l0 = __byte_perm(kLoLo, kLoHi, m), l1 = __byte_perm(kLoLo, kLoHi, m >> 16);
     uint32_t p[4];
-    p[0] = __byte_perm(l0, h0, 0x5140u) | (__byte_perm(sg4, sg, 0x4000u) & 0x80008000u);
-    p[1] = __byte_perm(l0, h0, 0x7362u) | (__byte_perm(sg4, sg, 0x5111u) & 0x80008000u);
-    p[2] = __byte_perm(l1, h1, 0x5140u) | (__byte_perm(sg4, sg, 0x6222u) & 0x80008000u);
-    p[3] = __byte_perm(l1, h1, 0x7362u) | (__byte_perm(sg4, sg, 0x7333u) & 0x80008000u);
+    p[0] = __byte_perm(l0, h0, 0x5140u);
+    p[1] = __byte_perm(l0, h0, 0x7362u);
+    p[2] = __byte_perm(l1, h1, 0x5140u);
+    p[3] = __byte_perm(l1, h1, 0x7362u);
     const uint32_t sb = (uint32_t)(127 + X) << 7;  // bf16 bits of 2^X
     const uint32_t sbits = sb | (sb << 16);
     __nv_bfloat162 sc;
