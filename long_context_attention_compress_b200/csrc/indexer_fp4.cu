@@ -86,22 +86,23 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
 // Eight E2M1 codes (word nibbles 0..7, element order) times 2^X -> eight bf16, packed in
 // pairs (o[k] = element 2k | element 2k+1 << 16).  The magnitudes come from byte
 // tables by byte permutes (bf16 bits of 0, 0.5, 1, 1.5, 2, 3, 4, 6: high bytes
-// 00 3F 3F 3F 40 40 40 40, low bytes 00 00 80 C0 00 40 80 C0; a permute reads only
-// the low 16 bits of its selector).  The signs (bit 3 of each nibble) join the high
-// bytes before the pairs are formed: byte k of (signs << 4) holds element 2k's sign in
-// its bit 7 and byte k of the signs element 2k+1's, so one permute per four elements
-// lines them up with the high bytes of those elements.  2^X is applied by one
+// 00 3F 3F 3F 40 40 40 40, low bytes 00 00 80 C0 00 40 80 C0; __byte_perm reads only
+// bits 0-2 of each of the four low selector nibbles, so the codes serve as selectors
+// as they are, sign bit included).  The signs (bit 3 of each nibble) join the high
+// bytes before the pairs are formed: byte k of (codes << 4) holds element 2k's sign in
+// its bit 7 and byte k of the codes element 2k+1's, so one permute per four elements
+// and a mask line them up with the high bytes of those elements.  2^X is applied by one
 // bf16x2 multiply, exact while every nonzero product stays a normal bf16
 // (|X| <= 125: 0.5 * 2^X .. 6 * 2^X); beyond that the values are formed in f32 (as
 // exact) and rounded once.
 __device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, int X, uint32_t* o) {
   constexpr uint32_t kHiLo = 0x3F3F3F00u, kHiHi = 0x40404040u, kLoLo = 0xC0800000u, kLoHi = 0xC0804000u;
   if (X >= -125 && X <= 125) {
-    const uint32_t m = w & 0x77777777u, sg = w & 0x88888888u, sg4 = sg << 4;
+    const uint32_t w4 = w << 4, wh = w >> 16;
     // high bytes of elements 0-3 and 4-7, signs included; low bytes likewise
-    const uint32_t h0 = __byte_perm(kHiLo, kHiHi, m) | (__byte_perm(sg4, sg, 0x5140u) & 0x80808080u);
-    const uint32_t h1 = __byte_perm(kHiLo, kHiHi, m >> 16) | (__byte_perm(sg4, sg, 0x7362u) & 0x80808080u);
-    const uint32_t l0 = __byte_perm(kLoLo, kLoHi, m), l1 = __byte_perm(kLoLo, kLoHi, m >> 16);
+    const uint32_t h0 = __byte_perm(kHiLo, kHiHi, w) | (__byte_perm(w4, w, 0x5140u) & 0x80808080u);
+    const uint32_t h1 = __byte_perm(kHiLo, kHiHi, wh) | (__byte_perm(w4, w, 0x7362u) & 0x80808080u);
+    const uint32_t l0 = __byte_perm(kLoLo, kLoHi, w), l1 = __byte_perm(kLoLo, kLoHi, wh);
     uint32_t p[4];
     p[0] = __byte_perm(l0, h0, 0x5140u);
     p[1] = __byte_perm(l0, h0, 0x7362u);
