@@ -205,6 +205,25 @@ __global__ void __launch_bounds__(256) mxfp4_roundtrip_kernel(const bf16* __rest
 
 __device__ unsigned int g_indexer_fp4_error = 0;
 
+namespace {
+// This CTA's (request r, tile t) items in order, from flat index g0 on: one division at
+// the start, then a carry into the next request; a request's visible entry count is
+// read once per request (every role of the kernel walks the same items).
+struct TileWalk {
+  int r, t, nvis;
+  __device__ __forceinline__ TileWalk(long long g0, int tiles, const int32_t* q_pos, int B, int rate, int N)
+      : r((int)(g0 / tiles)), t((int)(g0 % tiles)), nvis(0) {
+    if (r < B) nvis = n_visible(q_pos[r], rate, N);
+  }
+  __device__ __forceinline__ void next(int tiles, const int32_t* q_pos, int B, int rate, int N) {
+    if (++t == tiles) {
+      t = 0;
+      if (++r < B) nvis = n_visible(q_pos[r], rate, N);
+    }
+  }
+};
+}  // namespace
+
 __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
     const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_scales,
     const __grid_constant__ CUtensorMap tm_q, const float* __restrict__ w_idx, const int32_t* __restrict__ q_pos,
@@ -254,10 +273,11 @@ __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
       tc::tma_prefetch_desc(&tm_scales);
       tc::tma_prefetch_desc(&tm_q);
       int it = 0, rq = 0, cur_r = -1;
-      for (long long g = g0; g < g1; ++g) {
-        const int r = (int)(g / tiles_per_req);
-        const int row0 = (int)(g % tiles_per_req) * kFTile;
-        if (row0 >= n_visible(q_pos[r], rate, N)) continue;
+      TileWalk tw(g0, tiles_per_req, q_pos, B, rate, N);
+      for (long long g = g0; g < g1; ++g, tw.next(tiles_per_req, q_pos, B, rate, N)) {
+        const int r = tw.r;
+        const int row0 = tw.t * kFTile;
+        if (row0 >= tw.nvis) continue;
         if (r != cur_r) {
           const int qb = rq & 1;
           if (!tc::mbar_wait(&bars->qempty[qb], ((rq >> 1) & 1) ^ 1, abort)) break;
@@ -288,10 +308,11 @@ __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
       constexpr uint32_t idesc = tc::idesc_bf16_f32(kFTile, kFHeads, false, false);
       const uint32_t k_base = tc::smem_u32(k_smem), q_base = tc::smem_u32(q_smem);
       int it = 0, rq = 0, cur_r = -1, qb = 0;
-      for (long long g = g0; g < g1; ++g) {
-        const int r = (int)(g / tiles_per_req);
-        const int row0 = (int)(g % tiles_per_req) * kFTile;
-        if (row0 >= n_visible(q_pos[r], rate, N)) continue;
+      TileWalk tw(g0, tiles_per_req, q_pos, B, rate, N);
+      for (long long g = g0; g < g1; ++g, tw.next(tiles_per_req, q_pos, B, rate, N)) {
+        const int r = tw.r;
+        const int row0 = tw.t * kFTile;
+        if (row0 >= tw.nvis) continue;
         if (r != cur_r) {
           if (cur_r >= 0) tc::mma_commit(&bars->qempty[qb]);
           qb = rq & 1;
@@ -340,10 +361,11 @@ __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
       }
       tc::named_bar(1, 128);
     };
-    for (long long g = g0; g < g1; ++g) {
-      const int r = (int)(g / tiles_per_req);
-      const int row0 = (int)(g % tiles_per_req) * kFTile;
-      const int nvis = n_visible(q_pos[r], rate, N);
+    TileWalk tw(g0, tiles_per_req, q_pos, B, rate, N);
+    for (long long g = g0; g < g1; ++g, tw.next(tiles_per_req, q_pos, B, rate, N)) {
+      const int r = tw.r;
+      const int row0 = tw.t * kFTile;
+      const int nvis = tw.nvis;
       if (row0 >= nvis) continue;
       if (r != cur_r) {
         if (hist_g && cur_r >= 0) flush(cur_r);
@@ -388,10 +410,9 @@ __global__ void __launch_bounds__(kFThreads, 1) indexer_decode_fp4_kernel(
     const int ci = threadIdx.x - kFConv0;
     const int crw = ci & (kFTile - 1), chh = ci >> 7;
     int it = 0;
-    for (long long g = g0; g < g1; ++g) {
-      const int r = (int)(g / tiles_per_req);
-      const int row0 = (int)(g % tiles_per_req) * kFTile;
-      if (row0 >= n_visible(q_pos[r], rate, N)) continue;
+    TileWalk tw(g0, tiles_per_req, q_pos, B, rate, N);
+    for (long long g = g0; g < g1; ++g, tw.next(tiles_per_req, q_pos, B, rate, N)) {
+      if (tw.t * kFTile >= tw.nvis) continue;
       const int s = it % kFStages, b = it % kFBuf;
       if (!tc::warp_wait(&bars->sfull[s], (it / kFStages) & 1, abort)) break;
       if (!tc::warp_wait(&bars->bempty[b], ((it / kFBuf) & 1) ^ 1, abort)) break;
